@@ -1,0 +1,34 @@
+"""Reference oracle for the AWQ int4 weight-only decode step.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import anything
+from this package.  The product path (the CUDA library and its Python binding)
+never imports, links or executes it, and this package imports nothing from the
+product package: the two share no code, tables, constants or helpers.  Inputs
+reach both sides from the seeded generators only.
+
+Everything here is plain, slow and written to be checked by eye against the
+pages that define the method:
+
+* ``quant``  -- RTN min/max asymmetric int4 quantizer, canonical packing,
+  unpacking and exact dequantization
+  (ATLAS-OLMo-3-32B-Think-v4 model card, "Quantization recipe").
+* ``model``  -- the decoder definition in float64: RMSNorm, QK-norm over the
+  full projections, RoPE with YaRN on the full-attention layers, GQA with a
+  [SWA, SWA, SWA, full] layer pattern, SwiGLU, post-norm residuals, lm_head,
+  greedy argmax (ATLAS model card "Architecture deep-dive"; Olmo 3 32B,
+  "Every architecture field"; LLM Architecture KB "OLMo 3 32B", "Techniques
+  used"; archdb "Olmo-3-1125-32B" field list).
+* ``counts`` -- KV-cache bytes, decode/prefill FLOPs and parameter counts
+  (Olmo 3 32B, "Modelled costs"; archdb KV fields; ATLAS model card "Why the
+  3:1 SWA layout matters for serving").
+* ``brute``  -- a second, loop-by-loop float64 implementation of one layer on
+  tiny shapes, used to pin ``model`` against transposed operands, dropped
+  terms and wrong indices.
+
+Parity status per function is stated in each module header.  Every function is
+pinned by a ``-m "not gpu"`` test except the end-to-end logits, whose
+conventions (rotation pairing, YaRN ramp, final norm) are readings of pages
+that print no worked example: "parity unpinned" beyond the invariants listed in
+``model``.
+"""
