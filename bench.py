@@ -1,0 +1,347 @@
+"""Benchmark: batch-1 decode of the 64-layer OLMo-3-32B-shaped int4 model at 4K context.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl w4a|reference]
+
+One step = one decode token through the whole hot path (embedding, 64 x [QKV
+GEMV, QK-norm + RoPE/YaRN + KV append, GQA attention, O GEMV, post-norm,
+gate/up GEMV + SwiGLU, down GEMV, post-norm], final norm, lm_head, argmax), run
+as one persistent kernel launch.  Greedy: each step consumes the previous
+step's argmax on the device.  The KV cache is pre-filled with N(0,1) bf16 rows
+for positions 0..4095 (sliding-window rings full); timed steps decode positions
+4096 + warmup .. onward.  Weights are random-init (seeded), streamed from HBM
+every token (16.2 GB of int4 + 1.03 GB lm_head, far above the 126 MB L2).
+
+With --gpus N > 1 (launched by torchrun) every rank runs an independent replica
+(the method has no data-path exchange); value = total tokens / max-over-ranks
+device time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "decode tok/s @bs1, 32B-shape W4, 4K ctx; % of B200 HBM roofline"
+CTX = 4096
+SEED = 3
+NOMINAL_HBM_GBS = 8000.0
+
+
+def measured_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes of one decode token (the roofline numerator)
+# ---------------------------------------------------------------------------
+def w4_bytes(n, k):
+    return n * k // 2 + (k // 128) * n * 2 + (k // 128) * n // 2
+
+
+def step_bytes(cfg, pos: int) -> int:
+    """HBM bytes one batch-1 token must move: all int4 matrices (codes, fp16
+    scales, int4 zeros), the bf16 lm_head, K and V of every visible key, the new
+    K/V row per layer, norm gains and the embedding row."""
+    d = cfg.d_model
+    per_layer = (w4_bytes(cfg.qkv_dim, d) + w4_bytes(d, cfg.q_dim) + w4_bytes(2 * cfg.ffn, d)
+                 + w4_bytes(d, cfg.ffn))
+    kv_row = 2 * cfg.kv_dim * 2
+    kv = 0
+    for full in cfg.full_layers:
+        keys = pos + 1 if full else min(pos + 1, cfg.window)
+        kv += (keys - 1) * kv_row + kv_row          # read the old keys, write the new one
+    gains = cfg.n_layers * (cfg.q_dim + cfg.kv_dim + 2 * d) * 4 + d * 4
+    return cfg.n_layers * per_layer + cfg.vocab * d * 2 + kv + gains + d * 2
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU baseline: the oracle, as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+def cpu_baseline(cfg, layers_sample: int = 2):
+    """Time the float64 oracle on `layers_sample` layers of one decode step of
+    the same model at ctx 4096, plus the lm_head, and scale to a full token."""
+    import numpy as np
+    import torch
+    from oracle import model as om
+    from w4_weight_only_b200 import synth
+    sys.path.insert(0, str(ROOT / "tests"))
+    from helpers import oracle_config, np32, np64
+    ocfg = oracle_config(cfg)
+    layers = {}
+    for l in range(layers_sample):
+        raw = synth.layer_float(cfg, SEED, l, "cpu")
+        layers[l] = om.OracleLayer.from_float({k: np32(v) for k, v in raw.items()})
+    emb, head, fin = synth.embed_head(cfg, SEED, "cpu")
+    m = om.OracleModel(ocfg, np64(emb), np64(head), np64(fin), lambda l: layers[l], cache_dense=False)
+    kv = om.OracleKV(om.OracleConfig(**{**ocfg.__dict__, "n_layers": layers_sample,
+                                        "full_layers": ocfg.full_layers[:layers_sample]}), 1, CTX + 1)
+    for l in range(layers_sample):
+        k, v = synth.kv_rows(SEED, l, 0, cfg.n_kv_heads, CTX, cfg.head_dim, "cpu")
+        kv.fill(l, 0, 0, np64(k), np64(v))
+    x = np64(emb[1])
+    t0 = time.perf_counter()
+    for l in range(layers_sample):
+        x = om.layer_forward(ocfg, m.layer(l), l, x, kv, 0, CTX)
+    t_layers = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    om.head(m, x)
+    t_head = time.perf_counter() - t1
+    per_token = t_layers / layers_sample * cfg.n_layers + t_head
+    threads = torch.get_num_threads()
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        threads = max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        pass
+    return {"value": 1.0 / per_token, "unit": "tok/s", "cores": threads, "kind": "oracle",
+            "sample": f"{layers_sample} of {cfg.n_layers} layers of one ctx-{CTX} decode step (dequantize + "
+                      f"float64 matvecs + attention) plus the lm_head, timed, scaled to one token; "
+                      f"host has {len(os.sched_getaffinity(0))} cores"}
+
+
+# ---------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    """--impl reference: the oracle on this host's cores, same metric and config."""
+    from w4_weight_only_b200 import config as wc
+    if rank != 0:
+        return
+    cfg = wc.olmo3_32b()
+    base = cpu_baseline(cfg)
+    v = base["value"]
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "OLMo-3-32B-shaped int4 decode, 64 layers, batch 1, ctx 4096", "batch": 1,
+                       "ctx": CTX},
+            "cpu_baseline": base,
+            "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="w4a", choices=["w4a", "reference"])
+    ap.add_argument("--layers", type=int, default=64, help="model depth (64 = the benchmark model)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    from w4_weight_only_b200 import api, synth
+    from w4_weight_only_b200 import config as wc
+    cfg = wc.olmo3_32b(args.layers)
+
+    # ---- model and cache (not timed) ----
+    emb, head, fin = synth.embed_head(cfg, SEED, "cuda")
+
+    def layer_fn(l):
+        return synth.layer_float(cfg, SEED, l, "cuda")
+
+    model = api.Model.from_float(cfg, emb, head, fin, layer_fn)
+    del head
+    total = args.warmup + args.steps
+    max_ctx = ((CTX + total + 1 + 15) // 16) * 16
+    kv = api.KVCache(cfg, 1, max_ctx)
+    for l in range(cfg.n_layers):
+        k, v = synth.kv_rows(SEED, l, 0, cfg.n_kv_heads, CTX, cfg.head_dim, "cuda")
+        if cfg.full_layers[l]:
+            kv.write(l, 0, 0, k, v)
+        else:
+            W = cfg.window     # positions [0, 4096) fill the ring exactly once
+            kv.write(l, 0, 0, k[:, CTX - W:].contiguous(), v[:, CTX - W:].contiguous())
+        del k, v
+    torch.cuda.synchronize()
+    ws = model.workspace(1)
+    logits = torch.empty((1, cfg.vocab), dtype=torch.float32, device=dev)
+    toks = torch.zeros((total + 1,), dtype=torch.int32, device=dev)
+    toks[0] = 1
+    positions = torch.arange(CTX, CTX + total, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        model.decode_step(kv, toks[i:i + 1], positions[i:i + 1], logits=logits, next_token=toks[i + 1:i + 2])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    api.check(ws)
+
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.warmup, total):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    api.check(ws)
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    tok_s = world * args.steps / (ms_max / 1000.0)
+
+    # roofline of the (only) kernel: algorithmic bytes per launch / its device time
+    bytes_avg = sum(step_bytes(cfg, CTX + i) for i in range(args.warmup, total)) / args.steps
+    peak, peak_src = measured_peaks()
+    achieved = bytes_avg / (ms / args.steps / 1000.0) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_src,
+            "bytes_per_launch": int(bytes_avg), "frac_of_8000_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+            "kernel": "w4a_engine_kernel<1,128> (one launch per token)"}
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        h_tok = torch.zeros((1,), dtype=torch.int32).pin_memory()
+        h_pos = torch.zeros((1,), dtype=torch.int32).pin_memory()
+        h_next = torch.zeros((1,), dtype=torch.int32).pin_memory()
+        d_tok = torch.zeros((1,), dtype=torch.int32, device=dev)
+        d_pos = torch.zeros((1,), dtype=torch.int32, device=dev)
+        d_next = torch.zeros((1,), dtype=torch.int32, device=dev)
+        h_tok[0] = 1
+        n_e2e = args.steps
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(n_e2e):
+            h_pos[0] = CTX + i
+            d_tok.copy_(h_tok, non_blocking=True)
+            d_pos.copy_(h_pos, non_blocking=True)
+            model.decode_step(kv, d_tok, d_pos, logits=logits, next_token=d_next)
+            h_next.copy_(d_next, non_blocking=True)
+            stream.synchronize()
+            h_tok[0] = int(h_next[0])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * n_e2e / (float(te.item()) / 1000.0), "unit": "tok/s",
+               "h2d_bytes_per_step": 8, "d2h_bytes_per_step": 4}
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            base = cpu_baseline(cfg)
+        except Exception as ex:  # reported, never silently dropped
+            base = {"error": repr(ex)}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(tok_s, 2), "unit": "tok/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": f"OLMo-3-32B-shaped int4 (g128, fp16 scale, int4 zero) decode, "
+                                       f"{cfg.n_layers} layers, batch 1, ctx {CTX}..{CTX + total}, greedy",
+                           "batch": 1, "ctx": CTX, "layers": cfg.n_layers,
+                           "l2": "inputs larger than L2: 17.2 GB of weights streamed per token",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roof, "clocks": clk, "gpu_launches": args.steps,
+                "e2e": e2e, "cpu_baseline": base}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

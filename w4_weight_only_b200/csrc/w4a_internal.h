@@ -1,0 +1,130 @@
+// Internal definitions shared by the host entry points and the device engine.
+// Not part of the public C ABI (see include/w4a.h).
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/w4a.h"
+
+namespace w4a {
+
+// ---- engine geometry -------------------------------------------------------
+constexpr int NW = 16;                 // warps per CTA
+constexpr int NT = NW * 32;            // threads per CTA
+constexpr int NSLOT = 2;               // ring slots per warp
+constexpr int SLOT_BYTES = 4352;       // one unit (>= the largest unit below)
+constexpr int RB = 16;                 // output rows per unit (one m16 tile)
+constexpr int W4_KC = 512;             // k per int4 unit
+constexpr int BF_KC = 128;             // k per bf16 unit
+constexpr int GROUP = 128;             // quantization group (the only one supported)
+constexpr int W4_UNIT = RB * W4_KC / 2 + (W4_KC / GROUP) * RB * 2 + (W4_KC / GROUP) * RB / 2;  // 4256
+constexpr int BF_UNIT = RB * BF_KC * 2;                                                      // 4096
+constexpr int ATT_KEYS = 8;            // keys per warp unit
+constexpr int ATT_CTA_KEYS = ATT_KEYS * NW;  // keys per CTA unit (128)
+// Shared-memory budget per CTA (bytes).  x fragments shrink when two
+// 8-column batch tiles are in use, to make room for their split-K slots.
+__host__ __device__ constexpr int xs_cap(int nb) { return nb == 1 ? 57344 : 40960; }
+constexpr int XSUM_BYTES = 6912;       // per-128-group sums of x: [groups][8 * NB]
+__host__ __device__ constexpr int wsp_bytes(int nb) { return NW * 2 * 32 * 4 * nb * 4; }
+constexpr int MAX_B = 16;
+constexpr int MAX_LAYERS = 128;
+constexpr int MAX_GQ = 8;              // query heads per KV head supported by the attention tile
+
+static_assert(W4_UNIT == 4256, "int4 unit size");
+static_assert(W4_UNIT <= SLOT_BYTES && BF_UNIT <= SLOT_BYTES, "slot too small");
+
+// ---- device error word bits -----------------------------------------------
+enum : uint32_t {
+  EW_MBAR_TIMEOUT = 1u << 0,     // a ring slot never completed
+  EW_BARRIER_TIMEOUT = 1u << 1,  // a grid barrier never completed
+  EW_DRAIN_TIMEOUT = 1u << 2,    // in-flight copies did not land before exit
+  EW_BAD_SHAPE = 1u << 3,        // device-side shape check failed
+  EW_BAD_POS = 1u << 4,          // a position outside the cache
+};
+
+// ---- engine modes / phase kinds --------------------------------------------
+enum Mode : int { MODE_DECODE = 0, MODE_GEMV = 1, MODE_ATTN = 2 };
+enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_ATTN = 2, PK_ARGMAX = 3 };
+enum XSrc : int { XS_BF16 = 0, XS_EMBED = 1, XS_RESID = 2, XS_FINAL = 3 };
+enum Epi : int { EPI_Y = 0, EPI_Y_SUMSQ = 1, EPI_SILU = 2, EPI_LOGITS = 3 };
+
+struct LayerPtrs {
+  const uint8_t* qkv;
+  const uint8_t* o;
+  const uint8_t* gu;
+  const uint8_t* down;
+  const float* q_norm;
+  const float* k_norm;
+  const float* attn_norm;
+  const float* ffn_norm;
+};
+
+// Workspace carve-up (device pointers), filled on the host.
+struct Workspace {
+  uint32_t* ctl;        // [0] barrier, [1] exit, [2] error word, [3] argmax counter
+  uint32_t* seg_ctr;    // per-segment arrival counters
+  float* gpart;         // GEMV split pieces [NS][nrb][2][RB * 8 * NB]
+  float* apart;         // attention pieces [NC][2][MAX_GQ * (HD + 2)]
+  float* amax_val;      // argmax pieces [NC][B]
+  int32_t* amax_idx;
+  float* y_qkv;         // [B][qkv_dim]
+  uint16_t* o;          // [B][q_dim] bf16
+  float* a;             // [B][d]
+  uint16_t* h;          // [B][ffn] bf16
+  float* f;             // [B][d]
+  float* xA;            // [B][d]
+  float* xB;            // [B][d]
+  float* ss_qkv;        // [nrb_qkv][B]
+  float* ss_a;          // [nrb_d][B]
+  float* ss_f;          // [nrb_d][B]
+  int32_t* pos_seq;     // prefill positions [T]
+};
+
+struct EngineParams {
+  int mode;
+  int phase_begin, phase_end;
+  int nc;               // CTAs in the grid
+  // model dims
+  int d, nq, nkv, hd, ffn, vocab, window, n_layers;
+  float eps;
+  int final_norm;
+  double inv_freq[2][64];   // [0] sliding-window layers, [1] full layers
+  float mscale[2];
+  uint8_t full[MAX_LAYERS];
+  // weights
+  const uint16_t* embed;
+  const uint8_t* lm_head;
+  const float* final_gain;
+  LayerPtrs layers[MAX_LAYERS];
+  // KV cache
+  uint8_t* kv_base;
+  int kv_batch, max_ctx;
+  uint64_t kv_off[MAX_LAYERS];   // byte offset of layer l's K region (V follows it)
+  int kv_slots[MAX_LAYERS];
+  // step inputs / outputs
+  const int32_t* tokens;
+  const int32_t* pos;
+  int pos_const;        // >= 0: every sequence is at this position (prefill); else read pos[]
+  int B, seq0;
+  float* logits;
+  int32_t* next_token;
+  float* dump;
+  Workspace ws;
+  // standalone GEMV
+  const uint8_t* g_blob;
+  const uint16_t* g_x;
+  int g_n, g_k, g_epi;
+  void* g_out;
+  float* g_aux;
+  // standalone attention
+  const uint16_t* a_q;
+  const uint16_t* a_k;
+  const uint16_t* a_v;
+  uint16_t* a_out;
+  int a_slots, a_window;
+};
+
+// Slots of a layer's ring / linear cache.
+inline int64_t kv_slots(int full, int window, int max_ctx) { return full ? max_ctx : window; }
+
+}  // namespace w4a

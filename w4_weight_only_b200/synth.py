@@ -1,0 +1,91 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle runs.
+
+Holds none of the method's arithmetic: it only draws random numbers, so that
+the CUDA path and the oracle receive identical inputs.  Every tensor is drawn
+from its own ``torch.Generator`` seeded from (seed, name, index...) through
+SHA-256, so any single layer can be regenerated alone, on the CPU or on the GPU
+(the two devices give different streams; a test uses one device for both
+sides).
+
+Recipes (the pages' shapes with random-init values; no checkpoint is used):
+* linear weights  N(0, 0.02) fp32, quantized by the consumer;
+* norm gains      1 + N(0, 0.1) fp32;
+* embedding, lm_head N(0, 0.02) rounded to bf16;
+* prompts         uniform token ids in [0, vocab);
+* a pre-filled KV cache N(0, 1) bf16 (already-rotated keys);
+* GEMV activations N(0, 1) bf16; raw attention projections N(0, 1) fp32.
+"""
+from __future__ import annotations
+
+import hashlib
+
+import torch
+
+
+def seed_of(*keys) -> int:
+    h = hashlib.sha256(repr(keys).encode()).digest()
+    return int.from_bytes(h[:8], "little") & ((1 << 63) - 1)
+
+
+def _gen(device, *keys) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed_of(*keys))
+    return g
+
+
+def normal(shape, device, std: float, mean: float, *keys) -> torch.Tensor:
+    t = torch.randn(shape, generator=_gen(device, *keys), device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t
+
+
+def layer_float(cfg, seed: int, l: int, device="cpu") -> dict:
+    """fp32 weights of layer l: qkv [q+2kv, d] ([Q; K; V] rows), o [d, q],
+    gate_up [2 ffn, d] ([gate; up] rows), down [d, ffn] and the four gains."""
+    d, qd, kvd, f = cfg.d_model, cfg.n_heads * cfg.head_dim, cfg.n_kv_heads * cfg.head_dim, cfg.ffn
+    return {
+        "qkv": normal((qd + 2 * kvd, d), device, 0.02, 0.0, seed, "qkv", l),
+        "o": normal((d, qd), device, 0.02, 0.0, seed, "o", l),
+        "gate_up": normal((2 * f, d), device, 0.02, 0.0, seed, "gate_up", l),
+        "down": normal((d, f), device, 0.02, 0.0, seed, "down", l),
+        "q_norm": normal((qd,), device, 0.1, 1.0, seed, "q_norm", l),
+        "k_norm": normal((kvd,), device, 0.1, 1.0, seed, "k_norm", l),
+        "post_attn_norm": normal((d,), device, 0.1, 1.0, seed, "post_attn_norm", l),
+        "post_ffn_norm": normal((d,), device, 0.1, 1.0, seed, "post_ffn_norm", l),
+    }
+
+
+def embed_head(cfg, seed: int, device="cpu"):
+    """(embedding bf16 [V, d], lm_head bf16 [V, d], final norm gains fp32 [d])."""
+    e = normal((cfg.vocab, cfg.d_model), device, 0.02, 0.0, seed, "embed").to(torch.bfloat16)
+    h = normal((cfg.vocab, cfg.d_model), device, 0.02, 0.0, seed, "lm_head").to(torch.bfloat16)
+    g = normal((cfg.d_model,), device, 0.1, 1.0, seed, "final_norm")
+    return e, h, g
+
+
+def token_ids(seed: int, n: int, vocab: int, device="cpu", *keys) -> torch.Tensor:
+    return torch.randint(0, vocab, (n,), generator=_gen(device, seed, "tokens", *keys), device=device,
+                         dtype=torch.int64).to(torch.int32)
+
+
+def kv_rows(seed: int, l: int, b: int, n_kv: int, n: int, hd: int, device="cpu"):
+    """(K, V) bf16 [n_kv, n, hd] N(0, 1): pre-filled cache rows of sequence b, layer l."""
+    k = normal((n_kv, n, hd), device, 1.0, 0.0, seed, "kv_k", l, b).to(torch.bfloat16)
+    v = normal((n_kv, n, hd), device, 1.0, 0.0, seed, "kv_v", l, b).to(torch.bfloat16)
+    return k, v
+
+
+def gemv_case(seed: int, n: int, k: int, batch: int, device="cpu"):
+    """(W fp32 [n, k] N(0, 0.02), x bf16 [batch, k] N(0, 1))."""
+    W = normal((n, k), device, 0.02, 0.0, seed, "gemv_w", n, k)
+    x = normal((batch, k), device, 1.0, 0.0, seed, "gemv_x", n, k, batch).to(torch.bfloat16)
+    return W, x
+
+
+def weight_rows(seed: int, n: int, k: int, rows, device="cpu"):
+    """Selected rows of the gemv_case weight (same values, drawn in full on
+    ``device``; used when only a sample of rows is checked)."""
+    return gemv_case(seed, n, k, 1, device)[0][rows]
