@@ -1,10 +1,11 @@
 """GPU parity of QK-norm + rotation + KV append (w4a_qk_prep) and GQA decode
 attention (w4a_attn_decode) against the oracle.
 
-Tolerance.  The GPU rounds q and the new k, v to bf16 (2^-9 relative), feeds
-the softmax weights to the tensor core as bf16, and rounds o to bf16; each is
-an independent ~0.4% relative perturbation of o, so the max error over a head
-stays near 1-2% of RMS(o).  Bound used: 3e-2 * RMS(o_ref).
+Tolerance.  The cache holds k and v in bf16 (at most 2^-8 relative error
+per element) and the standalone q input is bf16; q and the softmax weights
+enter the tensor cores as hi + lo bf16 pairs and o is rounded to bf16 once.
+Each bf16 rounding is an independent <= 0.4% relative perturbation, so the
+max error over a head stays near 1-2% of RMS(o).  Bound: 3e-2 * RMS(o_ref).
 """
 import numpy as np
 import pytest
@@ -133,6 +134,8 @@ def test_qk_prep_append_matches_oracle(built_lib, cuda):
         _abi.call("w4a_kv_read", api._p(kc), api._p(vc), 1, nkv, hd, slots, 0, pos_v % slots, 1, api._p(k_rows),
                   api._p(v_rows), api._stream())
         qo, ko = om.qk_prep(oracle_config(cfg), np64(q_raw[0]), np64(k_raw[0]), np64(qg), np64(kg), pos_v, full)
-        assert max_rel_to_rms(np64(q[0]), qo) <= 1e-2
-        assert max_rel_to_rms(np64(k_rows[:, 0]), ko) <= 1e-2
+        # bf16 outputs: round-to-nearest error is at most 2^-8 of the value
+        for got, ref in ((np64(q[0]), qo), (np64(k_rows[:, 0]), ko)):
+            slack = 1e-5 * np.sqrt(np.mean(ref * ref))
+            assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + slack)
         assert np.array_equal(np64(v_rows[:, 0]).reshape(-1), np64(v_raw[0].to(torch.bfloat16)))

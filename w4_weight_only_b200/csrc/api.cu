@@ -583,6 +583,7 @@ int w4a_kv_layer(const W4AConfig* cfg, int batch, int max_ctx, int layer, size_t
 
 static int kv_copy(uint16_t* cache, const uint16_t* other, int batch, int nkv, int hd, int slots, int b, int slot0, int n,
                    int to_cache, void* stream) {
+  if (n == 0 && slot0 >= 0 && slot0 <= slots && b >= 0 && b < batch) return W4A_OK;  // nothing to copy
   if (!cache || !other) return fail(W4A_ERR_ARG, "null pointer");
   if (b < 0 || b >= batch || slot0 < 0 || n < 0 || slot0 + n > slots || nkv < 1 || hd % 8)
     return fail(W4A_ERR_SHAPE, "rows [%d, %d) of sequence %d outside the region", slot0, slot0 + n, b);

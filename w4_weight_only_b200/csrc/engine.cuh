@@ -12,9 +12,12 @@
 //
 // GEMV math: the int4 codes of a unit are laid out as mma.sync A fragments
 // (16 rows x 16 k per warp-wide word).  A LOP3 turns each nibble q into the
-// bf16 value 128 + q (exact), the tensor core accumulates sum_k (128+q) x_k
+// fp16 value 1024 + q (exact), the tensor core accumulates sum_k (1024+q) x_k
 // in fp32 per 128-group, and the group is closed in fp32 with
-// s * (acc - (128 + z) * sum_k x_k).  x is the mma B operand (batch = n).
+// s * (acc - (1024 + z) * sum_k x_k).  x is the mma B operand (batch = n),
+// held in fp16 (11-bit significand) after an exact power-of-two range
+// scaling that is undone when a partial leaves the warp.  The bf16 lm_head
+// takes bf16 x.
 //
 // Split-K is deterministic: pieces of one 16-row block computed by different
 // warps are summed in warp order in shared memory, pieces from different
@@ -74,6 +77,7 @@ struct PD {
   int rows_valid;
   // attention
   int type, newkv, slots, seqoff;
+  int out_f16;   // SiLU / attention outputs in fp16 (decode workspace) rather than bf16
   const uint8_t* kc;
   const uint8_t* vc;
   uint16_t* aout;
@@ -96,8 +100,11 @@ struct Lay {
   static constexpr int FLAGS = SST + 2 * (MAX_SEG + 1) * 4;
   static constexpr int TOTAL = FLAGS + 64;
   static constexpr int APW_BYTES = xs_cap(NB) + XSUM_BYTES + wsp_bytes(NB);  // attention warp partials
+  static constexpr int QF = XS + NW * MAX_GQ * (128 + 2) * 4;                 // q fragments (after the partials)
 };
 static_assert(Lay<1>::TOTAL <= 232448 && Lay<2>::TOTAL <= 232448, "shared memory budget");
+static_assert(Lay<1>::QF + 4096 <= Lay<1>::XS + Lay<1>::APW_BYTES, "q fragments overlap");
+static_assert(Lay<2>::QF + 4096 <= Lay<2>::XS + Lay<2>::APW_BYTES, "q fragments overlap");
 
 __device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
   return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
@@ -141,20 +148,20 @@ __device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint4* xs4, i
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t w = u4_word(i < 4 ? w0 : w1, i & 3);
-      const uint32_t a0 = lop3_and_or(w, 0x000F000Fu, 0x43004300u);
-      const uint32_t a1 = lop3_and_or(w >> 4, 0x000F000Fu, 0x43004300u);
-      const uint32_t a2 = lop3_and_or(w >> 8, 0x000F000Fu, 0x43004300u);
-      const uint32_t a3 = lop3_and_or(w >> 12, 0x000F000Fu, 0x43004300u);
+      const uint32_t a0 = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+      const uint32_t a1 = lop3_and_or(w >> 4, 0x000F000Fu, 0x64006400u);
+      const uint32_t a2 = lop3_and_or(w >> 8, 0x000F000Fu, 0x64006400u);
+      const uint32_t a3 = lop3_and_or(w >> 12, 0x000F000Fu, 0x64006400u);
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         const uint4& x = xv[nb][i >> 1];
-        mma_16816(c[nb], a0, a1, a2, a3, (i & 1) ? x.z : x.x, (i & 1) ? x.w : x.y);
+        mma_16816_f16(c[nb], a0, a1, a2, a3, (i & 1) ? x.z : x.x, (i & 1) ? x.w : x.y);
       }
     }
     const float sl = half_bits_to_f32(sc[grp * 16 + g]);
     const float sh = half_bits_to_f32(sc[grp * 16 + g + 8]);
-    const float zl = 128.f + float((zw[grp * 2] >> (4 * g)) & 15u);
-    const float zh = 128.f + float((zw[grp * 2 + 1] >> (4 * g)) & 15u);
+    const float zl = 1024.f + float((zw[grp * 2] >> (4 * g)) & 15u);
+    const float zh = 1024.f + float((zw[grp * 2 + 1] >> (4 * g)) & 15u);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       const float* xsr = xsum + (grp0 + grp) * (8 * NB) + nb * 8 + 2 * t;
@@ -230,6 +237,7 @@ struct Engine {
   __device__ float* wsp() const { return reinterpret_cast<float*>(sm + L::WSP); }
   __device__ float* apw() const { return reinterpret_cast<float*>(sm + L::XS); }
   __device__ float* qs() const { return reinterpret_cast<float*>(sm + L::QS); }
+  __device__ uint4* qf() const { return reinterpret_cast<uint4*>(sm + L::QF); }
   __device__ uint16_t* kn() const { return reinterpret_cast<uint16_t*>(sm + L::KNV); }
   __device__ uint16_t* vn() const { return reinterpret_cast<uint16_t*>(sm + L::KNV) + 128; }
   __device__ float* red() const { return reinterpret_cast<float*>(sm + L::RED); }
@@ -332,6 +340,7 @@ struct Engine {
       d.kc = P.kv_base + P.kv_off[l];
       d.vc = d.kc + (size_t)P.kv_batch * P.nkv * d.slots * HD * 2;
       d.aout = P.ws.o;
+      d.out_f16 = 1;
       return d;
     }
     d.kind = PK_GEMV_W4;
@@ -362,7 +371,7 @@ struct Engine {
       d.blob = lw.o;
       d.n = dm;
       d.k = P.nq * P.hd;
-      d.xsrc = XS_BF16;
+      d.xsrc = XS_F16;
       d.xbf = P.ws.o;
       d.xbf_stride = P.nq * P.hd;
       d.epi = EPI_Y_SUMSQ;
@@ -383,11 +392,12 @@ struct Engine {
       d.epi = EPI_SILU;
       d.hout = P.ws.h;
       d.hstride = P.ffn;
+      d.out_f16 = 1;
     } else {
       d.blob = lw.down;
       d.n = dm;
       d.k = P.ffn;
-      d.xsrc = XS_BF16;
+      d.xsrc = XS_F16;
       d.xbf = P.ws.h;
       d.xbf_stride = P.ffn;
       d.epi = EPI_Y_SUMSQ;
@@ -643,25 +653,59 @@ struct Engine {
       }
       __syncthreads();
     }
-    // x fragments for [kbase, kbase + klen)
+    // x fragments for [kbase, kbase + klen): fp16 for the int4 GEMVs, bf16 for the lm_head
+    const bool f16 = (d.kind == PK_GEMV_W4);
     uint16_t* xh = reinterpret_cast<uint16_t*>(xs());
+    uint32_t* xmax = reinterpret_cast<uint32_t*>(rd + 32);   // |x| max bits per batch row
+    float* xscale = rd + 48;                                 // 2^e per batch row
+    if (tid < MAX_B) {
+      xmax[tid] = 0u;
+      xscale[tid] = 1.f;
+    }
+    __syncthreads();
     const int xrow = klen / 2 + 16;
     const int total = B * klen;
-    for (int idx = tid; idx < total; idx += NT) {
-      const int bb = idx / klen, kl = idx - bb * klen, k = kbase + kl;
-      uint16_t hb;
-      if (d.xsrc == XS_BF16) {
-        hb = __ldcg(d.xbf + (size_t)bb * d.xbf_stride + k);
-      } else if (d.xsrc == XS_EMBED) {
-        int tok = P.tokens[bb];
-        tok = tok < 0 ? 0 : (tok >= P.vocab ? P.vocab - 1 : tok);
-        hb = P.embed[(size_t)tok * dm + k];
-      } else {
-        float x = __ldcg(d.xres + (size_t)bb * dm + k) + __ldcg(d.vres + (size_t)bb * dm + k) * rd[bb] * d.gain[k];
-        if (d.xsrc == XS_FINAL && d.gain2 != nullptr) x = x * rd[16 + bb] * d.gain2[k];
-        hb = f32_to_bf16(x);
+    {
+      int curb = -1;
+      float m = 0.f;
+      for (int idx = tid; idx < total; idx += NT) {
+        const int bb = idx / klen, kl = idx - bb * klen;
+        if (bb != curb) {
+          if (curb >= 0) atomicMax(xmax + curb, __float_as_uint(m));
+          curb = bb;
+          m = 0.f;
+        }
+        const float v = load_x(d, bb, kbase + kl);
+        m = fmaxf(m, fabsf(v));
+        xh[xfrag_half(bb, kl, xrow)] = f16 ? f32_to_f16(v) : f32_to_bf16(v);
       }
-      xh[xfrag_half(bb, kl, xrow)] = hb;
+      if (curb >= 0) atomicMax(xmax + curb, __float_as_uint(m));
+    }
+    __syncthreads();
+    if (f16) {
+      // fp16 range guard: rows whose max |x| reaches 2^15 are scaled by an exact
+      // power of two (undone on the partial sums in flush()).
+      bool any = false;
+      for (int bb = 0; bb < B; ++bb) any |= __uint_as_float(xmax[bb]) >= 32768.f;
+      if (any) {
+        for (int idx = tid; idx < total; idx += NT) {
+          const int bb = idx / klen, kl = idx - bb * klen;
+          const float mx = __uint_as_float(xmax[bb]);
+          if (!(mx >= 32768.f)) continue;
+          int ex;
+          frexpf(mx, &ex);
+          xh[xfrag_half(bb, kl, xrow)] = f32_to_f16(ldexpf(load_x(d, bb, kbase + kl), 15 - ex));
+        }
+        __syncthreads();
+        if (tid < B) {
+          const float mx = __uint_as_float(xmax[tid]);
+          if (mx >= 32768.f) {
+            int ex;
+            frexpf(mx, &ex);
+            xscale[tid] = ldexpf(1.f, ex - 15);
+          }
+        }
+      }
     }
     // residual copy and hidden-state dump (one CTA, the whole width)
     if (cta == 0 && (d.xdst != nullptr || d.dump != nullptr)) {
@@ -669,9 +713,7 @@ struct Engine {
         const int bb = idx / dm, k = idx - bb * dm;
         float x;
         if (d.xsrc == XS_EMBED) {
-          int tok = P.tokens[bb];
-          tok = tok < 0 ? 0 : (tok >= P.vocab ? P.vocab - 1 : tok);
-          x = bf16_to_f32(P.embed[(size_t)tok * dm + k]);
+          x = bf16_to_f32(P.embed[(size_t)clamp_token(bb) * dm + k]);
         } else {
           x = __ldcg(d.xres + idx) + __ldcg(d.vres + idx) * rd[bb] * d.gain[k];
         }
@@ -684,7 +726,7 @@ struct Engine {
         if (P.tokens[bb] < 0 || P.tokens[bb] >= P.vocab) set_error(EW_BAD_SHAPE);
     }
     __syncthreads();
-    // per-(batch, 128-group) sums of the bf16 x values (zero for unused columns)
+    // per-(batch, 128-group) sums of the x values as stored (zero for unused columns)
     float* xsm = xsum();
     const int ngr = klen / GROUP;
     for (int pr = warp; pr < ngr * 8 * NB; pr += NW) {
@@ -692,13 +734,40 @@ struct Engine {
       float s = 0.f;
       if (bb < B) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s += bf16_to_f32(xh[xfrag_half(bb, grp * GROUP + lane * 4 + e, xrow)]);
+        for (int e = 0; e < 4; ++e) {
+          const uint16_t hv = xh[xfrag_half(bb, grp * GROUP + lane * 4 + e, xrow)];
+          s += f16 ? half_bits_to_f32(hv) : bf16_to_f32(hv);
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (lane == 0) xsm[pr] = s;
     }
     __syncthreads();
+  }
+
+  __device__ int clamp_token(int bb) const {
+    const int tok = P.tokens[bb];
+    return tok < 0 ? 0 : (tok >= P.vocab ? P.vocab - 1 : tok);
+  }
+
+  // One activation of the GEMV input (fp32), from the phase's source.
+  __device__ float load_x(const PD& d, int bb, int k) const {
+    const int dm = P.d;
+    const float* rd = red();
+    switch (d.xsrc) {
+      case XS_BF16:
+        return bf16_to_f32(__ldcg(d.xbf + (size_t)bb * d.xbf_stride + k));
+      case XS_F16:
+        return half_bits_to_f32(__ldcg(d.xbf + (size_t)bb * d.xbf_stride + k));
+      case XS_EMBED:
+        return bf16_to_f32(P.embed[(size_t)clamp_token(bb) * dm + k]);
+      default: {
+        float x = __ldcg(d.xres + (size_t)bb * dm + k) + __ldcg(d.vres + (size_t)bb * dm + k) * rd[bb] * d.gain[k];
+        if (d.xsrc == XS_FINAL && d.gain2 != nullptr) x = x * rd[16 + bb] * d.gain2[k];
+        return x;
+      }
+    }
   }
 
   __device__ int expected_pieces(const PD& d, int rb) const {
@@ -727,12 +796,12 @@ struct Engine {
           const float s2 = v[nb][2] / (1.f + expf(-v[nb][2]));
           const float s3 = v[nb][3] / (1.f + expf(-v[nb][3]));
           if (b0 < B) {
-            d.hout[(size_t)b0 * d.hstride + j0] = f32_to_bf16(s0 * u0);
-            d.hout[(size_t)b0 * d.hstride + j1] = f32_to_bf16(s2 * u2);
+            d.hout[(size_t)b0 * d.hstride + j0] = d.out_f16 ? f32_to_f16(s0 * u0) : f32_to_bf16(s0 * u0);
+            d.hout[(size_t)b0 * d.hstride + j1] = d.out_f16 ? f32_to_f16(s2 * u2) : f32_to_bf16(s2 * u2);
           }
           if (b1 < B) {
-            d.hout[(size_t)b1 * d.hstride + j0] = f32_to_bf16(s1 * u1);
-            d.hout[(size_t)b1 * d.hstride + j1] = f32_to_bf16(s3 * u3);
+            d.hout[(size_t)b1 * d.hstride + j0] = d.out_f16 ? f32_to_f16(s1 * u1) : f32_to_bf16(s1 * u1);
+            d.hout[(size_t)b1 * d.hstride + j1] = d.out_f16 ? f32_to_f16(s3 * u3) : f32_to_bf16(s3 * u3);
           }
         }
       }
@@ -850,8 +919,20 @@ struct Engine {
     cta_combine(d, a, b);
   }
 
-  __device__ void flush(const PD& d, long long seg, const float (&acc)[NB][4], long long wa, long long wb,
+  __device__ void flush(const PD& d, long long seg, float (&acc)[NB][4], long long wa, long long wb,
                         float* my) {
+    if (d.kind == PK_GEMV_W4) {
+      const float* xscale = red() + 48;
+      const int t = lane & 3;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        const float s0 = xscale[nb * 8 + 2 * t], s1 = xscale[nb * 8 + 2 * t + 1];
+        acc[nb][0] *= s0;
+        acc[nb][1] *= s1;
+        acc[nb][2] *= s0;
+        acc[nb][3] *= s1;
+      }
+    }
     const long long u0 = seg * d.kps;
     if (u0 >= wa && u0 + d.kps <= wb) {
       piece_out(d, seg, acc);
@@ -979,6 +1060,18 @@ struct Engine {
       for (int idx = tid; idx < GQ * HD; idx += NT) q[idx] = bf16_to_f32(qin[idx]) * qscale;
     }
     __syncthreads();
+    // q as hi + lo bf16 mma A fragments: {a0 hi, a2 hi, a0 lo, a2 lo} per (k-step, lane)
+    if (tid < (HD / 16) * 32) {
+      const int s = tid >> 5, ln = tid & 31, gg = ln >> 2, t = ln & 3;
+      uint4 f = make_uint4(0u, 0u, 0u, 0u);
+      if (gg < GQ) {
+        const float* qr = q + gg * HD + 16 * s + 2 * t;
+        split_bf16x2(qr[0], qr[1], f.x, f.z);
+        split_bf16x2(qr[8], qr[9], f.y, f.w);
+      }
+      qf()[tid] = f;
+    }
+    __syncthreads();
   }
 
   __device__ void run_attn(const PD& d) {
@@ -1001,18 +1094,7 @@ struct Engine {
       const long long jnew = st[seg] + (sn_ >= 0 ? sn_ / ATT_CTA_KEYS : 0);
       const bool own_new = d.newkv && sn_ >= 0 && jnew >= u && jnew < run_end;
       attn_prologue(d, seg, own_new);
-      // this warp's query fragments
-      uint32_t qa0[HD / 16], qa2[HD / 16];
-      const float* q = qs();
-#pragma unroll
-      for (int s = 0; s < HD / 16; ++s) {
-        if (g < GQ) {
-          qa0[s] = pack_bf16x2(q[g * HD + 16 * s + 2 * t], q[g * HD + 16 * s + 2 * t + 1]);
-          qa2[s] = pack_bf16x2(q[g * HD + 16 * s + 2 * t + 8], q[g * HD + 16 * s + 2 * t + 9]);
-        } else {
-          qa0[s] = qa2[s] = 0u;
-        }
-      }
+      const uint4* qfr = qf();
       float m = -INFINITY, lsum = 0.f;
       float o[HD / 8][4];
 #pragma unroll
@@ -1040,8 +1122,11 @@ struct Engine {
         for (int s = 0; s < HD / 16; s += 2) {
           uint32_t k0, k1, k2, k3;
           ldsm_x4(k0, k1, k2, k3, Ks + r * HD * 2 + (((2 * s + mi) ^ r) << 4));
-          mma_16816(sc, qa0[s], 0u, qa2[s], 0u, k0, k1);
-          mma_16816(sc, qa0[s + 1], 0u, qa2[s + 1], 0u, k2, k3);
+          const uint4 f0 = qfr[s * 32 + lane], f1 = qfr[(s + 1) * 32 + lane];
+          mma_16816(sc, f0.x, 0u, f0.y, 0u, k0, k1);
+          mma_16816(sc, f0.z, 0u, f0.w, 0u, k0, k1);
+          mma_16816(sc, f1.x, 0u, f1.y, 0u, k2, k3);
+          mma_16816(sc, f1.z, 0u, f1.w, 0u, k2, k3);
         }
         const int ka = key0 + 2 * t;
         const float s0 = (ka < Lk) ? sc[0] : -INFINITY;
@@ -1059,15 +1144,20 @@ struct Engine {
           o[n][0] *= alpha;
           o[n][1] *= alpha;
         }
-        const uint32_t pa = pack_bf16x2(p0, p1);
+        uint32_t pa, pl;
+        split_bf16x2(p0, p1, pa, pl);
 #pragma unroll
         for (int q4 = 0; q4 < HD / 32; ++q4) {
           uint32_t v0, v1, v2, v3;
           ldsm_x4_t(v0, v1, v2, v3, Vs + r * HD * 2 + (((4 * q4 + mi) ^ r) << 4));
           mma_1688(o[4 * q4 + 0], pa, 0u, v0);
+          mma_1688(o[4 * q4 + 0], pl, 0u, v0);
           mma_1688(o[4 * q4 + 1], pa, 0u, v1);
+          mma_1688(o[4 * q4 + 1], pl, 0u, v1);
           mma_1688(o[4 * q4 + 2], pa, 0u, v2);
+          mma_1688(o[4 * q4 + 2], pl, 0u, v2);
           mma_1688(o[4 * q4 + 3], pa, 0u, v3);
+          mma_1688(o[4 * q4 + 3], pl, 0u, v3);
         }
         release_slot();
       }
@@ -1113,7 +1203,7 @@ struct Engine {
         os += e * wp[w * PW + h * (HD + 2) + dd];
       }
       if (!split) {
-        out[h * HD + dd] = f32_to_bf16(os / ls);
+        out[h * HD + dd] = d.out_f16 ? f32_to_f16(os / ls) : f32_to_bf16(os / ls);
       } else {
         piece[h * (HD + 2) + dd] = os;
         if (dd == 0) {
@@ -1150,7 +1240,7 @@ struct Engine {
         ls += e * __ldcg(pc + HD + 1);
         os += e * __ldcg(pc + dd);
       }
-      out[h * HD + dd] = f32_to_bf16(os / ls);
+      out[h * HD + dd] = d.out_f16 ? f32_to_f16(os / ls) : f32_to_bf16(os / ls);
     }
     if (tid == 0) P.ws.seg_ctr[seg] = 0u;
   }

@@ -45,7 +45,7 @@ enum : uint32_t {
 // ---- engine modes / phase kinds --------------------------------------------
 enum Mode : int { MODE_DECODE = 0, MODE_GEMV = 1, MODE_ATTN = 2 };
 enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_ATTN = 2, PK_ARGMAX = 3 };
-enum XSrc : int { XS_BF16 = 0, XS_EMBED = 1, XS_RESID = 2, XS_FINAL = 3 };
+enum XSrc : int { XS_BF16 = 0, XS_EMBED = 1, XS_RESID = 2, XS_FINAL = 3, XS_F16 = 4 };
 enum Epi : int { EPI_Y = 0, EPI_Y_SUMSQ = 1, EPI_SILU = 2, EPI_LOGITS = 3 };
 
 struct LayerPtrs {
@@ -68,9 +68,9 @@ struct Workspace {
   float* amax_val;      // argmax pieces [NC][B]
   int32_t* amax_idx;
   float* y_qkv;         // [B][qkv_dim]
-  uint16_t* o;          // [B][q_dim] bf16
+  uint16_t* o;          // [B][q_dim] fp16 (attention output)
   float* a;             // [B][d]
-  uint16_t* h;          // [B][ffn] bf16
+  uint16_t* h;          // [B][ffn] fp16 (SwiGLU output)
   float* f;             // [B][d]
   float* xA;            // [B][d]
   float* xB;            // [B][d]
