@@ -6,7 +6,8 @@ effects: per 128-group the tensor core sums products of size <= 143 |x| and the
 zero point is removed as (128 + z) * sum(x), cancelling about 7 bits; summed
 over K/128 groups this stays below 1e-4 relative to RMS(y).  The bound used,
 2e-3 * RMS(y_ref) on the max error, leaves a 20x margin.  SiLU*mul outputs are
-rounded to bf16 (2^-8 relative), so that epilogue gets 1e-2 * RMS.
+rounded to bf16, so that epilogue is checked element-wise: |err| <= 2^-8 |ref|
+plus 1e-3 * RMS(ref) for the GEMV error.
 """
 import numpy as np
 import pytest
@@ -88,7 +89,9 @@ def test_gemv_silu_mul_epilogue(built_lib, cuda, ffn, k, batch):
     gate = _ref_rows(W.cpu(), x.cpu(), js)
     up = _ref_rows(W.cpu(), x.cpu(), js + ffn)
     ref = gate / (1.0 + np.exp(-gate)) * up
-    assert max_rel_to_rms(h[:, js], ref) <= 1e-2
+    # bf16 output: round-to-nearest error <= 2^-8 of the value, plus the GEMV's own error
+    slack = 1e-3 * np.sqrt(np.mean(ref * ref))
+    assert np.all(np.abs(h[:, js] - ref) <= 2.0 ** -8 * np.abs(ref) + slack)
 
 
 def test_gemv_deterministic(built_lib, cuda):

@@ -343,6 +343,19 @@ class Model:
         check(ws)
 
 
+class Trace:
+    """Per-phase, per-CTA device timestamps of decode launches (w4a_trace)."""
+
+    def __init__(self, n_phases: int, device=None):
+        self.n_sms = torch.cuda.get_device_properties(device or 0).multi_processor_count
+        self.buf = torch.zeros((n_phases, self.n_sms, 4), dtype=torch.int64, device=device or "cuda")
+        call("w4a_trace", _p(self.buf), self.buf.numel() * 8)
+
+    def stop(self):
+        call("w4a_trace", None, 0)
+        return self.buf.cpu()
+
+
 def check(ws: torch.Tensor):
     """Synchronise and raise if the workspace's device error word is set."""
     call("w4a_check", _p(ws), ws.numel(), _stream())

@@ -92,6 +92,9 @@ static const void* engine_fn(int nb, int hd) {
 static int engine_smem(int nb) { return nb == 1 ? Lay<1>::TOTAL : Lay<2>::TOTAL; }
 static int nb_for(int batch) { return batch <= 8 ? 1 : 2; }
 
+static void* g_trace = nullptr;
+static size_t g_trace_bytes = 0;
+
 static int phases_per_launch() {
   const char* e = getenv("W4A_PHASES_PER_LAUNCH");
   if (!e || !*e) return 0;
@@ -120,6 +123,12 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
     }
   }
   P.nc = di->sms;
+  P.trace = nullptr;
+  P.trace_phases = 0;
+  if (g_trace && P.mode == MODE_DECODE) {
+    P.trace = static_cast<uint64_t*>(g_trace);
+    P.trace_phases = int(g_trace_bytes / ((size_t)P.nc * 32));
+  }
   const int begin = P.phase_begin, end = P.phase_end;
   int chunk = phases_per_launch();
   if (chunk <= 0) chunk = end - begin;
@@ -154,39 +163,59 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct GemvShape {
-  int64_t n, k;
-  int kcw;
-};
-
-static int64_t gpart_floats(const GemvShape& s, int B, int nb) {
-  const int nkc = int(s.k / s.kcw);
-  const int kps = choose_kps(nkc, s.kcw, B, nb);
-  if (kps <= 0) return -1;
-  const int64_t nrb = (s.n + RB - 1) / RB;
-  return (int64_t)(nkc / kps) * nrb * 2 * 32 * 4 * nb;
-}
-
 struct WsLayout {
-  size_t ctl, seg, gpart, apart, amax_v, amax_i, y_qkv, o, a, h, f, xA, xB, ss_qkv, ss_a, ss_f, total;
+  size_t ctl, seg, apart, amax_v, amax_i, y_part, o, a_part, gu_part, h, f_part, lg_part, xA, xB, g_part, total;
 };
 
 struct Dims {
   int d, nq, nkv, hd, ffn, vocab;
 };
 
-// decode != 0: all activations; shapes: the GEMVs the launch runs.
-static int ws_layout(int B, int nc, const Dims& dm, const GemvShape* shapes, int nshapes, int attn, int decode,
-                     WsLayout* L) {
+// A GEMV geometry the engine can run: some k-split fits shared memory and no
+// CTA's segments span more than two k-slabs.
+static int geo_check(const Geo& g, long long n, long long k, int B) {
+  if (g.ns <= 0) return fail(W4A_ERR_SHAPE, "no k-split of %lld x %lld fits shared memory at batch %d", n, k, B);
+  const long long upsl = (long long)g.nrb * g.kps;
+  for (int c = 0; c < g.nca; ++c) {
+    const long long a = rstart(g.nseg, g.nca, c) * g.kps, b = rstart(g.nseg, g.nca, c + 1) * g.kps;
+    if (a < b && (b - 1) / upsl - a / upsl > 1)
+      return fail(W4A_ERR_SHAPE, "%lld x %lld at batch %d needs more k-slabs per CTA than fit", n, k, B);
+  }
+  return W4A_OK;
+}
+
+// Geometries of the decode step's GEMVs: qkv, o, gate/up, down, lm_head.
+static int decode_geos(const Dims& dm, int B, int nc, Geo* g) {
   const int nb = nb_for(B);
-  int64_t gp = 0, ctr = MAX_SEG;
-  for (int i = 0; i < nshapes; ++i) {
-    const int64_t f = gpart_floats(shapes[i], B, nb);
-    if (f < 0) return fail(W4A_ERR_SHAPE, "no k-split of %lld x %lld fits shared memory at batch %d",
-                           (long long)shapes[i].n, (long long)shapes[i].k, B);
-    if (f > gp) gp = f;
-    const int64_t nrb = (shapes[i].n + RB - 1) / RB;
-    if (nrb > ctr) ctr = nrb;
+  const long long qd = (long long)dm.nq * dm.hd, qkv = (long long)(dm.nq + 2 * dm.nkv) * dm.hd;
+  const long long n[5] = {qkv, dm.d, 2LL * dm.ffn, dm.d, (dm.vocab + RB - 1) / RB * (long long)RB};
+  const long long k[5] = {dm.d, qd, dm.d, dm.ffn, dm.d};
+  // every CTA of the consuming phase reads the whole qkv, O, gate/up (counted
+  // as whole: one slab keeps the fused SiLU epilogue) and down outputs;
+  // argmax reads each logit once
+  const int readers[5] = {nc, nc, nc, nc, 1};
+  for (int i = 0; i < 5; ++i) {
+    g[i] = gemv_geo(n[i], k[i], i == 4 ? BF_KC : W4_KC, B, nb, nc, readers[i]);
+    const int rc = geo_check(g[i], n[i], k[i], B);
+    if (rc) return rc;
+  }
+  return W4A_OK;
+}
+
+// decode != 0: the decode step's activations; attn != 0: attention pieces;
+// gemv_n > 0: a standalone GEMV of gemv_n x gemv_k.
+static int ws_layout(int B, int nc, const Dims& dm, int attn, int decode, long long gemv_n, long long gemv_k,
+                     WsLayout* L) {
+  Geo g[5] = {};
+  if (decode) {
+    const int rc = decode_geos(dm, B, nc, g);
+    if (rc) return rc;
+  }
+  Geo gs = {};
+  if (gemv_n > 0) {
+    gs = gemv_geo(gemv_n, gemv_k, W4_KC, B, nb_for(B), nc, 1);
+    const int rc = geo_check(gs, gemv_n, gemv_k, B);
+    if (rc) return rc;
   }
   size_t off = 0;
   auto put = [&](size_t bytes) {
@@ -194,23 +223,22 @@ static int ws_layout(int B, int nc, const Dims& dm, const GemvShape* shapes, int
     off += al256(bytes);
     return o;
   };
+  const size_t qkv = (size_t)(dm.nq + 2 * dm.nkv) * dm.hd;
   L->ctl = put(256);
-  L->seg = put((size_t)ctr * 4);
-  L->gpart = put((size_t)gp * 4);
+  L->seg = put((size_t)MAX_SEG * 4);
   L->apart = put(attn ? (size_t)nc * 2 * MAX_GQ * (dm.hd + 2) * 4 : 0);
   L->amax_v = put(decode ? (size_t)nc * B * 4 : 0);
   L->amax_i = put(decode ? (size_t)nc * B * 4 : 0);
-  const int qkv = (dm.nq + 2 * dm.nkv) * dm.hd;
-  L->y_qkv = put(decode ? (size_t)B * qkv * 4 : 0);
+  L->y_part = put(decode ? (size_t)g[0].ns * B * qkv * 4 : 0);
   L->o = put(decode ? (size_t)B * dm.nq * dm.hd * 2 : 0);
-  L->a = put(decode ? (size_t)B * dm.d * 4 : 0);
+  L->a_part = put(decode ? (size_t)g[1].ns * B * dm.d * 4 : 0);
+  L->gu_part = put(decode && g[2].ns > 1 ? (size_t)g[2].ns * B * 2 * dm.ffn * 4 : 0);
   L->h = put(decode ? (size_t)B * dm.ffn * 2 : 0);
-  L->f = put(decode ? (size_t)B * dm.d * 4 : 0);
+  L->f_part = put(decode ? (size_t)g[3].ns * B * dm.d * 4 : 0);
+  L->lg_part = put(decode && g[4].ns > 1 ? (size_t)g[4].ns * B * dm.vocab * 4 : 0);
   L->xA = put(decode ? (size_t)B * dm.d * 4 : 0);
   L->xB = put(decode ? (size_t)B * dm.d * 4 : 0);
-  L->ss_qkv = put(decode ? (size_t)(qkv / RB) * B * 4 : 0);
-  L->ss_a = put(decode ? (size_t)(dm.d / RB) * B * 4 : 0);
-  L->ss_f = put(decode ? (size_t)(dm.d / RB) * B * 4 : 0);
+  L->g_part = put(gs.ns > 1 ? (size_t)gs.ns * B * gemv_n * 4 : 0);
   L->total = off;
   return W4A_OK;
 }
@@ -219,21 +247,19 @@ static void ws_bind(EngineParams& P, void* ws, const WsLayout& L) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   P.ws.ctl = reinterpret_cast<uint32_t*>(b + L.ctl);
   P.ws.seg_ctr = reinterpret_cast<uint32_t*>(b + L.seg);
-  P.ws.gpart = reinterpret_cast<float*>(b + L.gpart);
   P.ws.apart = reinterpret_cast<float*>(b + L.apart);
   P.ws.amax_val = reinterpret_cast<float*>(b + L.amax_v);
   P.ws.amax_idx = reinterpret_cast<int32_t*>(b + L.amax_i);
-  P.ws.y_qkv = reinterpret_cast<float*>(b + L.y_qkv);
+  P.ws.y_part = reinterpret_cast<float*>(b + L.y_part);
   P.ws.o = reinterpret_cast<uint16_t*>(b + L.o);
-  P.ws.a = reinterpret_cast<float*>(b + L.a);
+  P.ws.a_part = reinterpret_cast<float*>(b + L.a_part);
+  P.ws.gu_part = reinterpret_cast<float*>(b + L.gu_part);
   P.ws.h = reinterpret_cast<uint16_t*>(b + L.h);
-  P.ws.f = reinterpret_cast<float*>(b + L.f);
+  P.ws.f_part = reinterpret_cast<float*>(b + L.f_part);
+  P.ws.lg_part = reinterpret_cast<float*>(b + L.lg_part);
   P.ws.xA = reinterpret_cast<float*>(b + L.xA);
   P.ws.xB = reinterpret_cast<float*>(b + L.xB);
-  P.ws.ss_qkv = reinterpret_cast<float*>(b + L.ss_qkv);
-  P.ws.ss_a = reinterpret_cast<float*>(b + L.ss_a);
-  P.ws.ss_f = reinterpret_cast<float*>(b + L.ss_f);
-  P.ws.pos_seq = nullptr;
+  P.ws.g_part = reinterpret_cast<float*>(b + L.g_part);
 }
 
 static int nc_for_sizing(int* nc) {
@@ -313,15 +339,6 @@ static int check_config(const W4AConfig* c) {
 }
 
 static Dims dims_of(const W4AConfig& c) { return Dims{c.d_model, c.n_heads, c.n_kv_heads, c.head_dim, c.ffn, c.vocab}; }
-
-static void decode_shapes(const W4AConfig& c, GemvShape* s) {
-  const int qd = c.n_heads * c.head_dim, qkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
-  s[0] = {qkv, c.d_model, W4_KC};
-  s[1] = {c.d_model, qd, W4_KC};
-  s[2] = {2LL * c.ffn, c.d_model, W4_KC};
-  s[3] = {c.d_model, c.ffn, W4_KC};
-  s[4] = {(int64_t)(c.vocab + RB - 1) / RB * RB, c.d_model, BF_KC};
-}
 
 static int kv_regions(const W4AConfig* c, int batch, int max_ctx, uint64_t* off, int* slots, size_t* total) {
   size_t o = 0;
@@ -437,9 +454,8 @@ int w4a_gemv_workspace_bytes(const W4ATensor* W, int batch, size_t* bytes) {
   int nc;
   rc = nc_for_sizing(&nc);
   if (rc) return rc;
-  GemvShape s{W->n, W->k, W4_KC};
   WsLayout L;
-  rc = ws_layout(batch, nc, Dims{0, 0, 0, 128, 0, 0}, &s, 1, 0, 0, &L);
+  rc = ws_layout(batch, nc, Dims{0, 0, 0, 128, 0, 0}, 0, 0, W->n, W->k, &L);
   if (rc) return rc;
   *bytes = L.total;
   return W4A_OK;
@@ -460,16 +476,17 @@ int w4a_gemv(const W4ATensor* W, const uint16_t* x, int batch, void* out, int ep
   DevInfo* di;
   rc = device_info(&di);
   if (rc) return rc;
-  GemvShape s{W->n, W->k, W4_KC};
   WsLayout L;
-  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, 128, 0, 0}, &s, 1, 0, 0, &L);
+  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, 128, 0, 0}, 0, 0, W->n, W->k, &L);
   if (rc) return rc;
   if (ws_bytes < L.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   static thread_local EngineParams P;
   memset(&P, 0, sizeof(P));
   P.mode = MODE_GEMV;
   P.phase_begin = 0;
-  P.phase_end = 1;
+  // with K split into slabs a second phase sums them and applies the epilogue
+  P.geo[0] = gemv_geo(W->n, W->k, W4_KC, batch, nb_for(batch), di->sms, 1);
+  P.phase_end = P.geo[0].ns > 1 ? 2 : 1;
   P.B = batch;
   P.pos_const = -1;
   P.g_blob = static_cast<const uint8_t*>(W->qweight);
@@ -494,7 +511,7 @@ int w4a_attn_workspace_bytes(int batch, int n_heads, int n_kv_heads, int head_di
   int rc = nc_for_sizing(&nc);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, nc, Dims{0, 0, 0, head_dim, 0, 0}, nullptr, 0, 1, 0, &L);
+  rc = ws_layout(batch, nc, Dims{0, 0, 0, head_dim, 0, 0}, 1, 0, 0, 0, &L);
   if (rc) return rc;
   *bytes = L.total;
   return W4A_OK;
@@ -515,7 +532,7 @@ int w4a_attn_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* 
   int rc = device_info(&di);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, head_dim, 0, 0}, nullptr, 0, 1, 0, &L);
+  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, head_dim, 0, 0}, 1, 0, 0, 0, &L);
   if (rc) return rc;
   if (ws_bytes < L.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   static thread_local EngineParams P;
@@ -611,7 +628,9 @@ int w4a_model_create(const W4AConfig* cfg, const W4AModelWeights* w, W4AModel** 
   if (rc) return rc;
   if (!w || !out || !w->embed || !w->lm_head || !w->layers) return fail(W4A_ERR_ARG, "null pointer");
   if (cfg->final_norm && !w->final_norm) return fail(W4A_ERR_ARG, "final_norm gains missing");
-  if (!aligned16(w->lm_head)) return fail(W4A_ERR_ALIGN, "lm_head not 16-byte aligned");
+  if (!aligned16(w->lm_head) || !aligned16(w->embed) || (w->final_norm && !aligned16(w->final_norm)))
+    return fail(W4A_ERR_ALIGN, "embedding, lm_head and final norm must be 16-byte aligned");
+  if ((cfg->d_model * 2) % 16) return fail(W4A_ERR_SHAPE, "d_model must be a multiple of 8");
   W4AModel* m = static_cast<W4AModel*>(calloc(1, sizeof(W4AModel)));
   if (!m) return fail(W4A_ERR_ARG, "out of host memory");
   m->cfg = *cfg;
@@ -624,7 +643,9 @@ int w4a_model_create(const W4AConfig* cfg, const W4AModelWeights* w, W4AModel** 
       free(m);
       return fail(W4A_ERR_ARG, "layer %d: null weight pointer", l);
     }
-    if (!aligned16(L.qkv) || !aligned16(L.o) || !aligned16(L.gate_up) || !aligned16(L.down)) {
+    if (!aligned16(L.qkv) || !aligned16(L.o) || !aligned16(L.gate_up) || !aligned16(L.down) ||
+        !aligned16(L.q_norm) || !aligned16(L.k_norm) || !aligned16(L.post_attn_norm) ||
+        !aligned16(L.post_ffn_norm)) {
       free(m);
       return fail(W4A_ERR_ALIGN, "layer %d: weights not 16-byte aligned", l);
     }
@@ -648,10 +669,8 @@ int w4a_decode_workspace_bytes(const W4AModel* m, int batch, size_t* bytes) {
   int nc;
   int rc = nc_for_sizing(&nc);
   if (rc) return rc;
-  GemvShape s[5];
-  decode_shapes(m->cfg, s);
   WsLayout L;
-  rc = ws_layout(batch, nc, dims_of(m->cfg), s, 5, 1, 1, &L);
+  rc = ws_layout(batch, nc, dims_of(m->cfg), 1, 1, 0, 0, &L);
   if (rc) return rc;
   *bytes = L.total;
   return W4A_OK;
@@ -671,10 +690,8 @@ static int decode_common(W4AModel* m, const int32_t* tokens, const W4AKVCache* k
   DevInfo* di;
   int rc = device_info(&di);
   if (rc) return rc;
-  GemvShape s[5];
-  decode_shapes(c, s);
   WsLayout L;
-  rc = ws_layout(batch, di->sms, dims_of(c), s, 5, 1, 1, &L);
+  rc = ws_layout(batch, di->sms, dims_of(c), 1, 1, 0, 0, &L);
   if (rc) return rc;
   if (ws_bytes < L.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   static thread_local EngineParams P;
@@ -715,6 +732,8 @@ static int decode_common(W4AModel* m, const int32_t* tokens, const W4AKVCache* k
   P.next_token = next_token;
   P.dump = dump;
   ws_bind(P, ws, L);
+  rc = decode_geos(dims_of(c), batch, di->sms, P.geo);
+  if (rc) return rc;
   P.phase_begin = 0;
   P.phase_end = phase_end_kind;
   return launch_engine(P, nb_for(batch), c.head_dim, st);
@@ -725,8 +744,9 @@ int w4a_decode_step(W4AModel* m, const int32_t* token_ids, const W4AKVCache* kv,
                     size_t ws_bytes, void* stream) {
   if (!m || !pos || !logits) return fail(W4A_ERR_ARG, "null pointer");
   const int nl = m->cfg.n_layers;
-  return decode_common(m, token_ids, kv, seq0, batch, pos, -1, logits, next_token, hidden_dump,
-                       next_token ? 5 * nl + 2 : 5 * nl + 1, ws, ws_bytes, S(stream));
+  // the last phase also sums the lm_head's k-slabs into the logits when it is split
+  return decode_common(m, token_ids, kv, seq0, batch, pos, -1, logits, next_token, hidden_dump, 5 * nl + 2, ws,
+                       ws_bytes, S(stream));
 }
 
 int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv, int seq, int start_pos,
@@ -737,9 +757,16 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   for (int i = 0; i < T; ++i) {
     const bool last = (i == T - 1) && last_logits != nullptr;
     const int rc = decode_common(m, tokens + i, kv, seq, 1, nullptr, start_pos + i, last ? last_logits : nullptr,
-                                 nullptr, nullptr, last ? 5 * nl + 1 : 5 * nl, ws, ws_bytes, S(stream));
+                                 nullptr, nullptr, last ? 5 * nl + 2 : 5 * nl, ws, ws_bytes, S(stream));
     if (rc) return rc;
   }
+  return W4A_OK;
+}
+
+int w4a_trace(void* buf, size_t bytes) {
+  if (buf && !aligned16(buf)) return fail(W4A_ERR_ALIGN, "trace buffer not 16-byte aligned");
+  g_trace = buf;
+  g_trace_bytes = buf ? bytes : 0;
   return W4A_OK;
 }
 

@@ -44,9 +44,15 @@ enum : uint32_t {
 
 // ---- engine modes / phase kinds --------------------------------------------
 enum Mode : int { MODE_DECODE = 0, MODE_GEMV = 1, MODE_ATTN = 2 };
-enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_ATTN = 2, PK_ARGMAX = 3 };
-enum XSrc : int { XS_BF16 = 0, XS_EMBED = 1, XS_RESID = 2, XS_FINAL = 3, XS_F16 = 4 };
-enum Epi : int { EPI_Y = 0, EPI_Y_SUMSQ = 1, EPI_SILU = 2, EPI_LOGITS = 3 };
+enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_ATTN = 2, PK_ARGMAX = 3, PK_REDUCE = 4 };
+enum XSrc : int { XS_BF16 = 0, XS_EMBED = 1, XS_RESID = 2, XS_FINAL = 3, XS_F16 = 4, XS_SILU = 5 };
+enum Epi : int { EPI_Y = 0, EPI_Y_SUMSQ = 1, EPI_SILU = 2, EPI_PART = 3 };
+
+// Geometry of a GEMV phase: 16-row blocks, k-chunks, k-chunks per slab,
+// slabs, segments (= slabs x row blocks) and CTAs used.
+struct Geo {
+  int nrb, nkc, kps, ns, nseg, nca;
+};
 
 struct LayerPtrs {
   const uint8_t* qkv;
@@ -62,22 +68,20 @@ struct LayerPtrs {
 // Workspace carve-up (device pointers), filled on the host.
 struct Workspace {
   uint32_t* ctl;        // [0] barrier, [1] exit, [2] error word, [3] argmax counter
-  uint32_t* seg_ctr;    // per-segment arrival counters
-  float* gpart;         // GEMV split pieces [NS][nrb][2][RB * 8 * NB]
+  uint32_t* seg_ctr;    // attention arrival counters [MAX_SEG]
   float* apart;         // attention pieces [NC][2][MAX_GQ * (HD + 2)]
   float* amax_val;      // argmax pieces [NC][B]
   int32_t* amax_idx;
-  float* y_qkv;         // [B][qkv_dim]
-  uint16_t* o;          // [B][q_dim] fp16 (attention output)
-  float* a;             // [B][d]
-  uint16_t* h;          // [B][ffn] fp16 (SwiGLU output)
-  float* f;             // [B][d]
-  float* xA;            // [B][d]
-  float* xB;            // [B][d]
-  float* ss_qkv;        // [nrb_qkv][B]
-  float* ss_a;          // [nrb_d][B]
-  float* ss_f;          // [nrb_d][B]
-  int32_t* pos_seq;     // prefill positions [T]
+  float* y_part;        // QKV output, per k-slab [ns][B][qkv_dim]
+  uint16_t* o;          // attention output, fp16 [B][q_dim]
+  float* a_part;        // O output [ns][B][d]
+  float* gu_part;       // gate/up output when split [ns][B][2 ffn]
+  uint16_t* h;          // SwiGLU output, fp16 [B][ffn]
+  float* f_part;        // down output [ns][B][d]
+  float* lg_part;       // lm_head output when split [ns][B][vocab]
+  float* xA;            // residual at the layer input [B][d]
+  float* xB;            // residual after attention [B][d]
+  float* g_part;        // standalone GEMV output when split [ns][B][n]
 };
 
 struct EngineParams {
@@ -110,6 +114,7 @@ struct EngineParams {
   int32_t* next_token;
   float* dump;
   Workspace ws;
+  Geo geo[5];           // decode: qkv, o, gate/up, down, lm_head; GEMV: [0]
   // standalone GEMV
   const uint8_t* g_blob;
   const uint16_t* g_x;
@@ -122,6 +127,9 @@ struct EngineParams {
   const uint16_t* a_v;
   uint16_t* a_out;
   int a_slots, a_window;
+  // optional trace: [phase][cta][4] %globaltimer stamps (start, prologue done, units done, arrived)
+  uint64_t* trace;
+  int trace_phases;
 };
 
 // Slots of a layer's ring / linear cache.
