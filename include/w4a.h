@@ -254,10 +254,13 @@ W4A_API int w4a_prefill(W4AModel* model, const int32_t* tokens, int T, const W4A
 
 /* Profiling aid (off by default).  With a device buffer set, every later
  * w4a_decode_step / w4a_prefill launch writes, per phase p (5 per layer, then
- * lm_head and argmax) and CTA c, four %globaltimer stamps (ns) as uint64 at
- * buf[(p * n_sms + c) * 4 + {0: phase start, 1: inputs staged, 2: units
- * done, 3: arrived at the barrier}].  Phases beyond bytes / (32 * n_sms) are
- * not recorded.  buf = NULL turns tracing off.  Process-wide setting. */
+ * lm_head and argmax) and CTA c, eight %globaltimer stamps (ns) as uint64 at
+ * buf[(p * n_sms + c) * 8 + i]: i = 0 phase start, 1 phase descriptor ready,
+ * 2 first input pass done (norm statistics / raw inputs loaded), 3 inputs
+ * staged, 4 units done, 5 partial results combined, 6 arrived at the grid
+ * barrier, 7 unused.  A stamp the phase does not reach stays as it was.
+ * Phases beyond bytes / (64 * n_sms) are not recorded.  buf = NULL turns
+ * tracing off.  Process-wide setting. */
 W4A_API int w4a_trace(void* buf, size_t bytes);
 
 /* Synchronise `stream` and report the device error word of a workspace. */

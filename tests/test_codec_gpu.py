@@ -98,11 +98,49 @@ def test_tile_bf16_layout(built_lib, cuda):
             for s in range(8):
                 for lane in range(32):
                     g, t = lane // 4, lane % 4
-                    k0 = kc * 128 + s * 16 + 2 * t
+                    # k-step s = 2m + e of thread-in-quad t reads columns 32m + 8t + 4e .. +3
+                    k0 = kc * 128 + 32 * (s // 2) + 8 * t + 4 * (s % 2)
                     r0, r1 = rb * 16 + g, rb * 16 + g + 8
                     want = [full[r0, k0], full[r0, k0 + 1], full[r1, k0], full[r1, k0 + 1],
-                            full[r0, k0 + 8], full[r0, k0 + 9], full[r1, k0 + 8], full[r1, k0 + 9]]
+                            full[r0, k0 + 2], full[r0, k0 + 3], full[r1, k0 + 2], full[r1, k0 + 3]]
                     assert list(u[s, lane]) == want
+
+
+def test_tile_w4_layout(built_lib, cuda):
+    """Reassemble the documented int4 unit layout by hand (codes, scales, zeros)."""
+    api = _api()
+    n, k = 32, 1024
+    W, _ = synth.gemv_case(13, n, k, 1, "cpu")
+    qw, sc, qz = api.pack(W.to(cuda))
+    lin = api.tile(qw, sc, qz, n, k, row_interleave=False)
+    blob = lin.blob.cpu().numpy().view(np.uint8)
+    q, _, Z = quant.unpack(_as_u32(qw), _as_u16(sc), _as_u32(qz), n, k)   # codes [n, k], zeros [k/128, n]
+    S = _as_u16(sc)                                                       # fp16 bits [k/128, n]
+    nkc = k // 512
+    for rb in range(n // 16):
+        for kc in range(nkc):
+            u = blob[(rb * nkc + kc) * 4256:(rb * nkc + kc + 1) * 4256]
+            words = u[:4096].view(np.uint32).reshape(8, 32, 4)      # [s // 4][lane][s % 4]
+            for s in range(32):
+                for lane in range(32):
+                    g, t = lane // 4, lane % 4
+                    c = kc * 512 + 32 * (s // 2) + 8 * t + 4 * (s % 2)
+                    r0, r1 = rb * 16 + g, rb * 16 + g + 8
+                    # nibble j: row (j odd ? r1 : r0), column c + (2 if j & 2) + (1 if j & 4)
+                    want = 0
+                    for j in range(8):
+                        r = r1 if j & 1 else r0
+                        cc = c + (2 if j & 2 else 0) + (1 if j & 4 else 0)
+                        want |= int(q[r, cc]) << (4 * j)
+                    assert int(words[s // 4, lane, s % 4]) == want
+            scales = u[4096:4224].view(np.uint16).reshape(8, 4, 2)   # [row % 8][group][row / 8]
+            zeros = u[4224:4256].view(np.uint32).reshape(4, 2)       # [group][row / 8], nibble row % 8
+            for grp in range(4):
+                gi = kc * 4 + grp
+                for i in range(16):
+                    row = rb * 16 + i
+                    assert scales[i % 8, grp, i // 8] == S[gi, row]
+                    assert (int(zeros[grp, i // 8]) >> (4 * (i % 8))) & 15 == int(Z[gi, row])
 
 
 def test_kv_write_read_roundtrip(built_lib, cuda):

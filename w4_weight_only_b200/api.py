@@ -348,7 +348,7 @@ class Trace:
 
     def __init__(self, n_phases: int, device=None):
         self.n_sms = torch.cuda.get_device_properties(device or 0).multi_processor_count
-        self.buf = torch.zeros((n_phases, self.n_sms, 4), dtype=torch.int64, device=device or "cuda")
+        self.buf = torch.zeros((n_phases, self.n_sms, 8), dtype=torch.int64, device=device or "cuda")
         call("w4a_trace", _p(self.buf), self.buf.numel() * 8)
 
     def stop(self):

@@ -89,7 +89,7 @@ static const void* engine_fn(int nb, int hd) {
   if (nb == 2 && hd == 128) return reinterpret_cast<const void*>(&w4a_engine_kernel<2, 128>);
   return nullptr;
 }
-static int engine_smem(int nb) { return nb == 1 ? Lay<1>::TOTAL : Lay<2>::TOTAL; }
+static int engine_smem(int) { return SM_TOTAL; }
 static int nb_for(int batch) { return batch <= 8 ? 1 : 2; }
 
 static void* g_trace = nullptr;
@@ -127,7 +127,7 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
   P.trace_phases = 0;
   if (g_trace && P.mode == MODE_DECODE) {
     P.trace = static_cast<uint64_t*>(g_trace);
-    P.trace_phases = int(g_trace_bytes / ((size_t)P.nc * 32));
+    P.trace_phases = int(g_trace_bytes / ((size_t)P.nc * 64));
   }
   const int begin = P.phase_begin, end = P.phase_end;
   int chunk = phases_per_launch();
@@ -164,11 +164,12 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t ctl, seg, apart, amax_v, amax_i, y_part, o, a_part, gu_part, h, f_part, lg_part, xA, xB, g_part, total;
+  size_t ctl, seg, apart, amax_v, amax_i, y_part, o, a_part, gu_part, h, f_part, lg_part, xA, xB, g_part, plan,
+      total;
 };
 
 struct Dims {
-  int d, nq, nkv, hd, ffn, vocab;
+  int d, nq, nkv, hd, ffn, vocab, n_layers;
 };
 
 // A GEMV geometry the engine can run: some k-split fits shared memory and no
@@ -238,7 +239,9 @@ static int ws_layout(int B, int nc, const Dims& dm, int attn, int decode, long l
   L->lg_part = put(decode && g[4].ns > 1 ? (size_t)g[4].ns * B * dm.vocab * 4 : 0);
   L->xA = put(decode ? (size_t)B * dm.d * 4 : 0);
   L->xB = put(decode ? (size_t)B * dm.d * 4 : 0);
-  L->g_part = put(gs.ns > 1 ? (size_t)gs.ns * B * gemv_n * 4 : 0);
+  L->g_part = put(gemv_n > 0 ? (size_t)gs.ns * B * gemv_n * 4 : 0);
+  // phase descriptors: every phase of a decode step (standalone ops use at most two)
+  L->plan = put(decode ? (size_t)(5 * dm.n_layers + 2) * sizeof(PD) : 2 * sizeof(PD));
   L->total = off;
   return W4A_OK;
 }
@@ -260,6 +263,7 @@ static void ws_bind(EngineParams& P, void* ws, const WsLayout& L) {
   P.ws.xA = reinterpret_cast<float*>(b + L.xA);
   P.ws.xB = reinterpret_cast<float*>(b + L.xB);
   P.ws.g_part = reinterpret_cast<float*>(b + L.g_part);
+  P.ws.plan = b + L.plan;
 }
 
 static int nc_for_sizing(int* nc) {
@@ -338,7 +342,9 @@ static int check_config(const W4AConfig* c) {
   return W4A_OK;
 }
 
-static Dims dims_of(const W4AConfig& c) { return Dims{c.d_model, c.n_heads, c.n_kv_heads, c.head_dim, c.ffn, c.vocab}; }
+static Dims dims_of(const W4AConfig& c) {
+  return Dims{c.d_model, c.n_heads, c.n_kv_heads, c.head_dim, c.ffn, c.vocab, c.n_layers};
+}
 
 static int kv_regions(const W4AConfig* c, int batch, int max_ctx, uint64_t* off, int* slots, size_t* total) {
   size_t o = 0;
@@ -455,7 +461,7 @@ int w4a_gemv_workspace_bytes(const W4ATensor* W, int batch, size_t* bytes) {
   rc = nc_for_sizing(&nc);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, nc, Dims{0, 0, 0, 128, 0, 0}, 0, 0, W->n, W->k, &L);
+  rc = ws_layout(batch, nc, Dims{0, 0, 0, 128, 0, 0, 0}, 0, 0, W->n, W->k, &L);
   if (rc) return rc;
   *bytes = L.total;
   return W4A_OK;
@@ -477,7 +483,7 @@ int w4a_gemv(const W4ATensor* W, const uint16_t* x, int batch, void* out, int ep
   rc = device_info(&di);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, 128, 0, 0}, 0, 0, W->n, W->k, &L);
+  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, 128, 0, 0, 0}, 0, 0, W->n, W->k, &L);
   if (rc) return rc;
   if (ws_bytes < L.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   static thread_local EngineParams P;
@@ -486,7 +492,7 @@ int w4a_gemv(const W4ATensor* W, const uint16_t* x, int batch, void* out, int ep
   P.phase_begin = 0;
   // with K split into slabs a second phase sums them and applies the epilogue
   P.geo[0] = gemv_geo(W->n, W->k, W4_KC, batch, nb_for(batch), di->sms, 1);
-  P.phase_end = P.geo[0].ns > 1 ? 2 : 1;
+  P.phase_end = (P.geo[0].ns > 1 || epilogue == W4A_EPI_SUMSQ) ? 2 : 1;
   P.B = batch;
   P.pos_const = -1;
   P.g_blob = static_cast<const uint8_t*>(W->qweight);
@@ -511,7 +517,7 @@ int w4a_attn_workspace_bytes(int batch, int n_heads, int n_kv_heads, int head_di
   int rc = nc_for_sizing(&nc);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, nc, Dims{0, 0, 0, head_dim, 0, 0}, 1, 0, 0, 0, &L);
+  rc = ws_layout(batch, nc, Dims{0, 0, 0, head_dim, 0, 0, 0}, 1, 0, 0, 0, &L);
   if (rc) return rc;
   *bytes = L.total;
   return W4A_OK;
@@ -532,7 +538,7 @@ int w4a_attn_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* 
   int rc = device_info(&di);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, head_dim, 0, 0}, 1, 0, 0, 0, &L);
+  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, head_dim, 0, 0, 0}, 1, 0, 0, 0, &L);
   if (rc) return rc;
   if (ws_bytes < L.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   static thread_local EngineParams P;

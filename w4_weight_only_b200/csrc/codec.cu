@@ -75,6 +75,17 @@ __device__ inline uint32_t canon_code(const uint32_t* qw, int64_t k, int64_t row
   return (qw[row * (k / 8) + col / 8] >> (4 * (col % 8))) & 15u;
 }
 
+// Column order inside a unit.  Each 32-column slice is split in four runs of
+// eight, one per thread-in-quad t; the run of quad t feeds k-steps 2m (first
+// four columns) and 2m+1 (last four) of the m16n8k16 products, so the
+// activation fragments of a thread are 16 contiguous bytes of x.  Fragment
+// register a0 holds (row g, columns c, c+1), a1 (row g+8, c, c+1), a2 (row g,
+// c+2, c+3), a3 (row g+8, c+2, c+3) with c = 32m + 8t + 4e for k-step 2m+e.
+__host__ __device__ inline int64_t unit_col(int s, int t, int j) {
+  const int m = s >> 1, e = s & 1;
+  return 32 * m + 8 * t + 4 * e + j;  // j = 0..3: columns of a0/a1 (j < 2) and a2/a3 (j >= 2)
+}
+
 // One thread per 32-bit word of int4 codes in the tiled layout.
 __global__ void tile_codes_kernel(const uint32_t* __restrict__ qw, int64_t n, int64_t k, int interleave,
                                   uint8_t* __restrict__ out) {
@@ -83,18 +94,17 @@ __global__ void tile_codes_kernel(const uint32_t* __restrict__ qw, int64_t n, in
   const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= total) return;
   const int lane = int(id % 32);
-  const int64_t s = (id / 32) % (W4_KC / 16);
+  const int s = int((id / 32) % (W4_KC / 16));
   const int64_t unit = id / (32 * (W4_KC / 16));
   const int64_t rb = unit / nkc, kc = unit % nkc;
   const int g = lane >> 2, t = lane & 3;
   const int64_t r0 = canon_row(rb * RB + g, n, interleave), r1 = canon_row(rb * RB + g + 8, n, interleave);
-  const int64_t k0 = kc * W4_KC + s * 16 + 2 * t;
-  // nibble j of the word: row (j & 1 ? r1 : r0), column k0 + (j & 4 ? 1 : 0) + (j & 2 ? 8 : 0)
+  // nibble j of the word: row (j & 1 ? g + 8 : g), column unit_col(.., (j & 2 ? 2 : 0) + (j & 4 ? 1 : 0))
   uint32_t w = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int64_t row = (j & 1) ? r1 : r0;
-    const int64_t col = k0 + ((j & 4) ? 1 : 0) + ((j & 2) ? 8 : 0);
+    const int64_t col = kc * W4_KC + unit_col(s, t, ((j & 2) ? 2 : 0) + ((j & 4) ? 1 : 0));
     w |= canon_code(qw, k, row, col) << (4 * j);
   }
   uint8_t* u = out + unit * W4_UNIT;
@@ -115,7 +125,8 @@ __global__ void tile_meta_kernel(const uint16_t* __restrict__ sc, const uint32_t
   const int64_t gi = kc * 4 + grp;
   const int64_t row = canon_row(rb * RB + i, n, interleave);
   uint8_t* u = out + unit * W4_UNIT;
-  reinterpret_cast<uint16_t*>(u + 4096)[grp * RB + i] = sc[gi * n + row];
+  // scales ordered [row % 8][group][row / 8]: a thread's eight scales are 16 contiguous bytes
+  reinterpret_cast<uint16_t*>(u + 4096)[(i & 7) * 8 + grp * 2 + (i >> 3)] = sc[gi * n + row];
   if ((i & 7) == 0) {
     uint32_t zw = 0;
     for (int j = 0; j < 8; ++j) {
@@ -139,7 +150,7 @@ __global__ void tile_bf16_kernel(const uint16_t* __restrict__ W, int64_t n, int6
   const int64_t rb = unit / nkc, kc = unit % nkc;
   const int g = lane >> 2, t = lane & 3;
   const int64_t r0 = rb * RB + g, r1 = r0 + 8;
-  const int64_t k0 = kc * BF_KC + s * 16 + 2 * t;
+  const int64_t k0 = kc * BF_KC + unit_col(int(s), t, 0);
   auto pair = [&](int64_t r, int64_t c) -> uint32_t {
     if (r >= n) return 0u;
     return uint32_t(W[r * k + c]) | (uint32_t(W[r * k + c + 1]) << 16);
@@ -147,8 +158,8 @@ __global__ void tile_bf16_kernel(const uint16_t* __restrict__ W, int64_t n, int6
   uint4 v;
   v.x = pair(r0, k0);
   v.y = pair(r1, k0);
-  v.z = pair(r0, k0 + 8);
-  v.w = pair(r1, k0 + 8);
+  v.z = pair(r0, k0 + 2);
+  v.w = pair(r1, k0 + 2);
   reinterpret_cast<uint4*>(out + unit * BF_UNIT)[s * 32 + lane] = v;
 }
 
@@ -172,15 +183,16 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ qw, const uint16_t* _
     const int i = int(r % RB), g = i & 7, hi = i >> 3;
     const int64_t nkc = k / W4_KC, kc = col / W4_KC;
     const int kk = int(col % W4_KC);
-    const int s = kk / 16, within = kk % 16;
-    const int t = (within & 7) >> 1, e = within & 1, upper = within >> 3;
+    // inverse of unit_col: column kk = 32 m + 8 t + 4 e + j
+    const int m = kk / 32, t = (kk % 32) / 8, e = (kk % 8) / 4, j = kk % 4;
+    const int s = 2 * m + e;
     const int lane = g * 4 + t;
-    const int nib = (e ? 4 : 0) + (upper ? 2 : 0) + hi;
+    const int nib = ((j & 1) ? 4 : 0) + ((j & 2) ? 2 : 0) + hi;
     const uint8_t* u = tiled + (rb * nkc + kc) * W4_UNIT;
     const uint32_t w = reinterpret_cast<const uint32_t*>(u + ((s >> 2) * 32 + lane) * 16)[s & 3];
     q = (w >> (4 * nib)) & 15u;
     const int grp = kk / GROUP;
-    sb = reinterpret_cast<const uint16_t*>(u + 4096)[grp * RB + i];
+    sb = reinterpret_cast<const uint16_t*>(u + 4096)[g * 8 + grp * 2 + hi];
     z = (reinterpret_cast<const uint32_t*>(u + 4224)[grp * 2 + hi] >> (4 * g)) & 15u;
   }
   out[id] = float(int(q) - int(z)) * half_bits_to_f32(sb);

@@ -3,35 +3,46 @@
 // One CTA per SM, 16 warps.  A launch runs a list of phases (decode: per layer
 // QKV GEMV, GQA attention, O GEMV, gate/up GEMV, down GEMV; then lm_head and
 // argmax) separated by grid-wide barriers.  Every warp streams its own
-// contiguous range of 4 KB "units" (16 weight rows x 512 int4 columns, 16 rows
-// x 128 bf16 columns, or 8 keys of K and V) from HBM into a two-slot ring of
-// shared memory with bulk asynchronous copies completing on mbarriers, and
-// refills a slot with its next unit as soon as it has used it.  The stream
-// runs across phase boundaries: weights and old KV entries do not depend on
-// the activations, so the copies for phase p+1 are in flight while the CTA
-// waits at the barrier that ends phase p.
+// contiguous range of ~4 KB "units" (16 weight rows x 512 int4 columns, 16
+// rows x 128 bf16 columns, or 8 keys of K and V) from HBM into a two-slot ring
+// of shared memory with bulk asynchronous copies completing on mbarriers, and
+// refills a slot with its next unit as soon as it has used it.  A second
+// cursor runs a few units ahead of the ring and asks for those units to be
+// brought into L2, so HBM keeps streaming while the CTA sits in a barrier or
+// stages its inputs.  Both cursors run across phase boundaries: weights and
+// old KV entries do not depend on the activations.
 //
-// GEMV math: the int4 codes of a unit are laid out as mma.sync A fragments
-// (16 rows x 16 k per warp-wide word).  A LOP3 turns each nibble q into the
-// fp16 value 1024 + q (exact), the tensor core accumulates sum_k (1024+q) x_k
-// in fp32 per 128-group, and the group is closed in fp32 with
-// s * (acc - (1024 + z) * sum_k x_k).  x is the mma B operand (batch = n),
-// held in fp16 (11-bit significand) after an exact power-of-two range
-// scaling that is undone when a partial leaves the warp.  The bf16 lm_head
-// takes bf16 x.
+// Phase descriptors (what a phase reads, computes and writes) are built on the
+// device at launch, in parallel by one thread per phase, into a table in the
+// workspace; the CTA copies each descriptor into one of four shared-memory
+// slots two phases before it runs, so the unit streams can look ahead.
+//
+// GEMV math: the int4 codes of a unit are laid out as mma.sync A fragments.
+// A LOP3 turns each nibble q into the fp16 value 1024 + q (rows g) or
+// 1024 + 16 q (rows g + 8, no shift needed), the tensor core accumulates
+// sum_k (1024 + q) x_k in fp32 per 128-group, and the group is closed in fp32
+// with s * (acc - (1024 + z) * sum_k x_k) (the 16x rows with s / 16 and
+// 1024 + 16 z).  Within a unit the 512 columns are ordered so that each
+// thread's activation fragments are 16 contiguous bytes of x: the activations
+// are staged in shared memory in plain order, fp16 after an exact
+// power-of-two range scaling that is undone when a partial leaves the warp.
+// The bf16 lm_head takes bf16 x.
 //
 // Work split of a GEMV phase: K is cut into `ns` slabs; a "segment" is one
-// 16-row block of one slab.  Every CTA owns whole segments (so no segment is
-// shared between CTAs); its warps split the CTA's units and the pieces of a
-// segment held by different warps are summed in warp order in shared memory.
-// With one slab the CTA finishes the rows (plain store, sums of squares, or
-// SiLU * up); with several it stores one partial row per slab and the phase
-// that consumes the vector adds the slabs in order (and computes any RMSNorm
-// over the whole vector itself).  Every sum has a fixed order, so results are
-// bit-reproducible.
+// 16-row block of one slab.  Every CTA owns whole segments; its warps split
+// the CTA's units and the pieces of a segment held by different warps are
+// summed in warp order in shared memory.  With one slab the CTA finishes the
+// rows (plain store or SiLU * up); with several it stores one partial row per
+// slab and the phase that consumes the vector adds the slabs in order
+// (computing any RMSNorm over the whole vector itself).  Every sum has a fixed
+// order, so results are bit-reproducible.
 //
 // Attention splits each (sequence, KV head) over CTAs by keys; the last CTA to
 // arrive on a segment's counter merges the pieces in CTA order (no waiting).
+//
+// Nothing here lives in per-thread local memory: state that outlives a
+// function (ring cursors, descriptors, launch constants) is kept in shared
+// memory, and the hot loops keep theirs in registers.
 #pragma once
 #include <float.h>
 #include <math.h>
@@ -43,7 +54,8 @@ namespace w4a {
 
 constexpr long long WAIT_CYCLES = 4000000000LL;  // bound on any single wait (~2 s)
 constexpr int MAX_SEG = MAX_B * 16;              // attention segments (batch x kv heads)
-constexpr int NS_MAX = 8;                        // k-slabs a GEMV phase may use
+constexpr int NS_MAX = 8;                        // k-slabs a GEMV phase may choose
+constexpr int PF_AHEAD = 4;                      // units per warp requested into L2 ahead of the ring
 
 __host__ __device__ inline long long rstart(long long U, int n, int i) { return (U * i) / n; }
 // CTA (of n) whose range [rstart(c), rstart(c+1)) contains unit u.
@@ -51,14 +63,14 @@ __host__ __device__ inline int owner(long long U, int n, long long u) {
   return int(((u + 1) * n + U - 1) / U) - 1;
 }
 
-// x of klen columns for B rows fits the staging buffers (fragments and the
+// x of klen columns for B rows fits the staging buffers (values and the
 // per-group sums).
 __host__ __device__ inline bool x_fits(long long klen, int B, int nb) {
   return B * (klen * 2 + 64) <= xs_cap(nb) && (klen / GROUP) * 8 * nb * 4 <= XSUM_BYTES;
 }
 
-// Largest k-chunks per slab whose x fragments fit the shared-memory budget
-// (one slab when it fits whole, else two slabs must fit); 0 when none does.
+// Largest k-chunks per slab whose x fits the shared-memory budget (one slab
+// when it fits whole, else two slabs must fit); 0 when none does.
 __host__ __device__ inline int choose_kps(int nkc, int kcw, int B, int nb) {
   if (x_fits((long long)nkc * kcw, B, nb)) return nkc;
   for (int dv = nkc - 1; dv >= 1; --dv)
@@ -66,7 +78,6 @@ __host__ __device__ inline int choose_kps(int nkc, int kcw, int B, int nb) {
   return 0;
 }
 
-// The geometry the host computes for a GEMV phase (see Geo).
 // Chooses how many k-slabs a GEMV phase uses.  The phase lasts as long as its
 // busiest CTA, i.e. ceil(segments / CTAs) segments of kps units each; every
 // slab beyond the first makes the consuming phase read one more copy of the
@@ -105,114 +116,173 @@ inline Geo gemv_geo(long long n, long long k, int kcw, int B, int nb, int nc, in
   return g;
 }
 
-struct PD {
-  int kind, layer;
-  // GEMV
-  const uint8_t* blob;
-  int n, k, kcw, ub;
-  Geo g;
-  int xsrc;
-  const uint16_t* xbf;    // 16-bit input rows (XS_BF16 / XS_F16)
-  int xbf_stride;
-  const float* xres;      // residual (XS_RESID / XS_FINAL)
-  const float* vpart;     // branch output slabs [vns][B][vstride] (XS_RESID / XS_FINAL / XS_SILU)
-  int vns, vstride;
-  const float* gain;
-  const float* gain2;
-  float* xdst;
-  float* dump;
-  int epi;
-  float* yout;
-  int ystride;
-  uint16_t* hout;
-  int hstride;
-  int out_f16;
-  float* ssout;
-  int rows_valid;
-  float* part;            // EPI_PART target [ns][B][pstride]
-  int pstride;
-  // attention
-  int type, newkv, slots, seqoff;
-  const uint8_t* kc;
-  const uint8_t* vc;
-  uint16_t* aout;
-  const float* qpart;     // QKV output slabs (decode)
-  int qns;
-  // argmax
-  const float* lpart;
-  int lns;
+// ---------------------------------------------------------------------------
+// Phase descriptor (256 bytes; one per phase in the workspace plan)
+// ---------------------------------------------------------------------------
+struct alignas(16) PD {
+  int kind, layer, n, k;         // PK_*, layer, GEMV rows / columns
+  int kcw, ub, xsrc, epi;        // k per unit, unit bytes, XS_*, EPI_*
+  Geo g;                         // GEMV geometry (24 bytes)
+  int rows_valid, ostride;       // rows that exist; row stride of `out`
+  const uint8_t* blob;           // GEMV units
+  const uint16_t* xbf;           // 16-bit input rows (XS_BF16 / XS_F16; standalone attention: q)
+  const float* xres;             // residual (XS_RESID / XS_FINAL)
+  const float* vpart;            // producer slabs [vns][B][vstride] (XS_RESID / XS_FINAL / XS_SILU / reduce)
+  const float* gain;             // RMSNorm gain of the branch
+  const float* gain2;            // final RMSNorm gain (XS_FINAL)
+  float* xdst;                   // new residual copy
+  float* dump;                   // per-layer hidden dump
+  void* out;                     // EPI_PART: fp32 slab base [ns][B][ostride]; EPI_SILU: 16-bit [B][ostride]
+  float* aux;                    // reduce: per-16-row sums of squares
+  int xbf_stride, vns, vstride, out_f16;
+  int type, newkv, slots, seqoff;  // attention: layer type, append new k/v, cache slots, first sequence
+  const uint8_t* kc;             // attention K region
+  const uint8_t* vc;             // attention V region
+  uint16_t* aout;                // attention output [B][nq][hd]
+  const float* qpart;            // QKV slabs [qns][B][qkv_dim]
+  const float* lpart;            // lm_head slabs [lns][B][vocab]
+  const float* qnorm;            // QK-norm gains
+  const float* knorm;
+  int qns, lns, red_epi, pad_;
 };
+static_assert(sizeof(PD) == 256, "phase descriptor size");
 
-static_assert(sizeof(PD) <= 512, "phase descriptor slot");
+// Launch constants (shared memory).
+struct LC {
+  int B, d, nq, nkv, ffn, vocab, window, nc;
+  int mode, begin, end, n_layers, seq0, pos_const, trace_phases, max_ctx;
+  float eps, mscale0, mscale1;
+  int cur_phase;
+  int scaled;  // some x row of this phase is range-scaled
+  int final_norm, pad0, pad1;
+  uint32_t* ctl;
+  uint32_t* seg_ctr;
+  float* apart;
+  float* amax_val;
+  int32_t* amax_idx;
+  PD* plan;
+  uint64_t* trace;
+  const int32_t* tokens;
+  const uint16_t* embed;
+  float* logits;
+  int32_t* next_token;
+  const int32_t* pos;
+};
+static_assert(sizeof(LC) <= 256, "launch constants");
 
-struct Cursor {
-  int p;     // phase
-  int kind;  // PK_* of the phase, -1 past the last phase
-  int i, end;  // unit index in [i, end) (GEMV: phase order; attention: CTA unit)
-  // GEMV:      p0 = weights, x0 = unit bytes, x1 = k-chunks per row block,
-  //            x2 = k-chunks per slab, x3 = row blocks, x4 = slab, x5 = row
-  //            block, x6 = k-chunk within the slab (all of unit i)
-  // attention: p0 = K region, p1 = V region, x0 = slots, x1 = first sequence,
-  //            x2 = layer type, x3 = segment of unit i
+// A warp's position in its unit stream.
+//   GEMV:      p0 = units, x0 = unit bytes, x1 = k-chunks per row block, x2 =
+//              k-chunks per slab, x3 = row blocks, x4 / x5 / x6 = slab / row
+//              block / k-chunk of unit i
+//   attention: p0 / p1 = K / V regions, x0 = slots, x1 = first sequence, x2 =
+//              layer type, x3 = segment of unit i
+// kind: PK_* of phase p; CUR_DONE past the launch; CUR_WAIT when phase p's
+// descriptor is not in shared memory yet.
+constexpr int CUR_DONE = -1, CUR_WAIT = -2;
+struct alignas(16) Cursor {
+  int p, kind, i, end;
   const uint8_t* p0;
   const uint8_t* p1;
-  int x0, x1, x2, x3, x4, x5, x6;
+  int x0, x1, x2, x3, x4, x5, x6, pad_;
 };
+struct alignas(16) Ring {
+  uint32_t consumed, issued, pf_issued;
+  int bad;  // a wait of this warp timed out: stop waiting and issuing
+  Cursor ld;  // next unit to copy into the ring
+  Cursor pf;  // next unit to request into L2
+};
+static_assert(sizeof(Cursor) == 64 && sizeof(Ring) == 144, "ring state layout");
 
-// Ring state of a warp (a local value that only inlined code touches, so it
-// stays in registers through the unit loops).
-struct Stream {
-  uint32_t consumed, issued;
-  bool bad;   // this warp saw a timeout: stop waiting and issuing
-  Cursor ld;  // next unit to copy into the ring (kind < 0: none left)
-};
+// ---------------------------------------------------------------------------
+// Shared memory map
+// ---------------------------------------------------------------------------
+constexpr int SM_RING = 0;
+constexpr int SM_MBAR = SM_RING + NW * NSLOT * SLOT_BYTES;
+constexpr int PD_SLOTS = 4;                        // descriptor slots (phase p in slot p % 4)
+constexpr int PD_LEAD = 2;                         // descriptor p is copied at the start of phase p - 2
+constexpr int SM_PDBAR = SM_MBAR + NW * NSLOT * 8;
+constexpr int SM_XS = ((SM_PDBAR + PD_SLOTS * 8 + 127) / 128) * 128;
+constexpr int X_REGION = xs_cap(1) + XSUM_BYTES + wsp_bytes(1);
+static_assert(xs_cap(1) + wsp_bytes(1) == xs_cap(2) + wsp_bytes(2), "x region");
+__host__ __device__ constexpr int sm_xsum(int nb) { return SM_XS + xs_cap(nb); }
+__host__ __device__ constexpr int sm_wsp(int nb) { return sm_xsum(nb) + XSUM_BYTES; }
+constexpr int SM_QS = SM_XS + X_REGION;            // q of a head group, fp32 [MAX_GQ][128]
+constexpr int SM_KNV = SM_QS + MAX_GQ * 128 * 4;    // new k / v, bf16 [2][128]
+constexpr int SM_RED = SM_KNV + 512;                // 64 floats of block reductions
+constexpr int SM_POSB = SM_RED + 256;               // positions [MAX_B]
+constexpr int SM_LB = SM_POSB + MAX_B * 4;          // attended keys [2][MAX_B]
+constexpr int SM_SNEW = SM_LB + 2 * MAX_B * 4;      // slot of the new key [2][MAX_B]
+constexpr int SM_SST = SM_SNEW + 2 * MAX_B * 4;     // segment starts [2][MAX_SEG + 1]
+constexpr int SM_FLAGS = SM_SST + ((2 * (MAX_SEG + 1) * 4 + 15) / 16) * 16;
+constexpr int SM_LC = SM_FLAGS + 64;
+constexpr int SM_ROPE = SM_LC + 256;                // inverse frequencies, fp64 [2][64]
+constexpr int SM_PD = SM_ROPE + 2 * 64 * 8;         // descriptor slots
+constexpr int SM_WST = SM_PD + PD_SLOTS * (int)sizeof(PD);  // ring state per warp
+constexpr int SM_TOTAL = SM_WST + NW * (int)sizeof(Ring);
+static_assert(SM_TOTAL <= 232448, "shared memory budget");
+// attention views of the x region
+constexpr int ATT_PW = MAX_GQ * (128 + 2);                // floats of one warp's partial
+constexpr int SM_APW = SM_XS;                             // warp partials [NW][ATT_PW]
+constexpr int SM_QF = SM_XS + NW * ATT_PW * 4;            // q fragments (4 KB)
+constexpr int SM_ASCR = SM_QF + 4096;                     // k, v rows fp32 [2][128], sums [2][NW]
+static_assert(SM_ASCR + 2 * 128 * 4 + 2 * NW * 4 <= SM_XS + X_REGION, "attention scratch");
 
-// Per-warp ring addresses and ids, held in registers by the unit loops.
-struct RingCtx {
-  uint8_t* base;   // slot 0 of this warp's ring
-  uint64_t* bar;   // mbarrier of slot 0
-  uint32_t* err;   // device error word
-  int lane;
-};
+extern __shared__ __align__(128) uint8_t w4a_smem[];
 
-template <int NB>
-struct Acc {
-  float v[NB][4];
-};
+template <class T>
+__device__ __forceinline__ T* sm_at(int off) {
+  return reinterpret_cast<T*>(w4a_smem + off);
+}
+__device__ __forceinline__ LC& lc() { return *sm_at<LC>(SM_LC); }
+__device__ __forceinline__ PD& pd_slot(int p) {
+  return *sm_at<PD>(SM_PD + (p & (PD_SLOTS - 1)) * (int)sizeof(PD));
+}
+__device__ __forceinline__ uint64_t* pd_bar(int p) { return sm_at<uint64_t>(SM_PDBAR) + (p & (PD_SLOTS - 1)); }
+__device__ __forceinline__ Ring* ring_state(int w) { return sm_at<Ring>(SM_WST) + w; }
+__device__ __forceinline__ uint64_t* ring_bar(int w, int s) { return sm_at<uint64_t>(SM_MBAR) + w * NSLOT + s; }
+__device__ __forceinline__ uint8_t* ring_slot(int w, int s) {
+  return sm_at<uint8_t>(SM_RING + (w * NSLOT + s) * SLOT_BYTES);
+}
+__device__ __forceinline__ float* red() { return sm_at<float>(SM_RED); }
+__device__ __forceinline__ int* posb() { return sm_at<int>(SM_POSB); }
+__device__ __forceinline__ int* Lb(int type) { return sm_at<int>(SM_LB) + type * MAX_B; }
+__device__ __forceinline__ int* snew(int type) { return sm_at<int>(SM_SNEW) + type * MAX_B; }
+__device__ __forceinline__ int* sst(int type) { return sm_at<int>(SM_SST) + type * (MAX_SEG + 1); }
+__device__ __forceinline__ int* flags() { return sm_at<int>(SM_FLAGS); }
+__device__ __forceinline__ const double* rope_f(int type) { return sm_at<double>(SM_ROPE) + type * 64; }
 
-template <int NB>
-struct Lay {
-  static constexpr int RING = 0;
-  static constexpr int MBAR = RING + NW * NSLOT * SLOT_BYTES;
-  static constexpr int XS = MBAR + NW * NSLOT * 8;
-  static constexpr int XSUM = XS + xs_cap(NB);
-  static constexpr int WSP = XSUM + XSUM_BYTES;
-  static constexpr int QS = WSP + wsp_bytes(NB);
-  static constexpr int KNV = QS + MAX_GQ * 128 * 4;
-  static constexpr int RED = KNV + 512;
-  static constexpr int POSB = RED + 64 * 4;
-  static constexpr int LB = POSB + MAX_B * 4;
-  static constexpr int SNEW = LB + 2 * MAX_B * 4;
-  static constexpr int SST = SNEW + 2 * MAX_B * 4;
-  static constexpr int FLAGS = SST + 2 * (MAX_SEG + 1) * 4;
-  static constexpr int PDS = FLAGS + 64;
-  static constexpr int TOTAL = PDS + 512;
-  static constexpr int APW_BYTES = xs_cap(NB) + XSUM_BYTES + wsp_bytes(NB);  // attention warp partials
-  static constexpr int QF = XS + NW * MAX_GQ * (128 + 2) * 4;                 // q fragments (after the partials)
-};
-static_assert(Lay<1>::TOTAL <= 232448 && Lay<2>::TOTAL <= 232448, "shared memory budget");
-static_assert(Lay<1>::QF + 4096 <= Lay<1>::XS + Lay<1>::APW_BYTES, "q fragments overlap");
-static_assert(Lay<2>::QF + 4096 <= Lay<2>::XS + Lay<2>::APW_BYTES, "q fragments overlap");
+// Warp barrier that is also a compiler memory barrier: shared-memory state
+// written by one lane (under `if (lane == 0)`) must be re-read by the others
+// after it, never forwarded from a load the compiler hoisted above it.
+__device__ __forceinline__ void warp_sync() {
+  asm volatile("" ::: "memory");
+  __syncwarp();
+  asm volatile("" ::: "memory");
+}
+
+// barrier over the CTA's warps (named barrier 1)
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
+__device__ __forceinline__ void set_error(uint32_t bits) { atomicOr(lc().ctl + 2, bits); }
+
+__device__ __forceinline__ void mark(int slot) {
+  const LC& L = lc();
+  if (L.trace != nullptr && threadIdx.x == 0 && L.cur_phase < L.trace_phases)
+    L.trace[((size_t)L.cur_phase * L.nc + blockIdx.x) * 8 + slot] = globaltimer();
+}
 
 // cos / sin of the rotation angle pos * f, times the attention factor: the
 // angle is formed and reduced to [-pi, pi] in fp64, then evaluated in fp32.
-__device__ __forceinline__ void rope_cs(int pos, double f, float ms, float& c, float& s) {
+__device__ __noinline__ float2 rope_cs2(int pos, double f, float ms) {
   const double a = double(pos) * f;
   const double r = a - 6.283185307179586 * rint(a * 0.15915494309189535);
   float sn, cs;
   sincosf(float(r), &sn, &cs);
-  c = cs * ms;
-  s = sn * ms;
+  return make_float2(cs * ms, sn * ms);
+}
+__device__ __forceinline__ void rope_cs(int pos, double f, float ms, float& c, float& s) {
+  const float2 r = rope_cs2(pos, f, ms);
+  c = r.x;
+  s = r.y;
 }
 
 __device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
@@ -220,78 +290,1055 @@ __device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
 }
 
 // ---------------------------------------------------------------------------
-// Unit kernels (one warp, one unit)
+// Phase descriptors, built on the device from the launch parameters
 // ---------------------------------------------------------------------------
-template <int NB>
-__device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint4* xs4, int xrow4, int ks0,
-                                        const float* xsum, int grp0, float (&acc)[NB][4], int B, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const uint4* qw = reinterpret_cast<const uint4*>(slot);
-  const uint16_t* sc = reinterpret_cast<const uint16_t*>(slot + 4096);
-  const uint32_t* zw = reinterpret_cast<const uint32_t*>(slot + 4224);
-#pragma unroll
-  for (int grp = 0; grp < 4; ++grp) {
-    const uint4 w0 = qw[(grp * 2) * 32 + lane];
-    const uint4 w1 = qw[(grp * 2 + 1) * 32 + lane];
-    uint4 xv[NB][4];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const int bb = g + 8 * nb;
-#pragma unroll
-      for (int pr = 0; pr < 4; ++pr) {
-        const int ks = ks0 + grp * 8 + pr * 2;
-        xv[nb][pr] = (bb < B) ? xs4[bb * xrow4 + (ks >> 1) * 4 + t] : make_uint4(0u, 0u, 0u, 0u);
+__device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
+  uint4* z = reinterpret_cast<uint4*>(out);
+#pragma unroll 1
+  for (int i = 0; i < (int)(sizeof(PD) / 16); ++i) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  PD& d = *out;
+  const int B = P.B;
+  if (P.mode == MODE_GEMV) {
+    d.kind = (p == 0) ? PK_GEMV_W4 : PK_REDUCE;
+    d.blob = P.g_blob;
+    d.n = P.g_n;
+    d.k = P.g_k;
+    d.kcw = W4_KC;
+    d.ub = W4_UNIT;
+    d.xsrc = XS_BF16;
+    d.xbf = P.g_x;
+    d.xbf_stride = P.g_k;
+    d.rows_valid = P.g_n;
+    d.g = P.geo[0];
+    const bool direct_silu = P.g_epi == W4A_EPI_SILU_MUL && d.g.ns == 1;
+    const bool direct = P.g_epi == W4A_EPI_NONE && d.g.ns == 1;
+    if (direct_silu) {
+      d.epi = EPI_SILU;
+      d.out = P.g_out;
+      d.ostride = P.g_n / 2;
+    } else {
+      d.epi = EPI_PART;
+      d.out = direct ? P.g_out : P.ws.g_part;
+      d.ostride = P.g_n;
+    }
+    if (p == 1) {  // sum the slabs, then the requested epilogue
+      d.vpart = P.ws.g_part;
+      d.vns = d.g.ns;
+      d.out = P.g_out;
+      d.aux = P.g_aux;
+      d.red_epi = P.g_epi;
+    }
+    return;
+  }
+  if (P.mode == MODE_ATTN) {
+    d.kind = PK_ATTN;
+    d.slots = P.a_slots;
+    d.kc = reinterpret_cast<const uint8_t*>(P.a_k);
+    d.vc = reinterpret_cast<const uint8_t*>(P.a_v);
+    d.aout = P.a_out;
+    d.xbf = P.a_q;
+    return;
+  }
+  const int nl = P.n_layers, dm = P.d;
+  const int qd = P.nq * P.hd, qkv_dim = (P.nq + 2 * P.nkv) * P.hd;
+  const Geo& g_qkv = P.geo[0];
+  const Geo& g_o = P.geo[1];
+  const Geo& g_gu = P.geo[2];
+  const Geo& g_dn = P.geo[3];
+  const Geo& g_lm = P.geo[4];
+  if (p == 5 * nl) {
+    d.kind = PK_GEMV_BF16;
+    d.blob = P.lm_head;
+    d.n = (P.vocab + RB - 1) / RB * RB;
+    d.k = dm;
+    d.kcw = BF_KC;
+    d.ub = BF_UNIT;
+    d.g = g_lm;
+    d.xsrc = XS_FINAL;
+    d.xres = P.ws.xB;
+    d.vpart = P.ws.f_part;
+    d.vns = g_dn.ns;
+    d.vstride = dm;
+    d.gain = P.layers[nl - 1].ffn_norm;
+    d.gain2 = P.final_norm ? P.final_gain : nullptr;
+    d.dump = P.dump ? P.dump + (size_t)nl * B * dm : nullptr;
+    d.rows_valid = P.vocab;
+    d.epi = EPI_PART;
+    d.out = (g_lm.ns == 1) ? P.logits : P.ws.lg_part;
+    d.ostride = P.vocab;
+    return;
+  }
+  if (p == 5 * nl + 1) {
+    d.kind = PK_ARGMAX;
+    d.lpart = g_lm.ns > 1 ? P.ws.lg_part : nullptr;
+    d.lns = g_lm.ns;
+    return;
+  }
+  const int l = p / 5, sub = p % 5;
+  const LayerPtrs& lw = P.layers[l];
+  d.layer = l;
+  if (sub == 1) {
+    d.kind = PK_ATTN;
+    d.type = P.full[l] ? 1 : 0;
+    d.newkv = 1;
+    d.seqoff = P.seq0;
+    d.slots = P.kv_slots[l];
+    d.kc = P.kv_base + P.kv_off[l];
+    d.vc = d.kc + (size_t)P.kv_batch * P.nkv * d.slots * P.hd * 2;
+    d.aout = P.ws.o;
+    d.out_f16 = 1;
+    d.qpart = P.ws.y_part;
+    d.qns = g_qkv.ns;
+    d.qnorm = lw.q_norm;
+    d.knorm = lw.k_norm;
+    return;
+  }
+  d.kind = PK_GEMV_W4;
+  d.kcw = W4_KC;
+  d.ub = W4_UNIT;
+  d.rows_valid = 1 << 30;
+  d.epi = EPI_PART;
+  if (sub == 0) {
+    d.blob = lw.qkv;
+    d.n = qkv_dim;
+    d.k = dm;
+    d.g = g_qkv;
+    if (l == 0) {
+      d.xsrc = XS_EMBED;
+    } else {
+      d.xsrc = XS_RESID;
+      d.xres = P.ws.xB;
+      d.vpart = P.ws.f_part;
+      d.vns = g_dn.ns;
+      d.vstride = dm;
+      d.gain = P.layers[l - 1].ffn_norm;
+    }
+    d.xdst = P.ws.xA;
+    d.dump = P.dump ? P.dump + (size_t)l * B * dm : nullptr;
+    d.out = P.ws.y_part;
+    d.ostride = qkv_dim;
+  } else if (sub == 2) {
+    d.blob = lw.o;
+    d.n = dm;
+    d.k = qd;
+    d.g = g_o;
+    d.xsrc = XS_F16;
+    d.xbf = P.ws.o;
+    d.xbf_stride = qd;
+    d.out = P.ws.a_part;
+    d.ostride = dm;
+  } else if (sub == 3) {
+    d.blob = lw.gu;
+    d.n = 2 * P.ffn;
+    d.k = dm;
+    d.g = g_gu;
+    d.xsrc = XS_RESID;
+    d.xres = P.ws.xA;
+    d.vpart = P.ws.a_part;
+    d.vns = g_o.ns;
+    d.vstride = dm;
+    d.gain = lw.attn_norm;
+    d.xdst = P.ws.xB;
+    if (d.g.ns == 1) {
+      d.epi = EPI_SILU;
+      d.out = P.ws.h;
+      d.ostride = P.ffn;
+      d.out_f16 = 1;
+    } else {
+      d.out = P.ws.gu_part;
+      d.ostride = 2 * P.ffn;
+    }
+  } else {
+    d.blob = lw.down;
+    d.n = dm;
+    d.k = P.ffn;
+    d.g = g_dn;
+    if (g_gu.ns == 1) {
+      d.xsrc = XS_F16;
+      d.xbf = P.ws.h;
+      d.xbf_stride = P.ffn;
+    } else {
+      d.xsrc = XS_SILU;
+      d.vpart = P.ws.gu_part;
+      d.vns = g_gu.ns;
+      d.vstride = 2 * P.ffn;
+    }
+    d.out = P.ws.f_part;
+    d.ostride = dm;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Ranges
+// ---------------------------------------------------------------------------
+// A GEMV CTA owns whole segments: units [a, b) of the phase order.
+__device__ __forceinline__ void gemv_cta_range(const Geo& g, int cta, int& a, int& b) {
+  if (cta < g.nca) {
+    a = int(rstart(g.nseg, g.nca, cta)) * g.kps;
+    b = int(rstart(g.nseg, g.nca, cta + 1)) * g.kps;
+  } else {
+    a = b = 0;
+  }
+}
+__device__ __forceinline__ void warp_range(int a, int b, int w, int& wa, int& wb) {
+  wa = a + (b - a) * w / NW;
+  wb = a + (b - a) * (w + 1) / NW;
+}
+__device__ __forceinline__ void attn_cta_range(int type, int cta, int& a, int& b, int& nca) {
+  const LC& L = lc();
+  const int total = sst(type)[L.B * L.nkv];
+  nca = total < L.nc ? total : L.nc;
+  if (nca > 0 && cta < nca) {
+    a = int(rstart(total, nca, cta));
+    b = int(rstart(total, nca, cta + 1));
+  } else {
+    a = b = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Unit streams: cursors, the ring, the L2 prefetch
+// ---------------------------------------------------------------------------
+// Is phase q's descriptor in shared memory?  Descriptors begin .. begin +
+// PD_LEAD are built in shared memory at launch; descriptor q after them is
+// copied at the start of phase q - PD_LEAD (the k-th copy into its slot
+// completes mbarrier phase k).  `block`: wait for a copy under way (bounded);
+// else only test it.
+__device__ __noinline__ bool pd_ready(int q, bool block) {
+  const LC& L = lc();
+  if (q <= L.begin + PD_LEAD) return true;
+  if (L.cur_phase < q - PD_LEAD) return false;  // copy not issued yet
+  const uint32_t par = uint32_t((q - L.begin - PD_LEAD - 1) / PD_SLOTS) & 1u;
+  if (mbar_try_wait(pd_bar(q), par)) return true;
+  if (!block) return false;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(pd_bar(q), par)) {
+    if (clock64() - t0 > WAIT_CYCLES) {
+      set_error(EW_MBAR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Position cursor c at the first unit of warp w in phase q.
+__device__ __noinline__ void cur_enter(Cursor* c, int q, int w) {
+  const LC& L = lc();
+  c->p = q;
+  c->i = c->end = 0;
+  if (q >= L.end) {
+    c->kind = CUR_DONE;
+    return;
+  }
+  if (!pd_ready(q, false)) {
+    c->kind = CUR_WAIT;
+    return;
+  }
+  const PD& d = pd_slot(q);
+  c->kind = d.kind;
+  if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_BF16) {
+    int a, b, wa, wb;
+    gemv_cta_range(d.g, blockIdx.x, a, b);
+    warp_range(a, b, w, wa, wb);
+    c->p0 = d.blob;
+    c->x0 = d.ub;
+    c->x1 = d.g.nkc;
+    c->x2 = d.g.kps;
+    c->x3 = d.g.nrb;
+    c->i = wa;
+    c->end = wb;
+    const int upsl = d.g.nrb * d.g.kps;
+    c->x4 = wa / upsl;
+    const int r = wa - c->x4 * upsl;
+    c->x5 = r / d.g.kps;
+    c->x6 = r - c->x5 * d.g.kps;
+  } else if (d.kind == PK_ATTN) {
+    int a, b, nca;
+    attn_cta_range(d.type, blockIdx.x, a, b, nca);
+    c->i = a;
+    c->end = b;
+    c->p0 = d.kc;
+    c->p1 = d.vc;
+    c->x0 = d.slots;
+    c->x1 = d.seqoff;
+    c->x2 = d.type;
+    c->x3 = 0;
+  }
+}
+
+// Move c to warp w's next unit at or after its position (possibly in a later
+// phase).  Stops on CUR_DONE or CUR_WAIT.
+__device__ __noinline__ void cur_normalize(Cursor* c, int w) {
+  const LC& L = lc();
+#pragma unroll 1
+  for (;;) {
+    const int kind = c->kind;
+    if (kind == CUR_DONE) return;
+    if (kind == CUR_WAIT) {
+      if (!pd_ready(c->p, false)) return;
+      cur_enter(c, c->p, w);
+      continue;
+    }
+    if (kind == PK_GEMV_W4 || kind == PK_GEMV_BF16) {
+      if (c->i < c->end) return;
+    } else if (kind == PK_ATTN) {
+      const int* st = sst(c->x2);
+#pragma unroll 1
+      while (c->i < c->end) {
+        while (st[c->x3 + 1] <= c->i) ++c->x3;
+        const int key0 = (c->i - st[c->x3]) * ATT_CTA_KEYS + w * ATT_KEYS;
+        if (key0 < Lb(c->x2)[c->x3 / L.nkv]) return;
+        ++c->i;
       }
     }
+    cur_enter(c, c->p + 1, w);
+  }
+}
+
+__device__ __forceinline__ void cur_load(Cursor& c, const Cursor* s) {
+  const uint4* q = reinterpret_cast<const uint4*>(s);
+  const uint4 v0 = q[0], v1 = q[1], v2 = q[2], v3 = q[3];
+  c.p = int(v0.x);
+  c.kind = int(v0.y);
+  c.i = int(v0.z);
+  c.end = int(v0.w);
+  c.p0 = reinterpret_cast<const uint8_t*>((uint64_t(v1.y) << 32) | v1.x);
+  c.p1 = reinterpret_cast<const uint8_t*>((uint64_t(v1.w) << 32) | v1.z);
+  c.x0 = int(v2.x);
+  c.x1 = int(v2.y);
+  c.x2 = int(v2.z);
+  c.x3 = int(v2.w);
+  c.x4 = int(v3.x);
+  c.x5 = int(v3.y);
+  c.x6 = int(v3.z);
+  c.pad_ = 0;
+}
+__device__ __forceinline__ void cur_store(Cursor* s, const Cursor& c) {
+  uint4* q = reinterpret_cast<uint4*>(s);
+  const uint64_t a = reinterpret_cast<uint64_t>(c.p0), b = reinterpret_cast<uint64_t>(c.p1);
+  q[0] = make_uint4(uint32_t(c.p), uint32_t(c.kind), uint32_t(c.i), uint32_t(c.end));
+  q[1] = make_uint4(uint32_t(a), uint32_t(a >> 32), uint32_t(b), uint32_t(b >> 32));
+  q[2] = make_uint4(uint32_t(c.x0), uint32_t(c.x1), uint32_t(c.x2), uint32_t(c.x3));
+  q[3] = make_uint4(uint32_t(c.x4), uint32_t(c.x5), uint32_t(c.x6), 0u);
+}
+
+// Next unit of a register cursor (which = 0: ring cursor, 1: prefetch cursor);
+// the slow path goes through the warp's shared-memory copy.
+__device__ __forceinline__ void cur_next(Cursor& c, int which, int warp, int lane) {
+  if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
+    ++c.i;
+    if (++c.x6 == c.x2) {
+      c.x6 = 0;
+      if (++c.x5 == c.x3) {
+        c.x5 = 0;
+        ++c.x4;
+      }
+    }
+    if (c.i < c.end) return;
+  } else {
+    ++c.i;
+  }
+  Cursor* s = which ? &ring_state(warp)->pf : &ring_state(warp)->ld;
+  // lanes run independently between warp barriers: every lane must be done
+  // reading the shared copy before lane 0 rewrites it
+  warp_sync();
+  if (lane == 0) {
+    cur_store(s, c);
+    cur_normalize(s, warp);
+  }
+  warp_sync();
+  cur_load(c, s);
+}
+
+// Source range(s) of the unit under a cursor.
+__device__ __forceinline__ void cur_src(const Cursor& c, int warp, const uint8_t*& s1, const uint8_t*& s2,
+                                        uint32_t& bytes, int hd) {
+  if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
+    const uint32_t idx = uint32_t(c.x5 * c.x1 + c.x4 * c.x2 + c.x6);
+    s1 = c.p0 + (size_t)idx * uint32_t(c.x0);
+    s2 = nullptr;
+    bytes = uint32_t(c.x0);
+  } else {
+    const LC& L = lc();
+    const int* st = sst(c.x2);
+    const int bq = c.x3 / L.nkv, g = c.x3 - bq * L.nkv;
+    const int key0 = (c.i - st[c.x3]) * ATT_CTA_KEYS + warp * ATT_KEYS;
+    const size_t row = ((size_t)(c.x1 + bq) * L.nkv + g) * c.x0 + key0;
+    bytes = ATT_KEYS * hd * 2;
+    s1 = c.p0 + row * hd * 2;
+    s2 = c.p1 + row * hd * 2;
+  }
+}
+
+__device__ __forceinline__ void ring_load(Ring& R, int warp) {
+  const Ring* s = ring_state(warp);
+  const uint4 h = *reinterpret_cast<const uint4*>(s);
+  R.consumed = h.x;
+  R.issued = h.y;
+  R.pf_issued = h.z;
+  R.bad = int(h.w);
+  cur_load(R.ld, &s->ld);
+  cur_load(R.pf, &s->pf);
+}
+__device__ __forceinline__ void ring_store(const Ring& R, int warp, int lane) {
+  warp_sync();  // all lanes are done reading the shared copy
+  if (lane == 0) {
+    Ring* s = ring_state(warp);
+    *reinterpret_cast<uint4*>(s) = make_uint4(R.consumed, R.issued, R.pf_issued, uint32_t(R.bad));
+    cur_store(&s->ld, R.ld);
+    cur_store(&s->pf, R.pf);
+  }
+  warp_sync();
+}
+
+// Fill free ring slots (and keep the L2 requests PF_AHEAD units ahead).
+template <int HD>
+__device__ __forceinline__ void ring_fill(Ring& R, int warp, int lane) {
+#pragma unroll 1
+  while (!R.bad && R.ld.kind >= 0 && R.issued - R.consumed < uint32_t(NSLOT)) {
+#pragma unroll 1
+    while (R.pf.kind >= 0 && R.pf_issued < R.issued + 1u + uint32_t(PF_AHEAD)) {
+      const uint8_t *s1, *s2;
+      uint32_t bytes;
+      cur_src(R.pf, warp, s1, s2, bytes, HD);
+      if (lane == 0 && R.pf_issued > R.issued) {  // the ring's own next unit needs no request
+        bulk_prefetch_l2(s1, bytes);
+        if (s2) bulk_prefetch_l2(s2, bytes);
+      }
+      ++R.pf_issued;
+      cur_next(R.pf, 1, warp, lane);
+    }
+    const int sl = R.issued % NSLOT;
+    const uint8_t *s1, *s2;
+    uint32_t bytes;
+    cur_src(R.ld, warp, s1, s2, bytes, HD);
+    if (lane == 0) {
+      uint64_t* bar = ring_bar(warp, sl);
+      uint8_t* dst = ring_slot(warp, sl);
+      mbar_expect_tx(bar, s2 ? 2 * bytes : bytes);
+      bulk_g2s(dst, s1, bytes, bar);
+      if (s2) bulk_g2s(dst + bytes, s2, bytes, bar);
+    }
+    ++R.issued;
+    cur_next(R.ld, 0, warp, lane);
+  }
+}
+
+__device__ __forceinline__ uint8_t* ring_wait(Ring& R, int warp, int lane) {
+  const int sl = R.consumed % NSLOT;
+  const uint32_t par = (R.consumed / NSLOT) & 1u;
+  uint64_t* bar = ring_bar(warp, sl);
+  int late = 0;
+  if (!R.bad && !mbar_try_wait(bar, par)) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, par)) {
+      if (clock64() - t0 > WAIT_CYCLES) {
+        late = 1;
+        break;
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, late)) {  // keep the warp's ring state uniform
+    if (lane == 0) set_error(EW_MBAR_TIMEOUT);
+    R.bad = 1;
+  }
+  return ring_slot(warp, sl);
+}
+// Hand the slot back and refill the ring.
+template <int HD>
+__device__ __forceinline__ void ring_release(Ring& R, int warp, int lane, bool wrote_slot) {
+  // order generic accesses of the slot before the async re-fill (every lane
+  // when lanes wrote into the slot, else lane 0 after the warp's reads)
+  if (wrote_slot) fence_proxy_async();
+  warp_sync();
+  if (!wrote_slot && lane == 0) fence_proxy_async();
+  ++R.consumed;
+  ring_fill<HD>(R, warp, lane);
+}
+
+// Resume waiting cursors and fill the ring (phase start).
+template <int HD>
+__device__ __noinline__ void ring_top_up() {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Ring* s = ring_state(warp);
+  warp_sync();
+  if (lane == 0) {
+    if (s->ld.kind == CUR_WAIT) cur_normalize(&s->ld, warp);
+    if (s->pf.kind == CUR_WAIT) cur_normalize(&s->pf, warp);
+  }
+  warp_sync();
+  Ring R;
+  ring_load(R, warp);
+  ring_fill<HD>(R, warp, lane);
+  ring_store(R, warp, lane);
+}
+
+__device__ __noinline__ void ring_drain() {
+  const int warp = threadIdx.x >> 5;
+  const Ring* s = ring_state(warp);
+  uint32_t c = s->consumed;
+  const uint32_t iss = s->issued;
+#pragma unroll 1
+  while (c < iss) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(ring_bar(warp, c % NSLOT), (c / NSLOT) & 1u)) {
+      if (clock64() - t0 > WAIT_CYCLES) {
+        if ((threadIdx.x & 31) == 0) set_error(EW_DRAIN_TIMEOUT);
+        return;
+      }
+    }
+    ++c;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Grid barrier
+// ---------------------------------------------------------------------------
+__device__ __noinline__ bool grid_wait(uint32_t target) {
+  if (threadIdx.x == 0) {
+    const LC& L = lc();
+    int ok = 1;
+    const long long t0 = clock64();
+    while (ld_acquire(L.ctl) < target) {
+      if (ld_volatile_u32(L.ctl + 2) != 0u) {
+        ok = 0;
+        break;
+      }
+      if (clock64() - t0 > WAIT_CYCLES) {
+        set_error(EW_BARRIER_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+    flags()[0] = ok;
+  }
+  cbar();
+  return flags()[0] != 0;
+}
+__device__ __forceinline__ void grid_arrive() {
+  cbar();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    red_release_add(lc().ctl, 1u);
+  }
+}
+
+// Deterministic per-batch-row totals of per-warp partial sums wsum[warp][b].
+__device__ __forceinline__ void block_rows_total(const float* wsum, float* out, int B) {
+  cbar();
+  if ((int)threadIdx.x < B) {
+    float s = 0.f;
+#pragma unroll 1
+    for (int w = 0; w < NW; ++w) s += wsum[w * MAX_B + threadIdx.x];
+    out[threadIdx.x] = s;
+  }
+  cbar();
+}
+
+// ---------------------------------------------------------------------------
+// GEMV input staging
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+
+struct F8 {
+  float v[8];
+};
+__device__ __forceinline__ F8 f8(const float (&a)[8]) {
+  F8 r;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r.v[i] = a[i];
+  return r;
+}
+
+// Sum of `ns` slabs (stride sstride floats) at p[0 .. 8), in slab order, loads
+// of up to four slabs in flight.
+__device__ __noinline__ F8 slab_sum8v(const float* p, size_t sstride, int ns) {
+  F8 r;
+  float* v = r.v;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = 0.f;
+#pragma unroll 1
+  for (int s0 = 0; s0 < ns; s0 += 4) {
+    float4 a[4], b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[i] = b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s0 + i < ns) {
+        a[i] = ldcg4(p + (s0 + i) * sstride);
+        b[i] = ldcg4(p + (s0 + i) * sstride + 4);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (s0 + i < ns) {
+        v[0] += a[i].x;
+        v[1] += a[i].y;
+        v[2] += a[i].z;
+        v[3] += a[i].w;
+        v[4] += b[i].x;
+        v[5] += b[i].y;
+        v[6] += b[i].z;
+        v[7] += b[i].w;
+      }
+    }
+  }
+  return r;
+}
+__device__ __forceinline__ void slab_sum8(const float* p, size_t sstride, int ns, float (&v)[8]) {
+  const F8 r = slab_sum8v(p, sstride, ns);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = r.v[i];
+}
+
+__device__ __forceinline__ void cvt16(bool f16, const uint4& u, float (&v)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint16_t lo = uint16_t(w[i] & 0xffffu), hi = uint16_t(w[i] >> 16);
+    v[2 * i] = f16 ? half_bits_to_f32(lo) : bf16_to_f32(lo);
+    v[2 * i + 1] = f16 ? half_bits_to_f32(hi) : bf16_to_f32(hi);
+  }
+}
+
+// Store eight activations x[bb][kl0 .. kl0 + 8) (kl0 relative to the staged
+// range) as fp16 (f16) or bf16, times `scale`.  The 16 lanes of a half-warp
+// hold one 128-group, whose sum (of the stored, rounded values) and max |x|
+// they reduce here.  Warp-uniform: every lane calls it.
+template <int NB>
+__device__ __noinline__ void put8(bool valid, int bb, int kl0, int xrow_b, F8 vv, bool f16, float scale,
+                                  bool track_max) {
+  const float* v = vv.v;
+  const int lane = threadIdx.x & 31;
+  float s8 = 0.f, m8 = 0.f;
+  if (valid) {
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float a = v[2 * t] * scale, b = v[2 * t + 1] * scale;
+      if (f16) {
+        const uint16_t ha = f32_to_f16(a), hb = f32_to_f16(b);
+        w[t] = uint32_t(ha) | (uint32_t(hb) << 16);
+        s8 += half_bits_to_f32(ha) + half_bits_to_f32(hb);
+      } else {
+        const uint16_t ha = f32_to_bf16(a), hb = f32_to_bf16(b);
+        w[t] = uint32_t(ha) | (uint32_t(hb) << 16);
+        s8 += bf16_to_f32(ha) + bf16_to_f32(hb);
+      }
+      m8 = fmaxf(m8, fmaxf(fabsf(v[2 * t]), fabsf(v[2 * t + 1])));
+    }
+    *sm_at<uint4>(SM_XS + bb * xrow_b + kl0 * 2) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) {
+    s8 += __shfl_xor_sync(0xffffffffu, s8, o);
+    m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, o));
+  }
+  if (valid && (lane & 15) == 0) {
+    sm_at<float>(sm_xsum(NB))[(kl0 >> 7) * (8 * NB) + bb] = s8;
+    if (track_max) atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + bb, __float_as_uint(m8));
+  }
+}
+
+__device__ __forceinline__ void store8f(float* p, const float (&x)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+__device__ __forceinline__ void load8f(const float* p, float (&v)[8], bool ro) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+  const float4 a = ro ? __ldg(q) : __ldcg(q);
+  const float4 b = ro ? __ldg(q + 1) : __ldcg(q + 1);
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = a.z;
+  v[3] = a.w;
+  v[4] = b.x;
+  v[5] = b.y;
+  v[6] = b.z;
+  v[7] = b.w;
+}
+
+// Eight inputs of a 16-bit source or the SiLU(gate) * up source at k0.
+__device__ __noinline__ F8 src16_or_silu_v(const PD& d, int bb, int k0) {
+  F8 r;
+  float* v = r.v;
+  const LC& L = lc();
+  if (d.xsrc == XS_SILU) {
+    float ga[8], gb[8];
+    // tiled rows 2j (gate j), 2j + 1 (up j): columns [2 k0, 2 k0 + 16)
+    slab_sum8(d.vpart + (size_t)bb * d.vstride + 2 * k0, (size_t)L.B * d.vstride, d.vns, ga);
+    slab_sum8(d.vpart + (size_t)bb * d.vstride + 2 * k0 + 8, (size_t)L.B * d.vstride, d.vns, gb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[i] = ga[2 * i] / (1.f + expf(-ga[2 * i])) * ga[2 * i + 1];
+      v[4 + i] = gb[2 * i] / (1.f + expf(-gb[2 * i])) * gb[2 * i + 1];
+    }
+    return r;
+  }
+  int tok = 0;
+  if (d.xsrc == XS_EMBED) {
+    tok = L.tokens[bb];
+    tok = tok < 0 ? 0 : (tok >= L.vocab ? L.vocab - 1 : tok);
+  }
+  const uint4 u = (d.xsrc == XS_EMBED)
+                      ? __ldg(reinterpret_cast<const uint4*>(L.embed + (size_t)tok * L.d + k0))
+                      : __ldcg(reinterpret_cast<const uint4*>(d.xbf + (size_t)bb * d.xbf_stride + k0));
+  float w[8];
+  cvt16(d.xsrc == XS_F16, u, w);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = w[i];
+  return r;
+}
+__device__ __forceinline__ void src16_or_silu(const PD& d, int bb, int k0, float (&v)[8]) {
+  const F8 r = src16_or_silu_v(d, bb, k0);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = r.v[i];
+}
+
+// Residual update of one chunk: x = xres + v * r * gain.
+__device__ __forceinline__ void resid8(const float (&v)[8], const float (&xr)[8], const float (&g)[8], float r,
+                                       float (&x)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = fmaf(v[i] * r, g[i], xr[i]);
+}
+
+// Stage x for the CTA's k-range [kbase, kbase + klen) of a GEMV phase.
+template <int NB>
+__device__ __noinline__ void stage_x(const PD& d, int kbase, int klen) {
+  LC& L = lc();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = L.B, dm = L.d;
+  const bool f16 = (d.kind == PK_GEMV_W4);
+  float* rd = red();
+  float* xsm = sm_at<float>(sm_xsum(NB));
+#pragma unroll 1
+  for (int i = tid; i < XSUM_BYTES / 4; i += NT) xsm[i] = 0.f;
+  if (tid < MAX_B) {
+    reinterpret_cast<uint32_t*>(rd + 32)[tid] = 0u;
+    rd[48 + tid] = 1.f;
+  }
+  float* wsum = sm_at<float>(sm_wsp(NB));  // [NW][MAX_B] per-warp sums of squares
+  if (tid < NW * MAX_B) wsum[tid] = 0.f;
+  if (tid == 0) L.scaled = 0;
+  cbar();
+  const int xrow_b = klen * 2 + 64;
+  const bool has_out = (d.xdst != nullptr || d.dump != nullptr);
+  const int nout = B * dm / 8;
+  const int out_per = (nout + L.nc - 1) / L.nc;
+  const int o0 = blockIdx.x * out_per, o1 = min(nout, o0 + out_per);
+
+  if (d.xsrc == XS_RESID || d.xsrc == XS_FINAL) {
+    // Residual update over the whole width: v = sum of the branch slabs,
+    // x = xres + v * rsqrt(mean(v^2) + eps) * gain  [then the final norm].
+    // Chunks of 8; a warp iteration covers 32 consecutive chunks of one batch
+    // row (d % 256 == 0).  Up to two chunks per thread stay in registers.
+    const int n8 = dm / 8, total8 = B * n8;
+    const bool fin = (d.xsrc == XS_FINAL) && d.gain2 != nullptr;
+    const bool two = total8 <= 2 * NT;
+    const size_t sstride = (size_t)B * d.vstride;
+    const int c0 = warp * 32 + lane, c1 = c0 + NT;
+    const bool h0 = warp * 32 < total8, h1 = two && warp * 32 + NT < total8;
+    const int b0 = h0 ? (warp * 32) / n8 : 0, b1 = h1 ? (warp * 32 + NT) / n8 : 0;
+    const int k00 = (c0 - b0 * n8) * 8, k01 = (c1 - b1 * n8) * 8;
+    float v0[8], v1[8], x0[8], x1[8], g0[8], g1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v0[i] = v1[i] = x0[i] = x1[i] = g0[i] = g1[i] = 0.f;
+    // pass 1: branch sums (and, for up to two chunks, residual and gains in flight together)
+    if (two) {
+      if (h0) {
+        slab_sum8(d.vpart + (size_t)b0 * d.vstride + k00, sstride, d.vns, v0);
+        load8f(d.xres + (size_t)b0 * dm + k00, x0, false);
+        load8f(d.gain + k00, g0, true);
+      }
+      if (h1) {
+        slab_sum8(d.vpart + (size_t)b1 * d.vstride + k01, sstride, d.vns, v1);
+        load8f(d.xres + (size_t)b1 * dm + k01, x1, false);
+        load8f(d.gain + k01, g1, true);
+      }
+      float sq0 = 0.f, sq1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        sq0 = fmaf(v0[i], v0[i], sq0);
+        sq1 = fmaf(v1[i], v1[i], sq1);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sq0 += __shfl_xor_sync(0xffffffffu, sq0, o);
+        sq1 += __shfl_xor_sync(0xffffffffu, sq1, o);
+      }
+      if (lane == 0 && h0) wsum[warp * MAX_B + b0] += sq0;
+      if (lane == 0 && h1) wsum[warp * MAX_B + b1] += sq1;
+    } else {
+#pragma unroll 1
+      for (int j = 0; warp * 32 + j * NT < total8; ++j) {
+        const int c = warp * 32 + j * NT + lane, bb = (warp * 32 + j * NT) / n8;
+        float v[8];
+        slab_sum8(d.vpart + (size_t)bb * d.vstride + (c - bb * n8) * 8, sstride, d.vns, v);
+        float sq = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sq = fmaf(v[i], v[i], sq);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) wsum[warp * MAX_B + bb] += sq;
+      }
+    }
+    block_rows_total(wsum, rd, B);
+    if (tid < B) rd[tid] = rsqrtf(rd[tid] / float(dm) + L.eps);
+    cbar();
+    mark(2);
+    if (fin) {
+      // the final norm's sums of squares
+      if (tid < NW * MAX_B) wsum[tid] = 0.f;
+      cbar();
+#pragma unroll 1
+      for (int j = 0; warp * 32 + j * NT < total8; ++j) {
+        const int c = warp * 32 + j * NT + lane, bb = (warp * 32 + j * NT) / n8, k0 = (c - bb * n8) * 8;
+        float x[8];
+        if (two) {
+          if (j == 0)
+            resid8(v0, x0, g0, rd[bb], x);
+          else
+            resid8(v1, x1, g1, rd[bb], x);
+        } else {
+          float v[8], xr[8], g[8];
+          slab_sum8(d.vpart + (size_t)bb * d.vstride + k0, sstride, d.vns, v);
+          load8f(d.xres + (size_t)bb * dm + k0, xr, false);
+          load8f(d.gain + k0, g, true);
+          resid8(v, xr, g, rd[bb], x);
+        }
+        float sq = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sq = fmaf(x[i], x[i], sq);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) wsum[warp * MAX_B + bb] += sq;
+      }
+      block_rows_total(wsum, rd + 16, B);
+      if (tid < B) rd[16 + tid] = rsqrtf(rd[16 + tid] / float(dm) + L.eps);
+      cbar();
+    }
+    // convert the k-range, write the residual copy / dump slice
+#pragma unroll 1
+    for (int j = 0; warp * 32 + j * NT < total8; ++j) {
+      const int c = warp * 32 + j * NT + lane, bb = (warp * 32 + j * NT) / n8, k0 = (c - bb * n8) * 8;
+      float x[8];
+      if (two) {
+        if (j == 0)
+          resid8(v0, x0, g0, rd[bb], x);
+        else
+          resid8(v1, x1, g1, rd[bb], x);
+      } else {
+        float v[8], xr[8], g[8];
+        slab_sum8(d.vpart + (size_t)bb * d.vstride + k0, sstride, d.vns, v);
+        load8f(d.xres + (size_t)bb * dm + k0, xr, false);
+        load8f(d.gain + k0, g, true);
+        resid8(v, xr, g, rd[bb], x);
+      }
+      if (has_out && c >= o0 && c < o1) {
+        if (d.xdst) store8f(d.xdst + (size_t)bb * dm + k0, x);
+        if (d.dump) store8f(d.dump + (size_t)bb * dm + k0, x);
+      }
+      if (fin) {
+        float g2[8];
+        load8f(d.gain2 + k0, g2, true);
+        const float rf = rd[16 + bb];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = x[i] * rf * g2[i];
+      }
+      // half-warps are uniformly inside or outside (128-aligned k-range)
+      put8<NB>(k0 >= kbase && k0 < kbase + klen, bb, k0 - kbase, xrow_b, f8(x), f16, 1.f, f16);
+    }
+  } else {
+    // 16-bit / SiLU sources: the k-range only
+    const int n8 = klen / 8, total8 = B * n8;
+    if (d.xsrc != XS_SILU) {
+      constexpr int JU = 4;  // chunks per thread in flight
+#pragma unroll 1
+      for (int j0 = 0; warp * 32 + j0 * NT < total8; j0 += JU) {
+        uint4 raw[JU];
+#pragma unroll
+        for (int jj = 0; jj < JU; ++jj) {
+          const int c = warp * 32 + (j0 + jj) * NT + lane;
+          raw[jj] = make_uint4(0u, 0u, 0u, 0u);
+          if (c < total8) {
+            const int bb = c / n8;
+            const int k0 = kbase + (c - bb * n8) * 8;
+            if (d.xsrc == XS_EMBED) {
+              const int tok = max(0, min(L.vocab - 1, L.tokens[bb]));
+              raw[jj] = __ldg(reinterpret_cast<const uint4*>(L.embed + (size_t)tok * dm + k0));
+            } else {
+              raw[jj] = __ldcg(reinterpret_cast<const uint4*>(d.xbf + (size_t)bb * d.xbf_stride + k0));
+            }
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < JU; ++jj) {
+          const int cw = warp * 32 + (j0 + jj) * NT;
+          if (cw < total8) {  // warp-uniform (total8 % 32 == 0)
+            const int c = cw + lane, bb = cw / n8;
+            float v[8];
+            cvt16(d.xsrc == XS_F16, raw[jj], v);
+            put8<NB>(true, bb, (c - bb * n8) * 8, xrow_b, f8(v), f16, 1.f, f16);
+          }
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int j = 0; warp * 32 + j * NT < total8; ++j) {
+        const int cw = warp * 32 + j * NT, c = cw + lane, bb = cw / n8;
+        float v[8];
+        src16_or_silu(d, bb, kbase + (c - bb * n8) * 8, v);
+        put8<NB>(true, bb, (c - bb * n8) * 8, xrow_b, f8(v), f16, 1.f, f16);
+      }
+    }
+    mark(2);
+    // residual copy / dump of the embedding (first layer)
+    if (has_out) {
+#pragma unroll 1
+      for (int c = o0 + tid; c < o1; c += NT) {
+        const int bb = (c * 8) / dm, k0 = c * 8 - bb * dm;
+        float v[8];
+        src16_or_silu(d, bb, k0, v);
+        if (d.xdst) store8f(d.xdst + (size_t)bb * dm + k0, v);
+        if (d.dump) store8f(d.dump + (size_t)bb * dm + k0, v);
+      }
+    }
+    if (blockIdx.x == 0 && tid == 0 && d.xsrc == XS_EMBED) {
+#pragma unroll 1
+      for (int bb = 0; bb < B; ++bb)
+        if (L.tokens[bb] < 0 || L.tokens[bb] >= L.vocab) set_error(EW_BAD_SHAPE);
+    }
+  }
+  cbar();
+}
+
+// fp16 range guard: rows whose max |x| reaches 2^15 are re-staged scaled by an
+// exact power of two, undone on the partial sums when they leave the warp.
+template <int NB>
+__device__ __noinline__ void restage_scaled(const PD& d, int kbase, int klen) {
+  const LC& L = lc();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = L.B, dm = L.d;
+  float* rd = red();
+  const uint32_t* xmax = reinterpret_cast<const uint32_t*>(rd + 32);
+  const int n8 = klen / 8, total8 = B * n8;
+  const int xrow_b = klen * 2 + 64;
+#pragma unroll 1
+  for (int j = 0; warp * 32 + j * NT < total8; ++j) {
+    const int cw = warp * 32 + j * NT, c = cw + lane, bb = cw / n8;  // one batch row per warp iteration
+    const float mx = __uint_as_float(xmax[bb]);
+    if (!(mx >= 32768.f)) continue;  // warp-uniform
+    int ex;
+    frexpf(mx, &ex);
+    const int k0 = kbase + (c - bb * n8) * 8;
+    float v[8];
+    if (d.xsrc == XS_RESID || d.xsrc == XS_FINAL) {
+      float br[8], xr[8], g[8];
+      slab_sum8(d.vpart + (size_t)bb * d.vstride + k0, (size_t)B * d.vstride, d.vns, br);
+      load8f(d.xres + (size_t)bb * dm + k0, xr, false);
+      load8f(d.gain + k0, g, true);
+      resid8(br, xr, g, rd[bb], v);
+      if (d.xsrc == XS_FINAL && d.gain2 != nullptr) {
+        load8f(d.gain2 + k0, g, true);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] *= rd[16 + bb] * g[i];
+      }
+    } else {
+      src16_or_silu(d, bb, k0, v);
+    }
+    put8<NB>(true, bb, k0 - kbase, xrow_b, f8(v), true, ldexpf(1.f, 15 - ex), false);
+  }
+  cbar();
+  if (tid < B) {
+    const float mx = __uint_as_float(xmax[tid]);
+    if (mx >= 32768.f) {
+      int ex;
+      frexpf(mx, &ex);
+      rd[48 + tid] = ldexpf(1.f, ex - 15);
+    }
+  }
+  if (tid == 0) lc().scaled = 1;
+  cbar();
+}
+
+// ---------------------------------------------------------------------------
+// Unit kernels (one warp, one unit)
+// ---------------------------------------------------------------------------
+// int4 unit: codes [grp 4][half 2][lane 32][4 words], scales at +4096 ordered
+// [row % 8][grp][row / 8], zeros at +4224 [grp][row / 8] (nibble row % 8).
+// xl: this lane's x bytes (batch row g, + 16 t, + 2 koff); xsg: per-group sums
+// of x for the unit's first group, + 2 t.
+template <int NB>
+__device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint8_t* xl, int xrow_b, const float* xsg,
+                                        float (&acc)[NB][4], int B, int g, int lane) {
+  const uint4* qw = reinterpret_cast<const uint4*>(slot) + lane;
+  const uint4 sc = *reinterpret_cast<const uint4*>(slot + 4096 + g * 16);
+  const uint4 zA = *reinterpret_cast<const uint4*>(slot + 4224);
+  const uint4 zB = *reinterpret_cast<const uint4*>(slot + 4240);
+  const int sh = 4 * g;
+#pragma unroll
+  for (int grp = 0; grp < 4; ++grp) {
+    const uint4 w0 = qw[(grp * 2) * 32];
+    const uint4 w1 = qw[(grp * 2 + 1) * 32];
+    uint4 xv[NB][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int pr = 0; pr < 4; ++pr)
+        xv[nb][pr] = (g + 8 * nb < B)
+                         ? *reinterpret_cast<const uint4*>(xl + nb * 8 * xrow_b + grp * 256 + pr * 64)
+                         : make_uint4(0u, 0u, 0u, 0u);
     float c[NB][4];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) c[nb][0] = c[nb][1] = c[nb][2] = c[nb][3] = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t w = u4_word(i < 4 ? w0 : w1, i & 3);
-      const uint32_t a0 = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
-      const uint32_t a1 = lop3_and_or(w >> 4, 0x000F000Fu, 0x64006400u);
-      const uint32_t a2 = lop3_and_or(w >> 8, 0x000F000Fu, 0x64006400u);
-      const uint32_t a3 = lop3_and_or(w >> 12, 0x000F000Fu, 0x64006400u);
+      const uint32_t a0 = lop3_and_or(w, 0x000F000Fu, 0x64006400u);       // rows g:     1024 + q
+      const uint32_t a1 = lop3_and_or(w, 0x00F000F0u, 0x64006400u);       // rows g + 8: 1024 + 16 q
+      const uint32_t w8 = w >> 8;
+      const uint32_t a2 = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
+      const uint32_t a3 = lop3_and_or(w8, 0x00F000F0u, 0x64006400u);
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         const uint4& x = xv[nb][i >> 1];
         mma_16816_f16(c[nb], a0, a1, a2, a3, (i & 1) ? x.z : x.x, (i & 1) ? x.w : x.y);
       }
     }
-    const float sl = half_bits_to_f32(sc[grp * 16 + g]);
-    const float sh = half_bits_to_f32(sc[grp * 16 + g + 8]);
-    const float zl = 1024.f + float((zw[grp * 2] >> (4 * g)) & 15u);
-    const float zh = 1024.f + float((zw[grp * 2 + 1] >> (4 * g)) & 15u);
+    const uint32_t sw = u4_word(sc, grp);
+    const float sl = half_bits_to_f32(uint16_t(sw & 0xffffu));
+    const float shi = half_bits_to_f32(uint16_t(sw >> 16)) * 0.0625f;
+    const uint32_t zl_w = u4_word(grp < 2 ? zA : zB, (grp * 2) & 3);
+    const uint32_t zh_w = u4_word(grp < 2 ? zA : zB, (grp * 2 + 1) & 3);
+    // 1024 + z and 1024 + 16 z built in the fp32 significand (2^23 + m - (2^23 - 1024))
+    const float zl = __uint_as_float(0x4B000000u | ((zl_w >> sh) & 15u)) - 8387584.f;
+    const float zh = __uint_as_float(0x4B000000u | (((zh_w >> sh) & 15u) << 4)) - 8387584.f;
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      const float2 xs2 = *reinterpret_cast<const float2*>(xsum + (grp0 + grp) * (8 * NB) + nb * 8 + 2 * t);
-      acc[nb][0] = fmaf(sl, c[nb][0] - zl * xs2.x, acc[nb][0]);
-      acc[nb][1] = fmaf(sl, c[nb][1] - zl * xs2.y, acc[nb][1]);
-      acc[nb][2] = fmaf(sh, c[nb][2] - zh * xs2.x, acc[nb][2]);
-      acc[nb][3] = fmaf(sh, c[nb][3] - zh * xs2.y, acc[nb][3]);
+      const float2 xs2 = *reinterpret_cast<const float2*>(xsg + grp * (8 * NB) + nb * 8);
+      acc[nb][0] = fmaf(sl, fmaf(-zl, xs2.x, c[nb][0]), acc[nb][0]);
+      acc[nb][1] = fmaf(sl, fmaf(-zl, xs2.y, c[nb][1]), acc[nb][1]);
+      acc[nb][2] = fmaf(shi, fmaf(-zh, xs2.x, c[nb][2]), acc[nb][2]);
+      acc[nb][3] = fmaf(shi, fmaf(-zh, xs2.y, c[nb][3]), acc[nb][3]);
     }
   }
 }
 
+// bf16 unit: A fragments [k-step 8][lane 32][4 words].
 template <int NB>
-__device__ __forceinline__ void bf_unit(const uint8_t* slot, const uint4* xs4, int xrow4, int ks0,
-                                        float (&acc)[NB][4], int B, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const uint4* aw = reinterpret_cast<const uint4*>(slot);
+__device__ __forceinline__ void bf_unit(const uint8_t* slot, const uint8_t* xl, int xrow_b, float (&acc)[NB][4],
+                                        int B, int g, int lane) {
+  const uint4* aw = reinterpret_cast<const uint4*>(slot) + lane;
   uint4 xv[NB][4];
 #pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    const int bb = g + 8 * nb;
+  for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-    for (int pr = 0; pr < 4; ++pr) {
-      const int ks = ks0 + pr * 2;
-      xv[nb][pr] = (bb < B) ? xs4[bb * xrow4 + (ks >> 1) * 4 + t] : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
+    for (int pr = 0; pr < 4; ++pr)
+      xv[nb][pr] = (g + 8 * nb < B) ? *reinterpret_cast<const uint4*>(xl + nb * 8 * xrow_b + pr * 64)
+                                    : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint4 a = aw[i * 32 + lane];
+    const uint4 a = aw[i * 32];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       const uint4& x = xv[nb][i >> 1];
@@ -301,1644 +1348,909 @@ __device__ __forceinline__ void bf_unit(const uint8_t* slot, const uint4* xs4, i
 }
 
 // ---------------------------------------------------------------------------
-// The engine
+// GEMV outputs
 // ---------------------------------------------------------------------------
-template <int NB, int HD>
-struct Engine {
-  using L = Lay<NB>;
-  const EngineParams& P;
-  uint8_t* sm;
-  int tid, warp, lane, cta;
-  int cur_phase = 0;
+// Rows of 16-row block rb of slab s; fragment v[nb][0..3] = (row g, batch
+// nb*8 + 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
+template <int NB>
+struct Acc {
+  float v[NB][4];
+};
+template <int NB>
+__device__ __forceinline__ Acc<NB> acc_of(const float (&a)[NB][4]) {
+  Acc<NB> r;
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) r.v[nb][j] = a[nb][j];
+  return r;
+}
 
-  __device__ Engine(const EngineParams& p, uint8_t* s) : P(p), sm(s) {
-    tid = threadIdx.x;
-    warp = tid >> 5;
-    lane = tid & 31;
-    cta = blockIdx.x;
-  }
-
-  // ---- shared-memory views ----
-  __device__ uint64_t* fullb(int w, int sl) const {
-    return reinterpret_cast<uint64_t*>(sm + L::MBAR) + w * NSLOT + sl;
-  }
-  __device__ uint32_t* xs() const { return reinterpret_cast<uint32_t*>(sm + L::XS); }
-  __device__ float* xsum() const { return reinterpret_cast<float*>(sm + L::XSUM); }
-  __device__ float* wsp() const { return reinterpret_cast<float*>(sm + L::WSP); }
-  __device__ float* apw() const { return reinterpret_cast<float*>(sm + L::XS); }
-  __device__ float* qs() const { return reinterpret_cast<float*>(sm + L::QS); }
-  __device__ uint4* qf() const { return reinterpret_cast<uint4*>(sm + L::QF); }
-  __device__ uint16_t* kn() const { return reinterpret_cast<uint16_t*>(sm + L::KNV); }
-  __device__ uint16_t* vn() const { return reinterpret_cast<uint16_t*>(sm + L::KNV) + 128; }
-  __device__ float* red() const { return reinterpret_cast<float*>(sm + L::RED); }
-  __device__ int* posb() const { return reinterpret_cast<int*>(sm + L::POSB); }
-  __device__ int* Lb(int type) const { return reinterpret_cast<int*>(sm + L::LB) + type * MAX_B; }
-  __device__ int* snew(int type) const { return reinterpret_cast<int*>(sm + L::SNEW) + type * MAX_B; }
-  __device__ int* sst(int type) const { return reinterpret_cast<int*>(sm + L::SST) + type * (MAX_SEG + 1); }
-  __device__ int* flags() const { return reinterpret_cast<int*>(sm + L::FLAGS); }
-
-  __device__ void set_error(uint32_t bits) const { atomicOr(P.ws.ctl + 2, bits); }
-  // barrier over the CTA's warps (named barrier 1)
-  __device__ static __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
-
-  __device__ void mark(int slot) const {
-    if (P.trace != nullptr && tid == 0 && cur_phase < P.trace_phases)
-      P.trace[((size_t)cur_phase * P.nc + cta) * 4 + slot] = globaltimer();
-  }
-
-  // ---- phase descriptors ----
-  __device__ __noinline__ void get_phase(int p, PD& d) const {
-    memset(&d, 0, sizeof(PD));
-    const int B = P.B;
-    if (P.mode == MODE_GEMV) {
-      d.kind = PK_GEMV_W4;
-      d.blob = P.g_blob;
-      d.n = P.g_n;
-      d.k = P.g_k;
-      d.kcw = W4_KC;
-      d.ub = W4_UNIT;
-      d.xsrc = XS_BF16;
-      d.xbf = P.g_x;
-      d.xbf_stride = P.g_k;
-      d.rows_valid = P.g_n;
-      d.g = P.geo[0];
-      if (d.g.ns > 1) {
-        // partial rows, finished by the reduce phase
-        d.epi = EPI_PART;
-        d.part = P.ws.g_part;
-        d.pstride = P.g_n;
-      } else if (P.g_epi == W4A_EPI_SILU_MUL) {
-        d.epi = EPI_SILU;
-        d.hout = reinterpret_cast<uint16_t*>(P.g_out);
-        d.hstride = P.g_n / 2;
-      } else {
-        d.epi = (P.g_epi == W4A_EPI_SUMSQ) ? EPI_Y_SUMSQ : EPI_Y;
-        d.yout = reinterpret_cast<float*>(P.g_out);
-        d.ystride = P.g_n;
-        d.ssout = P.g_aux;
-      }
-      if (p == 1) d.kind = PK_REDUCE;
-      return;
-    }
-    if (P.mode == MODE_ATTN) {
-      d.kind = PK_ATTN;
-      d.slots = P.a_slots;
-      d.kc = reinterpret_cast<const uint8_t*>(P.a_k);
-      d.vc = reinterpret_cast<const uint8_t*>(P.a_v);
-      d.aout = P.a_out;
-      return;
-    }
-    const int nl = P.n_layers, dm = P.d;
-    const int qd = P.nq * P.hd, qkv_dim = (P.nq + 2 * P.nkv) * P.hd;
-    const Geo& g_qkv = P.geo[0];
-    const Geo& g_o = P.geo[1];
-    const Geo& g_gu = P.geo[2];
-    const Geo& g_dn = P.geo[3];
-    const Geo& g_lm = P.geo[4];
-    if (p == 5 * nl) {
-      d.kind = PK_GEMV_BF16;
-      d.blob = P.lm_head;
-      d.n = (P.vocab + RB - 1) / RB * RB;
-      d.k = dm;
-      d.kcw = BF_KC;
-      d.ub = BF_UNIT;
-      d.g = g_lm;
-      d.xsrc = XS_FINAL;
-      d.xres = P.ws.xB;
-      d.vpart = P.ws.f_part;
-      d.vns = g_dn.ns;
-      d.vstride = dm;
-      d.gain = P.layers[nl - 1].ffn_norm;
-      d.gain2 = P.final_norm ? P.final_gain : nullptr;
-      d.dump = P.dump ? P.dump + (size_t)nl * B * dm : nullptr;
-      d.rows_valid = P.vocab;
-      if (d.g.ns == 1) {
-        d.epi = EPI_Y;
-        d.yout = P.logits;
-        d.ystride = P.vocab;
-      } else {
-        d.epi = EPI_PART;
-        d.part = P.ws.lg_part;
-        d.pstride = P.vocab;
-      }
-      return;
-    }
-    if (p == 5 * nl + 1) {
-      d.kind = PK_ARGMAX;
-      d.lpart = g_lm.ns > 1 ? P.ws.lg_part : nullptr;
-      d.lns = g_lm.ns;
-      return;
-    }
-    const int l = p / 5, sub = p % 5;
-    const LayerPtrs& lw = P.layers[l];
-    d.layer = l;
-    if (sub == 1) {
-      d.kind = PK_ATTN;
-      d.type = P.full[l] ? 1 : 0;
-      d.newkv = 1;
-      d.seqoff = P.seq0;
-      d.slots = P.kv_slots[l];
-      d.kc = P.kv_base + P.kv_off[l];
-      d.vc = d.kc + (size_t)P.kv_batch * P.nkv * d.slots * HD * 2;
-      d.aout = P.ws.o;
-      d.out_f16 = 1;
-      d.qpart = P.ws.y_part;
-      d.qns = g_qkv.ns;
-      return;
-    }
-    d.kind = PK_GEMV_W4;
-    d.kcw = W4_KC;
-    d.ub = W4_UNIT;
-    d.rows_valid = 1 << 30;
-    d.epi = EPI_PART;
-    if (sub == 0) {
-      d.blob = lw.qkv;
-      d.n = qkv_dim;
-      d.k = dm;
-      d.g = g_qkv;
-      if (l == 0) {
-        d.xsrc = XS_EMBED;
-      } else {
-        d.xsrc = XS_RESID;
-        d.xres = P.ws.xB;
-        d.vpart = P.ws.f_part;
-        d.vns = g_dn.ns;
-        d.vstride = dm;
-        d.gain = P.layers[l - 1].ffn_norm;
-      }
-      d.xdst = P.ws.xA;
-      d.dump = P.dump ? P.dump + (size_t)l * B * dm : nullptr;
-      d.part = P.ws.y_part;
-      d.pstride = qkv_dim;
-    } else if (sub == 2) {
-      d.blob = lw.o;
-      d.n = dm;
-      d.k = qd;
-      d.g = g_o;
-      d.xsrc = XS_F16;
-      d.xbf = P.ws.o;
-      d.xbf_stride = qd;
-      d.part = P.ws.a_part;
-      d.pstride = dm;
-    } else if (sub == 3) {
-      d.blob = lw.gu;
-      d.n = 2 * P.ffn;
-      d.k = dm;
-      d.g = g_gu;
-      d.xsrc = XS_RESID;
-      d.xres = P.ws.xA;
-      d.vpart = P.ws.a_part;
-      d.vns = g_o.ns;
-      d.vstride = dm;
-      d.gain = lw.attn_norm;
-      d.xdst = P.ws.xB;
-      if (d.g.ns == 1) {
-        d.epi = EPI_SILU;
-        d.hout = P.ws.h;
-        d.hstride = P.ffn;
-        d.out_f16 = 1;
-      } else {
-        d.part = P.ws.gu_part;
-        d.pstride = 2 * P.ffn;
-      }
-    } else {
-      d.blob = lw.down;
-      d.n = dm;
-      d.k = P.ffn;
-      d.g = g_dn;
-      if (g_gu.ns == 1) {
-        d.xsrc = XS_F16;
-        d.xbf = P.ws.h;
-        d.xbf_stride = P.ffn;
-      } else {
-        d.xsrc = XS_SILU;
-        d.vpart = P.ws.gu_part;
-        d.vns = g_gu.ns;
-        d.vstride = 2 * P.ffn;
-      }
-      d.part = P.ws.f_part;
-      d.pstride = dm;
-    }
-  }
-
-  // ---- ranges ----
-  // A GEMV CTA owns whole segments: units [a, b) of the phase order.
-  __device__ void gemv_cta_range(const PD& d, long long& a, long long& b) const {
-    if (cta < d.g.nca) {
-      a = rstart(d.g.nseg, d.g.nca, cta) * d.g.kps;
-      b = rstart(d.g.nseg, d.g.nca, cta + 1) * d.g.kps;
-    } else {
-      a = b = 0;
-    }
-  }
-  __device__ static void warp_range(long long a, long long b, int w, long long& wa, long long& wb) {
-    wa = a + (b - a) * w / NW;
-    wb = a + (b - a) * (w + 1) / NW;
-  }
-  __device__ void attn_cta_range(const PD& d, long long& a, long long& b, int& nca) const {
-    const long long total = sst(d.type)[P.B * P.nkv];
-    nca = int(total < P.nc ? total : P.nc);
-    if (nca > 0 && cta < nca) {
-      a = rstart(total, nca, cta);
-      b = rstart(total, nca, cta + 1);
-    } else {
-      a = b = 0;
-    }
-  }
-
-  // ---- the loader ----
-  // Every warp walks its own unit stream across phases with a cursor and keeps
-  // its NSLOT-slot ring full: it refills a slot with its next unit as soon as
-  // it has consumed it, so copies for the next phase are already in flight
-  // while the CTA waits at a barrier.
-  __device__ __noinline__ Cursor cur_enter(int p, int w) const {
-    Cursor c;
-    memset(&c, 0, sizeof(c));
-    c.p = p;
-    if (p >= P.phase_end) {
-      c.kind = -1;
-      return c;
-    }
-    PD d;
-    get_phase(p, d);
-    c.kind = d.kind;
-    if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_BF16) {
-      long long a, b, wa, wb;
-      gemv_cta_range(d, a, b);
-      warp_range(a, b, w, wa, wb);
-      c.p0 = d.blob;
-      c.x0 = d.ub;
-      c.x1 = d.g.nkc;
-      c.x2 = d.g.kps;
-      c.x3 = d.g.nrb;
-      c.i = int(wa);
-      c.end = int(wb);
-      const int upsl = d.g.nrb * d.g.kps;
-      c.x4 = c.i / upsl;
-      const int r = c.i - c.x4 * upsl;
-      c.x5 = r / d.g.kps;
-      c.x6 = r - c.x5 * d.g.kps;
-    } else if (d.kind == PK_ATTN) {
-      long long a, b;
-      int nca;
-      attn_cta_range(d, a, b, nca);
-      c.i = int(a);
-      c.end = int(b);
-      c.p0 = d.kc;
-      c.p1 = d.vc;
-      c.x0 = d.slots;
-      c.x1 = d.seqoff;
-      c.x2 = d.type;
-      c.x3 = 0;
-    }
-    return c;
-  }
-  // The next unit of warp w's stream at or after c (possibly in a later
-  // phase); kind < 0 when the launch has no more.
-  __device__ __noinline__ Cursor cur_normalize(Cursor c, int w) const {
-    for (;;) {
-      if (c.kind < 0) return c;
-      if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
-        if (c.i < c.end) return c;
-      } else if (c.kind == PK_ATTN) {
-        const int* st = sst(c.x2);
-        while (c.i < c.end) {
-          while (st[c.x3 + 1] <= c.i) ++c.x3;
-          const int key0 = (c.i - st[c.x3]) * ATT_CTA_KEYS + w * ATT_KEYS;
-          if (key0 < Lb(c.x2)[c.x3 / P.nkv]) return c;
-          ++c.i;
-        }
-      }
-      c = cur_enter(c.p + 1, w);
-    }
-  }
-  __device__ __forceinline__ void cur_advance(Cursor& c) const {
-    ++c.i;
-    if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
-      if (++c.x6 == c.x2) {
-        c.x6 = 0;
-        if (++c.x5 == c.x3) {
-          c.x5 = 0;
-          ++c.x4;
-        }
-      }
-      if (c.i < c.end) return;  // fast path: same phase
-    }
-    c = cur_normalize(c, warp);
-  }
-  __device__ __forceinline__ void cur_src(const Cursor& c, const uint8_t*& s1, const uint8_t*& s2,
-                                          uint32_t& bytes) const {
-    if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
-      s1 = c.p0 + ((size_t)c.x5 * c.x1 + c.x4 * c.x2 + c.x6) * c.x0;
-      s2 = nullptr;
-      bytes = c.x0;
-    } else {
-      const int* st = sst(c.x2);
-      const int bq = c.x3 / P.nkv, g = c.x3 - bq * P.nkv;
-      const int key0 = (c.i - st[c.x3]) * ATT_CTA_KEYS + warp * ATT_KEYS;
-      const size_t row = ((size_t)(c.x1 + bq) * P.nkv + g) * c.x0 + key0;
-      bytes = ATT_KEYS * HD * 2;
-      s1 = c.p0 + row * HD * 2;
-      s2 = c.p1 + row * HD * 2;
-    }
-  }
-  __device__ __forceinline__ RingCtx ringctx() const {
-    RingCtx R;
-    R.base = sm + L::RING + warp * NSLOT * SLOT_BYTES;
-    R.bar = fullb(warp, 0);
-    R.err = P.ws.ctl + 2;
-    R.lane = lane;
-    return R;
-  }
-  __device__ __forceinline__ void loader_issue(const RingCtx& R, Stream& S) const {
-    const int sl = S.issued % NSLOT;
-    const uint8_t *s1, *s2;
-    uint32_t bytes;
-    cur_src(S.ld, s1, s2, bytes);
-    if (R.lane == 0) {
-      uint64_t* bar = R.bar + sl;
-      uint8_t* dst = R.base + sl * SLOT_BYTES;
-      mbar_expect_tx(bar, s2 ? 2 * bytes : bytes);
-      bulk_g2s(dst, s1, bytes, bar);
-      if (s2) bulk_g2s(dst + bytes, s2, bytes, bar);
-    }
-    ++S.issued;
-    cur_advance(S.ld);
-  }
-  __device__ Stream loader_start() const {
-    Stream S;
-    S.consumed = S.issued = 0;
-    S.bad = false;
-    S.ld = cur_normalize(cur_enter(P.phase_begin, warp), warp);
-    const RingCtx R = ringctx();
-    for (int i = 0; i < NSLOT && S.ld.kind >= 0; ++i) loader_issue(R, S);
-    return S;
-  }
-
-  // ---- ring consumption ----
-  __device__ __forceinline__ static const uint8_t* wait_slot(const RingCtx& R, Stream& S) {
-    const int sl = S.consumed % NSLOT;
-    const uint32_t par = (S.consumed / NSLOT) & 1u;
-    if (!S.bad && !mbar_try_wait(R.bar + sl, par)) {
-      const long long t0 = clock64();
-      while (!mbar_try_wait(R.bar + sl, par)) {
-        if (clock64() - t0 > WAIT_CYCLES) {
-          if (R.lane == 0) atomicOr(R.err, EW_MBAR_TIMEOUT);
-          S.bad = true;
-          break;
-        }
-      }
-    }
-    return R.base + sl * SLOT_BYTES;
-  }
-  // Hand the slot back and refill it with the warp's next unit.
-  __device__ __forceinline__ void release_slot(const RingCtx& R, Stream& S, bool wrote_slot = false) const {
-    // order generic accesses of the slot before the async re-fill (every lane
-    // when lanes wrote into the slot, else lane 0 after the warp's reads)
-    if (wrote_slot) fence_proxy_async();
-    __syncwarp();
-    if (!wrote_slot && R.lane == 0) fence_proxy_async();
-    ++S.consumed;
-    if (S.ld.kind >= 0 && !S.bad) loader_issue(R, S);
-  }
-  __device__ void drain(Stream& S) const {
-    const RingCtx R = ringctx();
-    while (S.consumed < S.issued) {
-      const int sl = S.consumed % NSLOT;
-      const uint32_t par = (S.consumed / NSLOT) & 1u;
-      const long long t0 = clock64();
-      while (!mbar_try_wait(R.bar + sl, par)) {
-        if (clock64() - t0 > WAIT_CYCLES) {
-          if (R.lane == 0) atomicOr(R.err, EW_DRAIN_TIMEOUT);
-          return;
-        }
-      }
-      ++S.consumed;
-    }
-  }
-
-  // ---- grid barrier ----
-  __device__ __noinline__ bool grid_wait(uint32_t target) {
-    if (tid == 0) {
-      int ok = 1;
-      const long long t0 = clock64();
-      while (ld_acquire(P.ws.ctl) < target) {
-        if (ld_volatile_u32(P.ws.ctl + 2) != 0u) {
-          ok = 0;
-          break;
-        }
-        if (clock64() - t0 > WAIT_CYCLES) {
-          set_error(EW_BARRIER_TIMEOUT);
-          ok = 0;
-          break;
-        }
-        __nanosleep(32);
-      }
-      flags()[0] = ok;
-    }
-    cbar();
-    return flags()[0] != 0;
-  }
-  __device__ void grid_arrive() {
-    cbar();
-    if (tid == 0) {
-      __threadfence();
-      red_release_add(P.ws.ctl, 1u);
-    }
-  }
-
-  // Deterministic per-batch-row totals of the per-warp slots wsum[warp][b].
-  __device__ void block_rows_total(const float* wsum, float* out, int B) const {
-    cbar();
-    if (tid < B) {
-      float s = 0.f;
-      for (int w = 0; w < NW; ++w) s += wsum[w * MAX_B + tid];
-      out[tid] = s;
-    }
-    cbar();
-  }
-
-  // ---- GEMV input staging ----
-  __device__ int clamp_token(int bb) const {
-    const int tok = P.tokens[bb];
-    return tok < 0 ? 0 : (tok >= P.vocab ? P.vocab - 1 : tok);
-  }
-  // Eight consecutive values x[bb][k0 .. k0 + 8) (k0 % 8 == 0) of a 16-bit source
-  // or of the SiLU(gate) * up source, in fp32.
-  __device__ void load_simple8(const PD& d, int bb, int k0, float (&v)[8]) const {
-    if (d.xsrc == XS_SILU) {
-      float g[8], u[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) g[i] = u[i] = 0.f;
-      for (int s0 = 0; s0 < d.vns; s0 += 2) {
-        float4 f[2][4];
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            f[i][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (s0 + i < d.vns)
-              f[i][q] = __ldcg(reinterpret_cast<const float4*>(
-                                   d.vpart + ((size_t)(s0 + i) * P.B + bb) * d.vstride + 2 * k0) + q);
-          }
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (s0 + i < d.vns) {  // tiled rows 2j (gate j), 2j+1 (up j)
-              g[2 * q] += f[i][q].x;
-              u[2 * q] += f[i][q].y;
-              g[2 * q + 1] += f[i][q].z;
-              u[2 * q + 1] += f[i][q].w;
-            }
-          }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = g[i] / (1.f + expf(-g[i])) * u[i];
-      return;
-    }
-    cvt16(d.xsrc == XS_F16, load_raw16(d, bb, k0), v);
-  }
-  // Eight 16-bit values of a bf16 / fp16 / embedding source, undecoded.
-  __device__ __forceinline__ uint4 load_raw16(const PD& d, int bb, int k0) const {
-    if (d.xsrc == XS_EMBED)
-      return __ldg(reinterpret_cast<const uint4*>(P.embed + (size_t)clamp_token(bb) * P.d + k0));
-    return __ldcg(reinterpret_cast<const uint4*>(d.xbf + (size_t)bb * d.xbf_stride + k0));
-  }
-  __device__ __forceinline__ static void cvt16(bool f16, const uint4& u, float (&v)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint16_t lo = uint16_t(w[i] & 0xffffu), hi = uint16_t(w[i] >> 16);
-      v[2 * i] = f16 ? half_bits_to_f32(lo) : bf16_to_f32(lo);
-      v[2 * i + 1] = f16 ? half_bits_to_f32(hi) : bf16_to_f32(hi);
-    }
-  }
-  // Sum of the branch slabs for x[bb][k0 .. k0 + 8), in slab order (loads of
-  // up to four slabs in flight at once).
-  __device__ void load_branch8(const PD& d, int bb, int k0, float (&v)[8]) const {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.f;
-    const float* base = d.vpart + (size_t)bb * d.vstride + k0;
-    const size_t sstride = (size_t)P.B * d.vstride;
-    for (int s0 = 0; s0 < d.vns; s0 += 4) {
-      float4 a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        a[i] = b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (s0 + i < d.vns) {
-          const float4* pr = reinterpret_cast<const float4*>(base + (s0 + i) * sstride);
-          a[i] = __ldcg(pr);
-          b[i] = __ldcg(pr + 1);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (s0 + i < d.vns) {
-          v[0] += a[i].x;
-          v[1] += a[i].y;
-          v[2] += a[i].z;
-          v[3] += a[i].w;
-          v[4] += b[i].x;
-          v[5] += b[i].y;
-          v[6] += b[i].z;
-          v[7] += b[i].w;
-        }
-      }
-    }
-  }
-  __device__ static void load8f(const float* p, float (&v)[8], bool ro) {
-    const float4* q = reinterpret_cast<const float4*>(p);
-    const float4 a = ro ? __ldg(q) : __ldcg(q);
-    const float4 b = ro ? __ldg(q + 1) : __ldcg(q + 1);
-    v[0] = a.x;
-    v[1] = a.y;
-    v[2] = a.z;
-    v[3] = a.w;
-    v[4] = b.x;
-    v[5] = b.y;
-    v[6] = b.z;
-    v[7] = b.w;
-  }
-
-  // Store a chunk of eight activations in fragment order.  The 16 lanes of a
-  // half-warp hold one 128-group, whose sum (of the stored, rounded values)
-  // and max |x| they reduce here.  Warp-uniform: every lane calls it.
-  __device__ void emit_chunk(bool valid, int bb, int kl0, int xrow, const float (&v)[8], bool f16, float scale,
-                             bool track_max) const {
-    uint32_t* xw = xs();
-    float s8 = 0.f, m8 = 0.f;
-    if (valid) {
-      const int ks = kl0 >> 4, hi = (kl0 >> 3) & 1;
-      const int base = bb * xrow + ((ks >> 1) * 4) * 4 + (ks & 1) * 2 + hi;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float a = v[2 * t] * scale, b = v[2 * t + 1] * scale;
-        uint32_t w;
-        if (f16) {
-          const uint16_t ha = f32_to_f16(a), hb = f32_to_f16(b);
-          w = uint32_t(ha) | (uint32_t(hb) << 16);
-          s8 += half_bits_to_f32(ha) + half_bits_to_f32(hb);
-        } else {
-          const uint16_t ha = f32_to_bf16(a), hb = f32_to_bf16(b);
-          w = uint32_t(ha) | (uint32_t(hb) << 16);
-          s8 += bf16_to_f32(ha) + bf16_to_f32(hb);
-        }
-        xw[base + t * 4] = w;
-        m8 = fmaxf(m8, fmaxf(fabsf(v[2 * t]), fabsf(v[2 * t + 1])));
-      }
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) {
-      s8 += __shfl_xor_sync(0xffffffffu, s8, o);
-      m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, o));
-    }
-    if (valid && (lane & 15) == 0) {
-      xsum()[(kl0 >> 7) * (8 * NB) + bb] = s8;
-      if (track_max) atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + bb, __float_as_uint(m8));
-    }
-  }
-
-  __device__ __noinline__ void fill_x(const PD& d, long long a, long long b, int& kbase, int& klen) {
-    const int B = P.B, dm = P.d;
-    kbase = 0;
-    klen = 0;
-    if (a < b) {
-      const long long upsl = (long long)d.g.nrb * d.g.kps;
-      const int KS = d.g.kps * d.kcw;
-      const int s0 = int(a / upsl), s1 = int((b - 1) / upsl);
-      kbase = s0 * KS;
-      klen = (s1 - s0 + 1) * KS;
-    }
-    if (!x_fits(klen, B, NB)) {  // the host sizes slabs so this never happens
-      if (tid == 0) set_error(EW_BAD_SHAPE);
-      klen = 0;
-    }
-    const bool f16 = (d.kind == PK_GEMV_W4);
-    float* rd = red();
-    float* xscale = rd + 48;  // 2^e per batch row
-    float* xsm = xsum();
-    for (int i = tid; i < XSUM_BYTES / 4; i += NT) xsm[i] = 0.f;
-    if (tid < MAX_B) {
-      reinterpret_cast<uint32_t*>(rd + 32)[tid] = 0u;
-      xscale[tid] = 1.f;
-    }
-    float* wsum = wsp();   // [NW][MAX_B] per-warp partial sums of squares
-    for (int w = tid; w < NW * MAX_B; w += NT) wsum[w] = 0.f;
-    cbar();
-    const int xrow = klen / 2 + 16;
-    const bool has_out = (d.xdst != nullptr || d.dump != nullptr);
-    const int nout = B * dm / 8;
-    const int out_per = (nout + P.nc - 1) / P.nc;
-    const int o0 = cta * out_per, o1 = min(nout, o0 + out_per);
-
-    if (d.xsrc == XS_RESID || d.xsrc == XS_FINAL) {
-      // Residual update over the whole width: v = sum of the branch slabs,
-      // x = xres + v * rsqrt(mean(v^2) + eps) * gain  [then the final norm].
-      const int n8 = dm / 8, total8 = B * n8;
-      const bool fin = (d.xsrc == XS_FINAL) && d.gain2 != nullptr;
-      // pass 1: sums of squares of v per batch row (a warp iteration covers 32
-      // consecutive chunks of one batch row since d % 256 == 0)
-      for (int j = 0; warp * 32 + j * NT < total8; ++j) {
-        const int cw = warp * 32 + j * NT, c = cw + lane;
-        const int bb = cw / n8;
-        const int k0 = (c - bb * n8) * 8;
-        float v[8];
-        load_branch8(d, bb, k0, v);
-        float sq = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sq = fmaf(v[i], v[i], sq);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        if (lane == 0) wsum[warp * MAX_B + bb] += sq;
-      }
-      block_rows_total(wsum, rd, B);
-      if (tid < B) rd[tid] = rsqrtf(rd[tid] / float(dm) + P.eps);
-      cbar();
-      // x = xres + v * r * gain (v re-read: the slabs are L2-resident)
-      auto x1_of = [&](int bb, int k0, float (&x)[8]) {
-        float v[8], xr[8], g[8];
-        load_branch8(d, bb, k0, v);
-        load8f(d.xres + (size_t)bb * dm + k0, xr, false);
-        load8f(d.gain + k0, g, true);
-        const float r = rd[bb];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = fmaf(v[i] * r, g[i], xr[i]);
-      };
-      if (fin) {
-        // pass 2: the final norm's sums of squares
-        for (int w = tid; w < NW * MAX_B; w += NT) wsum[w] = 0.f;
-        cbar();
-        for (int j = 0; warp * 32 + j * NT < total8; ++j) {
-          const int cw = warp * 32 + j * NT, c = cw + lane;
-          const int bb = cw / n8;
-          float x[8];
-          x1_of(bb, (c - bb * n8) * 8, x);
-          float sq = 0.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) sq = fmaf(x[i], x[i], sq);
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-          if (lane == 0) wsum[warp * MAX_B + bb] += sq;
-        }
-        block_rows_total(wsum, rd + 16, B);
-        if (tid < B) rd[16 + tid] = rsqrtf(rd[16 + tid] / float(dm) + P.eps);
-        cbar();
-      }
-      // pass 3: convert the k-range, write the residual copy / dump slice
-      for (int j = 0; warp * 32 + j * NT < total8; ++j) {
-        const int cw = warp * 32 + j * NT, c = cw + lane;
-        const int bb = cw / n8;
-        const int k0 = (c - bb * n8) * 8;
-        float x[8];
-        x1_of(bb, k0, x);
-        if (has_out && c >= o0 && c < o1) {
-          const size_t o = (size_t)bb * dm + k0;
-          const float4 lo = make_float4(x[0], x[1], x[2], x[3]), hi = make_float4(x[4], x[5], x[6], x[7]);
-          if (d.xdst) {
-            reinterpret_cast<float4*>(d.xdst + o)[0] = lo;
-            reinterpret_cast<float4*>(d.xdst + o)[1] = hi;
-          }
-          if (d.dump) {
-            reinterpret_cast<float4*>(d.dump + o)[0] = lo;
-            reinterpret_cast<float4*>(d.dump + o)[1] = hi;
-          }
-        }
-        if (fin) {
-          float g2[8];
-          load8f(d.gain2 + k0, g2, true);
-          const float rf = rd[16 + bb];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] = x[i] * rf * g2[i];
-        }
-        // half-warps are uniformly inside or outside (128-aligned k-range)
-        const bool inside = k0 >= kbase && k0 < kbase + klen;
-        emit_chunk(inside, bb, k0 - kbase, xrow, x, f16, 1.f, f16);
-      }
-    } else {
-      // 16-bit / SiLU sources: the k-range only, several chunks per thread in flight
-      const int n8 = klen / 8, total8 = B * n8;
-      if (d.xsrc != XS_SILU) {
-        constexpr int JU = 4;
-        for (int j0 = 0; warp * 32 + j0 * NT < total8; j0 += JU) {
-          uint4 raw[JU];
-#pragma unroll
-          for (int jj = 0; jj < JU; ++jj) {
-            const int c = warp * 32 + (j0 + jj) * NT + lane;
-            raw[jj] = make_uint4(0u, 0u, 0u, 0u);
-            if (c < total8) {
-              const int bb = c / n8;
-              raw[jj] = load_raw16(d, bb, kbase + (c - bb * n8) * 8);
-            }
-          }
-#pragma unroll
-          for (int jj = 0; jj < JU; ++jj) {
-            const int cw = warp * 32 + (j0 + jj) * NT;
-            if (cw < total8) {  // warp-uniform
-              const int c = cw + lane;
-              const int bb = c / n8;
-              float v[8];
-              cvt16(d.xsrc == XS_F16, raw[jj], v);
-              emit_chunk(c < total8, bb, (c - bb * n8) * 8, xrow, v, f16, 1.f, f16);
-            }
-          }
-        }
-      } else {
-        constexpr int JU = 2;
-        for (int j0 = 0; warp * 32 + j0 * NT < total8; j0 += JU) {
-          float v[JU][8];
-#pragma unroll
-          for (int jj = 0; jj < JU; ++jj) {
-            const int c = warp * 32 + (j0 + jj) * NT + lane;
-            if (c < total8) {
-              const int bb = c / n8;
-              load_simple8(d, bb, kbase + (c - bb * n8) * 8, v[jj]);
-            }
-          }
-#pragma unroll
-          for (int jj = 0; jj < JU; ++jj) {
-            const int cw = warp * 32 + (j0 + jj) * NT;
-            if (cw < total8) {  // warp-uniform
-              const int c = cw + lane;
-              const int bb = c / n8;
-              emit_chunk(c < total8, bb, (c - bb * n8) * 8, xrow, v[jj], f16, 1.f, f16);
-            }
-          }
-        }
-      }
-      // residual copy / dump of the embedding (first layer)
-      if (has_out) {
-        for (int c = o0 + tid; c < o1; c += NT) {
-          const int bb = (c * 8) / dm, k0 = c * 8 - bb * dm;
-          float v[8];
-          load_simple8(d, bb, k0, v);
-          const float4 lo = make_float4(v[0], v[1], v[2], v[3]), hi = make_float4(v[4], v[5], v[6], v[7]);
-          if (d.xdst) {
-            reinterpret_cast<float4*>(d.xdst + (size_t)bb * dm + k0)[0] = lo;
-            reinterpret_cast<float4*>(d.xdst + (size_t)bb * dm + k0)[1] = hi;
-          }
-          if (d.dump) {
-            reinterpret_cast<float4*>(d.dump + (size_t)bb * dm + k0)[0] = lo;
-            reinterpret_cast<float4*>(d.dump + (size_t)bb * dm + k0)[1] = hi;
-          }
-        }
-      }
-      if (cta == 0 && tid == 0 && d.xsrc == XS_EMBED) {
-        for (int bb = 0; bb < B; ++bb)
-          if (P.tokens[bb] < 0 || P.tokens[bb] >= P.vocab) set_error(EW_BAD_SHAPE);
-      }
-    }
-    cbar();
-    if (f16) {
-      // fp16 range guard: rows whose max |x| reaches 2^15 are re-staged scaled
-      // by an exact power of two, undone on the partial sums in flush().
-      const uint32_t* xmax = reinterpret_cast<const uint32_t*>(rd + 32);
-      bool any = false;
-      for (int bb = 0; bb < B; ++bb) any |= __uint_as_float(xmax[bb]) >= 32768.f;
-      if (any) restage_scaled(d, kbase, klen, xrow);
-    }
-  }
-
-  // Rare path of the fp16 range guard.
-  __device__ __noinline__ void restage_scaled(const PD& d, int kbase, int klen, int xrow) {
-    const int B = P.B, dm = P.d;
-    float* rd = red();
-    const uint32_t* xmax = reinterpret_cast<const uint32_t*>(rd + 32);
-    float* xscale = rd + 48;
-    const int n8 = klen / 8, total8 = B * n8;
-    for (int j = 0; warp * 32 + j * NT < total8; ++j) {
-      const int cw = warp * 32 + j * NT, c = cw + lane;
-      const int bb = cw / n8;  // n8 % 32 == 0: one batch row per warp iteration
-      const float mx = __uint_as_float(xmax[bb]);
-      if (!(mx >= 32768.f)) continue;  // warp-uniform
-      int ex;
-      frexpf(mx, &ex);
-      const int k0 = kbase + (c - bb * n8) * 8;
-      float v[8];
-      if (d.xsrc == XS_RESID || d.xsrc == XS_FINAL) {
-        float br[8], xr[8], g[8];
-        load_branch8(d, bb, k0, br);
-        load8f(d.xres + (size_t)bb * dm + k0, xr, false);
-        load8f(d.gain + k0, g, true);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = fmaf(br[i] * rd[bb], g[i], xr[i]);
-        if (d.xsrc == XS_FINAL && d.gain2 != nullptr) {
-          load8f(d.gain2 + k0, g, true);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] *= rd[16 + bb] * g[i];
-        }
-      } else {
-        load_simple8(d, bb, k0, v);
-      }
-      emit_chunk(true, bb, k0 - kbase, xrow, v, true, ldexpf(1.f, 15 - ex), false);
-    }
-    cbar();
-    if (tid < B) {
-      const float mx = __uint_as_float(xmax[tid]);
-      if (mx >= 32768.f) {
-        int ex;
-        frexpf(mx, &ex);
-        xscale[tid] = ldexpf(1.f, ex - 15);
-      }
-    }
-    cbar();
-  }
-
-  // ---- GEMV outputs ----
-  // Rows of 16-row block rb of slab s, fragment layout v[nb][0..3] = (row g,
-  // col 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1), columns = batch nb*8 + ...
-  __device__ __noinline__ void finalize(const PD& d, int s, int rb, Acc<NB> A) const {
-    const float (&v)[NB][4] = A.v;
-    const int g = lane >> 2, t = lane & 3, B = P.B;
-    const int r0 = rb * RB + g, r1 = r0 + 8;
-    if (d.epi == EPI_PART) {
-      float* base = d.part + (size_t)s * B * d.pstride;
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const int b0 = nb * 8 + 2 * t, b1 = b0 + 1;
-        if (r0 < d.rows_valid) {
-          if (b0 < B) base[(size_t)b0 * d.pstride + r0] = v[nb][0];
-          if (b1 < B) base[(size_t)b1 * d.pstride + r0] = v[nb][1];
-        }
-        if (r1 < d.rows_valid) {
-          if (b0 < B) base[(size_t)b0 * d.pstride + r1] = v[nb][2];
-          if (b1 < B) base[(size_t)b1 * d.pstride + r1] = v[nb][3];
-        }
-      }
-      return;
-    }
-    if (d.epi == EPI_SILU) {
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const float u0 = __shfl_down_sync(0xffffffffu, v[nb][0], 4);
-        const float u1 = __shfl_down_sync(0xffffffffu, v[nb][1], 4);
-        const float u2 = __shfl_down_sync(0xffffffffu, v[nb][2], 4);
-        const float u3 = __shfl_down_sync(0xffffffffu, v[nb][3], 4);
-        if ((g & 1) == 0) {
-          const int j0 = rb * 8 + g / 2, j1 = rb * 8 + (g + 8) / 2;
-          const int b0 = nb * 8 + 2 * t, b1 = b0 + 1;
-          const float h0 = v[nb][0] / (1.f + expf(-v[nb][0])) * u0;
-          const float h1 = v[nb][1] / (1.f + expf(-v[nb][1])) * u1;
-          const float h2 = v[nb][2] / (1.f + expf(-v[nb][2])) * u2;
-          const float h3 = v[nb][3] / (1.f + expf(-v[nb][3])) * u3;
-          if (b0 < B) {
-            d.hout[(size_t)b0 * d.hstride + j0] = d.out_f16 ? f32_to_f16(h0) : f32_to_bf16(h0);
-            d.hout[(size_t)b0 * d.hstride + j1] = d.out_f16 ? f32_to_f16(h2) : f32_to_bf16(h2);
-          }
-          if (b1 < B) {
-            d.hout[(size_t)b1 * d.hstride + j0] = d.out_f16 ? f32_to_f16(h1) : f32_to_bf16(h1);
-            d.hout[(size_t)b1 * d.hstride + j1] = d.out_f16 ? f32_to_f16(h3) : f32_to_bf16(h3);
-          }
-        }
-      }
-      return;
-    }
+template <int NB>
+__device__ __noinline__ void emit_rows(const PD& d, int s, int rb, Acc<NB> A, int B, int lane) {
+  const float (&v)[NB][4] = A.v;
+  const int g = lane >> 2, t = lane & 3;
+  if (d.epi == EPI_SILU) {
+    // rows 2j (gate) and 2j + 1 (up) sit in lanes g and g + 1 of a thread column
+    uint16_t* h = reinterpret_cast<uint16_t*>(d.out);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      const int b0 = nb * 8 + 2 * t, b1 = b0 + 1;
-      if (r0 < d.rows_valid) {
-        if (b0 < B) d.yout[(size_t)b0 * d.ystride + r0] = v[nb][0];
-        if (b1 < B) d.yout[(size_t)b1 * d.ystride + r0] = v[nb][1];
-      }
-      if (r1 < d.rows_valid) {
-        if (b0 < B) d.yout[(size_t)b0 * d.ystride + r1] = v[nb][2];
-        if (b1 < B) d.yout[(size_t)b1 * d.ystride + r1] = v[nb][3];
-      }
-      if (d.epi == EPI_Y_SUMSQ) {
-        float s0 = v[nb][0] * v[nb][0] + v[nb][2] * v[nb][2];
-        float s1 = v[nb][1] * v[nb][1] + v[nb][3] * v[nb][3];
+      float u[4];
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-          s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        }
-        if (g == 0) {
-          if (b0 < B) d.ssout[(size_t)rb * B + b0] = s0;
-          if (b1 < B) d.ssout[(size_t)rb * B + b1] = s1;
+      for (int j = 0; j < 4; ++j) u[j] = __shfl_down_sync(0xffffffffu, v[nb][j], 4);
+      if ((g & 1) == 0) {
+        const int j0 = rb * 8 + g / 2, j1 = j0 + 4;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int b = nb * 8 + 2 * t + (e & 1), j = (e & 2) ? j1 : j0;
+          const float x = v[nb][e];
+          const float hv = x / (1.f + expf(-x)) * u[e];
+          if (b < B) h[(size_t)b * d.ostride + j] = d.out_f16 ? f32_to_f16(hv) : f32_to_bf16(hv);
         }
       }
     }
+    return;
   }
-  __device__ void emit_segment(const PD& d, int seg, const Acc<NB>& A) const {
-    const int s = seg / d.g.nrb, rb = seg - s * d.g.nrb;
-    finalize(d, s, rb, A);
+  float* base = reinterpret_cast<float*>(d.out) + (size_t)s * B * d.ostride;
+  const int r0 = rb * RB + g, r1 = r0 + 8;
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int b0 = nb * 8 + 2 * t, b1 = b0 + 1;
+    if (r0 < d.rows_valid) {
+      if (b0 < B) base[(size_t)b0 * d.ostride + r0] = v[nb][0];
+      if (b1 < B) base[(size_t)b1 * d.ostride + r0] = v[nb][1];
+    }
+    if (r1 < d.rows_valid) {
+      if (b0 < B) base[(size_t)b0 * d.ostride + r1] = v[nb][2];
+      if (b1 < B) base[(size_t)b1 * d.ostride + r1] = v[nb][3];
+    }
   }
+}
 
-  __device__ static Acc<NB> to_acc(const float (&a)[NB][4]) {
-    Acc<NB> r;
+// A segment piece leaves the warp: undo the range scaling, then emit it
+// (segment wholly inside this warp) or park it in the warp's slot.
+template <int NB>
+__device__ __forceinline__ void seg_done(const PD& d, int seg, float (&acc)[NB][4], int wa, int wb, float* park,
+                                         int B, int lane) {
+  if (lc().scaled) {
+    const float* xscale = red() + 48;
+    const int t = lane & 3;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const float s0 = xscale[nb * 8 + 2 * t], s1 = xscale[nb * 8 + 2 * t + 1];
+      acc[nb][0] *= s0;
+      acc[nb][1] *= s1;
+      acc[nb][2] *= s0;
+      acc[nb][3] *= s1;
+    }
+  }
+  const int kps = d.g.kps, u0 = seg * kps;
+  if (u0 >= wa && u0 + kps <= wb) {
+    const int s = seg / d.g.nrb;
+    emit_rows<NB>(d, s, seg - s * d.g.nrb, acc_of<NB>(acc), B, lane);
+  } else {
+    float* q = park + ((seg == wa / kps) ? 0 : 32 * 4 * NB);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) r.v[nb][j] = a[nb][j];
-    return r;
+      reinterpret_cast<float4*>(q)[nb] = make_float4(acc[nb][0], acc[nb][1], acc[nb][2], acc[nb][3]);
   }
+}
 
-  // A segment piece leaves the warp: undo the range scaling, then emit it
-  // (segment wholly inside this warp) or park it in the warp's slot.
-  __device__ __noinline__ void flush(const PD& d, int seg, Acc<NB> A, int wa, int wb, float* my) const {
-    if (d.kind == PK_GEMV_W4) {
-      const float* xscale = red() + 48;
-      const int t = lane & 3;
+// Segments of this CTA split between warps: sum the pieces in warp order.
+template <int NB>
+__device__ __noinline__ void cta_combine(const PD& d, int a, int b) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kps = d.g.kps, B = lc().B;
+  const float* wsp = sm_at<float>(sm_wsp(NB));
+  int count = 0, last = -1;
+#pragma unroll 1
+  for (int w = 0; w < NW; ++w) {
+    int wa, wb;
+    warp_range(a, b, w, wa, wb);
+    if (wa >= wb) continue;
+    const int fs = wa / kps, ls = (wb - 1) / kps;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      const int S = which ? ls : fs;
+      if (which && ls == fs) break;
+      const bool complete = (S * kps >= wa) && (S * kps + kps <= wb);
+      if (complete || S == last) continue;
+      if (count % NW == warp) {
+        float sum[NB][4];
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const float s0 = xscale[nb * 8 + 2 * t], s1 = xscale[nb * 8 + 2 * t + 1];
-        A.v[nb][0] *= s0;
-        A.v[nb][1] *= s1;
-        A.v[nb][2] *= s0;
-        A.v[nb][3] *= s1;
-      }
-    }
-    const int u0 = seg * d.g.kps;
-    if (u0 >= wa && u0 + d.g.kps <= wb) {
-      emit_segment(d, seg, A);
-    } else {
-      const int sl = (seg == wa / d.g.kps) ? 0 : 1;
-      float* q = my + sl * (32 * 4 * NB) + lane * 4 * NB;
+        for (int nb = 0; nb < NB; ++nb) sum[nb][0] = sum[nb][1] = sum[nb][2] = sum[nb][3] = 0.f;
+#pragma unroll 1
+        for (int w2 = 0; w2 < NW; ++w2) {
+          int a2, b2;
+          warp_range(a, b, w2, a2, b2);
+          if (a2 >= b2 || S * kps >= b2 || S * kps + kps <= a2) continue;
+          const int sl = (S == a2 / kps) ? 0 : 1;
+          const float* q = wsp + w2 * (2 * 32 * 4 * NB) + sl * (32 * 4 * NB) + lane * 4 * NB;
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
-        reinterpret_cast<float4*>(q)[nb] = make_float4(A.v[nb][0], A.v[nb][1], A.v[nb][2], A.v[nb][3]);
-    }
-  }
-
-  // Segments of this CTA split between warps: sum the pieces in warp order.
-  __device__ __noinline__ void cta_combine(const PD& d, int a, int b) const {
-    const int kps = d.g.kps;
-    int count = 0, last = -1;
-    for (int w = 0; w < NW; ++w) {
-      long long wa64, wb64;
-      warp_range(a, b, w, wa64, wb64);
-      const int wa = int(wa64), wb = int(wb64);
-      if (wa >= wb) continue;
-      const int fs = wa / kps, ls = (wb - 1) / kps;
-      for (int which = 0; which < 2; ++which) {
-        const int S = which ? ls : fs;
-        if (which && ls == fs) break;
-        const bool complete = (S * kps >= wa) && (S * kps + kps <= wb);
-        if (complete || S == last) continue;
-        if (count % NW == warp) {
-          Acc<NB> sum;
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb) sum.v[nb][0] = sum.v[nb][1] = sum.v[nb][2] = sum.v[nb][3] = 0.f;
-          for (int w2 = 0; w2 < NW; ++w2) {
-            long long a2, b2;
-            warp_range(a, b, w2, a2, b2);
-            if (a2 >= b2 || S * kps >= b2 || S * kps + kps <= a2) continue;
-            const int sl = (S == int(a2) / kps) ? 0 : 1;
-            const float* q = wsp() + w2 * (2 * 32 * 4 * NB) + sl * (32 * 4 * NB) + lane * 4 * NB;
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-              const float4 f = reinterpret_cast<const float4*>(q)[nb];
-              sum.v[nb][0] += f.x;
-              sum.v[nb][1] += f.y;
-              sum.v[nb][2] += f.z;
-              sum.v[nb][3] += f.w;
-            }
+          for (int nb = 0; nb < NB; ++nb) {
+            const float4 f = reinterpret_cast<const float4*>(q)[nb];
+            sum[nb][0] += f.x;
+            sum[nb][1] += f.y;
+            sum[nb][2] += f.z;
+            sum[nb][3] += f.w;
           }
-          emit_segment(d, S, sum);
         }
-        ++count;
-        last = S;
+        const int s = S / d.g.nrb;
+        emit_rows<NB>(d, s, S - s * d.g.nrb, acc_of<NB>(sum), B, lane);
       }
+      ++count;
+      last = S;
     }
   }
+}
 
-  __device__ __forceinline__ void run_gemv(const PD& d, Stream& S) {
-    long long a, b;
-    gemv_cta_range(d, a, b);
-    int kbase, klen;
-    fill_x(d, a, b, kbase, klen);
-    mark(1);
-    if (a >= b) return;
-    long long wa64, wb64;
-    warp_range(a, b, warp, wa64, wb64);
-    S = gemv_loop(S, d, kbase, klen, int(wa64), int(wb64));
-    cbar();
-    mark(2);
-    cta_combine(d, int(a), int(b));
+template <int NB, int HD>
+__device__ __noinline__ void gemv_phase(const PD& d) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  int a, b;
+  gemv_cta_range(d.g, blockIdx.x, a, b);
+  int kbase = 0, klen = 0;
+  if (a < b) {
+    const int upsl = d.g.nrb * d.g.kps, KS = d.g.kps * d.kcw;
+    const int s0 = a / upsl, s1 = (b - 1) / upsl;
+    kbase = s0 * KS;
+    klen = (s1 - s0 + 1) * KS;
   }
-
-  // This warp's units [wa, wb) of a GEMV phase.  Its own (non-inlined) function
-  // so that the loop's registers are allocated for the loop alone.
-  __device__ __noinline__ Stream gemv_loop(Stream S, const PD& d, int kbase, int klen, int wa, int wb) const {
-    const RingCtx R = ringctx();
-    const uint4* xs4 = reinterpret_cast<const uint4*>(xs());
-    const int xrow4 = (klen / 2 + 16) / 4;
-    const float* xsm = xsum();
-    const int kps = d.g.kps, nrb = d.g.nrb, kcw = d.kcw, B = P.B;
-    const int upsl = nrb * kps;
-    int u = wa;
-    int s_ = u / upsl;
-    int rb = (u - s_ * upsl) / kps;
-    int kci = u - s_ * upsl - rb * kps;
-    float acc[NB][4];
-    int cur = -1;
-    float* my = wsp() + warp * (2 * 32 * 4 * NB);
+  if (!x_fits(klen, lc().B, NB)) {  // the host sizes slabs so this never happens
+    if (tid == 0) set_error(EW_BAD_SHAPE);
+    a = b = 0;
+    klen = 0;
+  }
+  stage_x<NB>(d, kbase, klen);
+  if (d.kind == PK_GEMV_W4) {
+    const uint32_t* xmax = reinterpret_cast<const uint32_t*>(red() + 32);
+    bool any = false;
+#pragma unroll 1
+    for (int bb = 0; bb < lc().B; ++bb) any |= __uint_as_float(xmax[bb]) >= 32768.f;
+    if (any) restage_scaled<NB>(d, kbase, klen);
+  }
+  mark(3);
+  if (a < b) {
+    int wa, wb;
+    warp_range(a, b, warp, wa, wb);
+    const int B = lc().B;
+    Ring R;
+    ring_load(R, warp);
+    const int kps = d.g.kps, nrb = d.g.nrb, upsl = nrb * kps, kcw = d.kcw;
     const bool w4 = (d.kind == PK_GEMV_W4);
-    const int ln = R.lane;
+    const int xrow_b = klen * 2 + 64;
+    const uint8_t* xl = sm_at<uint8_t>(SM_XS + g * xrow_b + t * 16);
+    const float* xsg = sm_at<float>(sm_xsum(NB)) + 2 * t;
+    float* park = sm_at<float>(sm_wsp(NB)) + warp * (2 * 32 * 4 * NB) + lane * 4 * NB;
+    int u = wa;
+    int sl = u / upsl;
+    int rb = (u - sl * upsl) / kps;
+    int kci = u - sl * upsl - rb * kps;
+    float acc[NB][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+    int cur = -1;
+#pragma unroll 1
     for (; u < wb; ++u) {
-      const int seg = s_ * nrb + rb;
+      const int seg = sl * nrb + rb;
       if (seg != cur) {
-        if (cur >= 0) flush(d, cur, to_acc(acc), wa, wb, my);
+        if (cur >= 0) seg_done<NB>(d, cur, acc, wa, wb, park, B, lane);
         cur = seg;
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
       }
-      const int koff = (s_ * kps + kci) * kcw - kbase;
-      const uint8_t* slot = wait_slot(R, S);
+      const int koff = (sl * kps + kci) * kcw - kbase;
+      const uint8_t* slot = ring_wait(R, warp, lane);
       if (w4)
-        w4_unit<NB>(slot, xs4, xrow4, koff >> 4, xsm, koff >> 7, acc, B, ln);
+        w4_unit<NB>(slot, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g, lane);
       else
-        bf_unit<NB>(slot, xs4, xrow4, koff >> 4, acc, B, ln);
-      release_slot(R, S);
+        bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
+      ring_release<HD>(R, warp, lane, false);
       if (++kci == kps) {
         kci = 0;
         if (++rb == nrb) {
           rb = 0;
-          ++s_;
+          ++sl;
         }
       }
     }
-    if (cur >= 0) flush(d, cur, to_acc(acc), wa, wb, my);
-    return S;
+    if (cur >= 0) seg_done<NB>(d, cur, acc, wa, wb, park, B, lane);
+    ring_store(R, warp, lane);
   }
+  cbar();
+  mark(4);
+  if (a < b) cta_combine<NB>(d, a, b);
+  mark(5);
+}
 
-  // Standalone GEMV with K split into slabs: y = sum of the slab rows in
-  // order, then the requested epilogue.
-  __device__ __noinline__ void run_reduce() const {
-    const int B = P.B, n = P.g_n;
-    const int ns = P.geo[0].ns;
-    const float* part = P.ws.g_part;
-    if (P.g_epi == W4A_EPI_SILU_MUL) {
-      const int nh = n / 2, total = B * nh;
-      for (int i = cta * NT + tid; i < total; i += P.nc * NT) {
-        const int bb = i / nh, j = i - bb * nh;
-        float gsum = 0.f, usum = 0.f;
-        for (int s = 0; s < ns; ++s) {
-          gsum += __ldcg(part + ((size_t)s * B + bb) * n + 2 * j);
-          usum += __ldcg(part + ((size_t)s * B + bb) * n + 2 * j + 1);
-        }
-        reinterpret_cast<uint16_t*>(P.g_out)[(size_t)bb * nh + j] = f32_to_bf16(gsum / (1.f + expf(-gsum)) * usum);
+// Standalone GEMV whose K was split into slabs (or with the SUMSQ epilogue):
+// y = sum of the slab rows in order, then the requested epilogue.
+__device__ __noinline__ void reduce_phase(const PD& d) {
+  const LC& L = lc();
+  const int B = L.B, n = d.n, ns = d.vns;
+  const float* part = d.vpart;
+  if (d.red_epi == W4A_EPI_SILU_MUL) {
+    const int nh = n / 2, total = B * nh;
+#pragma unroll 1
+    for (int i = blockIdx.x * NT + threadIdx.x; i < total; i += L.nc * NT) {
+      const int bb = i / nh, j = i - bb * nh;
+      float gs = 0.f, us = 0.f;
+#pragma unroll 1
+      for (int s = 0; s < ns; ++s) {
+        gs += __ldcg(part + ((size_t)s * B + bb) * n + 2 * j);
+        us += __ldcg(part + ((size_t)s * B + bb) * n + 2 * j + 1);
       }
-      return;
+      reinterpret_cast<uint16_t*>(d.out)[(size_t)bb * nh + j] = f32_to_bf16(gs / (1.f + expf(-gs)) * us);
     }
-    // one thread per (batch row, 16-row block): plain rows and their sum of squares
-    const int nrb = n / RB, total = B * nrb;
-    for (int i = cta * NT + tid; i < total; i += P.nc * NT) {
-      const int bb = i / nrb, rb = i - bb * nrb;
-      float ss = 0.f;
-      for (int r = rb * RB; r < rb * RB + RB; ++r) {
-        float y = 0.f;
-        for (int s = 0; s < ns; ++s) y += __ldcg(part + ((size_t)s * B + bb) * n + r);
-        reinterpret_cast<float*>(P.g_out)[(size_t)bb * n + r] = y;
-        ss = fmaf(y, y, ss);
-      }
-      if (P.g_epi == W4A_EPI_SUMSQ) P.g_aux[(size_t)rb * B + bb] = ss;
-    }
+    return;
   }
+  // one thread per (batch row, 16-row block): rows and their sum of squares
+  const int nrb = n / RB, total = B * nrb;
+#pragma unroll 1
+  for (int i = blockIdx.x * NT + threadIdx.x; i < total; i += L.nc * NT) {
+    const int bb = i / nrb, rb = i - bb * nrb;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int r = rb * RB; r < rb * RB + RB; ++r) {
+      float y = 0.f;
+#pragma unroll 1
+      for (int s = 0; s < ns; ++s) y += __ldcg(part + ((size_t)s * B + bb) * n + r);
+      reinterpret_cast<float*>(d.out)[(size_t)bb * n + r] = y;
+      ss = fmaf(y, y, ss);
+    }
+    if (d.red_epi == W4A_EPI_SUMSQ) d.aux[(size_t)rb * B + bb] = ss;
+  }
+}
 
-  // ---- attention phase ----
-  __device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
-    const int bq = seg / P.nkv, g = seg % P.nkv;
-    const int GQ = P.nq / P.nkv;
-    float* q = qs();
-    float* rd = red();
-    const float qscale = 1.4426950408889634f * rsqrtf(float(HD));
-    if (d.newkv) {
-      // q, k, v of this sequence are the sums of the QKV slabs (four-row
-      // chunks, several in flight per thread); the norms run over the whole Q
-      // and K projections.  This group's k and v rows go to scratch.
-      const int qd = P.nq * HD, kd = P.nkv * HD, qkv_dim = qd + 2 * kd;
-      const float* ybase = d.qpart + (size_t)bq * qkv_dim;
-      const size_t sstride = (size_t)P.B * qkv_dim;
-      float* kraw = wsp() + 64;
-      float* vraw = kraw + HD;
-      const int nq4 = qd / 4, nk4 = kd / 4;
-      const int total4 = nq4 + (own_new ? nk4 + HD / 4 : 0);
-      float sq = 0.f, sk = 0.f;
-      constexpr int JU = 4;
-      for (int c0 = tid; c0 < total4; c0 += JU * NT) {
-        int rows[JU];
-        float4 v[JU];
+// ---------------------------------------------------------------------------
+// Attention
+// ---------------------------------------------------------------------------
+template <int HD>
+__device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
+  const LC& L = lc();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bq = seg / L.nkv, g = seg % L.nkv;
+  const int GQ = L.nq / L.nkv;
+  float* q = sm_at<float>(SM_QS);
+  float* rd = red();
+  uint16_t* kn = sm_at<uint16_t>(SM_KNV);
+  uint16_t* vn = kn + 128;
+  const float qscale = 1.4426950408889634f * rsqrtf(float(HD));
+  if (d.newkv) {
+    // q, k, v of this sequence are the sums of the QKV slabs (four-row
+    // chunks, several in flight per thread); the norms run over the whole Q
+    // and K projections.  This group's k and v rows go to scratch.
+    const int qd = L.nq * HD, kd = L.nkv * HD, qkv_dim = qd + 2 * kd;
+    const float* ybase = d.qpart + (size_t)bq * qkv_dim;
+    const size_t sstride = (size_t)L.B * qkv_dim;
+    float* kraw = sm_at<float>(SM_ASCR);
+    float* vraw = kraw + 128;
+    float* wq = vraw + 128;
+    const int nq4 = qd / 4, nk4 = kd / 4;
+    const int total4 = nq4 + (own_new ? nk4 + HD / 4 : 0);
+    float sq = 0.f, sk = 0.f;
+    constexpr int JU = 4;
+#pragma unroll 1
+    for (int c0 = tid; c0 < total4; c0 += JU * NT) {
+      int rows[JU];
+      float4 v[JU];
+#pragma unroll
+      for (int j = 0; j < JU; ++j) {
+        const int c = c0 + j * NT;
+        rows[j] = c < nq4 + nk4 ? 4 * c : qd + kd + g * HD + 4 * (c - nq4 - nk4);
+        v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll 1
+      for (int sl = 0; sl < d.qns; ++sl) {
+        float4 t4[JU];
+#pragma unroll
+        for (int j = 0; j < JU; ++j)
+          t4[j] = (c0 + j * NT < total4) ? ldcg4(ybase + sl * sstride + rows[j]) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < JU; ++j) {
-          const int c = c0 + j * NT;
-          rows[j] = c < nq4 + nk4 ? 4 * c : qd + kd + g * HD + 4 * (c - nq4 - nk4);
-          v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        for (int sl = 0; sl < d.qns; ++sl) {
-          float4 t[JU];
-#pragma unroll
-          for (int j = 0; j < JU; ++j)
-            t[j] = (c0 + j * NT < total4) ? __ldcg(reinterpret_cast<const float4*>(ybase + sl * sstride + rows[j]))
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int j = 0; j < JU; ++j) {
-            v[j].x += t[j].x;
-            v[j].y += t[j].y;
-            v[j].z += t[j].z;
-            v[j].w += t[j].w;
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < JU; ++j) {
-          if (c0 + j * NT >= total4) continue;
-          const int r = rows[j];
-          const float ss = v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
-          float* dst = nullptr;
-          if (r < qd) {
-            sq += ss;
-            const int h = r / HD - g * GQ;
-            if (h >= 0 && h < GQ) dst = q + (r - g * GQ * HD);
-          } else if (r < qd + kd) {
-            sk += ss;
-            if ((r - qd) / HD == g) dst = kraw + (r - qd - g * HD);
-          } else {
-            dst = vraw + (r - qd - kd - g * HD);
-          }
-          if (dst) {
-            dst[0] = v[j].x;
-            dst[1] = v[j].y;
-            dst[2] = v[j].z;
-            dst[3] = v[j].w;
-          }
+          v[j].x += t4[j].x;
+          v[j].y += t4[j].y;
+          v[j].z += t4[j].z;
+          v[j].w += t4[j].w;
         }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        sq += __shfl_xor_sync(0xffffffffu, sq, o);
-        sk += __shfl_xor_sync(0xffffffffu, sk, o);
-      }
-      float* wq = wsp();
-      if (lane == 0) {
-        wq[warp] = sq;
-        wq[NW + warp] = sk;
-      }
-      cbar();
-      if (tid == 0) {
-        float a = 0.f, c = 0.f;
-        for (int w = 0; w < NW; ++w) {
-          a += wq[w];
-          c += wq[NW + w];
+      for (int j = 0; j < JU; ++j) {
+        if (c0 + j * NT >= total4) continue;
+        const int r = rows[j];
+        const float ss = v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+        float* dst = nullptr;
+        if (r < qd) {
+          sq += ss;
+          const int h = r / HD - g * GQ;
+          if (h >= 0 && h < GQ) dst = q + (r - g * GQ * HD);
+        } else if (r < qd + kd) {
+          sk += ss;
+          if ((r - qd) / HD == g) dst = kraw + (r - qd - g * HD);
+        } else {
+          dst = vraw + (r - qd - kd - g * HD);
         }
-        rd[32] = rsqrtf(a / float(qd) + P.eps);
-        rd[33] = rsqrtf(c / float(kd) + P.eps);
+        if (dst) *reinterpret_cast<float4*>(dst) = v[j];
       }
-      cbar();
-      const float rq = rd[32], rk = rd[33];
-      const int pos = posb()[bq];
-      const double* fr = P.inv_freq[d.type];
-      const float ms = P.mscale[d.type];
-      const float* qn = P.layers[d.layer].q_norm;
-      const float* kg = P.layers[d.layer].k_norm;
-      constexpr int H2 = HD / 2;
-      for (int idx = tid; idx < GQ * H2; idx += NT) {
-        const int h = idx / H2, i = idx - h * H2;
-        const int row = (g * GQ + h) * HD;
-        const float x1 = q[h * HD + i] * rq * qn[row + i];
-        const float x2 = q[h * HD + i + H2] * rq * qn[row + i + H2];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      sk += __shfl_xor_sync(0xffffffffu, sk, o);
+    }
+    mark(2);
+    if (lane == 0) {
+      wq[warp] = sq;
+      wq[NW + warp] = sk;
+    }
+    cbar();
+    if (tid == 0) {
+      float a = 0.f, c = 0.f;
+#pragma unroll 1
+      for (int w = 0; w < NW; ++w) {
+        a += wq[w];
+        c += wq[NW + w];
+      }
+      rd[32] = rsqrtf(a / float(qd) + L.eps);
+      rd[33] = rsqrtf(c / float(kd) + L.eps);
+    }
+    cbar();
+    const float rq = rd[32], rk = rd[33];
+    const int pos = posb()[bq];
+    const double* fr = rope_f(d.type);
+    const float ms = d.type ? L.mscale1 : L.mscale0;
+    constexpr int H2 = HD / 2;
+#pragma unroll 1
+    for (int idx = tid; idx < GQ * H2; idx += NT) {
+      const int h = idx / H2, i = idx - h * H2;
+      const int row = (g * GQ + h) * HD;
+      const float x1 = q[h * HD + i] * rq * d.qnorm[row + i];
+      const float x2 = q[h * HD + i + H2] * rq * d.qnorm[row + i + H2];
+      float c, s;
+      rope_cs(pos, fr[i], ms, c, s);
+      q[h * HD + i] = (x1 * c - x2 * s) * qscale;
+      q[h * HD + i + H2] = (x2 * c + x1 * s) * qscale;
+    }
+    if (own_new) {
+      if (tid < H2) {
+        const int i = tid;
+        const float x1 = kraw[i] * rk * d.knorm[g * HD + i];
+        const float x2 = kraw[i + H2] * rk * d.knorm[g * HD + i + H2];
         float c, s;
         rope_cs(pos, fr[i], ms, c, s);
-        q[h * HD + i] = (x1 * c - x2 * s) * qscale;
-        q[h * HD + i + H2] = (x2 * c + x1 * s) * qscale;
+        kn[i] = f32_to_bf16(x1 * c - x2 * s);
+        kn[i + H2] = f32_to_bf16(x2 * c + x1 * s);
       }
-      if (own_new) {
-        for (int i = tid; i < H2; i += NT) {
-          const float x1 = kraw[i] * rk * kg[g * HD + i];
-          const float x2 = kraw[i + H2] * rk * kg[g * HD + i + H2];
-          float c, s;
-          rope_cs(pos, fr[i], ms, c, s);
-          kn()[i] = f32_to_bf16(x1 * c - x2 * s);
-          kn()[i + H2] = f32_to_bf16(x2 * c + x1 * s);
-        }
-        for (int i = tid; i < HD; i += NT) vn()[i] = f32_to_bf16(vraw[i]);
-        cbar();
-        const int sn_ = snew(d.type)[bq];
-        const size_t row = ((size_t)(d.seqoff + bq) * P.nkv + g) * d.slots + sn_;
-        uint16_t* kd_ = reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(d.kc)) + row * HD;
-        uint16_t* vd_ = reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(d.vc)) + row * HD;
-        for (int i = tid; i < HD; i += NT) {
-          const int sw = (((i >> 3) ^ (sn_ & 7)) << 3) | (i & 7);
-          kd_[sw] = kn()[i];
-          vd_[sw] = vn()[i];
-        }
+      if (tid < HD) vn[tid] = f32_to_bf16(vraw[tid]);
+      cbar();
+      const int sn_ = snew(d.type)[bq];
+      const size_t row = ((size_t)(d.seqoff + bq) * L.nkv + g) * d.slots + sn_;
+      uint16_t* kd_ = reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(d.kc)) + row * HD;
+      uint16_t* vd_ = reinterpret_cast<uint16_t*>(const_cast<uint8_t*>(d.vc)) + row * HD;
+      if (tid < HD) {
+        const int i = tid;
+        const int sw = (((i >> 3) ^ (sn_ & 7)) << 3) | (i & 7);
+        kd_[sw] = kn[i];
+        vd_[sw] = vn[i];
       }
+    }
+  } else {
+    const uint16_t* qin = d.xbf + ((size_t)bq * L.nq + g * GQ) * HD;
+#pragma unroll 1
+    for (int idx = tid; idx < GQ * HD; idx += NT) q[idx] = bf16_to_f32(qin[idx]) * qscale;
+  }
+  cbar();
+  // q as hi + lo bf16 mma A fragments: {a0 hi, a2 hi, a0 lo, a2 lo} per (k-step, lane)
+  if (tid < (HD / 16) * 32) {
+    const int s = tid >> 5, ln = tid & 31, gg = ln >> 2, t = ln & 3;
+    uint4 f = make_uint4(0u, 0u, 0u, 0u);
+    if (gg < GQ) {
+      const float* qr = q + gg * HD + 16 * s + 2 * t;
+      split_bf16x2(qr[0], qr[1], f.x, f.z);
+      split_bf16x2(qr[8], qr[9], f.y, f.w);
+    }
+    sm_at<uint4>(SM_QF)[tid] = f;
+  }
+  cbar();
+}
+
+template <int HD>
+__device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, int nca) {
+  const LC& L = lc();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int* st = sst(d.type);
+  const int GQ = L.nq / L.nkv;
+  const int bq = seg / L.nkv, g = seg % L.nkv;
+  const bool split = (st[seg] < a) || (st[seg + 1] > b);
+  const float* wp = sm_at<float>(SM_APW);
+  uint16_t* out = d.aout + ((size_t)bq * L.nq + g * GQ) * HD;
+  const int pslot = (st[seg] < a) ? 0 : 1;
+  float* piece = L.apart + ((size_t)blockIdx.x * 2 + pslot) * ATT_PW;
+#pragma unroll 1
+  for (int idx = tid; idx < GQ * HD; idx += NT) {
+    const int h = idx / HD, dd = idx - h * HD;
+    float M = -INFINITY;
+#pragma unroll 1
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wp[w * ATT_PW + h * (HD + 2) + HD]);
+    float ls = 0.f, os = 0.f;
+#pragma unroll 1
+    for (int w = 0; w < NW; ++w) {
+      const float e = exp2f(wp[w * ATT_PW + h * (HD + 2) + HD] - M);
+      ls += e * wp[w * ATT_PW + h * (HD + 2) + HD + 1];
+      os += e * wp[w * ATT_PW + h * (HD + 2) + dd];
+    }
+    if (!split) {
+      out[h * HD + dd] = d.out_f16 ? f32_to_f16(os / ls) : f32_to_bf16(os / ls);
     } else {
-      const uint16_t* qin = P.a_q + ((size_t)bq * P.nq + g * GQ) * HD;
-      for (int idx = tid; idx < GQ * HD; idx += NT) q[idx] = bf16_to_f32(qin[idx]) * qscale;
-    }
-    cbar();
-    // q as hi + lo bf16 mma A fragments: {a0 hi, a2 hi, a0 lo, a2 lo} per (k-step, lane)
-    if (tid < (HD / 16) * 32) {
-      const int s = tid >> 5, ln = tid & 31, gg = ln >> 2, t = ln & 3;
-      uint4 f = make_uint4(0u, 0u, 0u, 0u);
-      if (gg < GQ) {
-        const float* qr = q + gg * HD + 16 * s + 2 * t;
-        split_bf16x2(qr[0], qr[1], f.x, f.z);
-        split_bf16x2(qr[8], qr[9], f.y, f.w);
+      piece[h * (HD + 2) + dd] = os;
+      if (dd == 0) {
+        piece[h * (HD + 2) + HD] = M;
+        piece[h * (HD + 2) + HD + 1] = ls;
       }
-      qf()[tid] = f;
-    }
-    cbar();
-  }
-
-  __device__ __forceinline__ void run_attn(const PD& d, Stream& S) {
-    long long a, b;
-    int nca;
-    attn_cta_range(d, a, b, nca);
-    if (a >= b) return;
-    const int* st = sst(d.type);
-    int seg = 0;
-    long long u = a;
-    while (u < b) {
-      while (st[seg + 1] <= u) ++seg;
-      const long long run_end = (b < st[seg + 1]) ? b : st[seg + 1];
-      const int bq = seg / P.nkv;
-      const int Lk = Lb(d.type)[bq];
-      const int sn_ = d.newkv ? snew(d.type)[bq] : -1;
-      const long long jnew = st[seg] + (sn_ >= 0 ? sn_ / ATT_CTA_KEYS : 0);
-      const bool own_new = d.newkv && sn_ >= 0 && jnew >= u && jnew < run_end;
-      attn_prologue(d, seg, own_new);
-      if (u == a) mark(1);
-      S = attn_loop(S, d, seg, u, run_end, Lk, sn_, own_new);
-      cbar();
-      if (run_end == b) mark(2);
-      attn_combine(d, seg, a, b, nca);
-      cbar();
-      u = run_end;
     }
   }
-
-  // This warp's keys of CTA units [u, run_end) of segment seg; writes the
-  // warp's (m, l, o) partial to shared memory.  Non-inlined for the same
-  // reason as gemv_loop.
-  __device__ __noinline__ Stream attn_loop(Stream S, const PD& d, int seg, long long u, long long run_end, int Lk,
-                                           int sn_, bool own_new) const {
-    const RingCtx R = ringctx();
-    const int* st = sst(d.type);
-    const int GQ = P.nq / P.nkv;
-    constexpr int PW = MAX_GQ * (HD + 2);
-    const int g = lane >> 2, t = lane & 3;
-    const uint4* qfr = qf();
-    float m = -INFINITY, lsum = 0.f;
-    // O^T tiles: o[j] covers dims [16 j, 16 j + 16) x query heads 0..7 of the group
-    float o[HD / 16][4];
+  if (!split) return;
+  __threadfence();
+  cbar();
+  const int total = st[L.B * L.nkv];
+  const int c0 = owner(total, nca, st[seg]);
+  const int c1 = owner(total, nca, st[seg + 1] - 1);
+  if (tid == 0) {
+    const uint32_t old = atomicAdd(L.seg_ctr + seg, 1u);
+    flags()[1] = (int(old) == c1 - c0) ? 1 : 0;
+  }
+  cbar();
+  if (!flags()[1]) return;
+  __threadfence();
+  // warp h combines query head h over the pieces c0..c1 (one piece per lane
+  // for the max and the denominators; shuffled weights for the outputs)
+  if (warp < GQ) {
+    const int h = warp;
+    auto piece_of = [&](int c) {
+      const int sl = (st[seg] < rstart(total, nca, c)) ? 0 : 1;
+      return L.apart + ((size_t)c * 2 + sl) * ATT_PW + h * (HD + 2);
+    };
+    float M = -INFINITY;
+#pragma unroll 1
+    for (int c = c0 + lane; c <= c1; c += 32) M = fmaxf(M, __ldcg(piece_of(c) + HD));
 #pragma unroll
-    for (int j = 0; j < HD / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    for (long long jc = u; jc < run_end; ++jc) {
-      const int key0 = int(jc - st[seg]) * ATT_CTA_KEYS + warp * ATT_KEYS;
-      if (key0 >= Lk) continue;
-      uint8_t* slot = const_cast<uint8_t*>(wait_slot(R, S));
-      uint8_t* Ks = slot;
-      uint8_t* Vs = slot + ATT_KEYS * HD * 2;
-      const bool patch = own_new && sn_ >= key0 && sn_ < key0 + ATT_KEYS;
-      if (patch) {
-        const int r = sn_ - key0;  // == sn_ & 7
-        uint16_t* kr = reinterpret_cast<uint16_t*>(Ks + r * HD * 2);
-        uint16_t* vr = reinterpret_cast<uint16_t*>(Vs + r * HD * 2);
-        for (int i = lane; i < HD; i += 32) {
-          const int sw = (((i >> 3) ^ r) << 3) | (i & 7);
-          kr[sw] = kn()[i];
-          vr[sw] = vn()[i];
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    constexpr int DPL = HD / 32;  // dims per lane
+    float acc[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+    float Lsum = 0.f;
+#pragma unroll 1
+    for (int cb = c0; cb <= c1; cb += 32) {
+      const int cl = cb + lane;
+      float ev = 0.f;
+      if (cl <= c1) {
+        const float* pc = piece_of(cl);
+        ev = exp2f(__ldcg(pc + HD) - M);
+        Lsum = fmaf(ev, __ldcg(pc + HD + 1), Lsum);
+      }
+      const int n = min(32, c1 - cb + 1);
+#pragma unroll 1
+      for (int i = 0; i < n; ++i) {
+        const float w = __shfl_sync(0xffffffffu, ev, i);
+        const float* pc = piece_of(cb + i) + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, __ldcg(pc + e), acc[e]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    const float inv = 1.f / Lsum;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) {
+      const float v = acc[e] * inv;
+      out[h * HD + lane * DPL + e] = d.out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
+    }
+  }
+  if (tid == 0) L.seg_ctr[seg] = 0u;
+}
+
+template <int HD>
+__device__ __noinline__ void attn_phase(const PD& d) {
+  const LC& L = lc();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int a, b, nca;
+  attn_cta_range(d.type, blockIdx.x, a, b, nca);
+  if (a >= b) return;
+  const int* st = sst(d.type);
+  const int GQ = L.nq / L.nkv;
+  int seg = 0;
+#pragma unroll 1
+  for (int u = a; u < b;) {
+    while (st[seg + 1] <= u) ++seg;
+    const int run_end = (b < st[seg + 1]) ? b : st[seg + 1];
+    const int bq = seg / L.nkv;
+    const int Lk = Lb(d.type)[bq];
+    const int sn_ = d.newkv ? snew(d.type)[bq] : -1;
+    const int jnew = st[seg] + (sn_ >= 0 ? sn_ / ATT_CTA_KEYS : 0);
+    const bool own_new = d.newkv && sn_ >= 0 && jnew >= u && jnew < run_end;
+    attn_prologue<HD>(d, seg, own_new);
+    if (u == a) mark(3);
+    {
+      // this warp's keys of CTA units [u, run_end); its (m, l, o) partial goes
+      // to shared memory
+      Ring R;
+      ring_load(R, warp);
+      const int g = lane >> 2, t = lane & 3;
+      const uint4* qfr = sm_at<uint4>(SM_QF);
+      const uint16_t* kn = sm_at<uint16_t>(SM_KNV);
+      const uint16_t* vn = kn + 128;
+      float m = -INFINITY, lsum = 0.f;
+      // O^T tiles: o[j] covers dims [16 j, 16 j + 16) x query heads 0..7 of the group
+      float o[HD / 16][4];
+#pragma unroll
+      for (int j = 0; j < HD / 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+#pragma unroll 1
+      for (int jc = u; jc < run_end; ++jc) {
+        const int key0 = (jc - st[seg]) * ATT_CTA_KEYS + warp * ATT_KEYS;
+        if (key0 >= Lk) continue;
+        uint8_t* slot = ring_wait(R, warp, lane);
+        uint8_t* Ks = slot;
+        uint8_t* Vs = slot + ATT_KEYS * HD * 2;
+        const bool patch = own_new && sn_ >= key0 && sn_ < key0 + ATT_KEYS;
+        if (patch) {
+          const int r = sn_ - key0;  // == sn_ & 7
+          uint16_t* kr = reinterpret_cast<uint16_t*>(Ks + r * HD * 2);
+          uint16_t* vr = reinterpret_cast<uint16_t*>(Vs + r * HD * 2);
+#pragma unroll 1
+          for (int i = lane; i < HD; i += 32) {
+            const int sw = (((i >> 3) ^ r) << 3) | (i & 7);
+            kr[sw] = kn[i];
+            vr[sw] = vn[i];
+          }
+          warp_sync();
         }
-        __syncwarp();
-      }
-      // S = Q K^T: rows = query heads (g), columns = the 8 keys (2t, 2t+1)
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int r = lane & 7, mi = lane >> 3;
+        // S = Q K^T: rows = query heads (g), columns = the 8 keys (2t, 2t+1)
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int r = lane & 7, mi = lane >> 3;
 #pragma unroll
-      for (int s = 0; s < HD / 16; s += 2) {
-        uint32_t k0, k1, k2, k3;
-        ldsm_x4(k0, k1, k2, k3, Ks + r * HD * 2 + (((2 * s + mi) ^ r) << 4));
-        const uint4 f0 = qfr[s * 32 + lane], f1 = qfr[(s + 1) * 32 + lane];
-        mma_16816(sc, f0.x, 0u, f0.y, 0u, k0, k1);
-        mma_16816(sc, f0.z, 0u, f0.w, 0u, k0, k1);
-        mma_16816(sc, f1.x, 0u, f1.y, 0u, k2, k3);
-        mma_16816(sc, f1.z, 0u, f1.w, 0u, k2, k3);
+        for (int s = 0; s < HD / 16; s += 2) {
+          uint32_t k0, k1, k2, k3;
+          ldsm_x4(k0, k1, k2, k3, Ks + r * HD * 2 + (((2 * s + mi) ^ r) << 4));
+          const uint4 f0 = qfr[s * 32 + lane], f1 = qfr[(s + 1) * 32 + lane];
+          mma_16816(sc, f0.x, 0u, f0.y, 0u, k0, k1);
+          mma_16816(sc, f0.z, 0u, f0.w, 0u, k0, k1);
+          mma_16816(sc, f1.x, 0u, f1.y, 0u, k2, k3);
+          mma_16816(sc, f1.z, 0u, f1.w, 0u, k2, k3);
+        }
+        const int ka = key0 + 2 * t;
+        const float s0 = (ka < Lk) ? sc[0] : -INFINITY;
+        const float s1 = (ka + 1 < Lk) ? sc[1] : -INFINITY;
+        float mx = fmaxf(s0, s1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m, mx);
+        const float alpha = exp2f(m - mn);
+        const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
+        lsum = lsum * alpha + p0 + p1;
+        m = mn;
+        // this lane's O^T columns are heads 2t and 2t+1: fetch their rescale factors
+        const float a_lo = __shfl_sync(0xffffffffu, alpha, (2 * t) * 4);
+        const float a_hi = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) * 4);
+#pragma unroll
+        for (int j = 0; j < HD / 16; ++j) {
+          o[j][0] *= a_lo;
+          o[j][1] *= a_hi;
+          o[j][2] *= a_lo;
+          o[j][3] *= a_hi;
+        }
+        // O^T += V^T P^T: A = V^T from transposed 8x8 loads, B = (p0, p1) as hi + lo bf16
+        uint32_t pa, pl;
+        split_bf16x2(p0, p1, pa, pl);
+#pragma unroll
+        for (int q4 = 0; q4 < HD / 32; ++q4) {
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_t(v0, v1, v2, v3, Vs + r * HD * 2 + (((4 * q4 + mi) ^ r) << 4));
+          mma_1688(o[2 * q4], v0, v1, pa);
+          mma_1688(o[2 * q4], v0, v1, pl);
+          mma_1688(o[2 * q4 + 1], v2, v3, pa);
+          mma_1688(o[2 * q4 + 1], v2, v3, pl);
+        }
+        ring_release<HD>(R, warp, lane, patch);
       }
-      const int ka = key0 + 2 * t;
-      const float s0 = (ka < Lk) ? sc[0] : -INFINITY;
-      const float s1 = (ka + 1 < Lk) ? sc[1] : -INFINITY;
-      float mx = fmaxf(s0, s1);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float mn = fmaxf(m, mx);
-      const float alpha = exp2f(m - mn);
-      const float p0 = exp2f(s0 - mn), p1 = exp2f(s1 - mn);
-      lsum = lsum * alpha + p0 + p1;
-      m = mn;
-      // this lane's O^T columns are heads 2t and 2t+1: fetch their rescale factors
-      const float a_lo = __shfl_sync(0xffffffffu, alpha, (2 * t) * 4);
-      const float a_hi = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) * 4);
+      ring_store(R, warp, lane);
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+      float* wp = sm_at<float>(SM_APW) + warp * ATT_PW;
 #pragma unroll
       for (int j = 0; j < HD / 16; ++j) {
-        o[j][0] *= a_lo;
-        o[j][1] *= a_hi;
-        o[j][2] *= a_lo;
-        o[j][3] *= a_hi;
-      }
-      // O^T += V^T P^T: A = V^T from transposed 8x8 loads, B = (p0, p1) as hi + lo bf16
-      uint32_t pa, pl;
-      split_bf16x2(p0, p1, pa, pl);
-#pragma unroll
-      for (int q4 = 0; q4 < HD / 32; ++q4) {
-        uint32_t v0, v1, v2, v3;
-        ldsm_x4_t(v0, v1, v2, v3, Vs + r * HD * 2 + (((4 * q4 + mi) ^ r) << 4));
-        mma_1688(o[2 * q4], v0, v1, pa);
-        mma_1688(o[2 * q4], v0, v1, pl);
-        mma_1688(o[2 * q4 + 1], v2, v3, pa);
-        mma_1688(o[2 * q4 + 1], v2, v3, pl);
-      }
-      release_slot(R, S, patch);
-    }
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-    float* wp = apw() + warp * PW;
-#pragma unroll
-    for (int j = 0; j < HD / 16; ++j) {
-      if (2 * t < GQ) {
-        wp[(2 * t) * (HD + 2) + 16 * j + g] = o[j][0];
-        wp[(2 * t) * (HD + 2) + 16 * j + 8 + g] = o[j][2];
-      }
-      if (2 * t + 1 < GQ) {
-        wp[(2 * t + 1) * (HD + 2) + 16 * j + g] = o[j][1];
-        wp[(2 * t + 1) * (HD + 2) + 16 * j + 8 + g] = o[j][3];
-      }
-    }
-    if (g < GQ && t == 0) {
-      wp[g * (HD + 2) + HD] = m;
-      wp[g * (HD + 2) + HD + 1] = lsum;
-    }
-    return S;
-  }
-
-  __device__ __noinline__ void attn_combine(const PD& d, int seg, long long a, long long b, int nca) {
-    constexpr int PW = MAX_GQ * (HD + 2);
-    const int* st = sst(d.type);
-    const int GQ = P.nq / P.nkv;
-    const int bq = seg / P.nkv, g = seg % P.nkv;
-    const bool split = (st[seg] < a) || (st[seg + 1] > b);
-    const float* wp = apw();
-    uint16_t* out = d.aout + ((size_t)bq * P.nq + g * GQ) * HD;
-    const int pslot = (st[seg] < a) ? 0 : 1;
-    float* piece = P.ws.apart + ((size_t)cta * 2 + pslot) * PW;
-    for (int idx = tid; idx < GQ * HD; idx += NT) {
-      const int h = idx / HD, dd = idx - h * HD;
-      float M = -INFINITY;
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, wp[w * PW + h * (HD + 2) + HD]);
-      float ls = 0.f, os = 0.f;
-      for (int w = 0; w < NW; ++w) {
-        const float e = exp2f(wp[w * PW + h * (HD + 2) + HD] - M);
-        ls += e * wp[w * PW + h * (HD + 2) + HD + 1];
-        os += e * wp[w * PW + h * (HD + 2) + dd];
-      }
-      if (!split) {
-        out[h * HD + dd] = d.out_f16 ? f32_to_f16(os / ls) : f32_to_bf16(os / ls);
-      } else {
-        piece[h * (HD + 2) + dd] = os;
-        if (dd == 0) {
-          piece[h * (HD + 2) + HD] = M;
-          piece[h * (HD + 2) + HD + 1] = ls;
+        if (2 * t < GQ) {
+          wp[(2 * t) * (HD + 2) + 16 * j + g] = o[j][0];
+          wp[(2 * t) * (HD + 2) + 16 * j + 8 + g] = o[j][2];
+        }
+        if (2 * t + 1 < GQ) {
+          wp[(2 * t + 1) * (HD + 2) + 16 * j + g] = o[j][1];
+          wp[(2 * t + 1) * (HD + 2) + 16 * j + 8 + g] = o[j][3];
         }
       }
-    }
-    if (!split) return;
-    __threadfence();
-    cbar();
-    const long long total = st[P.B * P.nkv];
-    const int c0 = owner(total, nca, st[seg]);
-    const int c1 = owner(total, nca, st[seg + 1] - 1);
-    if (tid == 0) {
-      const uint32_t old = atomicAdd(P.ws.seg_ctr + seg, 1u);
-      flags()[1] = (int(old) == c1 - c0) ? 1 : 0;
+      if (g < GQ && t == 0) {
+        wp[g * (HD + 2) + HD] = m;
+        wp[g * (HD + 2) + HD + 1] = lsum;
+      }
     }
     cbar();
-    if (!flags()[1]) return;
-    __threadfence();
-    // warp h combines query head h over the pieces c0..c1 (one piece per lane
-    // for the max and the denominators; shuffled weights for the outputs)
-    if (warp < GQ) {
-      const int h = warp;
-      auto piece_of = [&](int c) {
-        const int sl = (st[seg] < rstart(total, nca, c)) ? 0 : 1;
-        return P.ws.apart + ((size_t)c * 2 + sl) * PW + h * (HD + 2);
-      };
-      float M = -INFINITY;
-      for (int c = c0 + lane; c <= c1; c += 32) M = fmaxf(M, __ldcg(piece_of(c) + HD));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      constexpr int DPL = HD / 32;  // dims per lane
-      float acc[DPL];
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-      float Lsum = 0.f;
-      for (int cb = c0; cb <= c1; cb += 32) {
-        const int cl = cb + lane;
-        float ev = 0.f;
-        if (cl <= c1) {
-          const float* pc = piece_of(cl);
-          ev = exp2f(__ldcg(pc + HD) - M);
-          Lsum = fmaf(ev, __ldcg(pc + HD + 1), Lsum);
-        }
-        const int n = min(32, c1 - cb + 1);
-#pragma unroll 4
-        for (int i = 0; i < n; ++i) {
-          const float w = __shfl_sync(0xffffffffu, ev, i);
-          const float* pc = piece_of(cb + i) + lane * DPL;
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, __ldcg(pc + e), acc[e]);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
-      const float inv = 1.f / Lsum;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) {
-        const float v = acc[e] * inv;
-        out[h * HD + lane * DPL + e] = d.out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
-      }
-    }
-    if (tid == 0) P.ws.seg_ctr[seg] = 0u;
+    if (run_end == b) mark(4);
+    attn_combine<HD>(d, seg, a, b, nca);
+    cbar();
+    if (run_end == b) mark(5);
+    u = run_end;
   }
+}
 
-  // ---- argmax phase (and the sum of the lm_head slabs when K was split) ----
-  __device__ __noinline__ void run_argmax(const PD& d) {
-    const int V = P.vocab, B = P.B;
-    const int r0 = int(rstart(V, P.nc, cta)), r1 = int(rstart(V, P.nc, cta + 1));
-    if (d.lpart != nullptr) {
-      for (int bq = 0; bq < B; ++bq)
-        for (int r = r0 + tid; r < r1; r += NT) {
-          float y = 0.f;
-          for (int s0 = 0; s0 < d.lns; s0 += 4) {
-            float t[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              t[i] = (s0 + i < d.lns) ? __ldcg(d.lpart + ((size_t)(s0 + i) * B + bq) * V + r) : 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (s0 + i < d.lns) y += t[i];
-          }
-          P.logits[(size_t)bq * V + r] = y;
-        }
-      cbar();
-    }
-    if (P.next_token == nullptr) return;
-    float* rv = red();
-    int* ri = reinterpret_cast<int*>(red() + 32);
-    for (int bq = 0; bq < B; ++bq) {
-      float best = -INFINITY;
-      int bi = 0x7fffffff;
+// ---------------------------------------------------------------------------
+// Argmax (and the sum of the lm_head slabs when K was split)
+// ---------------------------------------------------------------------------
+__device__ __noinline__ void argmax_phase(const PD& d) {
+  const LC& L = lc();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int V = L.vocab, B = L.B;
+  const int r0 = int(rstart(V, L.nc, blockIdx.x)), r1 = int(rstart(V, L.nc, blockIdx.x + 1));
+  if (d.lpart != nullptr) {
+#pragma unroll 1
+    for (int bq = 0; bq < B; ++bq)
+#pragma unroll 1
       for (int r = r0 + tid; r < r1; r += NT) {
-        const float v = __ldcg(P.logits + (size_t)bq * V + r);
-        if (v > best || (v == best && r < bi)) {
-          best = v;
-          bi = r;
-        }
-      }
+        float y = 0.f;
+#pragma unroll 1
+        for (int s0 = 0; s0 < d.lns; s0 += 4) {
+          float t[4];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > best || (ov == best && oi < bi)) {
-          best = ov;
-          bi = oi;
+          for (int i = 0; i < 4; ++i)
+            t[i] = (s0 + i < d.lns) ? __ldcg(d.lpart + ((size_t)(s0 + i) * B + bq) * V + r) : 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (s0 + i < d.lns) y += t[i];
         }
+        L.logits[(size_t)bq * V + r] = y;
       }
-      if (lane == 0) {
-        rv[warp] = best;
-        ri[warp] = bi;
+    cbar();
+  }
+  if (L.next_token == nullptr) return;
+  float* rv = red();
+  int* ri = reinterpret_cast<int*>(red() + 32);
+#pragma unroll 1
+  for (int bq = 0; bq < B; ++bq) {
+    float best = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll 1
+    for (int r = r0 + tid; r < r1; r += NT) {
+      const float v = __ldcg(L.logits + (size_t)bq * V + r);
+      if (v > best || (v == best && r < bi)) {
+        best = v;
+        bi = r;
       }
-      cbar();
-      if (tid == 0) {
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > best || (ov == best && oi < bi)) {
+        best = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      rv[warp] = best;
+      ri[warp] = bi;
+    }
+    cbar();
+    if (tid == 0) {
+      float bb = -INFINITY;
+      int bbi = 0x7fffffff;
+#pragma unroll 1
+      for (int w = 0; w < NW; ++w)
+        if (rv[w] > bb || (rv[w] == bb && ri[w] < bbi)) {
+          bb = rv[w];
+          bbi = ri[w];
+        }
+      L.amax_val[(size_t)blockIdx.x * B + bq] = bb;
+      L.amax_idx[(size_t)blockIdx.x * B + bq] = bbi;
+    }
+    cbar();
+  }
+  if (tid == 0) {
+    __threadfence();
+    const uint32_t old = atomicAdd(L.ctl + 3, 1u);
+    if (int(old) == L.nc - 1) {
+      __threadfence();
+#pragma unroll 1
+      for (int bq = 0; bq < B; ++bq) {
         float bb = -INFINITY;
         int bbi = 0x7fffffff;
-        for (int w = 0; w < NW; ++w)
-          if (rv[w] > bb || (rv[w] == bb && ri[w] < bbi)) {
-            bb = rv[w];
-            bbi = ri[w];
+#pragma unroll 1
+        for (int c = 0; c < L.nc; ++c) {
+          const float v = __ldcg(L.amax_val + (size_t)c * B + bq);
+          const int i = __ldcg(L.amax_idx + (size_t)c * B + bq);
+          if (v > bb || (v == bb && i < bbi)) {
+            bb = v;
+            bbi = i;
           }
-        P.ws.amax_val[(size_t)cta * B + bq] = bb;
-        P.ws.amax_idx[(size_t)cta * B + bq] = bbi;
-      }
-      cbar();
-    }
-    if (tid == 0) {
-      __threadfence();
-      const uint32_t old = atomicAdd(P.ws.ctl + 3, 1u);
-      if (int(old) == P.nc - 1) {
-        __threadfence();
-        for (int bq = 0; bq < B; ++bq) {
-          float bb = -INFINITY;
-          int bbi = 0x7fffffff;
-          for (int c = 0; c < P.nc; ++c) {
-            const float v = __ldcg(P.ws.amax_val + (size_t)c * B + bq);
-            const int i = __ldcg(P.ws.amax_idx + (size_t)c * B + bq);
-            if (v > bb || (v == bb && i < bbi)) {
-              bb = v;
-              bbi = i;
-            }
-          }
-          P.next_token[bq] = (bbi == 0x7fffffff) ? 0 : bbi;
         }
-        P.ws.ctl[3] = 0u;
+        L.next_token[bq] = (bbi == 0x7fffffff) ? 0 : bbi;
       }
+      L.ctl[3] = 0u;
     }
   }
+}
 
-  // ---- launch-level setup ----
-  __device__ __noinline__ void setup() {
-    if (lane == 0) {
-      for (int s = 0; s < NSLOT; ++s) mbar_init(fullb(warp, s), 1u);
-      fence_mbar_init();
-    }
-    if (tid == 0) flags()[0] = 1;
-    const int B = P.B;
-    if (P.mode != MODE_GEMV && tid < B) posb()[tid] = (P.pos_const >= 0) ? P.pos_const : P.pos[tid];
-    __syncthreads();
-    if (P.mode != MODE_GEMV && tid < 2 * B) {
-      const int type = tid / B, bq = tid - type * B;
-      const int pos = posb()[bq];
-      int Lk = 0, sn = -1;
-      bool bad_pos = pos < 0;
-      if (P.mode == MODE_DECODE) {
-        if (type == 1) {
-          bad_pos |= pos >= P.max_ctx;
-          Lk = pos + 1;
-          sn = pos;
-        } else {
-          Lk = pos + 1 < P.window ? pos + 1 : P.window;
-          sn = pos % P.window;
-        }
-      } else if (type == 0) {
-        if (P.a_window == 0) {
-          bad_pos |= pos >= P.a_slots;
-          Lk = pos + 1;
-        } else {
-          Lk = pos + 1 < P.a_window ? pos + 1 : P.a_window;
-        }
-      }
-      if (bad_pos) {
-        if (cta == 0) set_error(EW_BAD_POS);
-        Lk = 0;
-        sn = -1;
-      }
-      Lb(type)[bq] = Lk;
-      snew(type)[bq] = sn;
-    }
-    __syncthreads();
-    if (P.mode != MODE_GEMV && tid < 2) {
-      int* st = sst(tid);
-      st[0] = 0;
-      for (int s = 0; s < B * P.nkv; ++s) {
-        const int Lk = Lb(tid)[s / P.nkv];
-        st[s + 1] = st[s] + (Lk + ATT_CTA_KEYS - 1) / ATT_CTA_KEYS;
-      }
-    }
-    __syncthreads();
+// ---------------------------------------------------------------------------
+// Launch setup, phase start, the kernel
+// ---------------------------------------------------------------------------
+__device__ __noinline__ void setup(const EngineParams& P) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cta = blockIdx.x;
+  LC& L = lc();
+  if (tid == 0) {
+    L.B = P.B;
+    L.d = P.d;
+    L.nq = P.nq;
+    L.nkv = P.nkv;
+    L.ffn = P.ffn;
+    L.vocab = P.vocab;
+    L.window = P.window;
+    L.nc = P.nc;
+    L.mode = P.mode;
+    L.begin = P.phase_begin;
+    L.end = P.phase_end;
+    L.n_layers = P.n_layers;
+    L.seq0 = P.seq0;
+    L.pos_const = P.pos_const;
+    L.trace_phases = P.trace_phases;
+    L.max_ctx = P.max_ctx;
+    L.eps = P.eps;
+    L.mscale0 = P.mscale[0];
+    L.mscale1 = P.mscale[1];
+    L.cur_phase = P.phase_begin;
+    L.scaled = 0;
+    L.final_norm = P.final_norm;
+    L.ctl = P.ws.ctl;
+    L.seg_ctr = P.ws.seg_ctr;
+    L.apart = P.ws.apart;
+    L.amax_val = P.ws.amax_val;
+    L.amax_idx = P.ws.amax_idx;
+    L.plan = reinterpret_cast<PD*>(P.ws.plan);
+    L.trace = P.trace;
+    L.tokens = P.tokens;
+    L.embed = P.embed;
+    L.logits = P.logits;
+    L.next_token = P.next_token;
+    L.pos = P.pos;
+#pragma unroll 1
+    for (int s = 0; s < PD_SLOTS; ++s) mbar_init(pd_bar(s), 1u);
   }
+  if (lane == 0) {
+#pragma unroll 1
+    for (int s = 0; s < NSLOT; ++s) mbar_init(ring_bar(warp, s), 1u);
+    fence_mbar_init();
+  }
+  if (tid < 128) sm_at<double>(SM_ROPE)[tid] = P.inv_freq[tid >> 6][tid & 63];
+  const int B = P.B;
+  if (P.mode != MODE_GEMV && tid < B) posb()[tid] = (P.pos_const >= 0) ? P.pos_const : P.pos[tid];
+  __syncthreads();
+  if (P.mode != MODE_GEMV && tid < 2 * B) {
+    const int type = tid / B, bq = tid - type * B;
+    const int pos = posb()[bq];
+    int Lk = 0, sn = -1;
+    bool bad_pos = pos < 0;
+    if (P.mode == MODE_DECODE) {
+      if (type == 1) {
+        bad_pos |= pos >= P.max_ctx;
+        Lk = pos + 1;
+        sn = pos;
+      } else {
+        Lk = pos + 1 < P.window ? pos + 1 : P.window;
+        sn = pos % P.window;
+      }
+    } else if (type == 0) {
+      if (P.a_window == 0) {
+        bad_pos |= pos >= P.a_slots;
+        Lk = pos + 1;
+      } else {
+        Lk = pos + 1 < P.a_window ? pos + 1 : P.a_window;
+      }
+    }
+    if (bad_pos) {
+      if (cta == 0) set_error(EW_BAD_POS);
+      Lk = 0;
+      sn = -1;
+    }
+    Lb(type)[bq] = Lk;
+    snew(type)[bq] = sn;
+  }
+  // phase descriptors: the first PD_LEAD + 1 into shared memory, the rest
+  // (one thread each) into the workspace plan
+  const int begin = P.phase_begin, end = P.phase_end;
+  if (lane == 0 && warp <= PD_LEAD && begin + warp < end) build_pd(P, begin + warp, &pd_slot(begin + warp));
+  if (lane == 0 && warp > PD_LEAD) {
+    const int q = begin + PD_LEAD + 1 + cta + P.nc * (warp - PD_LEAD - 1);
+    if (q < end) build_pd(P, q, reinterpret_cast<PD*>(P.ws.plan) + q);
+  }
+  __syncthreads();
+  if (P.mode != MODE_GEMV && tid < 2) {
+    int* st = sst(tid);
+    st[0] = 0;
+#pragma unroll 1
+    for (int s = 0; s < B * P.nkv; ++s) {
+      const int Lk = Lb(tid)[s / P.nkv];
+      st[s + 1] = st[s] + (Lk + ATT_CTA_KEYS - 1) / ATT_CTA_KEYS;
+    }
+  }
+  __syncthreads();
+  // ring state: both cursors at the warp's first unit
+  if (lane == 0) {
+    Ring* s = ring_state(warp);
+    *reinterpret_cast<uint4*>(s) = make_uint4(0u, 0u, 0u, 0u);
+    s->ld.kind = CUR_WAIT;
+    s->ld.p = begin;
+    cur_normalize(&s->ld, warp);
+    s->pf = s->ld;
+  }
+  warp_sync();
+}
 
-  __device__ void run() {
-    setup();
-    Stream S = loader_start();
-    for (int p = P.phase_begin; p < P.phase_end; ++p) {
-      if (p != P.phase_begin) {
-        if (!grid_wait(uint32_t(p - P.phase_begin) * uint32_t(P.nc))) break;
-      }
-      cur_phase = p;
-      mark(0);
-      // the phase descriptor lives in shared memory (read by every warp)
-      PD& d = *reinterpret_cast<PD*>(sm + L::PDS);
-      if (tid == 0) get_phase(p, d);
-      cbar();
-      if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_BF16)
-        run_gemv(d, S);
-      else if (d.kind == PK_ATTN)
-        run_attn(d, S);
-      else if (d.kind == PK_REDUCE)
-        run_reduce();
-      else
-        run_argmax(d);
-      grid_arrive();
-      mark(3);
-    }
-    drain(S);
-    cbar();
-    if (tid == 0) {
-      __threadfence();
-      const uint32_t old = atomicAdd(P.ws.ctl + 1, 1u);
-      if (int(old) == P.nc - 1) {
-        P.ws.ctl[0] = 0u;
-        P.ws.ctl[1] = 0u;
-        __threadfence();
-      }
+// Phase start: descriptor p ready in shared memory, the copy of descriptor
+// p + PD_LEAD under way, rings topped up.
+template <int HD>
+__device__ __forceinline__ void phase_start(int p) {
+  if (threadIdx.x == 0) {
+    LC& L = lc();
+    L.cur_phase = p;
+    pd_ready(p, true);
+    const int q = p + PD_LEAD;
+    if (q < L.end && q > L.begin + PD_LEAD) {
+      fence_proxy_async_all();
+      mbar_expect_tx(pd_bar(q), (uint32_t)sizeof(PD));
+      bulk_g2s(&pd_slot(q), L.plan + q, (uint32_t)sizeof(PD), pd_bar(q));
     }
   }
-};
+  cbar();
+  mark(1);
+  ring_top_up<HD>();
+}
 
 template <int NB, int HD>
 __global__ void __launch_bounds__(NT, 1) w4a_engine_kernel(const __grid_constant__ EngineParams P) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  Engine<NB, HD> e(P, smem_raw);
-  e.run();
+  setup(P);
+  const int begin = lc().begin, end = lc().end;
+  ring_top_up<HD>();
+#pragma unroll 1
+  for (int p = begin; p < end; ++p) {
+    if (p != begin) {
+      if (!grid_wait(uint32_t(p - begin) * uint32_t(lc().nc))) break;
+    }
+    if (threadIdx.x == 0) lc().cur_phase = p;
+    mark(0);
+    phase_start<HD>(p);
+    const PD& d = pd_slot(p);
+    const int kind = d.kind;
+    if (kind == PK_GEMV_W4 || kind == PK_GEMV_BF16)
+      gemv_phase<NB, HD>(d);
+    else if (kind == PK_ATTN)
+      attn_phase<HD>(d);
+    else if (kind == PK_REDUCE)
+      reduce_phase(d);
+    else
+      argmax_phase(d);
+    grid_arrive();
+    mark(6);
+  }
+  ring_drain();
+  cbar();
+  if (threadIdx.x == 0) {
+    uint32_t* ctl = lc().ctl;
+    __threadfence();
+    const uint32_t old = atomicAdd(ctl + 1, 1u);
+    if (int(old) == lc().nc - 1) {
+      ctl[0] = 0u;
+      ctl[1] = 0u;
+      __threadfence();
+    }
+  }
 }
 
 }  // namespace w4a

@@ -82,6 +82,7 @@ struct Workspace {
   float* xA;            // residual at the layer input [B][d]
   float* xB;            // residual after attention [B][d]
   float* g_part;        // standalone GEMV output when split [ns][B][n]
+  void* plan;           // phase descriptors, one per phase of the launch
 };
 
 struct EngineParams {
