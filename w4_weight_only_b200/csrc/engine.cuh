@@ -6,11 +6,10 @@
 // contiguous range of ~4 KB "units" (16 weight rows x 512 int4 columns, 16
 // rows x 128 bf16 columns, or 8 keys of K and V) from HBM into a two-slot ring
 // of shared memory with bulk asynchronous copies completing on mbarriers, and
-// refills a slot with its next unit as soon as it has used it.  A second
-// cursor runs a few units ahead of the ring and asks for those units to be
-// brought into L2, so HBM keeps streaming while the CTA sits in a barrier or
-// stages its inputs.  Both cursors run across phase boundaries: weights and
-// old KV entries do not depend on the activations.
+// refills a slot with its next unit as soon as it has copied the unit into
+// registers.  The stream runs across phase boundaries: weights and old KV
+// entries do not depend on the activations, so the copies for phase p + 1
+// are in flight while the CTA waits at the barrier that ends phase p.
 //
 // Phase descriptors (what a phase reads, computes and writes) are built on the
 // device at launch, in parallel by one thread per phase, into a table in the
@@ -55,7 +54,6 @@ namespace w4a {
 constexpr long long WAIT_CYCLES = 4000000000LL;  // bound on any single wait (~2 s)
 constexpr int MAX_SEG = MAX_B * 16;              // attention segments (batch x kv heads)
 constexpr int NS_MAX = 8;                        // k-slabs a GEMV phase may choose
-constexpr int PF_AHEAD = 4;                      // units per warp requested into L2 ahead of the ring
 
 __host__ __device__ inline long long rstart(long long U, int n, int i) { return (U * i) / n; }
 // CTA (of n) whose range [rstart(c), rstart(c+1)) contains unit u.
@@ -186,12 +184,11 @@ struct alignas(16) Cursor {
   int x0, x1, x2, x3, x4, x5, x6, pad_;
 };
 struct alignas(16) Ring {
-  uint32_t consumed, issued, pf_issued;
-  int bad;  // a wait of this warp timed out: stop waiting and issuing
+  uint32_t consumed, issued, pad_;
+  int bad;    // a wait of this warp timed out: stop waiting and issuing
   Cursor ld;  // next unit to copy into the ring
-  Cursor pf;  // next unit to request into L2
 };
-static_assert(sizeof(Cursor) == 64 && sizeof(Ring) == 144, "ring state layout");
+static_assert(sizeof(Cursor) == 64 && sizeof(Ring) == 80, "ring state layout");
 
 // ---------------------------------------------------------------------------
 // Shared memory map
@@ -622,9 +619,9 @@ __device__ __forceinline__ void cur_store(Cursor* s, const Cursor& c) {
   q[3] = make_uint4(uint32_t(c.x4), uint32_t(c.x5), uint32_t(c.x6), 0u);
 }
 
-// Next unit of a register cursor (which = 0: ring cursor, 1: prefetch cursor);
-// the slow path goes through the warp's shared-memory copy.
-__device__ __forceinline__ void cur_next(Cursor& c, int which, int warp, int lane) {
+// Next unit of the warp's register cursor; the slow path goes through the
+// warp's shared-memory copy.
+__device__ __forceinline__ void cur_next(Cursor& c, int warp, int lane) {
   if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
     ++c.i;
     if (++c.x6 == c.x2) {
@@ -638,7 +635,7 @@ __device__ __forceinline__ void cur_next(Cursor& c, int which, int warp, int lan
   } else {
     ++c.i;
   }
-  Cursor* s = which ? &ring_state(warp)->pf : &ring_state(warp)->ld;
+  Cursor* s = &ring_state(warp)->ld;
   // lanes run independently between warp barriers: every lane must be done
   // reading the shared copy before lane 0 rewrites it
   warp_sync();
@@ -675,39 +672,25 @@ __device__ __forceinline__ void ring_load(Ring& R, int warp) {
   const uint4 h = *reinterpret_cast<const uint4*>(s);
   R.consumed = h.x;
   R.issued = h.y;
-  R.pf_issued = h.z;
+  R.pad_ = 0u;
   R.bad = int(h.w);
   cur_load(R.ld, &s->ld);
-  cur_load(R.pf, &s->pf);
 }
 __device__ __forceinline__ void ring_store(const Ring& R, int warp, int lane) {
   warp_sync();  // all lanes are done reading the shared copy
   if (lane == 0) {
     Ring* s = ring_state(warp);
-    *reinterpret_cast<uint4*>(s) = make_uint4(R.consumed, R.issued, R.pf_issued, uint32_t(R.bad));
+    *reinterpret_cast<uint4*>(s) = make_uint4(R.consumed, R.issued, 0u, uint32_t(R.bad));
     cur_store(&s->ld, R.ld);
-    cur_store(&s->pf, R.pf);
   }
   warp_sync();
 }
 
-// Fill free ring slots (and keep the L2 requests PF_AHEAD units ahead).
+// Fill free ring slots.
 template <int HD>
 __device__ __forceinline__ void ring_fill(Ring& R, int warp, int lane) {
 #pragma unroll 1
   while (!R.bad && R.ld.kind >= 0 && R.issued - R.consumed < uint32_t(NSLOT)) {
-#pragma unroll 1
-    while (R.pf.kind >= 0 && R.pf_issued < R.issued + 1u + uint32_t(PF_AHEAD)) {
-      const uint8_t *s1, *s2;
-      uint32_t bytes;
-      cur_src(R.pf, warp, s1, s2, bytes, HD);
-      if (lane == 0 && R.pf_issued > R.issued) {  // the ring's own next unit needs no request
-        bulk_prefetch_l2(s1, bytes);
-        if (s2) bulk_prefetch_l2(s2, bytes);
-      }
-      ++R.pf_issued;
-      cur_next(R.pf, 1, warp, lane);
-    }
     const int sl = R.issued % NSLOT;
     const uint8_t *s1, *s2;
     uint32_t bytes;
@@ -720,7 +703,7 @@ __device__ __forceinline__ void ring_fill(Ring& R, int warp, int lane) {
       if (s2) bulk_g2s(dst + bytes, s2, bytes, bar);
     }
     ++R.issued;
-    cur_next(R.ld, 0, warp, lane);
+    cur_next(R.ld, warp, lane);
   }
 }
 
@@ -756,7 +739,7 @@ __device__ __forceinline__ void ring_release(Ring& R, int warp, int lane, bool w
   ring_fill<HD>(R, warp, lane);
 }
 
-// Resume waiting cursors and fill the ring (phase start).
+// Resume a waiting cursor and fill the ring (phase start).
 template <int HD>
 __device__ __noinline__ void ring_top_up() {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -764,7 +747,6 @@ __device__ __noinline__ void ring_top_up() {
   warp_sync();
   if (lane == 0) {
     if (s->ld.kind == CUR_WAIT) cur_normalize(&s->ld, warp);
-    if (s->pf.kind == CUR_WAIT) cur_normalize(&s->pf, warp);
   }
   warp_sync();
   Ring R;
@@ -1266,20 +1248,32 @@ __device__ __noinline__ void restage_scaled(const PD& d, int kbase, int klen) {
 // ---------------------------------------------------------------------------
 // int4 unit: codes [grp 4][half 2][lane 32][4 words], scales at +4096 ordered
 // [row % 8][grp][row / 8], zeros at +4224 [grp][row / 8] (nibble row % 8).
+// A warp copies its share of a unit into registers (w4_load) and hands the
+// ring slot back before the math (w4_math), so the slot refills while the
+// tensor cores work.
+struct W4Regs {
+  uint4 q[8];   // codes of this lane: [grp][half]
+  uint4 sc;     // scales of rows g, g + 8 for the four groups
+  uint4 zA, zB; // zero words [grp][row / 8]
+};
+__device__ __forceinline__ void w4_load(const uint8_t* slot, int g, int lane, W4Regs& r) {
+  const uint4* qw = reinterpret_cast<const uint4*>(slot) + lane;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r.q[i] = qw[i * 32];
+  r.sc = *reinterpret_cast<const uint4*>(slot + 4096 + g * 16);
+  r.zA = *reinterpret_cast<const uint4*>(slot + 4224);
+  r.zB = *reinterpret_cast<const uint4*>(slot + 4240);
+}
 // xl: this lane's x bytes (batch row g, + 16 t, + 2 koff); xsg: per-group sums
 // of x for the unit's first group, + 2 t.
 template <int NB>
-__device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint8_t* xl, int xrow_b, const float* xsg,
-                                        float (&acc)[NB][4], int B, int g, int lane) {
-  const uint4* qw = reinterpret_cast<const uint4*>(slot) + lane;
-  const uint4 sc = *reinterpret_cast<const uint4*>(slot + 4096 + g * 16);
-  const uint4 zA = *reinterpret_cast<const uint4*>(slot + 4224);
-  const uint4 zB = *reinterpret_cast<const uint4*>(slot + 4240);
+__device__ __forceinline__ void w4_math(const W4Regs& r, const uint8_t* xl, int xrow_b, const float* xsg,
+                                        float (&acc)[NB][4], int B, int g) {
   const int sh = 4 * g;
 #pragma unroll
   for (int grp = 0; grp < 4; ++grp) {
-    const uint4 w0 = qw[(grp * 2) * 32];
-    const uint4 w1 = qw[(grp * 2 + 1) * 32];
+    const uint4 w0 = r.q[grp * 2];
+    const uint4 w1 = r.q[grp * 2 + 1];
     uint4 xv[NB][4];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
@@ -1305,11 +1299,11 @@ __device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint8_t* xl, 
         mma_16816_f16(c[nb], a0, a1, a2, a3, (i & 1) ? x.z : x.x, (i & 1) ? x.w : x.y);
       }
     }
-    const uint32_t sw = u4_word(sc, grp);
+    const uint32_t sw = u4_word(r.sc, grp);
     const float sl = half_bits_to_f32(uint16_t(sw & 0xffffu));
     const float shi = half_bits_to_f32(uint16_t(sw >> 16)) * 0.0625f;
-    const uint32_t zl_w = u4_word(grp < 2 ? zA : zB, (grp * 2) & 3);
-    const uint32_t zh_w = u4_word(grp < 2 ? zA : zB, (grp * 2 + 1) & 3);
+    const uint32_t zl_w = u4_word(grp < 2 ? r.zA : r.zB, (grp * 2) & 3);
+    const uint32_t zh_w = u4_word(grp < 2 ? r.zA : r.zB, (grp * 2 + 1) & 3);
     // 1024 + z and 1024 + 16 z built in the fp32 significand (2^23 + m - (2^23 - 1024))
     const float zl = __uint_as_float(0x4B000000u | ((zl_w >> sh) & 15u)) - 8387584.f;
     const float zh = __uint_as_float(0x4B000000u | (((zh_w >> sh) & 15u) << 4)) - 8387584.f;
@@ -1323,12 +1317,26 @@ __device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint8_t* xl, 
     }
   }
 }
+template <int NB>
+__device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint8_t* xl, int xrow_b, const float* xsg,
+                                        float (&acc)[NB][4], int B, int g, int lane) {
+  W4Regs r;
+  w4_load(slot, g, lane, r);
+  w4_math<NB>(r, xl, xrow_b, xsg, acc, B, g);
+}
 
 // bf16 unit: A fragments [k-step 8][lane 32][4 words].
-template <int NB>
-__device__ __forceinline__ void bf_unit(const uint8_t* slot, const uint8_t* xl, int xrow_b, float (&acc)[NB][4],
-                                        int B, int g, int lane) {
+struct BfRegs {
+  uint4 a[8];
+};
+__device__ __forceinline__ void bf_load(const uint8_t* slot, int lane, BfRegs& r) {
   const uint4* aw = reinterpret_cast<const uint4*>(slot) + lane;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r.a[i] = aw[i * 32];
+}
+template <int NB>
+__device__ __forceinline__ void bf_math(const BfRegs& r, const uint8_t* xl, int xrow_b, float (&acc)[NB][4], int B,
+                                        int g) {
   uint4 xv[NB][4];
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb)
@@ -1338,13 +1346,20 @@ __device__ __forceinline__ void bf_unit(const uint8_t* slot, const uint8_t* xl, 
                                     : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint4 a = aw[i * 32];
+    const uint4& a = r.a[i];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       const uint4& x = xv[nb][i >> 1];
       mma_16816(acc[nb], a.x, a.y, a.z, a.w, (i & 1) ? x.z : x.x, (i & 1) ? x.w : x.y);
     }
   }
+}
+template <int NB>
+__device__ __forceinline__ void bf_unit(const uint8_t* slot, const uint8_t* xl, int xrow_b, float (&acc)[NB][4],
+                                        int B, int g, int lane) {
+  BfRegs r;
+  bf_load(slot, lane, r);
+  bf_math<NB>(r, xl, xrow_b, acc, B, g);
 }
 
 // ---------------------------------------------------------------------------
@@ -1542,11 +1557,25 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
       }
       const int koff = (sl * kps + kci) * kcw - kbase;
       const uint8_t* slot = ring_wait(R, warp, lane);
-      if (w4)
-        w4_unit<NB>(slot, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g, lane);
-      else
-        bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
-      ring_release<HD>(R, warp, lane, false);
+      if (NB > 1) {
+        // two batch tiles: the math reads the slot (registers are short)
+        if (w4)
+          w4_unit<NB>(slot, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g, lane);
+        else
+          bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
+        ring_release<HD>(R, warp, lane, false);
+      } else if (w4) {
+        // copy the unit to registers and hand the slot back before the math
+        W4Regs ur;
+        w4_load(slot, g, lane, ur);
+        ring_release<HD>(R, warp, lane, false);
+        w4_math<NB>(ur, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g);
+      } else {
+        BfRegs br;
+        bf_load(slot, lane, br);
+        ring_release<HD>(R, warp, lane, false);
+        bf_math<NB>(br, xl + koff * 2, xrow_b, acc, B, g);
+      }
       if (++kci == kps) {
         kci = 0;
         if (++rb == nrb) {
@@ -2181,14 +2210,13 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     }
   }
   __syncthreads();
-  // ring state: both cursors at the warp's first unit
+  // ring state: the cursor at the warp's first unit
   if (lane == 0) {
     Ring* s = ring_state(warp);
     *reinterpret_cast<uint4*>(s) = make_uint4(0u, 0u, 0u, 0u);
     s->ld.kind = CUR_WAIT;
     s->ld.p = begin;
     cur_normalize(&s->ld, warp);
-    s->pf = s->ld;
   }
   warp_sync();
 }
