@@ -833,18 +833,18 @@ __device__ __forceinline__ F8 f8(const float (&a)[8]) {
   return r;
 }
 
-// Sum of `ns` slabs (stride sstride floats) at p[0 .. 8), in slab order, loads
-// of up to four slabs in flight.
+// Sum of `ns` slabs (stride sstride floats) at p[0 .. 8), in slab order, the
+// loads of up to eight slabs in flight at once.
 __device__ __noinline__ F8 slab_sum8v(const float* p, size_t sstride, int ns) {
   F8 r;
   float* v = r.v;
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = 0.f;
 #pragma unroll 1
-  for (int s0 = 0; s0 < ns; s0 += 4) {
-    float4 a[4], b[4];
+  for (int s0 = 0; s0 < ns; s0 += 8) {
+    float4 a[8], b[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       a[i] = b[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (s0 + i < ns) {
         a[i] = ldcg4(p + (s0 + i) * sstride);
@@ -852,7 +852,7 @@ __device__ __noinline__ F8 slab_sum8v(const float* p, size_t sstride, int ns) {
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       if (s0 + i < ns) {
         v[0] += a[i].x;
         v[1] += a[i].y;
@@ -1028,15 +1028,15 @@ __device__ __noinline__ void stage_x(const PD& d, int kbase, int klen) {
     // pass 1: branch sums (and, for up to two chunks, residual and gains in flight together)
     if (two) {
       if (h0) {
-        slab_sum8(d.vpart + (size_t)b0 * d.vstride + k00, sstride, d.vns, v0);
         load8f(d.xres + (size_t)b0 * dm + k00, x0, false);
         load8f(d.gain + k00, g0, true);
       }
       if (h1) {
-        slab_sum8(d.vpart + (size_t)b1 * d.vstride + k01, sstride, d.vns, v1);
         load8f(d.xres + (size_t)b1 * dm + k01, x1, false);
         load8f(d.gain + k01, g1, true);
       }
+      if (h0) slab_sum8(d.vpart + (size_t)b0 * d.vstride + k00, sstride, d.vns, v0);
+      if (h1) slab_sum8(d.vpart + (size_t)b1 * d.vstride + k01, sstride, d.vns, v1);
       float sq0 = 0.f, sq1 = 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -1451,52 +1451,47 @@ __device__ __forceinline__ void seg_done(const PD& d, int seg, float (&acc)[NB][
   }
 }
 
-// Segments of this CTA split between warps: sum the pieces in warp order.
+// Segments of this CTA split between warps: the warp holding a segment's last
+// unit sums its pieces in warp order and emits the rows.
 template <int NB>
 __device__ __noinline__ void cta_combine(const PD& d, int a, int b) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kps = d.g.kps, B = lc().B;
+  int wa, wb;
+  warp_range(a, b, warp, wa, wb);
+  if (wa >= wb || wa % kps == 0) return;  // my first segment starts with me: no piece before mine
+  const int S = wa / kps;
+  if ((S + 1) * kps > wb) return;          // it goes on past my range: a later warp finishes it
+  int w0 = warp;
+#pragma unroll 1
+  while (w0 > 0) {
+    int pa, pb;
+    warp_range(a, b, w0 - 1, pa, pb);
+    if (pb <= S * kps) break;
+    --w0;
+  }
   const float* wsp = sm_at<float>(sm_wsp(NB));
-  int count = 0, last = -1;
-#pragma unroll 1
-  for (int w = 0; w < NW; ++w) {
-    int wa, wb;
-    warp_range(a, b, w, wa, wb);
-    if (wa >= wb) continue;
-    const int fs = wa / kps, ls = (wb - 1) / kps;
-#pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-      const int S = which ? ls : fs;
-      if (which && ls == fs) break;
-      const bool complete = (S * kps >= wa) && (S * kps + kps <= wb);
-      if (complete || S == last) continue;
-      if (count % NW == warp) {
-        float sum[NB][4];
+  float sum[NB][4];
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) sum[nb][0] = sum[nb][1] = sum[nb][2] = sum[nb][3] = 0.f;
+  for (int nb = 0; nb < NB; ++nb) sum[nb][0] = sum[nb][1] = sum[nb][2] = sum[nb][3] = 0.f;
 #pragma unroll 1
-        for (int w2 = 0; w2 < NW; ++w2) {
-          int a2, b2;
-          warp_range(a, b, w2, a2, b2);
-          if (a2 >= b2 || S * kps >= b2 || S * kps + kps <= a2) continue;
-          const int sl = (S == a2 / kps) ? 0 : 1;
-          const float* q = wsp + w2 * (2 * 32 * 4 * NB) + sl * (32 * 4 * NB) + lane * 4 * NB;
+  for (int w2 = w0; w2 <= warp; ++w2) {
+    int a2, b2;
+    warp_range(a, b, w2, a2, b2);
+    if (a2 >= b2) continue;
+    const int sl = (S == a2 / kps) ? 0 : 1;
+    const float* q = wsp + w2 * (2 * 32 * 4 * NB) + sl * (32 * 4 * NB) + lane * 4 * NB;
 #pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            const float4 f = reinterpret_cast<const float4*>(q)[nb];
-            sum[nb][0] += f.x;
-            sum[nb][1] += f.y;
-            sum[nb][2] += f.z;
-            sum[nb][3] += f.w;
-          }
-        }
-        const int s = S / d.g.nrb;
-        emit_rows<NB>(d, s, S - s * d.g.nrb, acc_of<NB>(sum), B, lane);
-      }
-      ++count;
-      last = S;
+    for (int nb = 0; nb < NB; ++nb) {
+      const float4 f = reinterpret_cast<const float4*>(q)[nb];
+      sum[nb][0] += f.x;
+      sum[nb][1] += f.y;
+      sum[nb][2] += f.z;
+      sum[nb][3] += f.w;
     }
   }
+  const int s = S / d.g.nrb;
+  emit_rows<NB>(d, s, S - s * d.g.nrb, acc_of<NB>(sum), B, lane);
 }
 
 template <int NB, int HD>
@@ -1671,18 +1666,23 @@ __device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
         v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll 1
-      for (int sl = 0; sl < d.qns; ++sl) {
-        float4 t4[JU];
+      for (int sl = 0; sl < d.qns; sl += 2) {  // two slabs' loads in flight together
+        float4 t4[2][JU];
 #pragma unroll
-        for (int j = 0; j < JU; ++j)
-          t4[j] = (c0 + j * NT < total4) ? ldcg4(ybase + sl * sstride + rows[j]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = 0; e < 2; ++e)
 #pragma unroll
-        for (int j = 0; j < JU; ++j) {
-          v[j].x += t4[j].x;
-          v[j].y += t4[j].y;
-          v[j].z += t4[j].z;
-          v[j].w += t4[j].w;
-        }
+          for (int j = 0; j < JU; ++j)
+            t4[e][j] = (c0 + j * NT < total4 && sl + e < d.qns) ? ldcg4(ybase + (sl + e) * sstride + rows[j])
+                                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+          for (int j = 0; j < JU; ++j) {
+            v[j].x += t4[e][j].x;
+            v[j].y += t4[e][j].y;
+            v[j].z += t4[e][j].z;
+            v[j].w += t4[e][j].w;
+          }
       }
 #pragma unroll
       for (int j = 0; j < JU; ++j) {
@@ -1832,13 +1832,14 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
   cbar();
   if (!flags()[1]) return;
   __threadfence();
-  // warp h combines query head h over the pieces c0..c1 (one piece per lane
-  // for the max and the denominators; shuffled weights for the outputs)
+  // warp h combines query head h over the pieces c0..c1: one piece per lane
+  // for the max and the denominators, then the outputs (four dims per lane)
+  // with the loads of eight pieces in flight.  CTA c0 filed its piece in its
+  // second slot (the segment is its last), the others in their first.
   if (warp < GQ) {
     const int h = warp;
     auto piece_of = [&](int c) {
-      const int sl = (st[seg] < rstart(total, nca, c)) ? 0 : 1;
-      return L.apart + ((size_t)c * 2 + sl) * ATT_PW + h * (HD + 2);
+      return L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
     };
     float M = -INFINITY;
 #pragma unroll 1
@@ -1861,11 +1862,20 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
       }
       const int n = min(32, c1 - cb + 1);
 #pragma unroll 1
-      for (int i = 0; i < n; ++i) {
-        const float w = __shfl_sync(0xffffffffu, ev, i);
-        const float* pc = piece_of(cb + i) + lane * DPL;
+      for (int i0 = 0; i0 < n; i0 += 8) {
+        float ov[8][DPL];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, __ldcg(pc + e), acc[e]);
+        for (int j = 0; j < 8; ++j) {
+          const float* pc = piece_of(min(cb + i0 + j, c1)) + lane * DPL;  // clamped: never past the last piece
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) ov[j][e] = (i0 + j < n) ? __ldcg(pc + e) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float w = __shfl_sync(0xffffffffu, ev, (i0 + j) & 31);
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, ov[j][e], acc[e]);
+        }
       }
     }
 #pragma unroll
