@@ -84,6 +84,8 @@ __host__ __device__ inline int choose_kps(int nkc, int kcw, int B, int nb) {
 // SM (an estimate: ~12 TB/s of L2 against 6.5 TB/s of HBM shared by the SMs).
 constexpr double L2_VS_SM_HBM = 270.0;
 inline Geo gemv_geo(long long n, long long k, int kcw, int B, int nb, int nc, int readers) {
+  // a consumer reading the whole vector loads at most four slabs per round trip
+  const int ns_cap = readers > 1 ? 4 : NS_MAX;
   Geo g;
   g.nrb = int((n + RB - 1) / RB);
   g.nkc = int(k / kcw);
@@ -94,7 +96,7 @@ inline Geo gemv_geo(long long n, long long k, int kcw, int B, int nb, int nc, in
   const int ub = kcw == W4_KC ? W4_UNIT : BF_UNIT;
   const double slab_cost = double(readers) * B * double(n) * 4.0 / L2_VS_SM_HBM;
   double best = 0.0;
-  for (int ns = ns0; ns <= g.nkc && (ns == ns0 || ns <= NS_MAX); ++ns) {
+  for (int ns = ns0; ns <= g.nkc && (ns == ns0 || ns <= ns_cap); ++ns) {
     if (g.nkc % ns) continue;
     const int kps = g.nkc / ns;
     if (!(ns == 1 ? x_fits((long long)g.nkc * kcw, B, nb) : x_fits(2LL * kps * kcw, B, nb))) continue;
@@ -481,9 +483,29 @@ __device__ __forceinline__ void warp_range(int a, int b, int w, int& wa, int& wb
   wa = a + (b - a) * w / NW;
   wb = a + (b - a) * (w + 1) / NW;
 }
+// Attention work split over CTAs.  When every segment (sequence, KV head)
+// has the same number of 128-key units n (the usual case: equal lengths),
+// each segment gets m = nc / segments CTAs of its own (at most n of them) and
+// no CTA spans two segments; otherwise the units are split contiguously.
+// amode / am / ameff per layer type live in flags()[4 + 3 type ..].
 __device__ __forceinline__ void attn_cta_range(int type, int cta, int& a, int& b, int& nca) {
   const LC& L = lc();
-  const int total = sst(type)[L.B * L.nkv];
+  const int* st = sst(type);
+  const int S = L.B * L.nkv;
+  const int total = st[S];
+  const int* am = flags() + 4 + 3 * type;
+  if (am[0]) {
+    const int m = am[1], meff = am[2], n = st[1] - st[0];
+    const int s = cta / m, j = cta - s * m;
+    nca = S * m;
+    if (s < S && j < meff) {
+      a = st[s] + n * j / meff;
+      b = st[s] + n * (j + 1) / meff;
+    } else {
+      a = b = 0;
+    }
+    return;
+  }
   nca = total < L.nc ? total : L.nc;
   if (nca > 0 && cta < nca) {
     a = int(rstart(total, nca, cta));
@@ -491,6 +513,19 @@ __device__ __forceinline__ void attn_cta_range(int type, int cta, int& a, int& b
   } else {
     a = b = 0;
   }
+}
+// CTAs c0 .. c1 holding the pieces of segment seg.
+__device__ __forceinline__ void attn_seg_ctas(int type, int seg, int nca, int& c0, int& c1) {
+  const int* st = sst(type);
+  const int* am = flags() + 4 + 3 * type;
+  if (am[0]) {
+    c0 = seg * am[1];
+    c1 = c0 + am[2] - 1;
+    return;
+  }
+  const int total = st[lc().B * lc().nkv];
+  c0 = owner(total, nca, st[seg]);
+  c1 = owner(total, nca, st[seg + 1] - 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -798,12 +833,11 @@ __device__ __noinline__ bool grid_wait(uint32_t target) {
   cbar();
   return flags()[0] != 0;
 }
+// The CTA barrier orders every thread's writes of the phase before thread
+// 0's release, and the release makes them visible to the acquiring CTAs.
 __device__ __forceinline__ void grid_arrive() {
   cbar();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    red_release_add(lc().ctl, 1u);
-  }
+  if (threadIdx.x == 0) red_release_add(lc().ctl, 1u);
 }
 
 // Deterministic per-batch-row totals of per-warp partial sums wsum[warp][b].
@@ -864,6 +898,48 @@ __device__ __noinline__ F8 slab_sum8v(const float* p, size_t sstride, int ns) {
         v[7] += b[i].w;
       }
     }
+  }
+  return r;
+}
+// The same for two chunks at once (p1 used when has1), four slabs of each in
+// flight per round.
+struct F16v {
+  float v[16];
+};
+__device__ __noinline__ F16v slab_sum8x2(const float* p0, const float* p1, bool has1, size_t sstride, int ns) {
+  F16v r;
+  float* v = r.v;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = 0.f;
+#pragma unroll 1
+  for (int s0 = 0; s0 < ns; s0 += 4) {
+    float4 a[2][4], b[2][4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[c][i] = b[c][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s0 + i < ns && (c == 0 || has1)) {
+          const float* p = (c ? p1 : p0) + (s0 + i) * sstride;
+          a[c][i] = ldcg4(p);
+          b[c][i] = ldcg4(p + 4);
+        }
+      }
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (s0 + i < ns) {
+          v[8 * c + 0] += a[c][i].x;
+          v[8 * c + 1] += a[c][i].y;
+          v[8 * c + 2] += a[c][i].z;
+          v[8 * c + 3] += a[c][i].w;
+          v[8 * c + 4] += b[c][i].x;
+          v[8 * c + 5] += b[c][i].y;
+          v[8 * c + 6] += b[c][i].z;
+          v[8 * c + 7] += b[c][i].w;
+        }
+      }
   }
   return r;
 }
@@ -1035,8 +1111,15 @@ __device__ __noinline__ void stage_x(const PD& d, int kbase, int klen) {
         load8f(d.xres + (size_t)b1 * dm + k01, x1, false);
         load8f(d.gain + k01, g1, true);
       }
-      if (h0) slab_sum8(d.vpart + (size_t)b0 * d.vstride + k00, sstride, d.vns, v0);
-      if (h1) slab_sum8(d.vpart + (size_t)b1 * d.vstride + k01, sstride, d.vns, v1);
+      if (h0) {
+        const F16v r = slab_sum8x2(d.vpart + (size_t)b0 * d.vstride + k00, d.vpart + (size_t)b1 * d.vstride + k01,
+                                   h1, sstride, d.vns);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v0[i] = r.v[i];
+          v1[i] = r.v[8 + i];
+        }
+      }
       float sq0 = 0.f, sq1 = 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -1820,18 +1903,16 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
     }
   }
   if (!split) return;
-  __threadfence();
   cbar();
-  const int total = st[L.B * L.nkv];
-  const int c0 = owner(total, nca, st[seg]);
-  const int c1 = owner(total, nca, st[seg + 1] - 1);
+  int c0, c1;
+  attn_seg_ctas(d.type, seg, nca, c0, c1);
   if (tid == 0) {
-    const uint32_t old = atomicAdd(L.seg_ctr + seg, 1u);
+    // release this CTA's piece, acquire the others' (last arriver)
+    const uint32_t old = atom_add_acqrel(L.seg_ctr + seg, 1u);
     flags()[1] = (int(old) == c1 - c0) ? 1 : 0;
   }
   cbar();
   if (!flags()[1]) return;
-  __threadfence();
   // warp h combines query head h over the pieces c0..c1: one piece per lane
   // for the max and the denominators, then the outputs (four dims per lane)
   // with the loads of eight pieces in flight.  CTA c0 filed its piece in its
@@ -2094,10 +2175,8 @@ __device__ __noinline__ void argmax_phase(const PD& d) {
     cbar();
   }
   if (tid == 0) {
-    __threadfence();
-    const uint32_t old = atomicAdd(L.ctl + 3, 1u);
+    const uint32_t old = atom_add_acqrel(L.ctl + 3, 1u);
     if (int(old) == L.nc - 1) {
-      __threadfence();
 #pragma unroll 1
       for (int bq = 0; bq < B; ++bq) {
         float bb = -INFINITY;
@@ -2213,11 +2292,19 @@ __device__ __noinline__ void setup(const EngineParams& P) {
   if (P.mode != MODE_GEMV && tid < 2) {
     int* st = sst(tid);
     st[0] = 0;
+    bool equal = true;
+    const int S = B * P.nkv;
 #pragma unroll 1
-    for (int s = 0; s < B * P.nkv; ++s) {
+    for (int s = 0; s < S; ++s) {
       const int Lk = Lb(tid)[s / P.nkv];
       st[s + 1] = st[s] + (Lk + ATT_CTA_KEYS - 1) / ATT_CTA_KEYS;
+      equal &= (st[s + 1] - st[s]) == st[1];
     }
+    int* am = flags() + 4 + 3 * tid;
+    const int n = st[1];
+    am[0] = (equal && n > 0 && S <= P.nc) ? 1 : 0;
+    am[1] = S > 0 ? P.nc / S : 0;
+    am[2] = min(am[1], n);
   }
   __syncthreads();
   // ring state: the cursor at the warp's first unit
