@@ -125,47 +125,95 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the CPU baseline: the oracle, as it stands, on a bounded sample
 # ---------------------------------------------------------------------------
-def cpu_baseline(cfg, layers_sample: int = 2):
-    """Time the float64 oracle on `layers_sample` layers of one decode step of
-    the same model at ctx 4096, plus the lm_head, and scale to a full token."""
-    import numpy as np
-    import torch
+SAMPLE_ROWS = 256
+
+
+def oracle_config_of(cfg):
     from oracle import model as om
-    from w4_weight_only_b200 import synth
-    sys.path.insert(0, str(ROOT / "tests"))
-    from helpers import oracle_config, np32, np64
-    ocfg = oracle_config(cfg)
-    layers = {}
-    for l in range(layers_sample):
-        raw = synth.layer_float(cfg, SEED, l, "cpu")
-        layers[l] = om.OracleLayer.from_float({k: np32(v) for k, v in raw.items()})
-    emb, head, fin = synth.embed_head(cfg, SEED, "cpu")
-    m = om.OracleModel(ocfg, np64(emb), np64(head), np64(fin), lambda l: layers[l], cache_dense=False)
-    kv = om.OracleKV(om.OracleConfig(**{**ocfg.__dict__, "n_layers": layers_sample,
-                                        "full_layers": ocfg.full_layers[:layers_sample]}), 1, CTX + 1)
-    for l in range(layers_sample):
-        k, v = synth.kv_rows(SEED, l, 0, cfg.n_kv_heads, CTX, cfg.head_dim, "cpu")
-        kv.fill(l, 0, 0, np64(k), np64(v))
-    x = np64(emb[1])
-    t0 = time.perf_counter()
-    for l in range(layers_sample):
-        x = om.layer_forward(ocfg, m.layer(l), l, x, kv, 0, CTX)
-    t_layers = time.perf_counter() - t0
-    t1 = time.perf_counter()
-    om.head(m, x)
-    t_head = time.perf_counter() - t1
-    per_token = t_layers / layers_sample * cfg.n_layers + t_head
-    threads = torch.get_num_threads()
+    return om.OracleConfig(d_model=cfg.d_model, n_layers=cfg.n_layers, n_heads=cfg.n_heads,
+                           n_kv_heads=cfg.n_kv_heads, head_dim=cfg.head_dim, ffn=cfg.ffn, vocab=cfg.vocab,
+                           window=cfg.window, full_layers=list(cfg.full_layers), rope_theta=cfg.rope_theta,
+                           yarn_factor=cfg.yarn_factor, yarn_orig_ctx=cfg.yarn_orig_ctx,
+                           beta_fast=cfg.yarn_beta_fast, beta_slow=cfg.yarn_beta_slow, eps=cfg.eps,
+                           group=cfg.group, final_norm=cfg.final_norm)
+
+
+class OracleSample:
+    """A bounded sample of one decode token through the float64 oracle: the
+    first SAMPLE_ROWS rows of each of a layer's four int4 GEMVs (dequantize +
+    matvec, the oracle's W4Matrix) and of the lm_head, one full-layer QK-prep +
+    GQA attention over 4096 cached keys; the per-token time scales each GEMV by
+    its rows / SAMPLE_ROWS and the layer by the layer count."""
+
+    def __init__(self, cfg):
+        import numpy as np
+        from oracle import model as om
+        from w4_weight_only_b200 import synth
+        self.cfg, self.om, self.np = cfg, om, np
+        self.ocfg = oracle_config_of(cfg)
+        d, qd, kvd, f = cfg.d_model, cfg.q_dim, cfg.kv_dim, cfg.ffn
+        shapes = {"qkv": (qd + 2 * kvd, d), "o": (d, qd), "gate_up": (2 * f, d), "down": (d, f)}
+        r = SAMPLE_ROWS
+        self.mats, self.xs, self.scale = {}, {}, {}
+        for name, (n, k) in shapes.items():
+            W = synth.normal((r, k), "cpu", 0.02, 0.0, SEED, "oracle_sample", name).numpy()
+            self.mats[name] = om.W4Matrix.from_float(W, cfg.group)
+            self.xs[name] = synth.normal((k,), "cpu", 1.0, 0.0, SEED, "oracle_sample_x", name).double().numpy()
+            self.scale[name] = n / r
+        self.head = synth.normal((r, d), "cpu", 0.02, 0.0, SEED, "oracle_sample", "head").to(
+            __import__("torch").bfloat16).double().numpy()
+        self.head_scale = cfg.vocab / r
+        self.x = self.xs["qkv"]
+        # one full layer's attention inputs at ctx 4096
+        kcfg = om.OracleConfig(**{**self.ocfg.__dict__, "n_layers": 1, "full_layers": [True]})
+        self.kv = om.OracleKV(kcfg, 1, CTX + 1)
+        k, v = synth.kv_rows(SEED, 0, 0, cfg.n_kv_heads, CTX, cfg.head_dim, "cpu")
+        self.kv.fill(0, 0, 0, k.double().numpy(), v.double().numpy())
+        self.qr = synth.normal((qd,), "cpu", 1.0, 0.0, SEED, "oracle_sample_q").double().numpy()
+        self.kr = synth.normal((kvd,), "cpu", 1.0, 0.0, SEED, "oracle_sample_k").double().numpy()
+        self.qg = synth.normal((qd,), "cpu", 0.1, 1.0, SEED, "oracle_sample_qg").double().numpy()
+        self.kg = synth.normal((kvd,), "cpu", 0.1, 1.0, SEED, "oracle_sample_kg").double().numpy()
+
+    def step(self) -> float:
+        """Seconds of one token, estimated from one pass over the sample."""
+        om, cfg = self.om, self.cfg
+        t_layer = 0.0
+        for name, W in self.mats.items():
+            t0 = time.perf_counter()
+            W.matvec(self.xs[name])
+            t_layer += (time.perf_counter() - t0) * self.scale[name]
+        t0 = time.perf_counter()
+        q, k = om.qk_prep(self.ocfg, self.qr, self.kr, self.qg, self.kg, CTX, True)
+        om.gqa_decode(self.ocfg, q, self.kv.K[0][0], self.kv.V[0][0], CTX - 1, True)
+        t_layer += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        _ = self.head @ self.x[: cfg.d_model]
+        t_head = (time.perf_counter() - t0) * self.head_scale
+        return cfg.n_layers * t_layer + t_head
+
+    def describe(self, steps: int) -> str:
+        return (f"{steps} passes over a sample of one ctx-{CTX} token: the first {SAMPLE_ROWS} rows of each "
+                f"int4 GEMV (dequantize + float64 matvec) and of the lm_head, one layer's QK-prep + GQA "
+                f"attention over {CTX} keys; scaled by rows and by {self.cfg.n_layers} layers")
+
+
+def oracle_threads() -> int:
     try:
         import threadpoolctl
         info = threadpoolctl.threadpool_info()
-        threads = max([i.get("num_threads", 1) for i in info] + [1])
+        return max([i.get("num_threads", 1) for i in info] + [1])
     except Exception:
-        pass
-    return {"value": 1.0 / per_token, "unit": "tok/s", "cores": threads, "kind": "oracle",
-            "sample": f"{layers_sample} of {cfg.n_layers} layers of one ctx-{CTX} decode step (dequantize + "
-                      f"float64 matvecs + attention) plus the lm_head, timed, scaled to one token; "
-                      f"host has {len(os.sched_getaffinity(0))} cores"}
+        import torch
+        return torch.get_num_threads()
+
+
+def cpu_baseline(cfg, steps: int = 3):
+    S = OracleSample(cfg)
+    S.step()
+    ts = [S.step() for _ in range(steps)]
+    per_token = statistics.median(ts)
+    return {"value": 1.0 / per_token, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": S.describe(steps) + f"; host has {len(os.sched_getaffinity(0))} cores"}
 
 
 # ---------------------------------------------------------------------------
@@ -174,17 +222,41 @@ def run_reference(args, rank, world):
     from w4_weight_only_b200 import config as wc
     if rank != 0:
         return
-    cfg = wc.olmo3_32b()
-    base = cpu_baseline(cfg)
-    v = base["value"]
+    cfg = wc.olmo3_32b(args.layers)
+    S = OracleSample(cfg)
+    for _ in range(args.warmup):
+        S.step()
+    ts = [S.step() for _ in range(args.steps)]
+    per_token = sum(ts) / len(ts)
+    v = 1.0 / per_token
+    base = {"value": v, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": S.describe(args.steps) + f"; host has {len(os.sched_getaffinity(0))} cores"}
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / v, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "OLMo-3-32B-shaped int4 decode, 64 layers, batch 1, ctx 4096", "batch": 1,
-                       "ctx": CTX},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * per_token,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"OLMo-3-32B-shaped int4 (g128, fp16 scale, int4 zero) decode, "
+                                   f"{cfg.n_layers} layers, batch 1, ctx {CTX}, greedy",
+                       "batch": 1, "ctx": CTX, "layers": cfg.n_layers, "parallelism": "host cores"},
             "cpu_baseline": base,
             "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of every rank's value (device time of the timed region);
+    every rank takes the same collective step."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tok_s(ms_max: float, steps: int, world: int) -> float:
+    """Whole-job throughput: every replica decodes `steps` tokens; the job
+    takes as long as its slowest rank."""
+    return world * steps / (ms_max / 1000.0)
 
 
 def main():
@@ -270,12 +342,9 @@ def main():
     clk = clocks.stop()
     api.check(ws)
     ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     ms_step = ms_max / args.steps
-    tok_s = world * args.steps / (ms_max / 1000.0)
+    tok_s = job_tok_s(ms_max, args.steps, world)
 
     # roofline of the (only) kernel: algorithmic bytes per launch / its device time
     bytes_avg = sum(step_bytes(cfg, CTX + i) for i in range(args.warmup, total)) / args.steps
@@ -313,10 +382,8 @@ def main():
             h_tok[0] = int(h_next[0])
         t1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * n_e2e / (float(te.item()) / 1000.0), "unit": "tok/s",
+        te = max_over_ranks(t0.elapsed_time(t1), world, dev)
+        e2e = {"value": job_tok_s(te, n_e2e, world), "unit": "tok/s",
                "h2d_bytes_per_step": 8, "d2h_bytes_per_step": 4}
 
     base = None
@@ -329,7 +396,7 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": round(tok_s, 2), "unit": "tok/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
                 "data": "synthetic",
                 "config": {"workload": f"OLMo-3-32B-shaped int4 (g128, fp16 scale, int4 zero) decode, "
                                        f"{cfg.n_layers} layers, batch 1, ctx {CTX}..{CTX + total}, greedy",
