@@ -37,6 +37,22 @@ SEED = 3
 NOMINAL_HBM_GBS = 8000.0
 
 
+# DRAM traffic of the engine from ncu (profiles/w4a_engine_decode_4layer_full.md):
+# 4- and 8-layer launches of the benchmark model at ctx 4096 give the bytes per
+# layer and the fixed part; valid only for the engine source they were taken on.
+TRAFFIC_ENGINE_SHA = "9784c0ffe744364c"
+TRAFFIC_FIXED = 1.0380e9
+TRAFFIC_PER_LAYER = 0.27187e9
+
+
+def measured_traffic(n_layers: int):
+    import hashlib
+    src = ROOT / "w4_weight_only_b200" / "csrc" / "engine.cuh"
+    if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:16] != TRAFFIC_ENGINE_SHA:
+        return None
+    return int(TRAFFIC_FIXED + n_layers * TRAFFIC_PER_LAYER)
+
+
 def measured_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -351,7 +367,7 @@ def main():
     peak, peak_src = measured_peaks()
     achieved = bytes_avg / (ms / args.steps / 1000.0) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_src,
+            "frac": round(achieved / peak, 4), "traffic": measured_traffic(cfg.n_layers), "peak_source": peak_src,
             "bytes_per_launch": int(bytes_avg), "frac_of_8000_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
             "kernel": "w4a_engine_kernel<1,128> (one launch per token)"}
 
