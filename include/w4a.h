@@ -179,6 +179,25 @@ W4A_API int w4a_gemv_workspace_bytes(const W4ATensor* W, int batch, size_t* byte
 W4A_API int w4a_gemv(const W4ATensor* W, const uint16_t* x, int batch, void* out, int epilogue,
              float* aux, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- GEMV without a caller workspace --------------------------------------
+ * This entry point is the library's own addition; the pages have no
+ * counterpart.  It computes exactly what w4a_gemv computes (same kernel, same
+ * split, bit-identical results) but takes no workspace and allocates nothing:
+ * its scratch is a fixed array of W4A_NOALLOC_SCRATCH_BYTES inside the
+ * library, one per device, whose address is looked up once per device.
+ *  - Returns W4A_ERR_WORKSPACE when the shape and batch need more scratch
+ *    than that (w4a_gemv_workspace_bytes tells how much they need).
+ *  - The scratch is shared by every call on a device: calls that overlap in
+ *    time (two streams, two host threads) race on it and give undefined
+ *    results; serialize them.
+ *  - The array keeps the last call's contents; each call first clears the
+ *    part that must start at zero (the control words: grid barrier counters
+ *    and the device error word) on `stream`.
+ * Arguments, layouts and the other errors are as for w4a_gemv. */
+#define W4A_NOALLOC_SCRATCH_BYTES 4194304
+W4A_API int w4a_gemv_noalloc(const W4ATensor* W, const uint16_t* x, int batch, void* out, int epilogue,
+                     float* aux, void* stream);
+
 /* ---- attention ----------------------------------------------------------- */
 
 W4A_API int w4a_attn_workspace_bytes(int batch, int n_heads, int n_kv_heads, int head_dim, size_t* bytes);

@@ -15,6 +15,7 @@ OK, ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR
 F32, BF16 = 0, 1
 LAYOUT_CANONICAL, LAYOUT_TILED = 0, 1
 EPI_NONE, EPI_SUMSQ, EPI_SILU_MUL = 0, 1, 2
+NOALLOC_SCRATCH_BYTES = 4194304
 
 ERROR_NAMES = {OK: "OK", ERR_ARG: "ERR_ARG", ERR_SHAPE: "ERR_SHAPE", ERR_ALIGN: "ERR_ALIGN",
                ERR_UNSUPPORTED: "ERR_UNSUPPORTED", ERR_CUDA: "ERR_CUDA", ERR_WORKSPACE: "ERR_WORKSPACE",
@@ -71,6 +72,7 @@ PROTOTYPES = {
     "w4a_tile_bf16": (_I, [_P, _I64, _I64, _P, _SZ, _P]),
     "w4a_gemv_workspace_bytes": (_I, [C.POINTER(W4ATensor), _I, _SZP]),
     "w4a_gemv": (_I, [C.POINTER(W4ATensor), _P, _I, _P, _I, _P, _P, _SZ, _P]),
+    "w4a_gemv_noalloc": (_I, [C.POINTER(W4ATensor), _P, _I, _P, _I, _P, _P]),
     "w4a_attn_workspace_bytes": (_I, [_I, _I, _I, _I, _SZP]),
     "w4a_attn_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "w4a_qk_prep": (_I, [C.POINTER(W4AConfig), _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P]),

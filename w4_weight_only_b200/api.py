@@ -158,6 +158,26 @@ def gemv(lin: W4Linear, x: torch.Tensor, epilogue: int = _abi.EPI_NONE, ws: Opti
     return (out, aux) if epilogue == _abi.EPI_SUMSQ else out
 
 
+def gemv_noalloc(lin: W4Linear, x: torch.Tensor, epilogue: int = _abi.EPI_NONE,
+                 out: Optional[torch.Tensor] = None, aux: Optional[torch.Tensor] = None):
+    """As gemv(), with the library's fixed scratch instead of a workspace
+    (w4a_gemv_noalloc): calls must not overlap in time."""
+    _need(x, torch.bfloat16, "x")
+    B = x.shape[0]
+    if x.shape[1] != lin.k:
+        raise ValueError("x has the wrong width")
+    if out is None:
+        if epilogue == _abi.EPI_SILU_MUL:
+            out = torch.empty((B, lin.n // 2), dtype=torch.bfloat16, device=x.device)
+        else:
+            out = torch.empty((B, lin.n), dtype=torch.float32, device=x.device)
+    if epilogue == _abi.EPI_SUMSQ and aux is None:
+        aux = torch.empty((lin.n // 16, B), dtype=torch.float32, device=x.device)
+    t = lin.tensor()
+    call("w4a_gemv_noalloc", C.byref(t), _p(x), B, _p(out), epilogue, _p(aux), _stream())
+    return (out, aux) if epilogue == _abi.EPI_SUMSQ else out
+
+
 # ---------------------------------------------------------------------------
 # attention
 # ---------------------------------------------------------------------------

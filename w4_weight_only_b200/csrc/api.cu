@@ -506,6 +506,41 @@ int w4a_gemv(const W4ATensor* W, const uint16_t* x, int batch, void* out, int ep
   return launch_engine(P, nb_for(batch), 128, S(stream));
 }
 
+// ---- GEMV with library-owned scratch -------------------------------------------------
+// A fixed scratch array per device (zero at module load) replaces the caller's
+// workspace; its device address is looked up once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A_NOALLOC_SCRATCH_BYTES];
+static void* g_noalloc_ptr[64];
+static std::mutex g_noalloc_mu;
+
+int w4a_gemv_noalloc(const W4ATensor* W, const uint16_t* x, int batch, void* out, int epilogue, float* aux,
+                     void* stream) {
+  int rc = check_tensor(W);
+  if (rc) return rc;
+  size_t need = 0;
+  rc = w4a_gemv_workspace_bytes(W, batch, &need);
+  if (rc) return rc;
+  if (need > (size_t)W4A_NOALLOC_SCRATCH_BYTES)
+    return fail(W4A_ERR_WORKSPACE, "%lld x %lld at batch %d needs %zu bytes of scratch (fixed scratch: %d)",
+                (long long)W->n, (long long)W->k, batch, need, W4A_NOALLOC_SCRATCH_BYTES);
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(W4A_ERR_UNSUPPORTED, "device index %d", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));  // with `dev` current
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  // the control words (barrier counters, error word) must start at zero
+  CK(cudaMemsetAsync(scratch, 0, 256, S(stream)));
+  return w4a_gemv(W, x, batch, out, epilogue, aux, scratch, W4A_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 // ---- attention ---------------------------------------------------------------------
 int w4a_attn_workspace_bytes(int batch, int n_heads, int n_kv_heads, int head_dim, size_t* bytes) {
   if (!bytes) return fail(W4A_ERR_ARG, "null output");
