@@ -117,7 +117,7 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
     if (!(di->attr_set & bit)) {
       CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
       int occ = 0;
-      CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NT, smem));
+      CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NTH, smem));
       if (occ < 1) return fail(W4A_ERR_UNSUPPORTED, "engine kernel does not fit on an SM");
       di->attr_set |= bit;
     }
@@ -137,7 +137,7 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
     P.phase_end = (p0 + chunk < end) ? p0 + chunk : end;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P.nc);
-    cfg.blockDim = dim3(NT);
+    cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

@@ -154,7 +154,9 @@ struct LC {
   float eps, mscale0, mscale1;
   int cur_phase;
   int scaled;  // some x row of this phase is range-scaled
-  int final_norm, pad0, pad1;
+  int final_norm;
+  int stop;  // the math warps have left the phase loop
+  int pad1;
   uint32_t* ctl;
   uint32_t* seg_ctr;
   float* apart;
@@ -186,9 +188,9 @@ struct alignas(16) Cursor {
   int x0, x1, x2, x3, x4, x5, x6, pad_;
 };
 struct alignas(16) Ring {
-  uint32_t consumed, issued, pad_;
-  int bad;    // a wait of this warp timed out: stop waiting and issuing
-  Cursor ld;  // next unit to copy into the ring
+  uint32_t consumed, pad0, pad1;  // units the math warp has taken
+  int bad;    // a wait of the math warp timed out: stop waiting
+  Cursor ld;  // the copy warp's cursor for this ring (its slow path)
 };
 static_assert(sizeof(Cursor) == 64 && sizeof(Ring) == 80, "ring state layout");
 
@@ -199,7 +201,8 @@ constexpr int SM_RING = 0;
 constexpr int SM_MBAR = SM_RING + NW * NSLOT * SLOT_BYTES;
 constexpr int PD_SLOTS = 4;                        // descriptor slots (phase p in slot p % 4)
 constexpr int PD_LEAD = 2;                         // descriptor p is copied at the start of phase p - 2
-constexpr int SM_PDBAR = SM_MBAR + NW * NSLOT * 8;
+constexpr int SM_EBAR = SM_MBAR + NW * NSLOT * 8;  // slot free again [NW][NSLOT]
+constexpr int SM_PDBAR = SM_EBAR + NW * NSLOT * 8;
 constexpr int SM_XS = ((SM_PDBAR + PD_SLOTS * 8 + 127) / 128) * 128;
 constexpr int X_REGION = xs_cap(1) + XSUM_BYTES + wsp_bytes(1);
 static_assert(xs_cap(1) + wsp_bytes(1) == xs_cap(2) + wsp_bytes(2), "x region");
@@ -239,6 +242,7 @@ __device__ __forceinline__ PD& pd_slot(int p) {
 __device__ __forceinline__ uint64_t* pd_bar(int p) { return sm_at<uint64_t>(SM_PDBAR) + (p & (PD_SLOTS - 1)); }
 __device__ __forceinline__ Ring* ring_state(int w) { return sm_at<Ring>(SM_WST) + w; }
 __device__ __forceinline__ uint64_t* ring_bar(int w, int s) { return sm_at<uint64_t>(SM_MBAR) + w * NSLOT + s; }
+__device__ __forceinline__ uint64_t* ring_ebar(int w, int s) { return sm_at<uint64_t>(SM_EBAR) + w * NSLOT + s; }
 __device__ __forceinline__ uint8_t* ring_slot(int w, int s) {
   return sm_at<uint8_t>(SM_RING + (w * NSLOT + s) * SLOT_BYTES);
 }
@@ -479,9 +483,16 @@ __device__ __forceinline__ void gemv_cta_range(const Geo& g, int cta, int& a, in
     a = b = 0;
   }
 }
+// A CTA's GEMV units split over its math warps.  Warp w runs on SM
+// sub-partition w % 4; the copy warp (warp NW = 15) shares sub-partition 3
+// with only three math warps, which therefore take 4/3 of the others' share
+// so that every sub-partition's tensor pipe gets the same work: warp w
+// starts at 3 w + floor(w / 4) of 48 parts.
+static_assert(NW == 15, "warp shares assume 15 math warps");
+__device__ __forceinline__ int warp_part(int w) { return 3 * w + (w >> 2); }
 __device__ __forceinline__ void warp_range(int a, int b, int w, int& wa, int& wb) {
-  wa = a + (b - a) * w / NW;
-  wb = a + (b - a) * (w + 1) / NW;
+  wa = a + (b - a) * warp_part(w) / 48;
+  wb = a + (b - a) * warp_part(w + 1) / 48;
 }
 // Attention work split over CTAs.  When every segment (sequence, KV head)
 // has the same number of 128-key units n (the usual case: equal lengths),
@@ -539,7 +550,7 @@ __device__ __forceinline__ void attn_seg_ctas(int type, int seg, int nca, int& c
 __device__ __noinline__ bool pd_ready(int q, bool block) {
   const LC& L = lc();
   if (q <= L.begin + PD_LEAD) return true;
-  if (L.cur_phase < q - PD_LEAD) return false;  // copy not issued yet
+  if (*reinterpret_cast<const volatile int*>(&L.cur_phase) < q - PD_LEAD) return false;  // copy not issued yet
   const uint32_t par = uint32_t((q - L.begin - PD_LEAD - 1) / PD_SLOTS) & 1u;
   if (mbar_try_wait(pd_bar(q), par)) return true;
   if (!block) return false;
@@ -654,9 +665,9 @@ __device__ __forceinline__ void cur_store(Cursor* s, const Cursor& c) {
   q[3] = make_uint4(uint32_t(c.x4), uint32_t(c.x5), uint32_t(c.x6), 0u);
 }
 
-// Next unit of the warp's register cursor; the slow path goes through the
-// warp's shared-memory copy.
-__device__ __forceinline__ void cur_next(Cursor& c, int warp, int lane) {
+// Next unit of a copy-warp lane's cursor: the common GEMV step in registers,
+// everything else through the lane's shared-memory copy.
+__device__ __forceinline__ void cur_adv(Cursor& c, int w) {
   if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
     ++c.i;
     if (++c.x6 == c.x2) {
@@ -670,15 +681,9 @@ __device__ __forceinline__ void cur_next(Cursor& c, int warp, int lane) {
   } else {
     ++c.i;
   }
-  Cursor* s = &ring_state(warp)->ld;
-  // lanes run independently between warp barriers: every lane must be done
-  // reading the shared copy before lane 0 rewrites it
-  warp_sync();
-  if (lane == 0) {
-    cur_store(s, c);
-    cur_normalize(s, warp);
-  }
-  warp_sync();
+  Cursor* s = &ring_state(w)->ld;
+  cur_store(s, c);
+  cur_normalize(s, w);
   cur_load(c, s);
 }
 
@@ -702,52 +707,34 @@ __device__ __forceinline__ void cur_src(const Cursor& c, int warp, const uint8_t
   }
 }
 
-__device__ __forceinline__ void ring_load(Ring& R, int warp) {
+// ---- consumer side of a warp's ring ----------------------------------------
+// Math warp w takes its units in order from slots w.0, w.1: it waits for the
+// slot's copy (full barrier) and hands the slot back (empty barrier) once its
+// lanes are done with it.  The copy warp refills it.
+struct Cons {
+  uint32_t consumed;
+  int bad;  // a wait of this warp timed out: stop waiting
+};
+__device__ __forceinline__ void cons_load(Cons& C, int warp) {
   const Ring* s = ring_state(warp);
-  const uint4 h = *reinterpret_cast<const uint4*>(s);
-  R.consumed = h.x;
-  R.issued = h.y;
-  R.pad_ = 0u;
-  R.bad = int(h.w);
-  cur_load(R.ld, &s->ld);
+  C.consumed = s->consumed;
+  C.bad = s->bad;
 }
-__device__ __forceinline__ void ring_store(const Ring& R, int warp, int lane) {
+__device__ __forceinline__ void cons_store(const Cons& C, int warp, int lane) {
   warp_sync();  // all lanes are done reading the shared copy
   if (lane == 0) {
     Ring* s = ring_state(warp);
-    *reinterpret_cast<uint4*>(s) = make_uint4(R.consumed, R.issued, 0u, uint32_t(R.bad));
-    cur_store(&s->ld, R.ld);
+    s->consumed = C.consumed;
+    s->bad = C.bad;
   }
   warp_sync();
 }
-
-// Fill free ring slots.
-template <int HD>
-__device__ __forceinline__ void ring_fill(Ring& R, int warp, int lane) {
-#pragma unroll 1
-  while (!R.bad && R.ld.kind >= 0 && R.issued - R.consumed < uint32_t(NSLOT)) {
-    const int sl = R.issued % NSLOT;
-    const uint8_t *s1, *s2;
-    uint32_t bytes;
-    cur_src(R.ld, warp, s1, s2, bytes, HD);
-    if (lane == 0) {
-      uint64_t* bar = ring_bar(warp, sl);
-      uint8_t* dst = ring_slot(warp, sl);
-      mbar_expect_tx(bar, s2 ? 2 * bytes : bytes);
-      bulk_g2s(dst, s1, bytes, bar);
-      if (s2) bulk_g2s(dst + bytes, s2, bytes, bar);
-    }
-    ++R.issued;
-    cur_next(R.ld, warp, lane);
-  }
-}
-
-__device__ __forceinline__ uint8_t* ring_wait(Ring& R, int warp, int lane) {
-  const int sl = R.consumed % NSLOT;
-  const uint32_t par = (R.consumed / NSLOT) & 1u;
+__device__ __forceinline__ uint8_t* cons_wait(Cons& C, int warp, int lane) {
+  const int sl = C.consumed % NSLOT;
+  const uint32_t par = (C.consumed / NSLOT) & 1u;
   uint64_t* bar = ring_bar(warp, sl);
   int late = 0;
-  if (!R.bad && !mbar_try_wait(bar, par)) {
+  if (!C.bad && !mbar_try_wait(bar, par)) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, par)) {
       if (clock64() - t0 > WAIT_CYCLES) {
@@ -756,55 +743,88 @@ __device__ __forceinline__ uint8_t* ring_wait(Ring& R, int warp, int lane) {
       }
     }
   }
-  if (__any_sync(0xffffffffu, late)) {  // keep the warp's ring state uniform
+  if (__any_sync(0xffffffffu, late)) {  // keep the warp's state uniform
     if (lane == 0) set_error(EW_MBAR_TIMEOUT);
-    R.bad = 1;
+    C.bad = 1;
   }
   return ring_slot(warp, sl);
 }
-// Hand the slot back and refill the ring.
-template <int HD>
-__device__ __forceinline__ void ring_release(Ring& R, int warp, int lane, bool wrote_slot) {
-  // order generic accesses of the slot before the async re-fill (every lane
-  // when lanes wrote into the slot, else lane 0 after the warp's reads)
+// Hand the slot back.  Lanes that wrote into it order those writes before
+// the copy engine's refill.
+__device__ __forceinline__ void cons_release(Cons& C, int warp, int lane, bool wrote_slot) {
   if (wrote_slot) fence_proxy_async();
-  warp_sync();
-  if (!wrote_slot && lane == 0) fence_proxy_async();
-  ++R.consumed;
-  ring_fill<HD>(R, warp, lane);
+  warp_sync();  // every lane is done with the slot
+  if (lane == 0) mbar_arrive(ring_ebar(warp, C.consumed % NSLOT));
+  ++C.consumed;
 }
 
-// Resume a waiting cursor and fill the ring (phase start).
+// ---- the copy warp -----------------------------------------------------------
+// Lane w (< NW) walks math warp w's unit stream through the phases of the
+// launch and issues each unit's bulk copy as soon as its slot is free; the
+// math warps never compute addresses or issue copies.  It stops past the last
+// phase, or when the math warps have left (error paths), and then waits for
+// its copies in flight so that none lands after the CTA has exited.
 template <int HD>
-__device__ __noinline__ void ring_top_up() {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  Ring* s = ring_state(warp);
-  warp_sync();
-  if (lane == 0) {
-    if (s->ld.kind == CUR_WAIT) cur_normalize(&s->ld, warp);
-  }
-  warp_sync();
-  Ring R;
-  ring_load(R, warp);
-  ring_fill<HD>(R, warp, lane);
-  ring_store(R, warp, lane);
-}
-
-__device__ __noinline__ void ring_drain() {
-  const int warp = threadIdx.x >> 5;
-  const Ring* s = ring_state(warp);
-  uint32_t c = s->consumed;
-  const uint32_t iss = s->issued;
+__device__ __noinline__ void copy_warp() {
+  const int lane = threadIdx.x & 31;
+  if (lane >= NW) return;
+  const int w = lane;
+  Cursor c;
+  cur_load(c, &ring_state(w)->ld);
+  uint32_t issued = 0;
+  long long idle0 = clock64();
 #pragma unroll 1
-  while (c < iss) {
+  for (;;) {
+    if (c.kind == CUR_DONE) break;
+    bool progress = false;
+    if (c.kind == CUR_WAIT) {
+      if (pd_ready(c.p, false)) {
+        Cursor* s = &ring_state(w)->ld;
+        cur_store(s, c);
+        cur_normalize(s, w);
+        cur_load(c, s);
+        progress = true;
+      }
+    } else {
+      const int sl = issued % NSLOT;
+      const uint32_t n = issued / NSLOT;
+      if (n == 0 || mbar_test_wait(ring_ebar(w, sl), (n - 1u) & 1u)) {
+        const uint8_t *s1, *s2;
+        uint32_t bytes;
+        cur_src(c, w, s1, s2, bytes, HD);
+        // the math warp's accesses of the slot (seen through the empty
+        // barrier) before the copy engine overwrites it
+        fence_proxy_async();
+        uint64_t* bar = ring_bar(w, sl);
+        uint8_t* dst = ring_slot(w, sl);
+        mbar_expect_tx(bar, s2 ? 2 * bytes : bytes);
+        bulk_g2s(dst, s1, bytes, bar);
+        if (s2) bulk_g2s(dst + bytes, s2, bytes, bar);
+        ++issued;
+        cur_adv(c, w);
+        progress = true;
+      }
+    }
+    if (progress) {
+      idle0 = clock64();
+      continue;
+    }
+    if (*reinterpret_cast<volatile int*>(&lc().stop) != 0) break;
+    if (clock64() - idle0 > 2 * WAIT_CYCLES) {
+      set_error(EW_MBAR_TIMEOUT);
+      break;
+    }
+  }
+  // copies in flight land before the lane leaves
+#pragma unroll 1
+  for (uint32_t j = issued > uint32_t(NSLOT) ? issued - NSLOT : 0u; j < issued; ++j) {
     const long long t0 = clock64();
-    while (!mbar_try_wait(ring_bar(warp, c % NSLOT), (c / NSLOT) & 1u)) {
+    while (!mbar_try_wait(ring_bar(w, j % NSLOT), (j / NSLOT) & 1u)) {
       if (clock64() - t0 > WAIT_CYCLES) {
-        if ((threadIdx.x & 31) == 0) set_error(EW_DRAIN_TIMEOUT);
+        set_error(EW_DRAIN_TIMEOUT);
         return;
       }
     }
-    ++c;
   }
 }
 
@@ -1608,8 +1628,8 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     int wa, wb;
     warp_range(a, b, warp, wa, wb);
     const int B = lc().B;
-    Ring R;
-    ring_load(R, warp);
+    Cons C;
+    cons_load(C, warp);
     const int kps = d.g.kps, nrb = d.g.nrb, upsl = nrb * kps, kcw = d.kcw;
     const bool w4 = (d.kind == PK_GEMV_W4);
     const int xrow_b = klen * 2 + 64;
@@ -1634,24 +1654,24 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
         for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
       }
       const int koff = (sl * kps + kci) * kcw - kbase;
-      const uint8_t* slot = ring_wait(R, warp, lane);
+      const uint8_t* slot = cons_wait(C, warp, lane);
       if (NB > 1) {
         // two batch tiles: the math reads the slot (registers are short)
         if (w4)
           w4_unit<NB>(slot, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g, lane);
         else
           bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
-        ring_release<HD>(R, warp, lane, false);
+        cons_release(C, warp, lane, false);
       } else if (w4) {
         // copy the unit to registers and hand the slot back before the math
         W4Regs ur;
         w4_load(slot, g, lane, ur);
-        ring_release<HD>(R, warp, lane, false);
+        cons_release(C, warp, lane, false);
         w4_math<NB>(ur, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g);
       } else {
         BfRegs br;
         bf_load(slot, lane, br);
-        ring_release<HD>(R, warp, lane, false);
+        cons_release(C, warp, lane, false);
         bf_math<NB>(br, xl + koff * 2, xrow_b, acc, B, g);
       }
       if (++kci == kps) {
@@ -1663,7 +1683,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
       }
     }
     if (cur >= 0) seg_done<NB>(d, cur, acc, wa, wb, park, B, lane);
-    ring_store(R, warp, lane);
+    cons_store(C, warp, lane);
   }
   cbar();
   mark(4);
@@ -1995,8 +2015,8 @@ __device__ __noinline__ void attn_phase(const PD& d) {
     {
       // this warp's keys of CTA units [u, run_end); its (m, l, o) partial goes
       // to shared memory
-      Ring R;
-      ring_load(R, warp);
+      Cons C;
+      cons_load(C, warp);
       const int g = lane >> 2, t = lane & 3;
       const uint4* qfr = sm_at<uint4>(SM_QF);
       const uint16_t* kn = sm_at<uint16_t>(SM_KNV);
@@ -2010,7 +2030,7 @@ __device__ __noinline__ void attn_phase(const PD& d) {
       for (int jc = u; jc < run_end; ++jc) {
         const int key0 = (jc - st[seg]) * ATT_CTA_KEYS + warp * ATT_KEYS;
         if (key0 >= Lk) continue;
-        uint8_t* slot = ring_wait(R, warp, lane);
+        uint8_t* slot = cons_wait(C, warp, lane);
         uint8_t* Ks = slot;
         uint8_t* Vs = slot + ATT_KEYS * HD * 2;
         const bool patch = own_new && sn_ >= key0 && sn_ < key0 + ATT_KEYS;
@@ -2072,9 +2092,9 @@ __device__ __noinline__ void attn_phase(const PD& d) {
           mma_1688(o[2 * q4 + 1], v2, v3, pa);
           mma_1688(o[2 * q4 + 1], v2, v3, pl);
         }
-        ring_release<HD>(R, warp, lane, patch);
+        cons_release(C, warp, lane, patch);
       }
-      ring_store(R, warp, lane);
+      cons_store(C, warp, lane);
       lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
       lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
       float* wp = sm_at<float>(SM_APW) + warp * ATT_PW;
@@ -2226,6 +2246,7 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     L.cur_phase = P.phase_begin;
     L.scaled = 0;
     L.final_norm = P.final_norm;
+    L.stop = 0;
     L.ctl = P.ws.ctl;
     L.seg_ctr = P.ws.seg_ctr;
     L.apart = P.ws.apart;
@@ -2241,9 +2262,12 @@ __device__ __noinline__ void setup(const EngineParams& P) {
 #pragma unroll 1
     for (int s = 0; s < PD_SLOTS; ++s) mbar_init(pd_bar(s), 1u);
   }
-  if (lane == 0) {
+  if (lane == 0 && warp < NW) {
 #pragma unroll 1
-    for (int s = 0; s < NSLOT; ++s) mbar_init(ring_bar(warp, s), 1u);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(ring_bar(warp, s), 1u);
+      mbar_init(ring_ebar(warp, s), 1u);
+    }
     fence_mbar_init();
   }
   if (tid < 128) sm_at<double>(SM_ROPE)[tid] = P.inv_freq[tid >> 6][tid & 63];
@@ -2306,16 +2330,14 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     am[1] = S > 0 ? P.nc / S : 0;
     am[2] = min(am[1], n);
   }
-  __syncthreads();
-  // ring state: the cursor at the warp's first unit
-  if (lane == 0) {
+  // ring state: nothing taken yet, the copy warp's cursor before the first phase
+  if (lane == 0 && warp < NW) {
     Ring* s = ring_state(warp);
     *reinterpret_cast<uint4*>(s) = make_uint4(0u, 0u, 0u, 0u);
     s->ld.kind = CUR_WAIT;
     s->ld.p = begin;
-    cur_normalize(&s->ld, warp);
   }
-  warp_sync();
+  __syncthreads();
 }
 
 // Phase start: descriptor p ready in shared memory, the copy of descriptor
@@ -2328,21 +2350,26 @@ __device__ __forceinline__ void phase_start(int p) {
     pd_ready(p, true);
     const int q = p + PD_LEAD;
     if (q < L.end && q > L.begin + PD_LEAD) {
-      fence_proxy_async_all();
+      // the plan was written with generic stores during setup and is read by
+      // the copy engine: one proxy fence before its first bulk read
+      if (q == L.begin + PD_LEAD + 1) fence_proxy_async_all();
       mbar_expect_tx(pd_bar(q), (uint32_t)sizeof(PD));
       bulk_g2s(&pd_slot(q), L.plan + q, (uint32_t)sizeof(PD), pd_bar(q));
     }
   }
   cbar();
   mark(1);
-  ring_top_up<HD>();
 }
 
+// NW math warps run the phases; warp NW is the copy warp.
 template <int NB, int HD>
-__global__ void __launch_bounds__(NT, 1) w4a_engine_kernel(const __grid_constant__ EngineParams P) {
+__global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constant__ EngineParams P) {
   setup(P);
+  if (threadIdx.x >= NT) {
+    copy_warp<HD>();
+    return;
+  }
   const int begin = lc().begin, end = lc().end;
-  ring_top_up<HD>();
 #pragma unroll 1
   for (int p = begin; p < end; ++p) {
     if (p != begin) {
@@ -2364,9 +2391,9 @@ __global__ void __launch_bounds__(NT, 1) w4a_engine_kernel(const __grid_constant
     grid_arrive();
     mark(6);
   }
-  ring_drain();
   cbar();
   if (threadIdx.x == 0) {
+    *reinterpret_cast<volatile int*>(&lc().stop) = 1;
     uint32_t* ctl = lc().ctl;
     __threadfence();
     const uint32_t old = atomicAdd(ctl + 1, 1u);

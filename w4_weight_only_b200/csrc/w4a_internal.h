@@ -9,8 +9,11 @@
 namespace w4a {
 
 // ---- engine geometry -------------------------------------------------------
-constexpr int NW = 16;                 // warps per CTA
-constexpr int NT = NW * 32;            // threads per CTA
+constexpr int NW = 15;                 // math warps per CTA
+constexpr int NT = NW * 32;            // threads of the math warps
+constexpr int NTH = NT + 32;           // threads per CTA: the math warps and the copy warp
+constexpr int ENGINE_REGS = 128;       // registers per thread (four warps per SM sub-partition)
+static_assert(NTH * ENGINE_REGS <= 65536, "register file");
 constexpr int NSLOT = 2;               // ring slots per warp
 constexpr int SLOT_BYTES = 4352;       // one unit (>= the largest unit below)
 constexpr int RB = 16;                 // output rows per unit (one m16 tile)
@@ -20,10 +23,10 @@ constexpr int GROUP = 128;             // quantization group (the only one suppo
 constexpr int W4_UNIT = RB * W4_KC / 2 + (W4_KC / GROUP) * RB * 2 + (W4_KC / GROUP) * RB / 2;  // 4256
 constexpr int BF_UNIT = RB * BF_KC * 2;                                                      // 4096
 constexpr int ATT_KEYS = 8;            // keys per warp unit
-constexpr int ATT_CTA_KEYS = ATT_KEYS * NW;  // keys per CTA unit (128)
+constexpr int ATT_CTA_KEYS = ATT_KEYS * NW;  // keys per CTA unit (120)
 // Shared-memory budget per CTA (bytes).  x fragments shrink when two
 // 8-column batch tiles are in use, to make room for their split-K slots.
-__host__ __device__ constexpr int xs_cap(int nb) { return nb == 1 ? 57344 : 40960; }
+__host__ __device__ constexpr int xs_cap(int nb) { return nb == 1 ? 58368 : 43008; }
 constexpr int XSUM_BYTES = 6912;       // per-128-group sums of x: [groups][8 * NB]
 __host__ __device__ constexpr int wsp_bytes(int nb) { return NW * 2 * 32 * 4 * nb * 4; }
 constexpr int MAX_B = 16;
