@@ -143,7 +143,8 @@ struct alignas(16) PD {
   const float* lpart;            // lm_head slabs [lns][B][vocab]
   const float* qnorm;            // QK-norm gains
   const float* knorm;
-  int qns, lns, red_epi, pad_;
+  int qns, lns, red_epi;
+  int gi;                        // GEMV: index of its geometry in the launch's table
 };
 static_assert(sizeof(PD) == 256, "phase descriptor size");
 
@@ -220,7 +221,8 @@ constexpr int SM_LC = SM_FLAGS + 64;
 constexpr int SM_ROPE = SM_LC + 256;                // inverse frequencies, fp64 [2][64]
 constexpr int SM_PD = SM_ROPE + 2 * 64 * 8;         // descriptor slots
 constexpr int SM_WST = SM_PD + PD_SLOTS * (int)sizeof(PD);  // ring state per warp
-constexpr int SM_TOTAL = SM_WST + NW * (int)sizeof(Ring);
+constexpr int SM_CTAB = SM_WST + NW * (int)sizeof(Ring);  // GEMV unit ranges [5 geometries][NW][2] int4
+constexpr int SM_TOTAL = SM_CTAB + 5 * NW * 32;
 static_assert(SM_TOTAL <= 232448, "shared memory budget");
 // attention views of the x region
 constexpr int ATT_PW = MAX_GQ * (128 + 2);                // floats of one warp's partial
@@ -241,6 +243,10 @@ __device__ __forceinline__ PD& pd_slot(int p) {
 }
 __device__ __forceinline__ uint64_t* pd_bar(int p) { return sm_at<uint64_t>(SM_PDBAR) + (p & (PD_SLOTS - 1)); }
 __device__ __forceinline__ Ring* ring_state(int w) { return sm_at<Ring>(SM_WST) + w; }
+// Unit range of math warp w under GEMV geometry gi, computed once per launch:
+// [0] = (first unit, end, slab, row block of the first unit), [1] = (its
+// k-chunk, the CTA's first unit, the CTA's end, 0).
+__device__ __forceinline__ const int4* ctab(int gi, int w) { return sm_at<int4>(SM_CTAB) + (gi * NW + w) * 2; }
 __device__ __forceinline__ uint64_t* ring_bar(int w, int s) { return sm_at<uint64_t>(SM_MBAR) + w * NSLOT + s; }
 __device__ __forceinline__ uint64_t* ring_ebar(int w, int s) { return sm_at<uint64_t>(SM_EBAR) + w * NSLOT + s; }
 __device__ __forceinline__ uint8_t* ring_slot(int w, int s) {
@@ -313,6 +319,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.xbf_stride = P.g_k;
     d.rows_valid = P.g_n;
     d.g = P.geo[0];
+    d.gi = 0;
     const bool direct_silu = P.g_epi == W4A_EPI_SILU_MUL && d.g.ns == 1;
     const bool direct = P.g_epi == W4A_EPI_NONE && d.g.ns == 1;
     if (direct_silu) {
@@ -357,6 +364,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.kcw = BF_KC;
     d.ub = BF_UNIT;
     d.g = g_lm;
+    d.gi = 4;
     d.xsrc = XS_FINAL;
     d.xres = P.ws.xB;
     d.vpart = P.ws.f_part;
@@ -406,6 +414,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.n = qkv_dim;
     d.k = dm;
     d.g = g_qkv;
+    d.gi = 0;
     if (l == 0) {
       d.xsrc = XS_EMBED;
     } else {
@@ -425,6 +434,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.n = dm;
     d.k = qd;
     d.g = g_o;
+    d.gi = 1;
     d.xsrc = XS_F16;
     d.xbf = P.ws.o;
     d.xbf_stride = qd;
@@ -435,6 +445,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.n = 2 * P.ffn;
     d.k = dm;
     d.g = g_gu;
+    d.gi = 2;
     d.xsrc = XS_RESID;
     d.xres = P.ws.xA;
     d.vpart = P.ws.a_part;
@@ -456,6 +467,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.n = dm;
     d.k = P.ffn;
     d.g = g_dn;
+    d.gi = 3;
     if (g_gu.ns == 1) {
       d.xsrc = XS_F16;
       d.xbf = P.ws.h;
@@ -485,14 +497,15 @@ __device__ __forceinline__ void gemv_cta_range(const Geo& g, int cta, int& a, in
 }
 // A CTA's GEMV units split over its math warps.  Warp w runs on SM
 // sub-partition w % 4; the copy warp (warp NW = 15) shares sub-partition 3
-// with only three math warps, which therefore take 4/3 of the others' share
-// so that every sub-partition's tensor pipe gets the same work: warp w
-// starts at 3 w + floor(w / 4) of 48 parts.
+// with only three math warps, which run a unit ~1.17x faster than the math
+// warps of the full sub-partitions (per-warp finish times of the 64-layer
+// decode step).  Shares: 6 parts per warp, 7 on sub-partition 3, of 93;
+// warp w starts at 6 w + floor(w / 4).
 static_assert(NW == 15, "warp shares assume 15 math warps");
-__device__ __forceinline__ int warp_part(int w) { return 3 * w + (w >> 2); }
+__device__ __forceinline__ int warp_part(int w) { return 6 * w + (w >> 2); }
 __device__ __forceinline__ void warp_range(int a, int b, int w, int& wa, int& wb) {
-  wa = a + (b - a) * warp_part(w) / 48;
-  wb = a + (b - a) * warp_part(w + 1) / 48;
+  wa = a + (b - a) * warp_part(w) / 93;
+  wb = a + (b - a) * warp_part(w + 1) / 93;
 }
 // Attention work split over CTAs.  When every segment (sequence, KV head)
 // has the same number of 128-key units n (the usual case: equal lengths),
@@ -580,21 +593,18 @@ __device__ __noinline__ void cur_enter(Cursor* c, int q, int w) {
   const PD& d = pd_slot(q);
   c->kind = d.kind;
   if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_BF16) {
-    int a, b, wa, wb;
-    gemv_cta_range(d.g, blockIdx.x, a, b);
-    warp_range(a, b, w, wa, wb);
+    const int4* e = ctab(d.gi, w);
+    const int4 e0 = e[0], e1 = e[1];
     c->p0 = d.blob;
     c->x0 = d.ub;
     c->x1 = d.g.nkc;
     c->x2 = d.g.kps;
     c->x3 = d.g.nrb;
-    c->i = wa;
-    c->end = wb;
-    const int upsl = d.g.nrb * d.g.kps;
-    c->x4 = wa / upsl;
-    const int r = wa - c->x4 * upsl;
-    c->x5 = r / d.g.kps;
-    c->x6 = r - c->x5 * d.g.kps;
+    c->i = e0.x;
+    c->end = e0.y;
+    c->x4 = e0.z;
+    c->x5 = e0.w;
+    c->x6 = e1.x;
   } else if (d.kind == PK_ATTN) {
     int a, b, nca;
     attn_cta_range(d.type, blockIdx.x, a, b, nca);
@@ -1601,8 +1611,8 @@ template <int NB, int HD>
 __device__ __noinline__ void gemv_phase(const PD& d) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  int a, b;
-  gemv_cta_range(d.g, blockIdx.x, a, b);
+  const int4 e0 = ctab(d.gi, warp)[0], e1 = ctab(d.gi, warp)[1];
+  int a = e1.y, b = e1.z;
   int kbase = 0, klen = 0;
   if (a < b) {
     const int upsl = d.g.nrb * d.g.kps, KS = d.g.kps * d.kcw;
@@ -1625,8 +1635,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
   }
   mark(3);
   if (a < b) {
-    int wa, wb;
-    warp_range(a, b, warp, wa, wb);
+    const int wa = e0.x, wb = e0.y;
     const int B = lc().B;
     Cons C;
     cons_load(C, warp);
@@ -1637,9 +1646,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     const float* xsg = sm_at<float>(sm_xsum(NB)) + 2 * t;
     float* park = sm_at<float>(sm_wsp(NB)) + warp * (2 * 32 * 4 * NB) + lane * 4 * NB;
     int u = wa;
-    int sl = u / upsl;
-    int rb = (u - sl * upsl) / kps;
-    int kci = u - sl * upsl - rb * kps;
+    int sl = e0.z, rb = e0.w, kci = e1.x;
     float acc[NB][4];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
@@ -2329,6 +2336,24 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     am[0] = (equal && n > 0 && S <= P.nc) ? 1 : 0;
     am[1] = S > 0 ? P.nc / S : 0;
     am[2] = min(am[1], n);
+  }
+  // GEMV unit ranges of this CTA and its warps, per geometry
+  if (tid < 5 * NW) {
+    const int gi = tid / NW, w = tid - gi * NW;
+    const Geo& g = P.geo[gi];
+    int a = 0, b = 0, wa = 0, wb = 0, x4 = 0, x5 = 0, x6 = 0;
+    if (g.nca > 0 && g.kps > 0 && g.nrb > 0) {
+      gemv_cta_range(g, cta, a, b);
+      warp_range(a, b, w, wa, wb);
+      const int upsl = g.nrb * g.kps;
+      x4 = wa / upsl;
+      const int r = wa - x4 * upsl;
+      x5 = r / g.kps;
+      x6 = r - x5 * g.kps;
+    }
+    int4* e = sm_at<int4>(SM_CTAB) + (gi * NW + w) * 2;
+    e[0] = make_int4(wa, wb, x4, x5);
+    e[1] = make_int4(x6, a, b, 0);
   }
   // ring state: nothing taken yet, the copy warp's cursor before the first phase
   if (lane == 0 && warp < NW) {
