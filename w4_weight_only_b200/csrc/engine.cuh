@@ -782,6 +782,9 @@ __device__ __noinline__ void copy_warp() {
   Cursor c;
   cur_load(c, &ring_state(w)->ld);
   uint32_t issued = 0;
+  // weights and old keys are read once per token: evict them first, so that
+  // the activations, residuals and gains the phase prologues read stay in L2
+  const uint64_t once = policy_evict_first();
   long long idle0 = clock64();
 #pragma unroll 1
   for (;;) {
@@ -808,8 +811,8 @@ __device__ __noinline__ void copy_warp() {
         uint64_t* bar = ring_bar(w, sl);
         uint8_t* dst = ring_slot(w, sl);
         mbar_expect_tx(bar, s2 ? 2 * bytes : bytes);
-        bulk_g2s(dst, s1, bytes, bar);
-        if (s2) bulk_g2s(dst + bytes, s2, bytes, bar);
+        bulk_g2s_hint(dst, s1, bytes, bar, once);
+        if (s2) bulk_g2s_hint(dst + bytes, s2, bytes, bar, once);
         ++issued;
         cur_adv(c, w);
         progress = true;
@@ -1024,7 +1027,9 @@ __device__ __noinline__ void put8(bool valid, int bb, int kl0, int xrow_b, F8 vv
   }
   if (valid && (lane & 15) == 0) {
     sm_at<float>(sm_xsum(NB))[(kl0 >> 7) * (8 * NB) + bb] = s8;
-    if (track_max) atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + bb, __float_as_uint(m8));
+    // the row maximum matters only once it reaches the fp16 guard, so only
+    // such groups post it (shared atomics on one word serialise across warps)
+    if (track_max && m8 >= 32768.f) atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + bb, __float_as_uint(m8));
   }
 }
 
@@ -1940,59 +1945,80 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
   }
   cbar();
   if (!flags()[1]) return;
-  // warp h combines query head h over the pieces c0..c1: one piece per lane
-  // for the max and the denominators, then the outputs (four dims per lane)
-  // with the loads of eight pieces in flight.  CTA c0 filed its piece in its
-  // second slot (the segment is its last), the others in their first.
-  if (warp < GQ) {
-    const int h = warp;
-    auto piece_of = [&](int c) {
-      return L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
+  // The pieces c0..c1 merge in one round of loads: warp w takes query head
+  // w % GQ and the w / GQ-th share of the pieces; every lane reads the maxima
+  // of all pieces (one piece per lane) while the loads of its share's outputs
+  // (four dims per lane), maxima and denominators are already in flight.  The
+  // shares then add up in shared memory in a fixed order.  CTA c0 filed its
+  // piece in its second slot (the segment is its last), the others in their
+  // first.
+  constexpr int DPL = HD / 32;  // dims per lane
+  constexpr int PB = 8;         // pieces per load batch
+  const int nparts = NW / GQ;
+  float* red_ws = sm_at<float>(SM_APW);  // [warp][lane][DPL + 1]; the warp partials are consumed
+  const int h = warp % GQ, part = warp / GQ;
+  const bool active = part < nparts;
+  auto piece_of = [&](int c) {
+    return L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
+  };
+  if (active) {
+    const int np = c1 - c0 + 1, per = (np + nparts - 1) / nparts;
+    const int p0 = c0 + part * per, p1 = min(c1 + 1, p0 + per);
+    float acc[DPL], Lsum = 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+    // first batch of this share in flight before the maxima
+    float ov[PB][DPL], mv[PB], lv[PB];
+    auto load_batch = [&](int cb) {
+#pragma unroll
+      for (int j = 0; j < PB; ++j) {
+        const bool ok = cb + j < p1;
+        const float* pc = piece_of(ok ? cb + j : c0);
+        mv[j] = ok ? __ldcg(pc + HD) : -INFINITY;
+        lv[j] = ok ? __ldcg(pc + HD + 1) : 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) ov[j][e] = ok ? __ldcg(pc + lane * DPL + e) : 0.f;
+      }
     };
+    load_batch(p0);
     float M = -INFINITY;
 #pragma unroll 1
     for (int c = c0 + lane; c <= c1; c += 32) M = fmaxf(M, __ldcg(piece_of(c) + HD));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    constexpr int DPL = HD / 32;  // dims per lane
-    float acc[DPL];
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-    float Lsum = 0.f;
 #pragma unroll 1
-    for (int cb = c0; cb <= c1; cb += 32) {
-      const int cl = cb + lane;
-      float ev = 0.f;
-      if (cl <= c1) {
-        const float* pc = piece_of(cl);
-        ev = exp2f(__ldcg(pc + HD) - M);
-        Lsum = fmaf(ev, __ldcg(pc + HD + 1), Lsum);
-      }
-      const int n = min(32, c1 - cb + 1);
-#pragma unroll 1
-      for (int i0 = 0; i0 < n; i0 += 8) {
-        float ov[8][DPL];
+    for (int cb = p0; cb < p1; cb += PB) {
+      if (cb != p0) load_batch(cb);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float* pc = piece_of(min(cb + i0 + j, c1)) + lane * DPL;  // clamped: never past the last piece
+      for (int j = 0; j < PB; ++j) {
+        const float w = exp2f(mv[j] - M);  // 0 for the padding (-inf)
+        Lsum = fmaf(w, lv[j], Lsum);
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) ov[j][e] = (i0 + j < n) ? __ldcg(pc + e) : 0.f;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float w = __shfl_sync(0xffffffffu, ev, (i0 + j) & 31);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, ov[j][e], acc[e]);
-        }
+        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, ov[j][e], acc[e]);
       }
     }
+    float* r = red_ws + (warp * 32 + lane) * (DPL + 1);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    for (int e = 0; e < DPL; ++e) r[e] = acc[e];
+    r[DPL] = Lsum;
+  }
+  cbar();
+  if (warp < GQ) {
+    float acc[DPL], Lsum = 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+#pragma unroll 1
+    for (int q = 0; q < nparts; ++q) {
+      const float* r = red_ws + ((q * GQ + warp) * 32 + lane) * (DPL + 1);
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] += r[e];
+      Lsum += r[DPL];
+    }
     const float inv = 1.f / Lsum;
 #pragma unroll
     for (int e = 0; e < DPL; ++e) {
       const float v = acc[e] * inv;
-      out[h * HD + lane * DPL + e] = d.out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
+      out[warp * HD + lane * DPL + e] = d.out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
     }
   }
   if (tid == 0) L.seg_ctr[seg] = 0u;
