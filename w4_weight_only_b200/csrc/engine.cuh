@@ -221,8 +221,8 @@ constexpr int SM_LC = SM_FLAGS + 64;
 constexpr int SM_ROPE = SM_LC + 256;                // inverse frequencies, fp64 [2][64]
 constexpr int SM_PD = SM_ROPE + 2 * 64 * 8;         // descriptor slots
 constexpr int SM_WST = SM_PD + PD_SLOTS * (int)sizeof(PD);  // ring state per warp
-constexpr int SM_CTAB = SM_WST + NW * (int)sizeof(Ring);  // GEMV unit ranges [5 geometries][NW][2] int4
-constexpr int SM_TOTAL = SM_CTAB + 5 * NW * 32;
+constexpr int SM_CTAB = SM_WST + NW * (int)sizeof(Ring);  // GEMV unit ranges [5 geometries][NW][4] int4
+constexpr int SM_TOTAL = SM_CTAB + 5 * NW * 64;
 static_assert(SM_TOTAL <= 232448, "shared memory budget");
 // attention views of the x region
 constexpr int ATT_PW = MAX_GQ * (128 + 2);                // floats of one warp's partial
@@ -245,8 +245,12 @@ __device__ __forceinline__ uint64_t* pd_bar(int p) { return sm_at<uint64_t>(SM_P
 __device__ __forceinline__ Ring* ring_state(int w) { return sm_at<Ring>(SM_WST) + w; }
 // Unit range of math warp w under GEMV geometry gi, computed once per launch:
 // [0] = (first unit, end, slab, row block of the first unit), [1] = (its
-// k-chunk, the CTA's first unit, the CTA's end, 0).
-__device__ __forceinline__ const int4* ctab(int gi, int w) { return sm_at<int4>(SM_CTAB) + (gi * NW + w) * 2; }
+// k-chunk, the CTA's first unit, the CTA's end, 0), [2] = the segment this
+// warp closes for the CTA: (1 + first warp holding a piece of it, or 0 when
+// the warp closes none; bit i: piece of warp first + i sits in that warp's
+// second park slot, bit 16 + i: warp first + i has no units; its slab; its
+// row block), [3] = (first column of the CTA's x range, its length, 0, 0).
+__device__ __forceinline__ const int4* ctab(int gi, int w) { return sm_at<int4>(SM_CTAB) + (gi * NW + w) * 4; }
 __device__ __forceinline__ uint64_t* ring_bar(int w, int s) { return sm_at<uint64_t>(SM_MBAR) + w * NSLOT + s; }
 __device__ __forceinline__ uint64_t* ring_ebar(int w, int s) { return sm_at<uint64_t>(SM_EBAR) + w * NSLOT + s; }
 __device__ __forceinline__ uint8_t* ring_slot(int w, int s) {
@@ -1517,7 +1521,7 @@ __device__ __noinline__ void emit_rows(const PD& d, int s, int rb, Acc<NB> A, in
         for (int e = 0; e < 4; ++e) {
           const int b = nb * 8 + 2 * t + (e & 1), j = (e & 2) ? j1 : j0;
           const float x = v[nb][e];
-          const float hv = x / (1.f + expf(-x)) * u[e];
+          const float hv = __fdividef(x, 1.f + __expf(-x)) * u[e];
           if (b < B) h[(size_t)b * d.ostride + j] = d.out_f16 ? f32_to_f16(hv) : f32_to_bf16(hv);
         }
       }
@@ -1542,9 +1546,11 @@ __device__ __noinline__ void emit_rows(const PD& d, int s, int rb, Acc<NB> A, in
 
 // A segment piece leaves the warp: undo the range scaling, then emit it
 // (segment wholly inside this warp) or park it in the warp's slot.
+// whole: the warp ran all of the segment's units; first: it is the warp's
+// first segment (its piece goes to park slot 0, a later one to slot 1).
 template <int NB>
-__device__ __forceinline__ void seg_done(const PD& d, int seg, float (&acc)[NB][4], int wa, int wb, float* park,
-                                         int B, int lane) {
+__device__ __forceinline__ void seg_done(const PD& d, int s, int rb, bool whole, bool first, float (&acc)[NB][4],
+                                         float* park, int B, int lane) {
   if (lc().scaled) {
     const float* xscale = red() + 48;
     const int t = lane & 3;
@@ -1557,12 +1563,10 @@ __device__ __forceinline__ void seg_done(const PD& d, int seg, float (&acc)[NB][
       acc[nb][3] *= s1;
     }
   }
-  const int kps = d.g.kps, u0 = seg * kps;
-  if (u0 >= wa && u0 + kps <= wb) {
-    const int s = seg / d.g.nrb;
-    emit_rows<NB>(d, s, seg - s * d.g.nrb, acc_of<NB>(acc), B, lane);
+  if (whole) {
+    emit_rows<NB>(d, s, rb, acc_of<NB>(acc), B, lane);
   } else {
-    float* q = park + ((seg == wa / kps) ? 0 : 32 * 4 * NB);
+    float* q = park + (first ? 0 : 32 * 4 * NB);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb)
       reinterpret_cast<float4*>(q)[nb] = make_float4(acc[nb][0], acc[nb][1], acc[nb][2], acc[nb][3]);
@@ -1572,32 +1576,19 @@ __device__ __forceinline__ void seg_done(const PD& d, int seg, float (&acc)[NB][
 // Segments of this CTA split between warps: the warp holding a segment's last
 // unit sums its pieces in warp order and emits the rows.
 template <int NB>
-__device__ __noinline__ void cta_combine(const PD& d, int a, int b) {
+__device__ __noinline__ void cta_combine(const PD& d) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kps = d.g.kps, B = lc().B;
-  int wa, wb;
-  warp_range(a, b, warp, wa, wb);
-  if (wa >= wb || wa % kps == 0) return;  // my first segment starts with me: no piece before mine
-  const int S = wa / kps;
-  if ((S + 1) * kps > wb) return;          // it goes on past my range: a later warp finishes it
-  int w0 = warp;
-#pragma unroll 1
-  while (w0 > 0) {
-    int pa, pb;
-    warp_range(a, b, w0 - 1, pa, pb);
-    if (pb <= S * kps) break;
-    --w0;
-  }
+  const int4 c = ctab(d.gi, warp)[2];
+  if (c.x == 0) return;
+  const int w0 = c.x - 1;
   const float* wsp = sm_at<float>(sm_wsp(NB));
   float sum[NB][4];
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) sum[nb][0] = sum[nb][1] = sum[nb][2] = sum[nb][3] = 0.f;
 #pragma unroll 1
   for (int w2 = w0; w2 <= warp; ++w2) {
-    int a2, b2;
-    warp_range(a, b, w2, a2, b2);
-    if (a2 >= b2) continue;
-    const int sl = (S == a2 / kps) ? 0 : 1;
+    if ((c.y >> (16 + w2 - w0)) & 1) continue;
+    const int sl = (c.y >> (w2 - w0)) & 1;
     const float* q = wsp + w2 * (2 * 32 * 4 * NB) + sl * (32 * 4 * NB) + lane * 4 * NB;
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
@@ -1608,8 +1599,7 @@ __device__ __noinline__ void cta_combine(const PD& d, int a, int b) {
       sum[nb][3] += f.w;
     }
   }
-  const int s = S / d.g.nrb;
-  emit_rows<NB>(d, s, S - s * d.g.nrb, acc_of<NB>(sum), B, lane);
+  emit_rows<NB>(d, c.z, c.w, acc_of<NB>(sum), lc().B, lane);
 }
 
 template <int NB, int HD>
@@ -1618,13 +1608,8 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
   const int g = lane >> 2, t = lane & 3;
   const int4 e0 = ctab(d.gi, warp)[0], e1 = ctab(d.gi, warp)[1];
   int a = e1.y, b = e1.z;
-  int kbase = 0, klen = 0;
-  if (a < b) {
-    const int upsl = d.g.nrb * d.g.kps, KS = d.g.kps * d.kcw;
-    const int s0 = a / upsl, s1 = (b - 1) / upsl;
-    kbase = s0 * KS;
-    klen = (s1 - s0 + 1) * KS;
-  }
+  const int4 e3 = ctab(d.gi, warp)[3];
+  int kbase = e3.x, klen = e3.y;
   if (!x_fits(klen, lc().B, NB)) {  // the host sizes slabs so this never happens
     if (tid == 0) set_error(EW_BAD_SHAPE);
     a = b = 0;
@@ -1644,7 +1629,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     const int B = lc().B;
     Cons C;
     cons_load(C, warp);
-    const int kps = d.g.kps, nrb = d.g.nrb, upsl = nrb * kps, kcw = d.kcw;
+    const int kps = d.g.kps, nrb = d.g.nrb, kcw = d.kcw;
     const bool w4 = (d.kind == PK_GEMV_W4);
     const int xrow_b = klen * 2 + 64;
     const uint8_t* xl = sm_at<uint8_t>(SM_XS + g * xrow_b + t * 16);
@@ -1655,16 +1640,21 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     float acc[NB][4];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-    int cur = -1;
+    // the segment in progress: its slab and row block, units run, first?
+    int cs = sl, crb = rb, cn = 0;
+    bool cfirst = true;
 #pragma unroll 1
     for (; u < wb; ++u) {
-      const int seg = sl * nrb + rb;
-      if (seg != cur) {
-        if (cur >= 0) seg_done<NB>(d, cur, acc, wa, wb, park, B, lane);
-        cur = seg;
+      if (sl != cs || rb != crb) {
+        seg_done<NB>(d, cs, crb, cn == kps, cfirst, acc, park, B, lane);
+        cs = sl;
+        crb = rb;
+        cn = 0;
+        cfirst = false;
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
       }
+      ++cn;
       const int koff = (sl * kps + kci) * kcw - kbase;
       const uint8_t* slot = cons_wait(C, warp, lane);
       if (NB > 1) {
@@ -1694,12 +1684,12 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
         }
       }
     }
-    if (cur >= 0) seg_done<NB>(d, cur, acc, wa, wb, park, B, lane);
+    seg_done<NB>(d, cs, crb, cn == kps, cfirst, acc, park, B, lane);
     cons_store(C, warp, lane);
   }
   cbar();
   mark(4);
-  if (a < b) cta_combine<NB>(d, a, b);
+  if (a < b) cta_combine<NB>(d);
   mark(5);
 }
 
@@ -2377,9 +2367,43 @@ __device__ __noinline__ void setup(const EngineParams& P) {
       x5 = r / g.kps;
       x6 = r - x5 * g.kps;
     }
-    int4* e = sm_at<int4>(SM_CTAB) + (gi * NW + w) * 2;
+    // the CTA-level close of a segment split between warps (the warp holding
+    // its last unit sums the pieces of warps w0..w in order)
+    int cw0 = 0, cmask = 0, cs = 0, crb = 0;
+    if (g.nca > 0 && g.kps > 0 && g.nrb > 0 && wa < wb && wa % g.kps != 0) {
+      const int S = wa / g.kps;
+      if ((S + 1) * g.kps <= wb) {
+        int w0 = w;
+        while (w0 > 0) {
+          int pa, pb;
+          warp_range(a, b, w0 - 1, pa, pb);
+          if (pb <= S * g.kps) break;
+          --w0;
+        }
+        for (int w2 = w0; w2 <= w; ++w2) {
+          int a2, b2;
+          warp_range(a, b, w2, a2, b2);
+          if (a2 >= b2) cmask |= 1 << (16 + w2 - w0);
+          else if (S != a2 / g.kps) cmask |= 1 << (w2 - w0);
+        }
+        cw0 = w0 + 1;
+        cs = S / g.nrb;
+        crb = S - cs * g.nrb;
+      }
+    }
+    // the CTA's x range: the slabs its segments touch
+    int kbase = 0, klen = 0;
+    if (a < b) {
+      const int upsl = g.nrb * g.kps, KS = g.kps * (gi == 4 ? BF_KC : W4_KC);
+      const int s0 = a / upsl, s1 = (b - 1) / upsl;
+      kbase = s0 * KS;
+      klen = (s1 - s0 + 1) * KS;
+    }
+    int4* e = sm_at<int4>(SM_CTAB) + (gi * NW + w) * 4;
     e[0] = make_int4(wa, wb, x4, x5);
     e[1] = make_int4(x6, a, b, 0);
+    e[2] = make_int4(cw0, cmask, cs, crb);
+    e[3] = make_int4(kbase, klen, 0, 0);
   }
   // ring state: nothing taken yet, the copy warp's cursor before the first phase
   if (lane == 0 && warp < NW) {
