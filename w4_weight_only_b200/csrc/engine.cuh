@@ -501,15 +501,15 @@ __device__ __forceinline__ void gemv_cta_range(const Geo& g, int cta, int& a, in
 }
 // A CTA's GEMV units split over its math warps.  Warp w runs on SM
 // sub-partition w % 4; the copy warp (warp NW = 15) shares sub-partition 3
-// with only three math warps, which run a unit ~1.17x faster than the math
+// with only three math warps, which run a unit ~1.09x faster than the math
 // warps of the full sub-partitions (per-warp finish times of the 64-layer
-// decode step).  Shares: 6 parts per warp, 7 on sub-partition 3, of 93;
-// warp w starts at 6 w + floor(w / 4).
+// decode step).  Shares: 11 parts per warp, 12 on sub-partition 3, of 168;
+// warp w starts at 11 w + floor(w / 4).
 static_assert(NW == 15, "warp shares assume 15 math warps");
-__device__ __forceinline__ int warp_part(int w) { return 6 * w + (w >> 2); }
+__device__ __forceinline__ int warp_part(int w) { return 11 * w + (w >> 2); }
 __device__ __forceinline__ void warp_range(int a, int b, int w, int& wa, int& wb) {
-  wa = a + (b - a) * warp_part(w) / 93;
-  wb = a + (b - a) * warp_part(w + 1) / 93;
+  wa = a + (b - a) * warp_part(w) / 168;
+  wb = a + (b - a) * warp_part(w + 1) / 168;
 }
 // Attention work split over CTAs.  When every segment (sequence, KV head)
 // has the same number of 128-key units n (the usual case: equal lengths),
@@ -1025,15 +1025,50 @@ __device__ __noinline__ void put8(bool valid, int bb, int kl0, int xrow_b, F8 vv
     *sm_at<uint4>(SM_XS + bb * xrow_b + kl0 * 2) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) {
-    s8 += __shfl_xor_sync(0xffffffffu, s8, o);
-    m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, o));
+  for (int o = 8; o > 0; o >>= 1) s8 += __shfl_xor_sync(0xffffffffu, s8, o);
+  if (valid && (lane & 15) == 0) sm_at<float>(sm_xsum(NB))[(kl0 >> 7) * (8 * NB) + bb] = s8;
+  // the row maximum matters only once it reaches the fp16 guard, so only the
+  // lanes past it post theirs (rare; shared atomics on one word serialise)
+  if (track_max && __any_sync(0xffffffffu, valid && m8 >= 32768.f) && valid && m8 >= 32768.f)
+    atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + bb, __float_as_uint(m8));
+}
+
+// Two fp16 chunks of eight at once (the residual paths hold up to two chunks
+// per thread): the conversions and the two group-sum reductions interleave.
+template <int NB>
+__device__ __forceinline__ void put8x2(bool va, int ba, int ka, const float (&xa)[8], bool vb, int bb, int kb,
+                                       const float (&xb)[8], int xrow_b) {
+  const int lane = threadIdx.x & 31;
+  float sa = 0.f, sb = 0.f, ma = 0.f, mb = 0.f;
+  uint32_t wa[4], wb[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint16_t a0 = f32_to_f16(xa[2 * t]), a1 = f32_to_f16(xa[2 * t + 1]);
+    const uint16_t b0 = f32_to_f16(xb[2 * t]), b1 = f32_to_f16(xb[2 * t + 1]);
+    wa[t] = uint32_t(a0) | (uint32_t(a1) << 16);
+    wb[t] = uint32_t(b0) | (uint32_t(b1) << 16);
+    sa += half_bits_to_f32(a0) + half_bits_to_f32(a1);
+    sb += half_bits_to_f32(b0) + half_bits_to_f32(b1);
+    ma = fmaxf(ma, fmaxf(fabsf(xa[2 * t]), fabsf(xa[2 * t + 1])));
+    mb = fmaxf(mb, fmaxf(fabsf(xb[2 * t]), fabsf(xb[2 * t + 1])));
   }
-  if (valid && (lane & 15) == 0) {
-    sm_at<float>(sm_xsum(NB))[(kl0 >> 7) * (8 * NB) + bb] = s8;
-    // the row maximum matters only once it reaches the fp16 guard, so only
-    // such groups post it (shared atomics on one word serialise across warps)
-    if (track_max && m8 >= 32768.f) atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + bb, __float_as_uint(m8));
+  if (!va) sa = 0.f;
+  if (!vb) sb = 0.f;
+  if (va) *sm_at<uint4>(SM_XS + ba * xrow_b + ka * 2) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+  if (vb) *sm_at<uint4>(SM_XS + bb * xrow_b + kb * 2) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    sb += __shfl_xor_sync(0xffffffffu, sb, o);
+  }
+  if ((lane & 15) == 0) {
+    if (va) sm_at<float>(sm_xsum(NB))[(ka >> 7) * (8 * NB) + ba] = sa;
+    if (vb) sm_at<float>(sm_xsum(NB))[(kb >> 7) * (8 * NB) + bb] = sb;
+  }
+  const bool pa = va && ma >= 32768.f, pb = vb && mb >= 32768.f;
+  if (__any_sync(0xffffffffu, pa || pb)) {  // rare: the fp16 guard
+    if (pa) atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + ba, __float_as_uint(ma));
+    if (pb) atomicMax(reinterpret_cast<uint32_t*>(red() + 32) + bb, __float_as_uint(mb));
   }
 }
 
@@ -1222,6 +1257,25 @@ __device__ __noinline__ void stage_x(const PD& d, int kbase, int klen) {
       cbar();
     }
     // convert the k-range, write the residual copy / dump slice
+    if (two && !fin) {
+      // this thread's (up to) two chunks, indexed in pass 1
+      float xa[8], xb[8];
+      resid8(v0, x0, g0, h0 ? rd[b0] : 0.f, xa);
+      resid8(v1, x1, g1, h1 ? rd[b1] : 0.f, xb);
+      if (has_out) {
+        if (h0 && c0 >= o0 && c0 < o1) {
+          if (d.xdst) store8f(d.xdst + (size_t)b0 * dm + k00, xa);
+          if (d.dump) store8f(d.dump + (size_t)b0 * dm + k00, xa);
+        }
+        if (h1 && c1 >= o0 && c1 < o1) {
+          if (d.xdst) store8f(d.xdst + (size_t)b1 * dm + k01, xb);
+          if (d.dump) store8f(d.dump + (size_t)b1 * dm + k01, xb);
+        }
+      }
+      // half-warps are uniformly inside or outside (128-aligned k-range)
+      put8x2<NB>(h0 && k00 >= kbase && k00 < kbase + klen, b0, k00 - kbase, xa,
+                 h1 && k01 >= kbase && k01 < kbase + klen, b1, k01 - kbase, xb, xrow_b);
+    } else
 #pragma unroll 1
     for (int j = 0; warp * 32 + j * NT < total8; ++j) {
       const int c = warp * 32 + j * NT + lane, bb = (warp * 32 + j * NT) / n8, k0 = (c - bb * n8) * 8;
