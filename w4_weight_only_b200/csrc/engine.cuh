@@ -878,13 +878,18 @@ __device__ __forceinline__ void grid_arrive() {
 }
 
 // Deterministic per-batch-row totals of per-warp partial sums wsum[warp][b].
+// Warp 0 sums the NW partials of each row with a fixed shuffle tree.
 __device__ __forceinline__ void block_rows_total(const float* wsum, float* out, int B) {
   cbar();
-  if ((int)threadIdx.x < B) {
-    float s = 0.f;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
 #pragma unroll 1
-    for (int w = 0; w < NW; ++w) s += wsum[w * MAX_B + threadIdx.x];
-    out[threadIdx.x] = s;
+    for (int b = 0; b < B; ++b) {
+      float s = lane < NW ? wsum[lane * MAX_B + b] : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) out[b] = s;
+    }
   }
   cbar();
 }
@@ -1813,6 +1818,19 @@ __device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
     const int nq4 = qd / 4, nk4 = kd / 4;
     const int total4 = nq4 + (own_new ? nk4 + HD / 4 : 0);
     float sq = 0.f, sk = 0.f;
+    // the norm gains of this thread's first rotation pair, in flight with the
+    // slab loads below
+    constexpr int H2 = HD / 2;
+    float qg1 = 0.f, qg2 = 0.f, kg1 = 0.f, kg2 = 0.f;
+    if (tid < GQ * H2) {
+      const int h = tid / H2, i = tid - h * H2, row = (g * GQ + h) * HD;
+      qg1 = __ldg(d.qnorm + row + i);
+      qg2 = __ldg(d.qnorm + row + i + H2);
+    }
+    if (own_new && tid < H2) {
+      kg1 = __ldg(d.knorm + g * HD + tid);
+      kg2 = __ldg(d.knorm + g * HD + tid + H2);
+    }
     constexpr int JU = 4;
 #pragma unroll 1
     for (int c0 = tid; c0 < total4; c0 += JU * NT) {
@@ -1873,28 +1891,30 @@ __device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
       wq[NW + warp] = sk;
     }
     cbar();
-    if (tid == 0) {
-      float a = 0.f, c = 0.f;
-#pragma unroll 1
-      for (int w = 0; w < NW; ++w) {
-        a += wq[w];
-        c += wq[NW + w];
+    if (tid < 32) {  // fixed shuffle tree over the warps' sums
+      float a = tid < NW ? wq[tid] : 0.f, c = tid < NW ? wq[NW + tid] : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
       }
-      rd[32] = rsqrtf(a / float(qd) + L.eps);
-      rd[33] = rsqrtf(c / float(kd) + L.eps);
+      if (tid == 0) {
+        rd[32] = rsqrtf(a / float(qd) + L.eps);
+        rd[33] = rsqrtf(c / float(kd) + L.eps);
+      }
     }
     cbar();
     const float rq = rd[32], rk = rd[33];
     const int pos = posb()[bq];
     const double* fr = rope_f(d.type);
     const float ms = d.type ? L.mscale1 : L.mscale0;
-    constexpr int H2 = HD / 2;
 #pragma unroll 1
     for (int idx = tid; idx < GQ * H2; idx += NT) {
       const int h = idx / H2, i = idx - h * H2;
       const int row = (g * GQ + h) * HD;
-      const float x1 = q[h * HD + i] * rq * d.qnorm[row + i];
-      const float x2 = q[h * HD + i + H2] * rq * d.qnorm[row + i + H2];
+      const bool first = idx == tid;
+      const float x1 = q[h * HD + i] * rq * (first ? qg1 : d.qnorm[row + i]);
+      const float x2 = q[h * HD + i + H2] * rq * (first ? qg2 : d.qnorm[row + i + H2]);
       float c, s;
       rope_cs(pos, fr[i], ms, c, s);
       q[h * HD + i] = (x1 * c - x2 * s) * qscale;
@@ -1903,8 +1923,8 @@ __device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
     if (own_new) {
       if (tid < H2) {
         const int i = tid;
-        const float x1 = kraw[i] * rk * d.knorm[g * HD + i];
-        const float x2 = kraw[i + H2] * rk * d.knorm[g * HD + i + H2];
+        const float x1 = kraw[i] * rk * kg1;
+        const float x2 = kraw[i + H2] * rk * kg2;
         float c, s;
         rope_cs(pos, fr[i], ms, c, s);
         kn[i] = f32_to_bf16(x1 * c - x2 * s);
@@ -1959,10 +1979,10 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
   for (int idx = tid; idx < GQ * HD; idx += NT) {
     const int h = idx / HD, dd = idx - h * HD;
     float M = -INFINITY;
-#pragma unroll 1
+#pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, wp[w * ATT_PW + h * (HD + 2) + HD]);
     float ls = 0.f, os = 0.f;
-#pragma unroll 1
+#pragma unroll
     for (int w = 0; w < NW; ++w) {
       const float e = exp2f(wp[w * ATT_PW + h * (HD + 2) + HD] - M);
       ls += e * wp[w * ATT_PW + h * (HD + 2) + HD + 1];
