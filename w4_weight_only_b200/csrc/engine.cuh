@@ -2009,81 +2009,45 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
   }
   cbar();
   if (!flags()[1]) return;
-  // The pieces c0..c1 merge in one round of loads: warp w takes query head
-  // w % GQ and the w / GQ-th share of the pieces; every lane reads the maxima
-  // of all pieces (one piece per lane) while the loads of its share's outputs
-  // (four dims per lane), maxima and denominators are already in flight.  The
-  // shares then add up in shared memory in a fixed order.  CTA c0 filed its
-  // piece in its second slot (the segment is its last), the others in their
-  // first.
-  constexpr int DPL = HD / 32;  // dims per lane
-  constexpr int PB = 8;         // pieces per load batch
-  const int nparts = NW / GQ;
-  float* red_ws = sm_at<float>(SM_APW);  // [warp][lane][DPL + 1]; the warp partials are consumed
-  const int h = warp % GQ, part = warp / GQ;
-  const bool active = part < nparts;
-  auto piece_of = [&](int c) {
-    return L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
-  };
-  if (active) {
-    const int np = c1 - c0 + 1, per = (np + nparts - 1) / nparts;
-    const int p0 = c0 + part * per, p1 = min(c1 + 1, p0 + per);
-    float acc[DPL], Lsum = 0.f;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-    // first batch of this share in flight before the maxima
-    float ov[PB][DPL], mv[PB], lv[PB];
-    auto load_batch = [&](int cb) {
+  // The pieces c0..c1 merge with one round of loads per batch of PB pieces:
+  // every output (head h, dim dd) has a thread that loads the batch's maxima,
+  // denominators and outputs together and folds them in piece order.  CTA c0
+  // filed its piece in its second slot (the segment is its last), the others
+  // in their first.
+  constexpr int PB = 24;
+  const int np = c1 - c0 + 1;
+#pragma unroll 1
+  for (int o = tid; o < GQ * HD; o += NT) {
+    const int h = o / HD, dd = o - h * HD;
+    float M = -INFINITY, acc = 0.f, Ls = 0.f;
+#pragma unroll 1
+    for (int cb = 0; cb < np; cb += PB) {
+      float mv[PB], lv[PB], ov[PB];
 #pragma unroll
       for (int j = 0; j < PB; ++j) {
-        const bool ok = cb + j < p1;
-        const float* pc = piece_of(ok ? cb + j : c0);
+        const bool ok = cb + j < np;
+        const int c = ok ? c0 + cb + j : c0;
+        const float* pc = L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
         mv[j] = ok ? __ldcg(pc + HD) : -INFINITY;
         lv[j] = ok ? __ldcg(pc + HD + 1) : 0.f;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) ov[j][e] = ok ? __ldcg(pc + lane * DPL + e) : 0.f;
+        ov[j] = ok ? __ldcg(pc + dd) : 0.f;
       }
-    };
-    load_batch(p0);
-    float M = -INFINITY;
-#pragma unroll 1
-    for (int c = c0 + lane; c <= c1; c += 32) M = fmaxf(M, __ldcg(piece_of(c) + HD));
+      float Mn = M;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-#pragma unroll 1
-    for (int cb = p0; cb < p1; cb += PB) {
-      if (cb != p0) load_batch(cb);
+      for (int j = 0; j < PB; ++j) Mn = fmaxf(Mn, mv[j]);
+      const float rs = exp2f(M - Mn);  // 0 on the first batch (M = -inf)
+      acc *= rs;
+      Ls *= rs;
 #pragma unroll
       for (int j = 0; j < PB; ++j) {
-        const float w = exp2f(mv[j] - M);  // 0 for the padding (-inf)
-        Lsum = fmaf(w, lv[j], Lsum);
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, ov[j][e], acc[e]);
+        const float w = exp2f(mv[j] - Mn);  // 0 for the padding
+        acc = fmaf(w, ov[j], acc);
+        Ls = fmaf(w, lv[j], Ls);
       }
+      M = Mn;
     }
-    float* r = red_ws + (warp * 32 + lane) * (DPL + 1);
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) r[e] = acc[e];
-    r[DPL] = Lsum;
-  }
-  cbar();
-  if (warp < GQ) {
-    float acc[DPL], Lsum = 0.f;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-#pragma unroll 1
-    for (int q = 0; q < nparts; ++q) {
-      const float* r = red_ws + ((q * GQ + warp) * 32 + lane) * (DPL + 1);
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] += r[e];
-      Lsum += r[DPL];
-    }
-    const float inv = 1.f / Lsum;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) {
-      const float v = acc[e] * inv;
-      out[warp * HD + lane * DPL + e] = d.out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
-    }
+    const float v = acc / Ls;
+    out[h * HD + dd] = d.out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
   }
   if (tid == 0) L.seg_ctr[seg] = 0u;
 }
