@@ -2453,25 +2453,27 @@ __device__ __noinline__ void setup(const EngineParams& P) {
   __syncthreads();
 }
 
-// Phase start: descriptor p ready in shared memory, the copy of descriptor
-// p + PD_LEAD under way, rings topped up.
-template <int HD>
-__device__ __forceinline__ void phase_start(int p) {
+// Copy descriptor q from the workspace plan into its shared-memory slot
+// (thread 0).  The plan was written with generic stores by every CTA during
+// setup and is read by the copy engine, so the first copy runs after the
+// first grid barrier and behind one proxy fence.
+__device__ __forceinline__ void pd_fetch(int q) {
+  LC& L = lc();
+  if (q == L.begin + PD_LEAD + 1) fence_proxy_async_all();
+  mbar_expect_tx(pd_bar(q), (uint32_t)sizeof(PD));
+  bulk_g2s(&pd_slot(q), L.plan + q, (uint32_t)sizeof(PD), pd_bar(q));
+}
+// Before the barrier into phase p (thread 0, while the other CTAs finish):
+// descriptor p ready in shared memory and the copy of descriptor p + PD_LEAD
+// under way; the barrier's CTA sync then publishes descriptor p.  The copy
+// for phase begin + 1 waits for the first barrier (see pd_fetch).
+__device__ __forceinline__ void phase_prep(int p) {
   if (threadIdx.x == 0) {
-    LC& L = lc();
-    L.cur_phase = p;
+    const LC& L = lc();
     pd_ready(p, true);
     const int q = p + PD_LEAD;
-    if (q < L.end && q > L.begin + PD_LEAD) {
-      // the plan was written with generic stores during setup and is read by
-      // the copy engine: one proxy fence before its first bulk read
-      if (q == L.begin + PD_LEAD + 1) fence_proxy_async_all();
-      mbar_expect_tx(pd_bar(q), (uint32_t)sizeof(PD));
-      bulk_g2s(&pd_slot(q), L.plan + q, (uint32_t)sizeof(PD), pd_bar(q));
-    }
+    if (q < L.end && q > L.begin + PD_LEAD + 1) pd_fetch(q);
   }
-  cbar();
-  mark(1);
 }
 
 // NW math warps run the phases; warp NW is the copy warp.
@@ -2488,9 +2490,12 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
     if (p != begin) {
       if (!grid_wait(uint32_t(p - begin) * uint32_t(lc().nc))) break;
     }
-    if (threadIdx.x == 0) lc().cur_phase = p;
+    if (threadIdx.x == 0) {
+      lc().cur_phase = p;
+      if (p == begin + 1 && p + PD_LEAD < end) pd_fetch(p + PD_LEAD);
+    }
     mark(0);
-    phase_start<HD>(p);
+    mark(1);
     const PD& d = pd_slot(p);
     const int kind = d.kind;
     if (kind == PK_GEMV_W4 || kind == PK_GEMV_BF16)
@@ -2503,6 +2508,7 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
       argmax_phase(d);
     grid_arrive();
     mark(6);
+    if (p + 1 < end) phase_prep(p + 1);
   }
   cbar();
   if (threadIdx.x == 0) {
