@@ -1966,7 +1966,7 @@ __device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
 template <int HD>
 __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, int nca) {
   const LC& L = lc();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int* st = sst(d.type);
   const int GQ = L.nq / L.nkv;
   const int bq = seg / L.nkv, g = seg % L.nkv;
