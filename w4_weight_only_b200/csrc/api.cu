@@ -178,7 +178,8 @@ static int geo_check(const Geo& g, long long n, long long k, int B) {
   if (g.ns <= 0) return fail(W4A_ERR_SHAPE, "no k-split of %lld x %lld fits shared memory at batch %d", n, k, B);
   const long long upsl = (long long)g.nrb * g.kps;
   for (int c = 0; c < g.nca; ++c) {
-    const long long a = rstart(g.nseg, g.nca, c) * g.kps, b = rstart(g.nseg, g.nca, c + 1) * g.kps;
+    int a, b;
+    gemv_cta_range(g, c, a, b);
     if (a < b && (b - 1) / upsl - a / upsl > 1)
       return fail(W4A_ERR_SHAPE, "%lld x %lld at batch %d needs more k-slabs per CTA than fit", n, k, B);
   }

@@ -89,7 +89,7 @@ inline Geo gemv_geo(long long n, long long k, int kcw, int B, int nb, int nc, in
   Geo g;
   g.nrb = int((n + RB - 1) / RB);
   g.nkc = int(k / kcw);
-  g.ns = g.kps = g.nseg = g.nca = 0;
+  g.ns = g.kps = g.nseg = g.nca = g.aligned = 0;
   const int kmax = choose_kps(g.nkc, kcw, B, nb);
   if (kmax <= 0 || nc <= 0) return g;
   const int ns0 = g.nkc / kmax;
@@ -112,6 +112,16 @@ inline Geo gemv_geo(long long n, long long k, int kcw, int B, int nb, int nc, in
       g.nseg = int(nseg);
       g.nca = int(nca);
     }
+  }
+  // slab-aligned CTA groups when that keeps the busiest CTA's segment count
+  if (g.ns > 1 && g.nca >= g.ns) {
+    const long long per = (g.nseg + g.nca - 1) / g.nca;
+    long long per_al = 0;
+    for (int s = 0; s < g.ns; ++s) {
+      const long long cnt = rstart(g.nca, g.ns, s + 1) - rstart(g.nca, g.ns, s);
+      per_al = per_al > (g.nrb + cnt - 1) / cnt ? per_al : (g.nrb + cnt - 1) / cnt;
+    }
+    if (per_al <= per) g.aligned = 1;
   }
   return g;
 }
@@ -491,12 +501,19 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
 // Ranges
 // ---------------------------------------------------------------------------
 // A GEMV CTA owns whole segments: units [a, b) of the phase order.
-__device__ __forceinline__ void gemv_cta_range(const Geo& g, int cta, int& a, int& b) {
-  if (cta < g.nca) {
+__host__ __device__ inline void gemv_cta_range(const Geo& g, int cta, int& a, int& b) {
+  if (cta >= g.nca) {
+    a = b = 0;
+  } else if (g.aligned) {
+    // CTA group s of slab s: its CTAs share the slab's row blocks
+    int s = 0;
+    while (s + 1 < g.ns && rstart(g.nca, g.ns, s + 1) <= cta) ++s;
+    const int c0 = int(rstart(g.nca, g.ns, s)), cnt = int(rstart(g.nca, g.ns, s + 1)) - c0;
+    a = (s * g.nrb + int(rstart(g.nrb, cnt, cta - c0))) * g.kps;
+    b = (s * g.nrb + int(rstart(g.nrb, cnt, cta - c0 + 1))) * g.kps;
+  } else {
     a = int(rstart(g.nseg, g.nca, cta)) * g.kps;
     b = int(rstart(g.nseg, g.nca, cta + 1)) * g.kps;
-  } else {
-    a = b = 0;
   }
 }
 // A CTA's GEMV units split over its math warps.  Warp w runs on SM

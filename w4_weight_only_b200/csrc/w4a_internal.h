@@ -55,6 +55,9 @@ enum Epi : int { EPI_Y = 0, EPI_Y_SUMSQ = 1, EPI_SILU = 2, EPI_PART = 3 };
 // slabs, segments (= slabs x row blocks) and CTAs used.
 struct Geo {
   int nrb, nkc, kps, ns, nseg, nca;
+  // 1: the CTAs are split into ns groups, one per k-slab, so that no CTA's
+  // segments span two slabs (it stages one slab of x)
+  int aligned;
 };
 
 struct LayerPtrs {
