@@ -227,7 +227,7 @@ static int ws_layout(int B, int nc, const Dims& dm, int attn, int decode, long l
   };
   const size_t qkv = (size_t)(dm.nq + 2 * dm.nkv) * dm.hd;
   L->ctl = put(256);
-  L->seg = put((size_t)MAX_SEG * 4);
+  L->seg = put((size_t)2 * MAX_SEG * 4);  // last-arriver counters, then equal-split counters
   L->apart = put(attn ? (size_t)nc * 2 * MAX_GQ * (dm.hd + 2) * 4 : 0);
   L->amax_v = put(decode ? (size_t)nc * B * 4 : 0);
   L->amax_i = put(decode ? (size_t)nc * B * 4 : 0);

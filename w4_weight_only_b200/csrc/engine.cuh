@@ -167,7 +167,7 @@ struct LC {
   int scaled;  // some x row of this phase is range-scaled
   int final_norm;
   int stop;  // the math warps have left the phase loop
-  int pad1;
+  uint32_t seg_target;  // arrivals each equal-split attention segment counter has reached
   uint32_t* ctl;
   uint32_t* seg_ctr;
   float* apart;
@@ -1980,6 +1980,49 @@ __device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
   cbar();
 }
 
+// Outputs [lo, hi) of a split segment (head o / HD, dim o % HD) from the
+// pieces of CTAs c0 .. c0 + np - 1, one round of loads per batch of PB
+// pieces: every output's thread loads the batch's maxima, denominators and
+// values together and folds them in piece order.  CTA c0 filed its piece in
+// its second slot (the segment is its last), the others in their first.
+template <int HD>
+__device__ __forceinline__ void merge_pieces(const LC& L, int c0, int np, int lo, int hi, uint16_t* out, int out_f16) {
+  constexpr int PB = 24;
+#pragma unroll 1
+  for (int o = lo + (int)threadIdx.x; o < hi; o += NT) {
+    const int h = o / HD, dd = o - h * HD;
+    float M = -INFINITY, acc = 0.f, Ls = 0.f;
+#pragma unroll 1
+    for (int cb = 0; cb < np; cb += PB) {
+      float mv[PB], lv[PB], ov[PB];
+#pragma unroll
+      for (int j = 0; j < PB; ++j) {
+        const bool ok = cb + j < np;
+        const int c = ok ? c0 + cb + j : c0;
+        const float* pc = L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
+        mv[j] = ok ? __ldcg(pc + HD) : -INFINITY;
+        lv[j] = ok ? __ldcg(pc + HD + 1) : 0.f;
+        ov[j] = ok ? __ldcg(pc + dd) : 0.f;
+      }
+      float Mn = M;
+#pragma unroll
+      for (int j = 0; j < PB; ++j) Mn = fmaxf(Mn, mv[j]);
+      const float rs = exp2f(M - Mn);  // 0 on the first batch (M = -inf)
+      acc *= rs;
+      Ls *= rs;
+#pragma unroll
+      for (int j = 0; j < PB; ++j) {
+        const float w = exp2f(mv[j] - Mn);  // 0 for the padding
+        acc = fmaf(w, ov[j], acc);
+        Ls = fmaf(w, lv[j], Ls);
+      }
+      M = Mn;
+    }
+    const float v = acc / Ls;
+    out[o] = out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
+  }
+}
+
 template <int HD>
 __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, int nca) {
   const LC& L = lc();
@@ -2019,6 +2062,34 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
   cbar();
   int c0, c1;
   attn_seg_ctas(d.type, seg, nca, c0, c1);
+  const int* am = flags() + 4 + 3 * d.type;
+  if (am[0]) {
+    // Equal split (each CTA in one segment): every CTA of the segment
+    // publishes its piece, waits until all of them have, then merges its
+    // share of the outputs.  The counters only grow during a launch (the
+    // target advances by the pieces per segment each attention phase) and
+    // are cleared when the launch ends.
+    if (tid == 0) {
+      uint32_t* ctr = L.seg_ctr + MAX_SEG + seg;
+      const uint32_t target = L.seg_target + uint32_t(c1 - c0 + 1);
+      red_release_add(ctr, 1u);
+      int ok = 1;
+      const long long t0 = clock64();
+      while (ld_acquire(ctr) < target) {
+        if (clock64() - t0 > WAIT_CYCLES) {
+          set_error(EW_BARRIER_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+      flags()[1] = ok;
+    }
+    cbar();
+    if (!flags()[1]) return;
+    const int np = c1 - c0 + 1, j = blockIdx.x - c0, nout = GQ * HD;
+    merge_pieces<HD>(L, c0, np, nout * j / np, nout * (j + 1) / np, out, d.out_f16);
+    return;
+  }
   if (tid == 0) {
     // release this CTA's piece, acquire the others' (last arriver)
     const uint32_t old = atom_add_acqrel(L.seg_ctr + seg, 1u);
@@ -2026,46 +2097,7 @@ __device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, in
   }
   cbar();
   if (!flags()[1]) return;
-  // The pieces c0..c1 merge with one round of loads per batch of PB pieces:
-  // every output (head h, dim dd) has a thread that loads the batch's maxima,
-  // denominators and outputs together and folds them in piece order.  CTA c0
-  // filed its piece in its second slot (the segment is its last), the others
-  // in their first.
-  constexpr int PB = 24;
-  const int np = c1 - c0 + 1;
-#pragma unroll 1
-  for (int o = tid; o < GQ * HD; o += NT) {
-    const int h = o / HD, dd = o - h * HD;
-    float M = -INFINITY, acc = 0.f, Ls = 0.f;
-#pragma unroll 1
-    for (int cb = 0; cb < np; cb += PB) {
-      float mv[PB], lv[PB], ov[PB];
-#pragma unroll
-      for (int j = 0; j < PB; ++j) {
-        const bool ok = cb + j < np;
-        const int c = ok ? c0 + cb + j : c0;
-        const float* pc = L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
-        mv[j] = ok ? __ldcg(pc + HD) : -INFINITY;
-        lv[j] = ok ? __ldcg(pc + HD + 1) : 0.f;
-        ov[j] = ok ? __ldcg(pc + dd) : 0.f;
-      }
-      float Mn = M;
-#pragma unroll
-      for (int j = 0; j < PB; ++j) Mn = fmaxf(Mn, mv[j]);
-      const float rs = exp2f(M - Mn);  // 0 on the first batch (M = -inf)
-      acc *= rs;
-      Ls *= rs;
-#pragma unroll
-      for (int j = 0; j < PB; ++j) {
-        const float w = exp2f(mv[j] - Mn);  // 0 for the padding
-        acc = fmaf(w, ov[j], acc);
-        Ls = fmaf(w, lv[j], Ls);
-      }
-      M = Mn;
-    }
-    const float v = acc / Ls;
-    out[h * HD + dd] = d.out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
-  }
+  merge_pieces<HD>(L, c0, c1 - c0 + 1, 0, GQ * HD, out, d.out_f16);
   if (tid == 0) L.seg_ctr[seg] = 0u;
 }
 
@@ -2325,6 +2357,7 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     L.scaled = 0;
     L.final_norm = P.final_norm;
     L.stop = 0;
+    L.seg_target = 0u;
     L.ctl = P.ws.ctl;
     L.seg_ctr = P.ws.seg_ctr;
     L.apart = P.ws.apart;
@@ -2517,8 +2550,13 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
     const int kind = d.kind;
     if (kind == PK_GEMV_W4 || kind == PK_GEMV_BF16)
       gemv_phase<NB, HD>(d);
-    else if (kind == PK_ATTN)
+    else if (kind == PK_ATTN) {
       attn_phase<HD>(d);
+      // every CTA advances the equal-split counters' target (see attn_combine);
+      // segments of one CTA (meff = 1) are not split and touch no counter
+      const int* am = flags() + 4 + 3 * d.type;
+      if (threadIdx.x == 0 && am[0] && am[2] > 1) lc().seg_target += uint32_t(am[2]);
+    }
     else if (kind == PK_REDUCE)
       reduce_phase(d);
     else
@@ -2536,6 +2574,8 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
     if (int(old) == lc().nc - 1) {
       ctl[0] = 0u;
       ctl[1] = 0u;
+#pragma unroll 1
+      for (int i = 0; i < MAX_SEG; ++i) lc().seg_ctr[MAX_SEG + i] = 0u;  // equal-split attention counters
       __threadfence();
     }
   }

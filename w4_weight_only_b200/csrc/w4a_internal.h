@@ -74,7 +74,7 @@ struct LayerPtrs {
 // Workspace carve-up (device pointers), filled on the host.
 struct Workspace {
   uint32_t* ctl;        // [0] barrier, [1] exit, [2] error word, [3] argmax counter
-  uint32_t* seg_ctr;    // attention arrival counters [MAX_SEG]
+  uint32_t* seg_ctr;    // attention arrival counters [2][MAX_SEG]
   float* apart;         // attention pieces [NC][2][MAX_GQ * (HD + 2)]
   float* amax_val;      // argmax pieces [NC][B]
   int32_t* amax_idx;
