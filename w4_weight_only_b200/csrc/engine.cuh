@@ -295,7 +295,7 @@ __device__ __forceinline__ void mark(int slot) {
 
 // cos / sin of the rotation angle pos * f, times the attention factor: the
 // angle is formed and reduced to [-pi, pi] in fp64, then evaluated in fp32.
-__device__ __noinline__ float2 rope_cs2(int pos, double f, float ms) {
+__device__ __forceinline__ float2 rope_cs2(int pos, double f, float ms) {
   const double a = double(pos) * f;
   const double r = a - 6.283185307179586 * rint(a * 0.15915494309189535);
   float sn, cs;
@@ -581,7 +581,7 @@ __device__ __forceinline__ void attn_seg_ctas(int type, int seg, int nca, int& c
 // copied at the start of phase q - PD_LEAD (the k-th copy into its slot
 // completes mbarrier phase k).  `block`: wait for a copy under way (bounded);
 // else only test it.
-__device__ __noinline__ bool pd_ready(int q, bool block) {
+__device__ __forceinline__ bool pd_ready(int q, bool block) {
   const LC& L = lc();
   if (q <= L.begin + PD_LEAD) return true;
   if (*reinterpret_cast<const volatile int*>(&L.cur_phase) < q - PD_LEAD) return false;  // copy not issued yet
@@ -599,7 +599,7 @@ __device__ __noinline__ bool pd_ready(int q, bool block) {
 }
 
 // Position cursor c at the first unit of warp w in phase q.
-__device__ __noinline__ void cur_enter(Cursor* c, int q, int w) {
+__device__ __forceinline__ void cur_enter(Cursor* c, int q, int w) {
   const LC& L = lc();
   c->p = q;
   c->i = c->end = 0;
@@ -642,7 +642,7 @@ __device__ __noinline__ void cur_enter(Cursor* c, int q, int w) {
 
 // Move c to warp w's next unit at or after its position (possibly in a later
 // phase).  Stops on CUR_DONE or CUR_WAIT.
-__device__ __noinline__ void cur_normalize(Cursor* c, int w) {
+__device__ __forceinline__ void cur_normalize(Cursor* c, int w) {
   const LC& L = lc();
 #pragma unroll 1
   for (;;) {
@@ -865,7 +865,7 @@ __device__ __noinline__ void copy_warp() {
 // ---------------------------------------------------------------------------
 // Grid barrier
 // ---------------------------------------------------------------------------
-__device__ __noinline__ bool grid_wait(uint32_t target) {
+__device__ __forceinline__ bool grid_wait(uint32_t target) {
   if (threadIdx.x == 0) {
     const LC& L = lc();
     int ok = 1;
@@ -965,7 +965,7 @@ __device__ __noinline__ F8 slab_sum8v(const float* p, size_t sstride, int ns) {
 struct F16v {
   float v[16];
 };
-__device__ __noinline__ F16v slab_sum8x2(const float* p0, const float* p1, bool has1, size_t sstride, int ns) {
+__device__ __forceinline__ F16v slab_sum8x2(const float* p0, const float* p1, bool has1, size_t sstride, int ns) {
   F16v r;
   float* v = r.v;
 #pragma unroll
@@ -1023,7 +1023,7 @@ __device__ __forceinline__ void cvt16(bool f16, const uint4& u, float (&v)[8]) {
 // hold one 128-group, whose sum (of the stored, rounded values) and max |x|
 // they reduce here.  Warp-uniform: every lane calls it.
 template <int NB>
-__device__ __noinline__ void put8(bool valid, int bb, int kl0, int xrow_b, F8 vv, bool f16, float scale,
+__device__ __forceinline__ void put8(bool valid, int bb, int kl0, int xrow_b, F8 vv, bool f16, float scale,
                                   bool track_max) {
   const float* v = vv.v;
   const int lane = threadIdx.x & 31;
@@ -1158,7 +1158,7 @@ __device__ __forceinline__ void resid8(const float (&v)[8], const float (&xr)[8]
 
 // Stage x for the CTA's k-range [kbase, kbase + klen) of a GEMV phase.
 template <int NB>
-__device__ __noinline__ void stage_x(const PD& d, int kbase, int klen) {
+__device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
   LC& L = lc();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = L.B, dm = L.d;
@@ -1580,7 +1580,7 @@ __device__ __forceinline__ Acc<NB> acc_of(const float (&a)[NB][4]) {
 }
 
 template <int NB>
-__device__ __noinline__ void emit_rows(const PD& d, int s, int rb, Acc<NB> A, int B, int lane) {
+__device__ __forceinline__ void emit_rows(const PD& d, int s, int rb, Acc<NB> A, int B, int lane) {
   const float (&v)[NB][4] = A.v;
   const int g = lane >> 2, t = lane & 3;
   if (d.epi == EPI_SILU) {
@@ -1652,7 +1652,7 @@ __device__ __forceinline__ void seg_done(const PD& d, int s, int rb, bool whole,
 // Segments of this CTA split between warps: the warp holding a segment's last
 // unit sums its pieces in warp order and emits the rows.
 template <int NB>
-__device__ __noinline__ void cta_combine(const PD& d) {
+__device__ __forceinline__ void cta_combine(const PD& d) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int4 c = ctab(d.gi, warp)[2];
   if (c.x == 0) return;
@@ -1812,7 +1812,7 @@ __device__ __noinline__ void reduce_phase(const PD& d) {
 // Attention
 // ---------------------------------------------------------------------------
 template <int HD>
-__device__ __noinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
+__device__ __forceinline__ void attn_prologue(const PD& d, int seg, bool own_new) {
   const LC& L = lc();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bq = seg / L.nkv, g = seg % L.nkv;
@@ -2024,7 +2024,7 @@ __device__ __forceinline__ void merge_pieces(const LC& L, int c0, int np, int lo
 }
 
 template <int HD>
-__device__ __noinline__ void attn_combine(const PD& d, int seg, int a, int b, int nca) {
+__device__ __forceinline__ void attn_combine(const PD& d, int seg, int a, int b, int nca) {
   const LC& L = lc();
   const int tid = threadIdx.x;
   const int* st = sst(d.type);
