@@ -1156,13 +1156,13 @@ __device__ __forceinline__ void resid8(const float (&v)[8], const float (&xr)[8]
   for (int i = 0; i < 8; ++i) x[i] = fmaf(v[i] * r, g[i], xr[i]);
 }
 
-// Stage x for the CTA's k-range [kbase, kbase + klen) of a GEMV phase.
+// Scratch a GEMV phase's staging starts from: group sums, row maxima, row
+// scales, per-warp sums of squares.  Runs between phases (after the CTA's
+// arrival at the grid barrier, before the wait's CTA sync), so the staging
+// itself starts with loads.
 template <int NB>
-__device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
-  LC& L = lc();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int B = L.B, dm = L.d;
-  const bool f16 = (d.kind == PK_GEMV_W4);
+__device__ __forceinline__ void stage_reset() {
+  const int tid = threadIdx.x;
   float* rd = red();
   float* xsm = sm_at<float>(sm_xsum(NB));
 #pragma unroll 1
@@ -1171,10 +1171,21 @@ __device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
     reinterpret_cast<uint32_t*>(rd + 32)[tid] = 0u;
     rd[48 + tid] = 1.f;
   }
-  float* wsum = sm_at<float>(sm_wsp(NB));  // [NW][MAX_B] per-warp sums of squares
+  float* wsum = sm_at<float>(sm_wsp(NB));
   if (tid < NW * MAX_B) wsum[tid] = 0.f;
-  if (tid == 0) L.scaled = 0;
-  cbar();
+  if (tid == 0) lc().scaled = 0;
+}
+
+// Stage x for the CTA's k-range [kbase, kbase + klen) of a GEMV phase.  The
+// scratch was reset by stage_reset.
+template <int NB>
+__device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
+  LC& L = lc();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = L.B, dm = L.d;
+  const bool f16 = (d.kind == PK_GEMV_W4);
+  float* rd = red();
+  float* wsum = sm_at<float>(sm_wsp(NB));  // [NW][MAX_B] per-warp sums of squares (reset by stage_reset)
   const int xrow_b = klen * 2 + 64;
   const bool has_out = (d.xdst != nullptr || d.dump != nullptr);
   const int nout = B * dm / 8;
@@ -2535,6 +2546,8 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
     return;
   }
   const int begin = lc().begin, end = lc().end;
+  stage_reset<NB>();
+  cbar();
 #pragma unroll 1
   for (int p = begin; p < end; ++p) {
     if (p != begin) {
@@ -2563,6 +2576,7 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
       argmax_phase(d);
     grid_arrive();
     mark(6);
+    stage_reset<NB>();  // the phase's shared scratch is free once every warp has arrived
     if (p + 1 < end) phase_prep(p + 1);
   }
   cbar();
