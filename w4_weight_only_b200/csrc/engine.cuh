@@ -2252,12 +2252,19 @@ __device__ __noinline__ void argmax_phase(const PD& d) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int V = L.vocab, B = L.B;
   const int r0 = int(rstart(V, L.nc, blockIdx.x)), r1 = int(rstart(V, L.nc, blockIdx.x + 1));
-  if (d.lpart != nullptr) {
+  const bool pick = L.next_token != nullptr;
+  float* rv = red();
+  int* ri = reinterpret_cast<int*>(red() + 32);
+  // one pass over the CTA's rows: the logit (sum of the lm_head slabs, or
+  // the finished row) and this CTA's greedy candidate (ties: lowest index)
 #pragma unroll 1
-    for (int bq = 0; bq < B; ++bq)
+  for (int bq = 0; bq < B; ++bq) {
+    float best = -INFINITY;
+    int bi = 0x7fffffff;
 #pragma unroll 1
-      for (int r = r0 + tid; r < r1; r += NT) {
-        float y = 0.f;
+    for (int r = r0 + tid; r < r1; r += NT) {
+      float y = 0.f;
+      if (d.lpart != nullptr) {
 #pragma unroll 1
         for (int s0 = 0; s0 < d.lns; s0 += 4) {
           float t[4];
@@ -2269,24 +2276,15 @@ __device__ __noinline__ void argmax_phase(const PD& d) {
             if (s0 + i < d.lns) y += t[i];
         }
         L.logits[(size_t)bq * V + r] = y;
+      } else if (pick) {
+        y = __ldcg(L.logits + (size_t)bq * V + r);
       }
-    cbar();
-  }
-  if (L.next_token == nullptr) return;
-  float* rv = red();
-  int* ri = reinterpret_cast<int*>(red() + 32);
-#pragma unroll 1
-  for (int bq = 0; bq < B; ++bq) {
-    float best = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll 1
-    for (int r = r0 + tid; r < r1; r += NT) {
-      const float v = __ldcg(L.logits + (size_t)bq * V + r);
-      if (v > best || (v == best && r < bi)) {
-        best = v;
+      if (y > best || (y == best && r < bi)) {
+        best = y;
         bi = r;
       }
     }
+    if (!pick) continue;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, best, o);
@@ -2315,27 +2313,39 @@ __device__ __noinline__ void argmax_phase(const PD& d) {
     }
     cbar();
   }
-  if (tid == 0) {
-    const uint32_t old = atom_add_acqrel(L.ctl + 3, 1u);
-    if (int(old) == L.nc - 1) {
+  if (!pick || warp != 0) return;
+  // the last CTA to file its candidates picks the token: warp 0 reduces
+  // the CTAs' candidates (lanes over CTAs, then shuffles)
+  int last = 0;
+  if (lane == 0) last = int(atom_add_acqrel(L.ctl + 3, 1u)) == L.nc - 1;
+  last = __shfl_sync(0xffffffffu, last, 0);
+  __syncwarp();  // orders the lanes' reads after lane 0's acquire
+  if (!last) return;
 #pragma unroll 1
-      for (int bq = 0; bq < B; ++bq) {
-        float bb = -INFINITY;
-        int bbi = 0x7fffffff;
+  for (int bq = 0; bq < B; ++bq) {
+    float bb = -INFINITY;
+    int bbi = 0x7fffffff;
 #pragma unroll 1
-        for (int c = 0; c < L.nc; ++c) {
-          const float v = __ldcg(L.amax_val + (size_t)c * B + bq);
-          const int i = __ldcg(L.amax_idx + (size_t)c * B + bq);
-          if (v > bb || (v == bb && i < bbi)) {
-            bb = v;
-            bbi = i;
-          }
-        }
-        L.next_token[bq] = (bbi == 0x7fffffff) ? 0 : bbi;
+    for (int c = lane; c < L.nc; c += 32) {
+      const float v = __ldcg(L.amax_val + (size_t)c * B + bq);
+      const int i = __ldcg(L.amax_idx + (size_t)c * B + bq);
+      if (v > bb || (v == bb && i < bbi)) {
+        bb = v;
+        bbi = i;
       }
-      L.ctl[3] = 0u;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bb, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bbi, o);
+      if (ov > bb || (ov == bb && oi < bbi)) {
+        bb = ov;
+        bbi = oi;
+      }
+    }
+    if (lane == 0) L.next_token[bq] = (bbi == 0x7fffffff) ? 0 : bbi;
   }
+  if (lane == 0) L.ctl[3] = 0u;
 }
 
 // ---------------------------------------------------------------------------
