@@ -1210,11 +1210,16 @@ __device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
     for (int i = 0; i < 8; ++i) v0[i] = v1[i] = x0[i] = x1[i] = g0[i] = g1[i] = 0.f;
     // pass 1: branch sums (and, for up to two chunks, residual and gains in flight together)
     if (two) {
-      if (h0) {
+      // the residual and gain only where this CTA uses x: its k-range and
+      // its share of the residual copy (all of it for the final norm); the
+      // sums of squares need every branch value
+      const bool u0 = fin || (k00 >= kbase && k00 < kbase + klen) || (c0 >= o0 && c0 < o1);
+      const bool u1 = fin || (k01 >= kbase && k01 < kbase + klen) || (c1 >= o0 && c1 < o1);
+      if (h0 && u0) {
         load8f(d.xres + (size_t)b0 * dm + k00, x0, false);
         load8f(d.gain + k00, g0, true);
       }
-      if (h1) {
+      if (h1 && u1) {
         load8f(d.xres + (size_t)b1 * dm + k01, x1, false);
         load8f(d.gain + k01, g1, true);
       }
@@ -2550,7 +2555,11 @@ __device__ __forceinline__ void phase_prep(int p) {
 // NW math warps run the phases; warp NW is the copy warp.
 template <int NB, int HD>
 __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constant__ EngineParams P) {
+  const uint64_t t_entry = P.trace != nullptr ? globaltimer() : 0ull;
   setup(P);
+  // trace: the CTA's start in stamp 7 of the first phase (setup = stamp 0 - stamp 7)
+  if (threadIdx.x == 0 && P.trace != nullptr && P.phase_begin < P.trace_phases)
+    P.trace[((size_t)P.phase_begin * P.nc + blockIdx.x) * 8 + 7] = t_entry;
   if (threadIdx.x >= NT) {
     copy_warp<HD>();
     return;

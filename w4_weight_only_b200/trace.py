@@ -113,6 +113,11 @@ def main():
     print(f"step: {untraced:.3f} ms untraced, {e0.elapsed_time(e1):.3f} ms traced "
           f"({cfg.n_layers} layers, batch {B}, ctx {ctx})")
     print("per phase kind: span, then median/max over CTAs of each step, us")
+    t0 = t.double()
+    ok = (t0[0, :, 7] > 0) & (t0[0, :, 0] > 0)
+    if ok.any():
+        su = (t0[0, ok, 0] - t0[0, ok, 7]) / 1000
+        print(f"setup (CTA start to its first phase): median {su.median().item():.2f} us, max {su.max().item():.2f} us")
     print(f"{'kind':8s} {'n':>3s} {'span':>7s} " + " ".join(f"{s:>13s}" for s in STEPS))
     for k, (n, span, st) in phase_table(t, cfg.n_layers).items():
         print(f"{k:8s} {n:3d} {span:7.2f} " + " ".join(f"{a:6.2f}/{b:6.2f}" for a, b in st))
