@@ -116,3 +116,73 @@ def test_tiny_seq_offset_and_determinism(tiny_pair):
     pos3 = torch.tensor([40, 41, 42], dtype=torch.int32, device="cuda")
     c, _ = P.gpu.decode_step(kv, toks3, pos3)
     assert float((c[2] - a[0]).abs().max()) <= 1e-3
+
+
+# ---------------------------------------------------------------------------
+# The persistent engine at the full OLMo-3-32B shape, in the launch
+# configuration the benchmark times (all SMs, the 32B geometries, the
+# equal-split attention): a sliding-window layer and a full-attention (YaRN)
+# layer, the bf16 lm_head over 100,278 logits and the greedy pick, against
+# the oracle.  The oracle quantizes and dequantizes the layers itself.
+# ---------------------------------------------------------------------------
+def _cfg32_two_layers():
+    c = wc.olmo3_32b(2)
+    c.full_layers = [False, True]
+    return c
+
+
+@pytest.fixture(scope="module")
+def pair32(built_lib, cuda):
+    return Pair(_cfg32_two_layers(), seed=5, gen_device="cuda", oracle_cache=True)
+
+
+def _fill_kv(P, kv, okv, lens):
+    cfg = P.cfg
+    for l in range(cfg.n_layers):
+        for b, n in enumerate(lens):
+            k, v = synth.kv_rows(P.seed, l, b, cfg.n_kv_heads, n, cfg.head_dim, "cuda")
+            kv.write(l, b, 0, k, v)
+            okv.fill(l, b, 0, k.to("cpu").to(torch.float64).numpy(), v.to("cpu").to(torch.float64).numpy())
+
+
+def test_engine_32b_shape_batch1_ctx4096(pair32):
+    """The benchmark's step at batch 1 with 4,096 cached positions: hidden
+    state after each layer, all logits and the greedy token."""
+    from w4_weight_only_b200 import api
+    P = pair32
+    cfg = P.cfg
+    ctx = 4096
+    kv = api.KVCache(cfg, 1, ctx + 16)  # capacity: a multiple of 16 slots
+    okv = om.OracleKV(P.ocfg, 1, ctx + 16)
+    _fill_kv(P, kv, okv, [ctx])
+    tok = int(synth.token_ids(P.seed, 1, cfg.vocab, "cpu")[0])
+    dump = torch.zeros((cfg.n_layers + 1, 1, cfg.d_model), dtype=torch.float32, device="cuda")
+    lg, nxt = P.gpu.decode_step(kv, torch.tensor([tok], dtype=torch.int32, device="cuda"),
+                                torch.tensor([ctx], dtype=torch.int32, device="cuda"), hidden_dump=dump)
+    ref_lg, ref_hid = om.decode_step(P.oracle, okv, [tok], [ctx])
+    P.gpu.check()
+    _check_step(cfg, lg[0].cpu().numpy(), dump[:, 0].cpu().numpy(), ref_lg[0], ref_hid[:, 0], "32b b1")
+    top2 = np.sort(ref_lg[0])[-2:]
+    if top2[1] - top2[0] >= 2 * LOGIT_TOL:
+        assert int(nxt[0]) == int(om.argmax(ref_lg[0]))
+
+
+def test_engine_32b_shape_batch16_ragged(pair32):
+    """Sixteen sequences with different cached lengths (the two-tile batch
+    path of the engine, unequal attention segments) in one step."""
+    from w4_weight_only_b200 import api
+    P = pair32
+    cfg = P.cfg
+    lens = [5 + 61 * b for b in range(16)]
+    cap = (max(lens) + 16) // 16 * 16
+    kv = api.KVCache(cfg, 16, cap)
+    okv = om.OracleKV(P.ocfg, 16, cap)
+    _fill_kv(P, kv, okv, lens)
+    toks = [int(t) for t in synth.token_ids(P.seed + 1, 16, cfg.vocab, "cpu")]
+    dump = torch.zeros((cfg.n_layers + 1, 16, cfg.d_model), dtype=torch.float32, device="cuda")
+    lg, nxt = P.gpu.decode_step(kv, torch.tensor(toks, dtype=torch.int32, device="cuda"),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), hidden_dump=dump)
+    ref_lg, ref_hid = om.decode_step(P.oracle, okv, toks, lens)
+    P.gpu.check(16)
+    for b in range(16):
+        _check_step(cfg, lg[b].cpu().numpy(), dump[:, b].cpu().numpy(), ref_lg[b], ref_hid[:, b], f"32b seq {b}")
