@@ -239,6 +239,7 @@ constexpr int ATT_PW = MAX_GQ * (128 + 2);                // floats of one warp'
 constexpr int SM_APW = SM_XS;                             // warp partials [NW][ATT_PW]
 constexpr int SM_QF = SM_XS + NW * ATT_PW * 4;            // q fragments (4 KB)
 constexpr int SM_ASCR = SM_QF + 4096;                     // k, v rows fp32 [2][128], sums [2][NW]
+static_assert(NW * 64 * 3 * 4 <= NW * ATT_PW * 4, "piece-merge scratch inside the warp partials");
 static_assert(SM_ASCR + 2 * 128 * 4 + 2 * NW * 4 <= SM_XS + X_REGION, "attention scratch");
 
 extern __shared__ __align__(128) uint8_t w4a_smem[];
@@ -2039,6 +2040,79 @@ __device__ __forceinline__ void merge_pieces(const LC& L, int c0, int np, int lo
   }
 }
 
+// The same merge for a short output range (hi - lo <= 64, one to two
+// outputs per lane): warp w takes pieces w, w + NW, ..., so the pieces'
+// loads spread over all warps; each warp folds its pieces per output into
+// shared memory and the range's threads fold the NW warp results in warp
+// order.  Every thread of the CTA calls it (one CTA sync).
+template <int HD>
+__device__ __forceinline__ void merge_pieces_warps(const LC& L, int c0, int np, int lo, int hi, uint16_t* out,
+                                                   int out_f16) {
+  constexpr int RMAX = 64, PB = 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* sc = sm_at<float>(SM_APW);  // [NW][RMAX][3]: maximum, weighted sum, denominator
+#pragma unroll
+  for (int ob = 0; ob < RMAX; ob += 32) {
+    const int o = lo + ob + lane;
+    const bool live = o < hi;
+    const int oc = live ? o : lo;
+    const int h = oc / HD, dd = oc - h * HD;
+    float M = -INFINITY, acc = 0.f, Ls = 0.f;
+#pragma unroll 1
+    for (int j0 = warp; j0 < np; j0 += PB * NW) {
+      float mv[PB], lv[PB], vv[PB];
+#pragma unroll
+      for (int i = 0; i < PB; ++i) {
+        const int j = j0 + i * NW;
+        const bool ok = live && j < np;
+        const int c = c0 + (j < np ? j : 0);
+        const float* pc = L.apart + ((size_t)c * 2 + (c == c0 ? 1 : 0)) * ATT_PW + h * (HD + 2);
+        mv[i] = ok ? __ldcg(pc + HD) : -INFINITY;
+        lv[i] = ok ? __ldcg(pc + HD + 1) : 0.f;
+        vv[i] = ok ? __ldcg(pc + dd) : 0.f;
+      }
+      float Mn = M;
+#pragma unroll
+      for (int i = 0; i < PB; ++i) Mn = fmaxf(Mn, mv[i]);
+      if (Mn != -INFINITY) {
+        const float rs = exp2f(M - Mn);  // 0 while M = -inf
+        acc *= rs;
+        Ls *= rs;
+#pragma unroll
+        for (int i = 0; i < PB; ++i) {
+          const float w = exp2f(mv[i] - Mn);  // 0 for the padding
+          acc = fmaf(w, vv[i], acc);
+          Ls = fmaf(w, lv[i], Ls);
+        }
+        M = Mn;
+      }
+    }
+    float* e = sc + (warp * RMAX + ob + lane) * 3;
+    e[0] = M;
+    e[1] = acc;
+    e[2] = Ls;
+  }
+  cbar();
+  const int t = threadIdx.x;
+  if (t < hi - lo) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sc[(w * RMAX + t) * 3]);
+    float acc = 0.f, Ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float* e = sc + (w * RMAX + t) * 3;
+      if (e[0] != -INFINITY) {
+        const float f = exp2f(e[0] - M);
+        acc = fmaf(f, e[1], acc);
+        Ls = fmaf(f, e[2], Ls);
+      }
+    }
+    const float v = acc / Ls;
+    out[lo + t] = out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
+  }
+}
+
 template <int HD>
 __device__ __forceinline__ void attn_combine(const PD& d, int seg, int a, int b, int nca) {
   const LC& L = lc();
@@ -2103,7 +2177,11 @@ __device__ __forceinline__ void attn_combine(const PD& d, int seg, int a, int b,
     cbar();
     if (!flags()[1]) return;
     const int np = c1 - c0 + 1, j = blockIdx.x - c0, nout = GQ * HD;
-    merge_pieces<HD>(L, c0, np, nout * j / np, nout * (j + 1) / np, out, d.out_f16);
+    const int lo = nout * j / np, hi = nout * (j + 1) / np;
+    if (hi - lo <= 64)  // the same for every thread of the CTA
+      merge_pieces_warps<HD>(L, c0, np, lo, hi, out, d.out_f16);
+    else
+      merge_pieces<HD>(L, c0, np, lo, hi, out, d.out_f16);
     return;
   }
   if (tid == 0) {
