@@ -40,9 +40,9 @@ NOMINAL_HBM_GBS = 8000.0
 # DRAM traffic of the engine from ncu (profiles/w4a_engine_decode_4layer_full.md):
 # 4- and 8-layer launches of the benchmark model at ctx 4096 give the bytes per
 # layer and the fixed part; valid only for the engine source they were taken on.
-TRAFFIC_ENGINE_SHA = "5e8aaa7f1478d44c"
-TRAFFIC_FIXED = 1.03330e9
-TRAFFIC_PER_LAYER = 0.271389e9
+TRAFFIC_ENGINE_SHA = "14ce3df424fd41f0"
+TRAFFIC_FIXED = 1.03557e9
+TRAFFIC_PER_LAYER = 0.270234e9
 
 
 def measured_traffic(n_layers: int):
