@@ -39,16 +39,28 @@ NOMINAL_HBM_GBS = 8000.0
 
 # DRAM traffic of the engine from ncu (profiles/w4a_engine_decode_4layer_full.md):
 # 4- and 8-layer launches of the benchmark model at ctx 4096 give the bytes per
-# layer and the fixed part; valid only for the engine source they were taken on.
-TRAFFIC_ENGINE_SHA = "14ce3df424fd41f0"
+# layer and the fixed part; valid only for the engine code they were taken on
+# (its hash with comments and whitespace stripped).
+TRAFFIC_ENGINE_CODE = "6ff7029416b7a011"
 TRAFFIC_FIXED = 1.03557e9
 TRAFFIC_PER_LAYER = 0.270234e9
 
 
-def measured_traffic(n_layers: int):
+def engine_code_hash(text: str) -> str:
+    """sha256 prefix of the engine source without // comments and whitespace:
+    edits of comments or layout do not change the kernel."""
     import hashlib
+    import re
+    kept = []
+    for line in text.splitlines():
+        i = line.find("//")
+        kept.append(re.sub(r"\s+", "", line if i < 0 else line[:i]))
+    return hashlib.sha256("".join(kept).encode()).hexdigest()[:16]
+
+
+def measured_traffic(n_layers: int):
     src = ROOT / "w4_weight_only_b200" / "csrc" / "engine.cuh"
-    if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:16] != TRAFFIC_ENGINE_SHA:
+    if not src.exists() or engine_code_hash(src.read_text()) != TRAFFIC_ENGINE_CODE:
         return None
     return int(TRAFFIC_FIXED + n_layers * TRAFFIC_PER_LAYER)
 

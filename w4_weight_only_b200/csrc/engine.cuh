@@ -1,15 +1,17 @@
 // The persistent decode engine.
 //
-// One CTA per SM, 16 warps.  A launch runs a list of phases (decode: per layer
-// QKV GEMV, GQA attention, O GEMV, gate/up GEMV, down GEMV; then lm_head and
-// argmax) separated by grid-wide barriers.  Every warp streams its own
-// contiguous range of ~4 KB "units" (16 weight rows x 512 int4 columns, 16
-// rows x 128 bf16 columns, or 8 keys of K and V) from HBM into a two-slot ring
-// of shared memory with bulk asynchronous copies completing on mbarriers, and
-// refills a slot with its next unit as soon as it has copied the unit into
-// registers.  The stream runs across phase boundaries: weights and old KV
-// entries do not depend on the activations, so the copies for phase p + 1
-// are in flight while the CTA waits at the barrier that ends phase p.
+// One CTA per SM, 16 warps: 15 math warps and a copy warp.  A launch runs a
+// list of phases (decode: per layer QKV GEMV, GQA attention, O GEMV, gate/up
+// GEMV, down GEMV; then lm_head and argmax) separated by grid-wide barriers.
+// Every math warp consumes its own contiguous range of ~4 KB "units" (16
+// weight rows x 512 int4 columns, 16 rows x 128 bf16 columns, or 8 keys of K
+// and V) from a two-slot ring of shared memory; lane w of the copy warp walks
+// math warp w's unit stream and issues each unit's bulk asynchronous copy
+// (completing on an mbarrier) as soon as its slot is free, which the math
+// warp signals once it has copied the unit into registers.  The stream runs
+// across phase boundaries: weights and old KV entries do not depend on the
+// activations, so the copies for phase p + 1 are in flight while the CTA
+// waits at the barrier that ends phase p.
 //
 // Phase descriptors (what a phase reads, computes and writes) are built on the
 // device at launch, in parallel by one thread per phase, into a table in the
@@ -36,12 +38,18 @@
 // (computing any RMSNorm over the whole vector itself).  Every sum has a fixed
 // order, so results are bit-reproducible.
 //
-// Attention splits each (sequence, KV head) over CTAs by keys; the last CTA to
-// arrive on a segment's counter merges the pieces in CTA order (no waiting).
+// Attention splits each (sequence, KV head) over CTAs by keys.  When every
+// segment has the same number of CTAs, each CTA posts its piece, waits on the
+// segment's counter and merges its share of the segment's outputs; otherwise
+// the last CTA to arrive merges the whole segment (no waiting).  Pieces are
+// folded in a fixed order.
 //
-// Nothing here lives in per-thread local memory: state that outlives a
-// function (ring cursors, descriptors, launch constants) is kept in shared
-// memory, and the hot loops keep theirs in registers.
+// State that outlives a function (ring cursors, descriptors, launch
+// constants, unit tables) is kept in shared memory; the hot loops keep theirs
+// in registers and touch no local memory.  The helpers on the phase
+// boundaries and the copy warp's cursor walk are inlined: a call to a
+// non-inlined device function there costs far more than its body.  The
+// phase bodies, the launch setup and the rare paths stay out of line.
 #pragma once
 #include <float.h>
 #include <math.h>
