@@ -186,3 +186,24 @@ def test_engine_32b_shape_batch16_ragged(pair32):
     P.gpu.check(16)
     for b in range(16):
         _check_step(cfg, lg[b].cpu().numpy(), dump[:, b].cpu().numpy(), ref_lg[b], ref_hid[:, b], f"32b seq {b}")
+
+
+def test_engine_32b_shape_batch4_ragged(pair32):
+    """Batch 4 at the full shape, ragged cached lengths: the geometry changes
+    with the batch (the down projection in nine k-slabs)."""
+    from w4_weight_only_b200 import api
+    P = pair32
+    cfg = P.cfg
+    lens = [4096, 3001, 100, 2049]
+    cap = (max(lens) + 16) // 16 * 16
+    kv = api.KVCache(cfg, 4, cap)
+    okv = om.OracleKV(P.ocfg, 4, cap)
+    _fill_kv(P, kv, okv, lens)
+    toks = [int(t) for t in synth.token_ids(P.seed + 2, 4, cfg.vocab, "cpu")]
+    dump = torch.zeros((cfg.n_layers + 1, 4, cfg.d_model), dtype=torch.float32, device="cuda")
+    lg, nxt = P.gpu.decode_step(kv, torch.tensor(toks, dtype=torch.int32, device="cuda"),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), hidden_dump=dump)
+    ref_lg, ref_hid = om.decode_step(P.oracle, okv, toks, lens)
+    P.gpu.check(4)
+    for b in range(4):
+        _check_step(cfg, lg[b].cpu().numpy(), dump[:, b].cpu().numpy(), ref_lg[b], ref_hid[:, b], f"32b b4 seq {b}")
