@@ -141,7 +141,7 @@ def _fill_kv(P, kv, okv, lens):
     for l in range(cfg.n_layers):
         for b, n in enumerate(lens):
             k, v = synth.kv_rows(P.seed, l, b, cfg.n_kv_heads, n, cfg.head_dim, "cuda")
-            kv.write(l, b, 0, k, v)
+            kv.fill_history(l, b, k, v)
             okv.fill(l, b, 0, k.to("cpu").to(torch.float64).numpy(), v.to("cpu").to(torch.float64).numpy())
 
 
@@ -207,3 +207,25 @@ def test_engine_32b_shape_batch4_ragged(pair32):
     P.gpu.check(4)
     for b in range(4):
         _check_step(cfg, lg[b].cpu().numpy(), dump[:, b].cpu().numpy(), ref_lg[b], ref_hid[:, b], f"32b b4 seq {b}")
+
+
+def test_engine_32b_shape_batch16_ctx16k(pair32):
+    """Batch 16 at 16,384 cached positions with an independent random cache
+    per sequence: the full layer attends to all of them, the sliding-window
+    layer to the last 4,096 (its 4,096-slot ring has wrapped four times)."""
+    from w4_weight_only_b200 import api
+    P = pair32
+    cfg = P.cfg
+    ctx = 16384
+    lens = [ctx] * 16
+    kv = api.KVCache(cfg, 16, ctx + 16)
+    okv = om.OracleKV(P.ocfg, 16, ctx + 16)
+    _fill_kv(P, kv, okv, lens)
+    toks = [int(t) for t in synth.token_ids(P.seed + 3, 16, cfg.vocab, "cpu")]
+    dump = torch.zeros((cfg.n_layers + 1, 16, cfg.d_model), dtype=torch.float32, device="cuda")
+    lg, nxt = P.gpu.decode_step(kv, torch.tensor(toks, dtype=torch.int32, device="cuda"),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), hidden_dump=dump)
+    ref_lg, ref_hid = om.decode_step(P.oracle, okv, toks, lens)
+    P.gpu.check(16)
+    for b in range(16):
+        _check_step(cfg, lg[b].cpu().numpy(), dump[:, b].cpu().numpy(), ref_lg[b], ref_hid[:, b], f"32b 16k seq {b}")

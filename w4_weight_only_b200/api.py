@@ -256,6 +256,22 @@ class KVCache:
         call("w4a_kv_write", _p(kc), _p(vc), self.batch, cfg.n_kv_heads, cfg.head_dim, self.slots(layer), b, slot0,
              k.shape[1], _p(k), _p(v), _stream())
 
+    def fill_history(self, layer: int, b: int, k: torch.Tensor, v: torch.Tensor):
+        """Store the rows of positions 0 .. n-1 (k, v bf16 [n_kv, n, hd]) of
+        sequence b as the cache holds them: at their own slots in a layer with
+        room for all of them, else (a sliding-window ring) the last `slots`
+        positions at slot position % slots."""
+        n, sl = k.shape[1], self.slots(layer)
+        if n <= sl:
+            self.write(layer, b, 0, k, v)
+            return
+        p0 = n - sl  # first position still held
+        s0 = p0 % sl
+        first = sl - s0  # positions p0 .. p0 + first - 1 go to slots s0 .. sl - 1
+        self.write(layer, b, s0, k[:, p0:p0 + first].contiguous(), v[:, p0:p0 + first].contiguous())
+        if first < sl:
+            self.write(layer, b, 0, k[:, p0 + first:].contiguous(), v[:, p0 + first:].contiguous())
+
     def read(self, layer: int, b: int, slot0: int, n: int):
         cfg = self.cfg
         k = torch.empty((cfg.n_kv_heads, n, cfg.head_dim), dtype=torch.bfloat16, device=self.mem.device)

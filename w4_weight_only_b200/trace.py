@@ -86,7 +86,7 @@ def main():
     for l in range(cfg.n_layers):
         for b in range(B):
             k, v = synth.kv_rows(args.seed, l, b, cfg.n_kv_heads, ctx, cfg.head_dim, "cuda")
-            kv.write(l, b, 0, k, v)
+            kv.fill_history(l, b, k, v)
     tok = torch.ones(B, dtype=torch.int32, device="cuda")
     nxt = torch.zeros(B, dtype=torch.int32, device="cuda")
 
