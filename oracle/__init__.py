@@ -25,6 +25,10 @@ pages that define the method:
 * ``brute``  -- a second, loop-by-loop float64 implementation of one layer on
   tiny shapes, used to pin ``model`` against transposed operands, dropped
   terms and wrong indices.
+* ``sampling`` -- temperature / top-p (nucleus) sampling of one token with the
+  draw passed in (ATLAS model card, "Benchmarks" and "Prompting guide for
+  Think models": temperature 0.6, top-p 0.95); the device side is not built
+  yet.
 
 Parity status per function is stated in each module header.  Every function is
 pinned by a ``-m "not gpu"`` test except the end-to-end logits, whose
