@@ -277,10 +277,32 @@ W4A_API int w4a_prefill(W4AModel* model, const int32_t* tokens, int T, const W4A
  * buf[(p * n_sms + c) * 8 + i]: i = 0 phase start, 1 phase descriptor ready,
  * 2 first input pass done (norm statistics / raw inputs loaded), 3 inputs
  * staged, 4 units done, 5 partial results combined, 6 arrived at the grid
- * barrier, 7 unused.  A stamp the phase does not reach stays as it was.
+ * barrier, 7 unused except in the launch's first phase, where it holds the
+ * CTA's start (before the launch setup).  A stamp the phase does not reach
+ * stays as it was.
  * Phases beyond bytes / (64 * n_sms) are not recorded.  buf = NULL turns
  * tracing off.  Process-wide setting. */
 W4A_API int w4a_trace(void* buf, size_t bytes);
+
+/* ---- sampling --------------------------------------------------------------
+ * Temperature / top-p (nucleus) sampling of one token per row, the sampling
+ * of the ATLAS-OLMo-3-32B-Think-v4 model card ("Benchmarks", "Prompting guide
+ * for Think models": temperature 0.6, top-p 0.95), with the uniform draws
+ * given so that results are reproducible: p = softmax(logits / temperature);
+ * tokens ordered by logit, largest first, equal logits by the lower index;
+ * the nucleus is the shortest prefix of that order whose mass reaches top_p;
+ * the token is the first of the nucleus whose cumulative mass, divided by the
+ * nucleus mass, exceeds u[row].
+ *   logits  fp32 [batch, vocab] (device, finite)
+ *   u       fp32 [batch] (device), each in [0, 1)
+ *   tokens  int32 [batch] (device), written
+ *   ws      device scratch of w4a_sample_workspace_bytes() bytes (no zeroing
+ *           needed), 16-byte aligned
+ * temperature > 0, 0 < top_p <= 1; W4A_ERR_ARG / _SHAPE / _ALIGN /
+ * _WORKSPACE on bad arguments.  Masses are float64 sums in a fixed order. */
+W4A_API int w4a_sample_workspace_bytes(int batch, int vocab, size_t* bytes);
+W4A_API int w4a_sample(const float* logits, int batch, int vocab, float temperature, float top_p,
+               const float* u, int32_t* tokens, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream` and report the device error word of a workspace. */
 W4A_API int w4a_check(const void* ws, size_t ws_bytes, void* stream);

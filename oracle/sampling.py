@@ -10,7 +10,8 @@ the random draw passed in, so that a device implementation can be compared
 token for token:
 
 * p = softmax(z / T) over the vocabulary, in float64;
-* the tokens are ordered by p, largest first, equal p by the lower index;
+* the tokens are ordered by logit z, largest first (the order of p), equal
+  logits by the lower index;
 * the nucleus is the shortest prefix of that order whose mass reaches top_p
   (at least one token);
 * with u uniform in [0, 1), the token is the first of the nucleus whose
@@ -35,19 +36,21 @@ def probabilities(logits, temperature: float) -> np.ndarray:
     return e / np.sum(e)
 
 
-def order(probs) -> np.ndarray:
-    """Token indices by probability, largest first; equal probabilities by index."""
-    p = np.asarray(probs, dtype=np.float64)
-    # lexsort sorts by the last key first: -p descending, then index ascending
-    return np.lexsort((np.arange(p.size), -p))
+def order(keys) -> np.ndarray:
+    """Token indices by key (logit or probability), largest first; equal keys
+    by index."""
+    k = np.asarray(keys, dtype=np.float64)
+    # lexsort sorts by the last key first: -key descending, then index ascending
+    return np.lexsort((np.arange(k.size), -k))
 
 
-def nucleus(probs, top_p: float):
-    """(tokens of the nucleus in sampling order, their probabilities)."""
+def nucleus(probs, top_p: float, keys=None):
+    """(tokens of the nucleus in sampling order, their probabilities); the
+    order follows `keys` (the logits) when given, else the probabilities."""
     if not (0.0 < top_p <= 1.0):
         raise ValueError("top_p must be in (0, 1]")
     p = np.asarray(probs, dtype=np.float64)
-    idx = order(p)
+    idx = order(p if keys is None else keys)
     cum = np.cumsum(p[idx])
     # shortest prefix whose mass reaches top_p; float round-off may leave the
     # full sum a hair below 1, so the whole vocabulary is the fallback
@@ -60,7 +63,7 @@ def sample(logits, temperature: float, top_p: float, u: float) -> int:
     """The token drawn with u in [0, 1)."""
     if not (0.0 <= u < 1.0):
         raise ValueError("u must be in [0, 1)")
-    toks, pk = nucleus(probabilities(logits, temperature), top_p)
+    toks, pk = nucleus(probabilities(logits, temperature), top_p, keys=logits)
     cum = np.cumsum(pk) / np.sum(pk)
     j = int(np.searchsorted(cum, u, side="right"))  # first cumulative mass > u
     return int(toks[min(j, toks.size - 1)])

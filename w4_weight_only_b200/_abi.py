@@ -87,6 +87,8 @@ PROTOTYPES = {
     "w4a_prefill": (_I, [_P, _P, _I, C.POINTER(W4AKVCache), _I, _I, _P, _P, _SZ, _P]),
     "w4a_trace": (_I, [_P, _SZ]),
     "w4a_check": (_I, [_P, _SZ, _P]),
+    "w4a_sample_workspace_bytes": (_I, [_I, _I, C.POINTER(C.c_size_t)]),
+    "w4a_sample": (_I, [_P, _I, _I, C.c_float, C.c_float, _P, _P, _P, _SZ, _P]),
 }
 
 _LIB = None

@@ -395,3 +395,16 @@ class Trace:
 def check(ws: torch.Tensor):
     """Synchronise and raise if the workspace's device error word is set."""
     call("w4a_check", _p(ws), ws.numel(), _stream())
+
+
+def sample(logits: torch.Tensor, temperature: float, top_p: float, u: torch.Tensor) -> torch.Tensor:
+    """Temperature / top-p sampling of one token per row (w4a_sample): logits
+    fp32 [B, V], draws u fp32 [B] in [0, 1); returns int32 [B]."""
+    _need(logits, torch.float32, "logits")
+    _need(u, torch.float32, "u")
+    B, V = logits.shape
+    ws = torch.empty(_size_out("w4a_sample_workspace_bytes", B, V), dtype=torch.uint8, device=logits.device)
+    out = torch.empty((B,), dtype=torch.int32, device=logits.device)
+    call("w4a_sample", _p(logits), B, V, C.c_float(temperature), C.c_float(top_p), _p(u), _p(out), _p(ws), ws.numel(),
+         _stream())
+    return out

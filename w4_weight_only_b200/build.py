@@ -15,7 +15,7 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libw4a.so"
-SOURCES = ["api.cu", "codec.cu"]
+SOURCES = ["api.cu", "codec.cu", "sample.cu"]
 HEADERS = ["engine.cuh", "ptx.cuh", "w4a_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

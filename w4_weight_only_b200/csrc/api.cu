@@ -22,6 +22,7 @@ cudaError_t launch_kv_copy(uint16_t*, const uint16_t*, int, int, int, int, int, 
 cudaError_t launch_qk_prep(int, int, int, int, float, const double*, float, const float*, const float*, const float*,
                            const float*, const float*, const int32_t*, uint16_t*, uint16_t*, uint16_t*, int,
                            cudaStream_t);
+cudaError_t launch_sample(const float*, int, int, float, float, const float*, int32_t*, double*, cudaStream_t);
 }  // namespace w4a
 
 using namespace w4a;
@@ -809,6 +810,27 @@ int w4a_trace(void* buf, size_t bytes) {
   if (buf && !aligned16(buf)) return fail(W4A_ERR_ALIGN, "trace buffer not 16-byte aligned");
   g_trace = buf;
   g_trace_bytes = buf ? bytes : 0;
+  return W4A_OK;
+}
+
+// ---- sampling ------------------------------------------------------------------------
+int w4a_sample_workspace_bytes(int batch, int vocab, size_t* bytes) {
+  if (!bytes) return fail(W4A_ERR_ARG, "null output");
+  if (batch < 1 || vocab < 1) return fail(W4A_ERR_SHAPE, "batch %d vocab %d", batch, vocab);
+  *bytes = (size_t)batch * vocab * sizeof(double);
+  return W4A_OK;
+}
+
+int w4a_sample(const float* logits, int batch, int vocab, float temperature, float top_p, const float* u,
+               int32_t* tokens, void* ws, size_t ws_bytes, void* stream) {
+  if (!logits || !u || !tokens || !ws) return fail(W4A_ERR_ARG, "null pointer");
+  if (batch < 1 || vocab < 1) return fail(W4A_ERR_SHAPE, "batch %d vocab %d", batch, vocab);
+  if (!(temperature > 0.f) || !isfinite(temperature)) return fail(W4A_ERR_ARG, "temperature %g", temperature);
+  if (!(top_p > 0.f && top_p <= 1.f)) return fail(W4A_ERR_ARG, "top_p %g", top_p);
+  if (!aligned16(ws)) return fail(W4A_ERR_ALIGN, "workspace not 16-byte aligned");
+  if (ws_bytes < (size_t)batch * vocab * sizeof(double))
+    return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, (size_t)batch * vocab * sizeof(double));
+  CK(launch_sample(logits, batch, vocab, temperature, top_p, u, tokens, static_cast<double*>(ws), S(stream)));
   return W4A_OK;
 }
 

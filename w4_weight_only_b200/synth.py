@@ -89,3 +89,14 @@ def weight_rows(seed: int, n: int, k: int, rows, device="cpu"):
     """Selected rows of the gemv_case weight (same values, drawn in full on
     ``device``; used when only a sample of rows is checked)."""
     return gemv_case(seed, n, k, 1, device)[0][rows]
+
+
+def logits_rows(seed: int, batch: int, vocab: int, scale: float = 3.0, device="cpu") -> torch.Tensor:
+    """fp32 [batch, vocab] N(0, scale^2): rows of logits for the sampler."""
+    return normal((batch, vocab), device, scale, 0.0, seed, "logits")
+
+
+def uniforms(seed: int, n: int, device="cpu") -> torch.Tensor:
+    """fp32 [n] uniform in [0, 1): the draws of the sampler."""
+    g = _gen(device, seed, "uniform")
+    return torch.rand((n,), generator=g, device=device, dtype=torch.float32)
