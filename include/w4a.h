@@ -193,6 +193,10 @@ W4A_API int w4a_gemv(const W4ATensor* W, const uint16_t* x, int batch, void* out
  *  - The array keeps the last call's contents; each call first clears the
  *    part that must start at zero (the control words: grid barrier counters
  *    and the device error word) on `stream`.
+ *  - Device-side failures (a bounded wait that ran out) land in the array's
+ *    error word like in a workspace: w4a_check(NULL, 0, stream) reads it for
+ *    the current device.  Call it after a call and before the next one on
+ *    that device, since the next call clears the word.
  * Arguments, layouts and the other errors are as for w4a_gemv. */
 #define W4A_NOALLOC_SCRATCH_BYTES 4194304
 W4A_API int w4a_gemv_noalloc(const W4ATensor* W, const uint16_t* x, int batch, void* out, int epilogue,
@@ -304,7 +308,16 @@ W4A_API int w4a_sample_workspace_bytes(int batch, int vocab, size_t* bytes);
 W4A_API int w4a_sample(const float* logits, int batch, int vocab, float temperature, float top_p,
                const float* u, int32_t* tokens, void* ws, size_t ws_bytes, void* stream);
 
-/* Synchronise `stream` and report the device error word of a workspace. */
+/* Synchronise `stream` and report the device error word of a workspace:
+ * W4A_OK, W4A_ERR_TIMEOUT (a bounded wait ran out) or W4A_ERR_KERNEL (a
+ * device-side check failed: a position outside the cache, a bad shape).
+ * ws == NULL reads the fixed scratch of w4a_gemv_noalloc on the current
+ * device instead (ws_bytes is then ignored; W4A_ERR_ARG before the first
+ * w4a_gemv_noalloc call on that device).
+ * Debugging: the environment variable W4A_BARRIER_WAIT_CYCLES, when set to a
+ * positive number of SM cycles at a launch, bounds that launch's waits for
+ * other CTAs (default ~2 s); a wait that runs out yields W4A_ERR_TIMEOUT
+ * here, and the workspace must be zeroed again before its next use. */
 W4A_API int w4a_check(const void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus

@@ -39,15 +39,26 @@ class Pair:
     'cuda' for the 32B shape).  The oracle receives host copies.
     """
 
-    def __init__(self, cfg: wc.Config, seed: int, gen_device: str = "cpu", oracle_cache: bool = True):
+    def __init__(self, cfg: wc.Config, seed: int, gen_device: str = "cpu", oracle_cache: bool = True,
+                 embed_scale: float = 1.0, weight_scale: dict = None):
+        """embed_scale, weight_scale {name: factor}: powers of two that scale
+        the embedding and the named float matrices exactly (range tests)."""
         from w4_weight_only_b200 import api
         self.cfg, self.seed, self.gen_device = cfg, seed, gen_device
         emb, head, fin = synth.embed_head(cfg, seed, gen_device)
+        if embed_scale != 1.0:
+            emb = (emb.float() * embed_scale).to(torch.bfloat16)
         self.emb, self.head, self.fin = emb, head, fin
+        wscale = dict(weight_scale or {})
+
+        def layer_float(l):
+            raw = synth.layer_float(cfg, seed, l, gen_device)
+            for name, f in wscale.items():
+                raw[name] = raw[name] * f
+            return raw
 
         def layer_gpu(l):
-            raw = synth.layer_float(cfg, seed, l, gen_device)
-            return {k: v.to("cuda") for k, v in raw.items()}
+            return {k: v.to("cuda") for k, v in layer_float(l).items()}
 
         self.gpu = api.Model.from_float(cfg, emb.to("cuda"), head.to("cuda"),
                                         fin.to("cuda") if cfg.final_norm else None, layer_gpu)
@@ -55,8 +66,7 @@ class Pair:
         self.ocfg = oracle_config(cfg)
 
         def layer_oracle(l):
-            raw = synth.layer_float(cfg, seed, l, gen_device)
-            return om.OracleLayer.from_float({k: np32(v) for k, v in raw.items()}, cfg.group)
+            return om.OracleLayer.from_float({k: np32(v) for k, v in layer_float(l).items()}, cfg.group)
 
         self.oracle = om.OracleModel(self.ocfg, np64(emb), np64(head), np64(fin) if cfg.final_norm else None,
                                      layer_oracle, cache_dense=oracle_cache)

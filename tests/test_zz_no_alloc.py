@@ -25,7 +25,7 @@ def test_noalloc_equals_workspace_gemv_twice(built_lib, cuda, n, k, batch, epi):
     ref = api.gemv(lin, x, epilogue=epi)
     for _ in range(2):
         got = api.gemv_noalloc(lin, x, epilogue=epi)
-        torch.cuda.synchronize()
+        api.check_noalloc()  # the scratch's error word: no wait ran out
         if epi == abi.EPI_SUMSQ:
             assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
         else:
@@ -45,3 +45,25 @@ def test_noalloc_rejects_oversized_scratch(built_lib, cuda):
     assert e.value.code == abi.ERR_WORKSPACE
     ref = api.gemv(lin, x[:1])
     assert torch.equal(api.gemv_noalloc(lin, x[:1]), ref)
+    api.check_noalloc()
+
+
+def test_noalloc_error_word_is_readable(built_lib, cuda, monkeypatch):
+    """A wait that runs out inside w4a_gemv_noalloc lands in the fixed
+    scratch's error word, which w4a_check(NULL, 0, stream) reads; the next
+    call clears it and succeeds.  (The waits of a CTA for the others are
+    bounded to a few dozen cycles here, so the grid barrier between the GEMV
+    and its reduction cannot complete in time.)"""
+    api, abi = _api()
+    W, x = synth.gemv_case(32, 1024, 1536, 3, "cuda")
+    lin = api.quantize_linear(W)
+    ref = api.gemv(lin, x, epilogue=abi.EPI_SUMSQ)
+    monkeypatch.setenv("W4A_BARRIER_WAIT_CYCLES", "32")
+    api.gemv_noalloc(lin, x, epilogue=abi.EPI_SUMSQ)
+    with pytest.raises(abi.W4AError) as e:
+        api.check_noalloc()
+    assert e.value.code == abi.ERR_TIMEOUT
+    monkeypatch.delenv("W4A_BARRIER_WAIT_CYCLES")
+    got = api.gemv_noalloc(lin, x, epilogue=abi.EPI_SUMSQ)
+    api.check_noalloc()
+    assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])

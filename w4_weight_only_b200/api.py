@@ -397,6 +397,13 @@ def check(ws: torch.Tensor):
     call("w4a_check", _p(ws), ws.numel(), _stream())
 
 
+def check_noalloc():
+    """Synchronise and raise if the error word of the fixed scratch that
+    gemv_noalloc uses on the current device is set (w4a_check with no
+    workspace).  Call it after a gemv_noalloc call and before the next one."""
+    call("w4a_check", None, 0, _stream())
+
+
 def sample(logits: torch.Tensor, temperature: float, top_p: float, u: torch.Tensor) -> torch.Tensor:
     """Temperature / top-p sampling of one token per row (w4a_sample): logits
     fp32 [B, V], draws u fp32 [B] in [0, 1); returns int32 [B]."""

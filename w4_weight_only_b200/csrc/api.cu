@@ -103,8 +103,21 @@ static int phases_per_launch() {
   return v > 0 ? v : 0;
 }
 
-// Runs phases [P.phase_begin, P.phase_end); multi-phase launches are
-// cooperative so that every CTA is resident for the grid barriers.
+// Debugging knob: W4A_BARRIER_WAIT_CYCLES bounds every wait of a CTA for the
+// other CTAs (the grid barrier, the attention segment merge); unset or <= 0
+// keeps the default of ~2 s.  A wait that runs out sets the timeout bit of
+// the workspace's error word and the launch unwinds.
+static long long barrier_wait_cycles() {
+  const char* e = getenv("W4A_BARRIER_WAIT_CYCLES");
+  if (!e || !*e) return 0;
+  const long long v = atoll(e);
+  return v > 0 ? v : 0;
+}
+
+// Runs phases [P.phase_begin, P.phase_end).  Every launch is cooperative, so
+// that all CTAs are resident together: the grid barriers between phases and
+// the attention merge of a segment split over CTAs (which waits for the
+// segment's other CTAs even inside one phase) depend on it.
 static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
   DevInfo* di;
   int rc = device_info(&di);
@@ -124,6 +137,7 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
     }
   }
   P.nc = di->sms;
+  P.wait_bar = barrier_wait_cycles();
   P.trace = nullptr;
   P.trace_phases = 0;
   if (g_trace && P.mode == MODE_DECODE) {
@@ -145,7 +159,7 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = (P.phase_end - P.phase_begin > 1) ? 1 : 0;
+    cfg.numAttrs = 1;
     void* args[] = {&P};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
     if (e != cudaSuccess) {
@@ -835,13 +849,27 @@ int w4a_sample(const float* logits, int batch, int vocab, float temperature, flo
 }
 
 int w4a_check(const void* ws, size_t ws_bytes, void* stream) {
-  if (!ws || ws_bytes < 256) return fail(W4A_ERR_ARG, "null or short workspace");
+  if (!ws) {
+    // the fixed scratch of w4a_gemv_noalloc on the current device
+    int dev = 0;
+    CK(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(W4A_ERR_UNSUPPORTED, "device index %d", dev);
+    {
+      std::lock_guard<std::mutex> lk(g_noalloc_mu);
+      ws = g_noalloc_ptr[dev];
+    }
+    if (!ws) return fail(W4A_ERR_ARG, "no w4a_gemv_noalloc call on device %d yet", dev);
+    ws_bytes = W4A_NOALLOC_SCRATCH_BYTES;
+  }
+  if (ws_bytes < 256) return fail(W4A_ERR_ARG, "short workspace");
   CK(cudaStreamSynchronize(S(stream)));
   uint32_t ctl[4];
   CK(cudaMemcpy(ctl, ws, sizeof(ctl), cudaMemcpyDeviceToHost));
   const uint32_t e = ctl[2];
   if (e & (EW_MBAR_TIMEOUT | EW_BARRIER_TIMEOUT | EW_DRAIN_TIMEOUT))
     return fail(W4A_ERR_TIMEOUT, "device wait timed out (error word 0x%x)", e);
+  if (e & EW_RANGE)
+    return fail(W4A_ERR_KERNEL, "an fp16 intermediate (SwiGLU or attention output) overflowed (error word 0x%x)", e);
   if (e) return fail(W4A_ERR_KERNEL, "device error word 0x%x", e);
   return W4A_OK;
 }

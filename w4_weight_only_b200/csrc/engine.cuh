@@ -176,6 +176,8 @@ struct LC {
   int final_norm;
   int stop;  // the math warps have left the phase loop
   uint32_t seg_target;  // arrivals each equal-split attention segment counter has reached
+  long long wait_bar;   // bound (cycles) on a wait for other CTAs: grid barrier, attention segment
+  int pd_hi;            // last phase whose descriptor copy was issued (thread 0)
   uint32_t* ctl;
   uint32_t* seg_ctr;
   float* apart;
@@ -295,6 +297,17 @@ __device__ __forceinline__ void warp_sync() {
 // barrier over the CTA's warps (named barrier 1)
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
 __device__ __forceinline__ void set_error(uint32_t bits) { atomicOr(lc().ctl + 2, bits); }
+
+// A phase output carried between phases as 16 bits: bf16, or fp16 (the
+// SwiGLU output h and the attention output o of the decode step).  fp16 holds
+// |v| < 65504; a value beyond it (or a NaN) sets EW_RANGE instead of passing
+// an infinity on silently.
+__device__ __forceinline__ uint16_t out16(float v, bool f16) {
+  if (!f16) return f32_to_bf16(v);
+  const uint16_t h = f32_to_f16(v);
+  if ((h & 0x7c00u) == 0x7c00u) set_error(EW_RANGE);
+  return h;
+}
 
 __device__ __forceinline__ void mark(int slot) {
   const LC& L = lc();
@@ -884,7 +897,7 @@ __device__ __forceinline__ bool grid_wait(uint32_t target) {
         ok = 0;
         break;
       }
-      if (clock64() - t0 > WAIT_CYCLES) {
+      if (clock64() - t0 > L.wait_bar) {
         set_error(EW_BARRIER_TIMEOUT);
         ok = 0;
         break;
@@ -1623,7 +1636,7 @@ __device__ __forceinline__ void emit_rows(const PD& d, int s, int rb, Acc<NB> A,
           const int b = nb * 8 + 2 * t + (e & 1), j = (e & 2) ? j1 : j0;
           const float x = v[nb][e];
           const float hv = __fdividef(x, 1.f + __expf(-x)) * u[e];
-          if (b < B) h[(size_t)b * d.ostride + j] = d.out_f16 ? f32_to_f16(hv) : f32_to_bf16(hv);
+          if (b < B) h[(size_t)b * d.ostride + j] = out16(hv, d.out_f16);
         }
       }
     }
@@ -2044,7 +2057,7 @@ __device__ __forceinline__ void merge_pieces(const LC& L, int c0, int np, int lo
       M = Mn;
     }
     const float v = acc / Ls;
-    out[o] = out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
+    out[o] = out16(v, out_f16);
   }
 }
 
@@ -2117,7 +2130,7 @@ __device__ __forceinline__ void merge_pieces_warps(const LC& L, int c0, int np, 
       }
     }
     const float v = acc / Ls;
-    out[lo + t] = out_f16 ? f32_to_f16(v) : f32_to_bf16(v);
+    out[lo + t] = out16(v, out_f16);
   }
 }
 
@@ -2147,7 +2160,7 @@ __device__ __forceinline__ void attn_combine(const PD& d, int seg, int a, int b,
       os += e * wp[w * ATT_PW + h * (HD + 2) + dd];
     }
     if (!split) {
-      out[h * HD + dd] = d.out_f16 ? f32_to_f16(os / ls) : f32_to_bf16(os / ls);
+      out[h * HD + dd] = out16(os / ls, d.out_f16);
     } else {
       piece[h * (HD + 2) + dd] = os;
       if (dd == 0) {
@@ -2174,7 +2187,11 @@ __device__ __forceinline__ void attn_combine(const PD& d, int seg, int a, int b,
       int ok = 1;
       const long long t0 = clock64();
       while (ld_acquire(ctr) < target) {
-        if (clock64() - t0 > WAIT_CYCLES) {
+        if (ld_volatile_u32(L.ctl + 2) != 0u) {  // another CTA gave up: its piece may never come
+          ok = 0;
+          break;
+        }
+        if (clock64() - t0 > L.wait_bar) {
           set_error(EW_BARRIER_TIMEOUT);
           ok = 0;
           break;
@@ -2470,6 +2487,8 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     L.final_norm = P.final_norm;
     L.stop = 0;
     L.seg_target = 0u;
+    L.wait_bar = P.wait_bar > 0 ? P.wait_bar : WAIT_CYCLES;
+    L.pd_hi = P.phase_begin + PD_LEAD;
     L.ctl = P.ws.ctl;
     L.seg_ctr = P.ws.seg_ctr;
     L.apart = P.ws.apart;
@@ -2624,6 +2643,27 @@ __device__ __forceinline__ void pd_fetch(int q) {
   if (q == L.begin + PD_LEAD + 1) fence_proxy_async_all();
   mbar_expect_tx(pd_bar(q), (uint32_t)sizeof(PD));
   bulk_g2s(&pd_slot(q), L.plan + q, (uint32_t)sizeof(PD), pd_bar(q));
+  L.pd_hi = q;
+}
+// Before the CTA exits (thread 0): the descriptor copies still in flight land
+// first.  On the normal path every issued copy has been waited for already;
+// a launch that leaves its phase loop early (a wait ran out) may have issued
+// up to PD_LEAD copies that no phase consumed.  The last PD_SLOTS copies are
+// one per slot, so each one's mbarrier phase is the one to wait for.
+__device__ __noinline__ void pd_drain() {
+  const LC& L = lc();
+  const int q0 = max(L.begin + PD_LEAD + 1, L.pd_hi - PD_SLOTS + 1);
+#pragma unroll 1
+  for (int q = q0; q <= L.pd_hi; ++q) {
+    const uint32_t par = uint32_t((q - L.begin - PD_LEAD - 1) / PD_SLOTS) & 1u;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(pd_bar(q), par)) {
+      if (clock64() - t0 > WAIT_CYCLES) {
+        set_error(EW_DRAIN_TIMEOUT);
+        return;
+      }
+    }
+  }
 }
 // Before the barrier into phase p (thread 0, while the other CTAs finish):
 // descriptor p ready in shared memory and the copy of descriptor p + PD_LEAD
@@ -2686,6 +2726,7 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
   }
   cbar();
   if (threadIdx.x == 0) {
+    pd_drain();
     *reinterpret_cast<volatile int*>(&lc().stop) = 1;
     uint32_t* ctl = lc().ctl;
     __threadfence();

@@ -43,6 +43,7 @@ enum : uint32_t {
   EW_DRAIN_TIMEOUT = 1u << 2,    // in-flight copies did not land before exit
   EW_BAD_SHAPE = 1u << 3,        // device-side shape check failed
   EW_BAD_POS = 1u << 4,          // a position outside the cache
+  EW_RANGE = 1u << 5,            // a value carried in fp16 (SwiGLU or attention output) overflowed
 };
 
 // ---- engine modes / phase kinds --------------------------------------------
@@ -95,6 +96,7 @@ struct EngineParams {
   int mode;
   int phase_begin, phase_end;
   int nc;               // CTAs in the grid
+  long long wait_bar;   // bound in cycles on waits for other CTAs (<= 0: the default, ~2 s)
   // model dims
   int d, nq, nkv, hd, ffn, vocab, window, n_layers;
   float eps;
