@@ -275,7 +275,9 @@ class OracleModel:
     """Embedding, lm_head, final norm gains and a layer provider.
 
     ``layers`` is either a list of OracleLayer or a callable l -> OracleLayer
-    (built on demand, so a 64-layer model never sits dequantized in memory).
+    (built on demand, so a 64-layer model never sits dequantized in memory);
+    a provider may also return the layer already dequantized (the
+    attributes of DenseLayer, as ``fast.dense_layer`` builds them).
     """
 
     def __init__(self, cfg: OracleConfig, embed, lm_head, final_norm, layers,
@@ -291,7 +293,7 @@ class OracleModel:
         if self._dense is not None and l in self._dense:
             return self._dense[l]
         src = self._layers(l) if callable(self._layers) else self._layers[l]
-        d = DenseLayer(src)
+        d = src if hasattr(src, "Wqkv") else DenseLayer(src)   # already dense (oracle.fast)
         if self._dense is not None:
             self._dense[l] = d
         return d
@@ -402,6 +404,52 @@ def prefill(model: OracleModel, kv: OracleKV, tokens, b: int = 0, start_pos: int
         lg, _ = decode_step_one(model, kv, int(t), b, start_pos + i)
         logits = lg
     return logits
+
+
+def prefill_layers(model: OracleModel, kv: OracleKV, tokens, b: int = 0, start_pos: int = 0,
+                   n_layers: Optional[int] = None, keep_hidden: bool = False):
+    """Prefill computed one layer at a time for all T tokens.
+
+    The same numbers as ``prefill`` (sequential decode over positions
+    start_pos + i): token i's key and value at layer l depend only on its own
+    input to layer l, and its attention reads keys of positions <= its own,
+    so every token's projection at layer l can be formed first (one matrix
+    product over the tokens), then each position attends.  Rounding differs
+    from ``prefill`` only by the order of float64 sums.
+
+    Returns (last token's logits, or None when stopping early; the residual
+    after each layer [n + 1, T, d] when keep_hidden, else None)."""
+    cfg = model.cfg
+    n = cfg.n_layers if n_layers is None else n_layers
+    tokens = [int(t) for t in tokens]
+    T = len(tokens)
+    X = model.embed[tokens].copy()                       # [T, d]
+    hidden = np.zeros((n + 1, T, cfg.d_model)) if keep_hidden else None
+    if keep_hidden:
+        hidden[0] = X
+    for l in range(n):
+        L = model.layer(l)
+        full = bool(cfg.full_layers[l])
+        Y = X @ L.Wqkv.T                                 # [T, qkv_dim]
+        Q = np.zeros((T, cfg.n_heads, cfg.head_dim))
+        for i in range(T):
+            pos = start_pos + i
+            q, k = qk_prep(cfg, Y[i, :cfg.q_dim], Y[i, cfg.q_dim:cfg.q_dim + cfg.kv_dim], L.q_norm, L.k_norm,
+                           pos, full)
+            Q[i] = q
+            kv.K[l][b, :, pos] = k
+            kv.V[l][b, :, pos] = Y[i, cfg.q_dim + cfg.kv_dim:].reshape(cfg.n_kv_heads, cfg.head_dim)
+        O = np.zeros((T, cfg.q_dim))
+        for i in range(T):
+            O[i] = gqa_decode(cfg, Q[i], kv.K[l][b], kv.V[l][b], start_pos + i, full).reshape(-1)
+        X = X + rmsnorm(O @ L.Wo.T, L.post_attn_norm, cfg.eps)
+        GU = X @ L.Wgu.T
+        H = silu(GU[:, :cfg.ffn]) * GU[:, cfg.ffn:]
+        X = X + rmsnorm(H @ L.Wd.T, L.post_ffn_norm, cfg.eps)
+        if keep_hidden:
+            hidden[l + 1] = X
+    logits = head(model, X[-1]) if n == cfg.n_layers else None
+    return logits, hidden
 
 
 def decode_step_one(model: OracleModel, kv: OracleKV, token: int, b: int, pos: int):

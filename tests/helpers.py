@@ -40,9 +40,10 @@ class Pair:
     """
 
     def __init__(self, cfg: wc.Config, seed: int, gen_device: str = "cpu", oracle_cache: bool = True,
-                 embed_scale: float = 1.0, weight_scale: dict = None):
+                 embed_scale: float = 1.0, weight_scale: dict = None, oracle_fast: bool = False):
         """embed_scale, weight_scale {name: factor}: powers of two that scale
-        the embedding and the named float matrices exactly (range tests)."""
+        the embedding and the named float matrices exactly (range tests).
+        oracle_fast: the oracle quantizes with oracle.fast (all host cores)."""
         from w4_weight_only_b200 import api
         self.cfg, self.seed, self.gen_device = cfg, seed, gen_device
         emb, head, fin = synth.embed_head(cfg, seed, gen_device)
@@ -66,6 +67,9 @@ class Pair:
         self.ocfg = oracle_config(cfg)
 
         def layer_oracle(l):
+            if oracle_fast:
+                from oracle import fast
+                return fast.dense_layer({k: v.cpu() for k, v in layer_float(l).items()}, cfg.group)
             return om.OracleLayer.from_float({k: np32(v) for k, v in layer_float(l).items()}, cfg.group)
 
         self.oracle = om.OracleModel(self.ocfg, np64(emb), np64(head), np64(fin) if cfg.final_norm else None,

@@ -193,3 +193,40 @@ def test_batched_decode_equals_single_and_prefill_is_sequential():
 
 def test_argmax_ties_to_lowest_index():
     assert model.argmax(np.array([[1.0, 3.0, 3.0, 2.0]]))[0] == 1
+
+
+@pytest.mark.parametrize("start", [0, 5])
+def test_layer_at_a_time_prefill_equals_sequential(start):
+    """prefill_layers (all tokens' projections as one matrix product per
+    layer, then attention per position) gives what sequential decode gives:
+    the last logits, every K/V it wrote, and the residual after each layer of
+    every token; the window of 4 wraps within the 11 tokens, and start > 0
+    continues from a pre-filled history."""
+    cfg = micro_config()
+    m = micro_model(cfg, seed=21)
+    r = np.random.default_rng(22)
+    toks = list(r.integers(0, cfg.vocab, size=11))
+    cap = start + len(toks) + 1
+    kv_a = model.OracleKV(cfg, 2, cap)
+    kv_b = model.OracleKV(cfg, 2, cap)
+    for l in range(cfg.n_layers):
+        hk = r.standard_normal((cfg.n_kv_heads, start, cfg.head_dim))
+        hv = r.standard_normal((cfg.n_kv_heads, start, cfg.head_dim))
+        kv_a.fill(l, 1, 0, hk, hv)
+        kv_b.fill(l, 1, 0, hk, hv)
+    seq_hidden = []
+    for i, t in enumerate(toks):
+        lg_seq, h = model.decode_step_one(m, kv_a, int(t), 1, start + i)
+        seq_hidden.append(h)
+    lg_lay, hid = model.prefill_layers(m, kv_b, toks, b=1, start_pos=start, keep_hidden=True)
+    assert np.allclose(lg_lay, lg_seq, rtol=1e-12, atol=1e-12)
+    assert np.allclose(hid, np.stack(seq_hidden, axis=1), rtol=1e-12, atol=1e-12)
+    for l in range(cfg.n_layers):
+        assert np.allclose(kv_a.K[l], kv_b.K[l], rtol=1e-12, atol=1e-12)
+        assert np.allclose(kv_a.V[l], kv_b.V[l], rtol=1e-12, atol=1e-12)
+    # early stop: the first two layers' residuals only
+    kv_c = model.OracleKV(cfg, 2, cap)
+    for l in range(cfg.n_layers):
+        kv_c.K[l][:], kv_c.V[l][:] = kv_b.K[l], kv_b.V[l]
+    none, hid2 = model.prefill_layers(m, kv_c, toks, b=1, start_pos=start, n_layers=2, keep_hidden=True)
+    assert none is None and np.allclose(hid2, hid[:3], rtol=1e-12, atol=1e-12)
