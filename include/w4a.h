@@ -46,7 +46,7 @@ enum {
   W4A_ERR_UNSUPPORTED = -4,  /* valid request this build does not implement */
   W4A_ERR_CUDA = -5,         /* a CUDA runtime call failed */
   W4A_ERR_WORKSPACE = -6,    /* workspace too small */
-  W4A_ERR_KERNEL = -7,       /* device error word set (bad shape / position) */
+  W4A_ERR_KERNEL = -7,       /* device error word set (bad shape / position / fp16 overflow) */
   W4A_ERR_TIMEOUT = -8       /* a bounded device wait ran out */
 };
 
@@ -268,12 +268,56 @@ W4A_API int w4a_decode_step(W4AModel* model, const int32_t* token_ids, const W4A
                     void* stream);
 
 /* Prefill T tokens (device int32 [T]) of sequence `seq` at positions
- * start_pos .. start_pos + T - 1: defined as T sequential decode steps
- * (model card "Limitations & roadmap": prefill runs token by token through the
- * decode path).  last_logits: fp32 [vocab] of the last token, or NULL. */
+ * start_pos .. start_pos + T - 1: what T sequential decode steps compute
+ * (their K / V written to the cache, the last token's logits), with the
+ * prompt's tokens taken through each layer together (model card
+ * "Limitations & roadmap": batched / tiled prefill, GEMV -> GEMM): the int4
+ * projections as tcgen05 GEMMs on weights expanded to fp16, causal attention
+ * with the sliding window as a flash-attention kernel, the last token as one
+ * decode step.  Prompts of fewer than 9 tokens run token by token.
+ * last_logits: fp32 [vocab] of the last token, or NULL.  ws: device scratch
+ * of w4a_prefill_workspace_bytes(model, T) bytes, zero-filled once before its
+ * first use (its leading part is a decode workspace, whose error word
+ * w4a_check reads).  Full-attention layers need start_pos + T <= max_ctx. */
+W4A_API int w4a_prefill_workspace_bytes(const W4AModel* model, int T, size_t* bytes);
 W4A_API int w4a_prefill(W4AModel* model, const int32_t* tokens, int T, const W4AKVCache* kv,
                 int seq, int start_pos, float* last_logits, void* ws, size_t ws_bytes,
                 void* stream);
+
+/* ---- prompt-time building blocks -------------------------------------------
+ * int4 GEMM for many tokens: out = x . W~^T for x fp16 [M, k] (row-major,
+ * 16-byte aligned rows), W TILED.  The weights are first expanded to fp16
+ * (q - z) * s (rounded to nearest) in the workspace, then multiplied on the
+ * tcgen05 tensor cores with fp32 accumulation.  row_scale: fp32 [M] or NULL;
+ * row m of the product is multiplied by row_scale[m] (an fp16 range scaling
+ * of x undone).  Epilogues: W4A_EPI_NONE out fp32 [M, n]; W4A_EPI_SILU_MUL (W
+ * tiled with row_interleave = 1) out fp16 [M, n / 2] = silu(gate) * up, an
+ * fp16 overflow is reported by w4a_check as W4A_ERR_KERNEL.  ws: device
+ * scratch of w4a_gemm_workspace_bytes() bytes, its first 256 bytes zeroed
+ * once (error word).  Source: model card "Limitations & roadmap" (GEMV ->
+ * GEMM for prefill). */
+W4A_API int w4a_gemm_workspace_bytes(const W4ATensor* W, size_t* bytes);
+W4A_API int w4a_gemm(const W4ATensor* W, const uint16_t* x, int M, const float* row_scale, void* out,
+             int epilogue, void* ws, size_t ws_bytes, void* stream);
+
+/* Causal GQA attention of T prompt tokens at positions start_pos .. start_pos
+ * + T - 1.  q bf16 [T, n_heads, head_dim] (normed and rotated); the prompt's
+ * own keys and values k_new / v_new bf16 [n_kv_heads, T, head_dim] in plain
+ * order; the positions before the prompt from one layer's cache regions
+ * k_cache / v_cache (see W4AKVCache) of a cache of `batch` sequences,
+ * sequence `seq`, which is only read (a ring of `window` slots cannot hold
+ * the windows of two consecutive prompt tokens, so the prompt's rows are
+ * appended to it afterwards).  window == 0: full attention over positions
+ * 0 .. p (slot = position, start_pos + T <= slots); window == slots (a
+ * multiple of 64): the last `window` positions, slot = position % window.
+ * out fp16 [T, n_heads, head_dim] = softmax(q K^T / sqrt(head_dim)) V per
+ * query head h over KV head h / (n_heads / n_kv_heads).  ws: >= 256 device
+ * bytes, zeroed once (error word).  Source: model card "Architecture
+ * deep-dive" (GQA 40/8, SWA 4,096). */
+W4A_API int w4a_attn_prefill(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache, int batch,
+                     int seq, int n_heads, int n_kv_heads, int head_dim, int slots, int window,
+                     int start_pos, int T, const uint16_t* k_new, const uint16_t* v_new, uint16_t* out,
+                     void* ws, size_t ws_bytes, void* stream);
 
 /* Profiling aid (off by default).  With a device buffer set, every later
  * w4a_decode_step / w4a_prefill launch writes, per phase p (5 per layer, then

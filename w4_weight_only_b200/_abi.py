@@ -85,6 +85,10 @@ PROTOTYPES = {
     "w4a_decode_workspace_bytes": (_I, [_P, _I, _SZP]),
     "w4a_decode_step": (_I, [_P, _P, C.POINTER(W4AKVCache), _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "w4a_prefill": (_I, [_P, _P, _I, C.POINTER(W4AKVCache), _I, _I, _P, _P, _SZ, _P]),
+    "w4a_prefill_workspace_bytes": (_I, [_P, _I, _SZP]),
+    "w4a_gemm_workspace_bytes": (_I, [C.POINTER(W4ATensor), _SZP]),
+    "w4a_gemm": (_I, [C.POINTER(W4ATensor), _P, _I, _P, _P, _I, _P, _SZ, _P]),
+    "w4a_attn_prefill": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "w4a_trace": (_I, [_P, _SZ]),
     "w4a_check": (_I, [_P, _SZ, _P]),
     "w4a_sample_workspace_bytes": (_I, [_I, _I, C.POINTER(C.c_size_t)]),

@@ -364,11 +364,22 @@ class Model:
              _p(next_token) if want_next else None, _p(hidden_dump), _p(ws), ws.numel(), _stream())
         return logits, next_token
 
+    def prefill_workspace(self, T: int) -> torch.Tensor:
+        """Zero-filled scratch for w4a_prefill of T tokens (kept and reused
+        while large enough; its leading part is a batch-1 decode workspace)."""
+        out = C.c_size_t(0)
+        call("w4a_prefill_workspace_bytes", self.handle, T, C.byref(out))
+        cur = getattr(self, "_pf_ws", None)
+        if cur is None or cur.numel() < out.value:
+            self._pf_ws = None
+            self._pf_ws = zeros_workspace(out.value, self.embed.device)
+        return self._pf_ws
+
     def prefill(self, kv: KVCache, tokens: torch.Tensor, seq: int = 0, start_pos: int = 0,
                 want_logits: bool = True) -> Optional[torch.Tensor]:
         _need(tokens, torch.int32, "tokens")
         last = torch.empty((self.cfg.vocab,), dtype=torch.float32, device=tokens.device) if want_logits else None
-        ws = self.workspace(1)
+        ws = self.prefill_workspace(tokens.shape[0])
         kvc = kv.c()
         call("w4a_prefill", self.handle, _p(tokens), tokens.shape[0], C.byref(kvc), seq, start_pos, _p(last),
              _p(ws), ws.numel(), _stream())
@@ -377,6 +388,8 @@ class Model:
     def check(self, batch: int = 1):
         ws = self.workspace(batch)
         check(ws)
+        if batch == 1 and getattr(self, "_pf_ws", None) is not None:
+            check(self._pf_ws)
 
 
 class Trace:
@@ -390,6 +403,53 @@ class Trace:
     def stop(self):
         call("w4a_trace", None, 0)
         return self.buf.cpu()
+
+
+def gemm_workspace(lin: W4Linear) -> torch.Tensor:
+    t = lin.tensor()
+    return zeros_workspace(_size_out("w4a_gemm_workspace_bytes", C.byref(t)), lin.blob.device)
+
+
+def gemm(lin: W4Linear, x16: torch.Tensor, epilogue: int = _abi.EPI_NONE, row_scale: Optional[torch.Tensor] = None,
+         ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out = x16 . W~^T for many tokens (w4a_gemm): x16 fp16 [M, k]; fp32
+    [M, n] out, or fp16 [M, n/2] silu(gate) * up with EPI_SILU_MUL."""
+    _need(x16, torch.float16, "x16")
+    M = x16.shape[0]
+    if x16.shape[1] != lin.k:
+        raise ValueError("x has the wrong width")
+    if row_scale is not None:
+        _need(row_scale, torch.float32, "row_scale")
+    if ws is None:
+        ws = gemm_workspace(lin)
+    if out is None:
+        if epilogue == _abi.EPI_SILU_MUL:
+            out = torch.empty((M, lin.n // 2), dtype=torch.float16, device=x16.device)
+        else:
+            out = torch.empty((M, lin.n), dtype=torch.float32, device=x16.device)
+    t = lin.tensor()
+    call("w4a_gemm", C.byref(t), _p(x16), M, _p(row_scale), _p(out), epilogue, _p(ws), ws.numel(), _stream())
+    return out
+
+
+def attn_prefill(q: torch.Tensor, k_region: torch.Tensor, v_region: torch.Tensor, k_new: torch.Tensor,
+                 v_new: torch.Tensor, batch: int, seq: int, slots: int, window: int, start_pos: int,
+                 ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Causal GQA attention of a prompt (w4a_attn_prefill): q bf16 [T, nq,
+    hd], the prompt's keys / values k_new, v_new bf16 [n_kv, T, hd], the
+    history in a layer's cache regions; returns fp16 [T, nq, hd]."""
+    _need(q, torch.bfloat16, "q")
+    _need(k_new, torch.bfloat16, "k_new")
+    _need(v_new, torch.bfloat16, "v_new")
+    T, nq, hd = q.shape
+    n_kv = k_new.shape[0]
+    if ws is None:
+        ws = zeros_workspace(256, q.device)
+    if out is None:
+        out = torch.empty((T, nq, hd), dtype=torch.float16, device=q.device)
+    call("w4a_attn_prefill", _p(q), _p(k_region), _p(v_region), batch, seq, nq, n_kv, hd, slots, window,
+         start_pos, T, _p(k_new), _p(v_new), _p(out), _p(ws), ws.numel(), _stream())
+    return out
 
 
 def check(ws: torch.Tensor):

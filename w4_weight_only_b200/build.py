@@ -15,8 +15,8 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libw4a.so"
-SOURCES = ["api.cu", "codec.cu", "sample.cu"]
-HEADERS = ["engine.cuh", "ptx.cuh", "w4a_internal.h"]
+SOURCES = ["api.cu", "codec.cu", "sample.cu", "prefill.cu"]
+HEADERS = ["engine.cuh", "ptx.cuh", "tc.cuh", "w4a_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-Xptxas", "-v"]

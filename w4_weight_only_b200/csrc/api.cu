@@ -23,6 +23,18 @@ cudaError_t launch_qk_prep(int, int, int, int, float, const double*, float, cons
                            const float*, const float*, const int32_t*, uint16_t*, uint16_t*, uint16_t*, int,
                            cudaStream_t);
 cudaError_t launch_sample(const float*, int, int, float, float, const float*, int32_t*, double*, cudaStream_t);
+cudaError_t launch_dequant_f16(const uint8_t*, int64_t, int64_t, uint16_t*, cudaStream_t);
+cudaError_t launch_gemm_f16(const uint16_t*, const uint16_t*, int, int, int, int, void*, int, const float*, uint32_t*,
+                            int, cudaStream_t);
+cudaError_t launch_flash_prefill(const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*,
+                                 uint16_t*, int, int, int, int, int, int, int, int, uint32_t*, cudaStream_t);
+cudaError_t launch_kv_append(uint16_t*, uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int, int, int, int,
+                             cudaStream_t);
+cudaError_t launch_embed_rows(const int32_t*, int, const uint16_t*, int, int, float*, uint16_t*, float*, uint32_t*,
+                              cudaStream_t);
+cudaError_t launch_resid_rows(const float*, const float*, int, int, float, float*, uint16_t*, float*, cudaStream_t);
+cudaError_t launch_qk_rows(const float*, const float*, const float*, uint16_t*, uint16_t*, uint16_t*, const double*,
+                           float, float, int, int, int, int, int, cudaStream_t);
 }  // namespace w4a
 
 using namespace w4a;
@@ -806,17 +818,208 @@ int w4a_decode_step(W4AModel* m, const int32_t* token_ids, const W4AKVCache* kv,
                        ws_bytes, S(stream));
 }
 
+// ---- dense prefill -------------------------------------------------------------
+// Workspace: the batch-1 decode workspace (its control words, error word
+// included, come first; the prompt's last token runs as a decode step), then
+// the prefill buffers for Tp = T - 1 tokens.
+struct PfLayout {
+  size_t dec, X, X16, scale, Y, Q16, O16, H16, Kn, Vn, W16, total;
+};
+static int pf_layout(const W4AConfig& c, int T, int nc, PfLayout* P) {
+  WsLayout L;
+  int rc = ws_layout(1, nc, dims_of(c), 1, 1, 0, 0, &L);
+  if (rc) return rc;
+  const size_t Tp = T > 1 ? (size_t)(T - 1) : 0;
+  const size_t d = c.d_model, qd = (size_t)c.n_heads * c.head_dim, kvd = (size_t)c.n_kv_heads * c.head_dim;
+  const size_t qkv = qd + 2 * kvd, ffn = c.ffn;
+  size_t off = 0;
+  auto put = [&](size_t bytes) {
+    const size_t o = off;
+    off += al256(bytes);
+    return o;
+  };
+  P->dec = put(L.total);
+  P->X = put(Tp * d * 4);
+  P->X16 = put(Tp * d * 2);
+  P->scale = put(Tp * 4);
+  P->Y = put(Tp * (qkv > d ? qkv : d) * 4);
+  P->Q16 = put(Tp * qd * 2);
+  P->O16 = put(Tp * qd * 2);
+  P->H16 = put(Tp * ffn * 2);
+  P->Kn = put(Tp * kvd * 2);
+  P->Vn = put(Tp * kvd * 2);
+  size_t w = qkv * d;
+  if (d * qd > w) w = d * qd;
+  if (2 * ffn * d > w) w = 2 * ffn * d;
+  if (d * ffn > w) w = d * ffn;
+  P->W16 = put(Tp ? w * 2 : 0);
+  P->total = off;
+  return W4A_OK;
+}
+
+// Prompts shorter than this run token by token through the decode launch
+// (expanding the weights to fp16 costs about as much as a few decode steps).
+static const int PF_MIN_DENSE = 8;
+
+int w4a_prefill_workspace_bytes(const W4AModel* m, int T, size_t* bytes) {
+  if (!m || !bytes) return fail(W4A_ERR_ARG, "null pointer");
+  if (T < 0) return fail(W4A_ERR_SHAPE, "T %d", T);
+  int nc;
+  int rc = nc_for_sizing(&nc);
+  if (rc) return rc;
+  PfLayout P;
+  rc = pf_layout(m->cfg, T - 1 >= PF_MIN_DENSE ? T : 1, nc, &P);
+  if (rc) return rc;
+  *bytes = P.total;
+  return W4A_OK;
+}
+
 int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv, int seq, int start_pos,
                 float* last_logits, void* ws, size_t ws_bytes, void* stream) {
-  if (!m || !tokens) return fail(W4A_ERR_ARG, "null pointer");
+  if (!m || !tokens || !kv || !kv->base || !ws) return fail(W4A_ERR_ARG, "null pointer");
   if (T < 0 || start_pos < 0) return fail(W4A_ERR_SHAPE, "T %d start_pos %d", T, start_pos);
-  const int nl = m->cfg.n_layers;
-  for (int i = 0; i < T; ++i) {
-    const bool last = (i == T - 1) && last_logits != nullptr;
-    const int rc = decode_common(m, tokens + i, kv, seq, 1, nullptr, start_pos + i, last ? last_logits : nullptr,
-                                 nullptr, nullptr, last ? 5 * nl + 2 : 5 * nl, ws, ws_bytes, S(stream));
-    if (rc) return rc;
+  if (T == 0) return W4A_OK;
+  const W4AConfig& c = m->cfg;
+  if (seq < 0 || seq >= kv->batch) return fail(W4A_ERR_SHAPE, "sequence %d outside a cache of %d", seq, kv->batch);
+  if ((long long)start_pos + T > kv->max_ctx && [&] {
+        for (int l = 0; l < c.n_layers; ++l)
+          if (c.full_layers[l]) return true;
+        return false;
+      }())
+    return fail(W4A_ERR_SHAPE, "positions up to %d do not fit a cache of %d", start_pos + T - 1, kv->max_ctx);
+  if (!aligned16(ws)) return fail(W4A_ERR_ALIGN, "workspace not 16-byte aligned");
+  DevInfo* di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  const int nl = c.n_layers;
+  const int Tp = T - 1;
+  const bool dense = Tp >= PF_MIN_DENSE;
+  PfLayout P;
+  rc = pf_layout(c, dense ? T : 1, di->sms, &P);
+  if (rc) return rc;
+  if (ws_bytes < P.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, P.total);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const size_t dec_bytes = P.X - P.dec;
+  cudaStream_t st = S(stream);
+  if (!dense) {
+    for (int i = 0; i < T; ++i) {
+      const bool last = (i == T - 1) && last_logits != nullptr;
+      rc = decode_common(m, tokens + i, kv, seq, 1, nullptr, start_pos + i, last ? last_logits : nullptr, nullptr,
+                         nullptr, last ? 5 * nl + 2 : 5 * nl, b + P.dec, dec_bytes, st);
+      if (rc) return rc;
+    }
+    return W4A_OK;
   }
+  uint32_t* err = reinterpret_cast<uint32_t*>(b + P.dec) + 2;  // the decode workspace's error word
+  float* X = reinterpret_cast<float*>(b + P.X);
+  uint16_t* X16 = reinterpret_cast<uint16_t*>(b + P.X16);
+  float* scale = reinterpret_cast<float*>(b + P.scale);
+  float* Y = reinterpret_cast<float*>(b + P.Y);
+  uint16_t* Q16 = reinterpret_cast<uint16_t*>(b + P.Q16);
+  uint16_t* O16 = reinterpret_cast<uint16_t*>(b + P.O16);
+  uint16_t* H16 = reinterpret_cast<uint16_t*>(b + P.H16);
+  uint16_t* W16 = reinterpret_cast<uint16_t*>(b + P.W16);
+  uint16_t* Kn = reinterpret_cast<uint16_t*>(b + P.Kn);
+  uint16_t* Vn = reinterpret_cast<uint16_t*>(b + P.Vn);
+  const int d = c.d_model, nq = c.n_heads, nkv = c.n_kv_heads, hd = c.head_dim;
+  const int qd = nq * hd, qkv = qd + 2 * nkv * hd, ffn = c.ffn;
+  uint64_t off[MAX_LAYERS];
+  int slots[MAX_LAYERS];
+  size_t total;
+  rc = kv_regions(&c, kv->batch, kv->max_ctx, off, slots, &total);
+  if (rc) return rc;
+  const float eps = float(c.eps);
+  CK(launch_embed_rows(tokens, Tp, m->embed, c.vocab, d, X, X16, scale, err, st));
+  for (int l = 0; l < nl; ++l) {
+    const LayerPtrs& L = m->layers[l];
+    const int full = c.full_layers[l] ? 1 : 0;
+    const int win = full ? 0 : c.window;
+    uint16_t* kc = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(kv->base) + off[l]);
+    uint16_t* vc = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(kc) +
+                                               al256((size_t)kv->batch * nkv * slots[l] * hd * 2));
+    CK(launch_dequant_f16(L.qkv, qkv, d, W16, st));
+    CK(launch_gemm_f16(X16, W16, Tp, qkv, d, 0, Y, qkv, scale, err, di->sms, st));
+    CK(launch_qk_rows(Y, L.q_norm, L.k_norm, Q16, Kn, Vn, m->inv_freq[full], m->ms[full], eps, Tp, nq, nkv, hd,
+                      start_pos, st));
+    CK(launch_flash_prefill(Q16, kc, vc, Kn, Vn, O16, Tp, nq, nkv, hd, slots[l], win, start_pos, seq, err, st));
+    CK(launch_kv_append(kc, vc, Kn, Vn, nkv, hd, slots[l], win, seq, start_pos, Tp, st));
+    CK(launch_dequant_f16(L.o, d, qd, W16, st));
+    CK(launch_gemm_f16(O16, W16, Tp, d, qd, 0, Y, d, nullptr, err, di->sms, st));
+    CK(launch_resid_rows(Y, L.attn_norm, Tp, d, eps, X, X16, scale, st));
+    CK(launch_dequant_f16(L.gu, 2LL * ffn, d, W16, st));
+    CK(launch_gemm_f16(X16, W16, Tp, 2 * ffn, d, 1, H16, ffn, scale, err, di->sms, st));
+    CK(launch_dequant_f16(L.down, d, ffn, W16, st));
+    CK(launch_gemm_f16(H16, W16, Tp, d, ffn, 0, Y, d, nullptr, err, di->sms, st));
+    CK(launch_resid_rows(Y, L.ffn_norm, Tp, d, eps, X, X16, scale, st));
+  }
+  // the last token: one decode step over the cache the prompt has filled
+  // (its K / V appended, the final norm, the lm_head)
+  const bool want = last_logits != nullptr;
+  return decode_common(m, tokens + Tp, kv, seq, 1, nullptr, start_pos + Tp, want ? last_logits : nullptr, nullptr,
+                       nullptr, want ? 5 * nl + 2 : 5 * nl, b + P.dec, dec_bytes, st);
+}
+
+// ---- int4 GEMM (the prefill's projections) ---------------------------------------
+int w4a_gemm_workspace_bytes(const W4ATensor* W, size_t* bytes) {
+  int rc = check_tensor(W);
+  if (rc) return rc;
+  if (!bytes) return fail(W4A_ERR_ARG, "null output");
+  *bytes = 256 + al256((size_t)W->n * W->k * 2);
+  return W4A_OK;
+}
+
+int w4a_gemm(const W4ATensor* W, const uint16_t* x, int M, const float* row_scale, void* out, int epilogue, void* ws,
+             size_t ws_bytes, void* stream) {
+  int rc = check_tensor(W);
+  if (rc) return rc;
+  if (W->layout != W4A_LAYOUT_TILED) return fail(W4A_ERR_ARG, "w4a_gemm takes a tiled tensor (see w4a_tile)");
+  if (!x || !out || !ws) return fail(W4A_ERR_ARG, "null pointer");
+  if (M < 1) return fail(W4A_ERR_SHAPE, "M %d", M);
+  if (epilogue != W4A_EPI_NONE && epilogue != W4A_EPI_SILU_MUL) return fail(W4A_ERR_ARG, "epilogue %d", epilogue);
+  if (epilogue == W4A_EPI_SILU_MUL && !W->row_interleave)
+    return fail(W4A_ERR_ARG, "W4A_EPI_SILU_MUL needs a row-interleaved (gate/up) tensor");
+  if (!aligned16(x) || !aligned16(out) || !aligned16(ws)) return fail(W4A_ERR_ALIGN, "x / out / ws not 16-byte aligned");
+  size_t need = 0;
+  rc = w4a_gemm_workspace_bytes(W, &need);
+  if (rc) return rc;
+  if (ws_bytes < need) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  DevInfo* di;
+  rc = device_info(&di);
+  if (rc) return rc;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  uint16_t* W16 = reinterpret_cast<uint16_t*>(b + 256);
+  uint32_t* err = reinterpret_cast<uint32_t*>(b) + 2;
+  cudaStream_t st = S(stream);
+  CK(launch_dequant_f16(static_cast<const uint8_t*>(W->qweight), W->n, W->k, W16, st));
+  const int silu = epilogue == W4A_EPI_SILU_MUL ? 1 : 0;
+  CK(launch_gemm_f16(x, W16, M, int(W->n), int(W->k), silu, out, silu ? int(W->n / 2) : int(W->n), row_scale, err,
+                     di->sms, st));
+  return W4A_OK;
+}
+
+// ---- attention over a prompt ------------------------------------------------------
+int w4a_attn_prefill(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache, int batch, int seq,
+                     int n_heads, int n_kv_heads, int head_dim, int slots, int window, int start_pos, int T,
+                     const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, void* ws, size_t ws_bytes,
+                     void* stream) {
+  if (!q || !k_cache || !v_cache || !k_new || !v_new || !out || !ws) return fail(W4A_ERR_ARG, "null pointer");
+  if (head_dim != 64 && head_dim != 128) return fail(W4A_ERR_UNSUPPORTED, "head_dim %d", head_dim);
+  if (n_kv_heads < 1 || n_heads % n_kv_heads) return fail(W4A_ERR_SHAPE, "heads %d / kv heads %d", n_heads, n_kv_heads);
+  if (batch < 1 || seq < 0 || seq >= batch || T < 1 || start_pos < 0)
+    return fail(W4A_ERR_SHAPE, "batch %d seq %d T %d start %d", batch, seq, T, start_pos);
+  if (window == 0) {
+    if ((long long)start_pos + T > slots) return fail(W4A_ERR_SHAPE, "positions beyond the %d slots", slots);
+  } else if (window != slots || window % 64) {
+    return fail(W4A_ERR_SHAPE, "window must equal slots and be a multiple of 64");
+  }
+  if (slots < 16 || slots % 16) return fail(W4A_ERR_SHAPE, "slots %d (multiple of 16)", slots);
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || !aligned16(out) || !aligned16(ws) ||
+      !aligned16(k_new) || !aligned16(v_new))
+    return fail(W4A_ERR_ALIGN, "misaligned pointer");
+  if (ws_bytes < 256) return fail(W4A_ERR_WORKSPACE, "workspace %zu < 256 bytes", ws_bytes);
+  uint32_t* err = static_cast<uint32_t*>(ws) + 2;
+  CK(launch_flash_prefill(q, k_cache, v_cache, k_new, v_new, out, T, n_heads, n_kv_heads, head_dim, slots, window,
+                          start_pos, seq, err, S(stream)));
   return W4A_OK;
 }
 

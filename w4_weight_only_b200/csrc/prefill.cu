@@ -1,0 +1,841 @@
+// Dense prefill: the prompt's tokens go through each layer together, so the
+// int4 projections become matrix products (T tokens x K) . W~^T and run on the
+// tcgen05 tensor cores; attention over the prompt is causal (with the sliding
+// window on the SWA layers) and runs as a flash-attention kernel.
+//
+// Per layer (ATLAS-OLMo-3-32B-Think-v4 model card, "Architecture deep-dive";
+// "Limitations & roadmap": batched / tiled prefill, GEMV -> GEMM):
+//   Y  = X16 . Wqkv~^T                     (GEMM, fp32 out)
+//   q, k <- RMSNorm over the whole projection, gains, RoPE / YaRN; K, V -> cache
+//   O  = causal GQA attention              (fp16 out)
+//   A  = O . Wo~^T;   X += RMSNorm(A) g_pa (fp32 residual), X16 = fp16(X)
+//   H  = silu(G) * U, [G; U] = X16 . Wgu~^T (GEMM with the SwiGLU epilogue)
+//   F  = H . Wd~^T;   X += RMSNorm(F) g_pf
+//
+// The int4 weights are expanded, one matrix at a time, to fp16 (q - z) * s
+// rounded to nearest (the product of a 4-bit code and an fp16 scale needs up
+// to 15 significant bits; fp16 keeps 11) in the rows' tiled order, so the
+// gate / up rows alternate and the GEMM epilogue finds each pair side by
+// side.  Activations are fp16 with a per-token power-of-two scale that keeps
+// every row's magnitude below 2^15 (undone in the GEMM epilogue).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+#include "tc.cuh"
+#include "w4a_internal.h"
+
+namespace w4a {
+
+constexpr long long PF_WAIT = 4000000000LL;  // bound on any single wait (~2 s)
+
+__device__ __forceinline__ void pf_error(uint32_t* err, uint32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+__device__ __forceinline__ uint16_t f16_checked(float v, uint32_t* err) {
+  const uint16_t h = f32_to_f16(v);
+  if ((h & 0x7c00u) == 0x7c00u) pf_error(err, EW_RANGE);
+  return h;
+}
+
+// ---------------------------------------------------------------------------
+// int4 tiled units -> fp16 [n, k] (tiled row order)
+// ---------------------------------------------------------------------------
+// One thread per (unit, 32-column slice m, lane): the two code words of
+// k-steps 2m and 2m + 1 hold rows g and g + 8 at columns 32 m + 8 t .. + 7.
+__global__ void dequant_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n, int64_t k,
+                                   uint16_t* __restrict__ out) {
+  const int64_t nkc = k / W4_KC;
+  const int64_t total = (n / RB) * nkc * 16 * 32;
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= total) return;
+  const int lane = int(id & 31);
+  const int m = int((id >> 5) & 15);
+  const int64_t unit = id >> 9;
+  const int64_t rb = unit / nkc, kc = unit - rb * nkc;
+  const int g = lane >> 2, t = lane & 3;
+  const uint8_t* u = tiled + unit * W4_UNIT;
+  const int s0 = 2 * m, s1 = 2 * m + 1;
+  const uint32_t w0 = reinterpret_cast<const uint32_t*>(u + ((s0 >> 2) * 32 + lane) * 16)[s0 & 3];
+  const uint32_t w1 = reinterpret_cast<const uint32_t*>(u + ((s1 >> 2) * 32 + lane) * 16)[s1 & 3];
+  const int grp = m >> 2;
+  const uint16_t* sc = reinterpret_cast<const uint16_t*>(u + 4096);
+  const uint32_t* zw = reinterpret_cast<const uint32_t*>(u + 4224);
+  const float s_lo = half_bits_to_f32(sc[g * 8 + grp * 2 + 0]), s_hi = half_bits_to_f32(sc[g * 8 + grp * 2 + 1]);
+  const int z_lo = int((zw[grp * 2 + 0] >> (4 * g)) & 15u), z_hi = int((zw[grp * 2 + 1] >> (4 * g)) & 15u);
+  // nibble j of a word: row g (+8 when j odd), column offset 2 [j & 2] + [j & 4]
+  uint16_t lo[8], hi[8];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const uint32_t w = e ? w1 : w0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int q = int((w >> (4 * j)) & 15u);
+      const int c = 4 * e + ((j & 2) ? 2 : 0) + ((j & 4) ? 1 : 0);
+      if (j & 1)
+        hi[c] = f32_to_f16(float(q - z_hi) * s_hi);
+      else
+        lo[c] = f32_to_f16(float(q - z_lo) * s_lo);
+    }
+  }
+  const int64_t col = kc * W4_KC + 32 * m + 8 * t;
+  const int64_t r0 = rb * RB + g;
+  uint4 a, b;
+  a.x = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
+  a.y = uint32_t(lo[2]) | (uint32_t(lo[3]) << 16);
+  a.z = uint32_t(lo[4]) | (uint32_t(lo[5]) << 16);
+  a.w = uint32_t(lo[6]) | (uint32_t(lo[7]) << 16);
+  b.x = uint32_t(hi[0]) | (uint32_t(hi[1]) << 16);
+  b.y = uint32_t(hi[2]) | (uint32_t(hi[3]) << 16);
+  b.z = uint32_t(hi[4]) | (uint32_t(hi[5]) << 16);
+  b.w = uint32_t(hi[6]) | (uint32_t(hi[7]) << 16);
+  *reinterpret_cast<uint4*>(out + r0 * k + col) = a;
+  *reinterpret_cast<uint4*>(out + (r0 + 8) * k + col) = b;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM on the tcgen05 tensor cores: D[M, N] = A[M, K] . B[N, K]^T, fp16 in,
+// fp32 accumulation in tensor memory
+// ---------------------------------------------------------------------------
+// Persistent: one CTA per SM walks output tiles of 128 x 256 (M-blocks of one
+// N-column consecutive, so the CTAs running together share the B panels in
+// L2).  Warp 0 (one thread) issues the TMA loads of a 4-stage ring of
+// 64-column K slices, warp 1 (one thread) issues the MMAs (four of K = 16 per
+// slice) and owns the 512 tensor-memory columns (two 256-column accumulators,
+// so the epilogue of a tile overlaps the MMAs of the next), warps 2..5 read
+// an accumulator back (each its own 32 TMEM lanes = 32 rows) and write it.
+constexpr int GM_BM = 128, GM_BN = 256, GM_BK = 64, GM_ST = 4;
+constexpr int GM_A_BYTES = GM_BM * GM_BK * 2;
+constexpr int GM_B_BYTES = GM_BN * GM_BK * 2;
+constexpr int GM_STAGE_BYTES = GM_A_BYTES + GM_B_BYTES;
+constexpr int GM_THREADS = 192;
+constexpr int GM_SMEM = GM_ST * GM_STAGE_BYTES + 256 + 1024;  // ring, barriers, alignment slack
+constexpr uint32_t GM_IDESC = umma_idesc_f16(GM_BM, GM_BN, false);
+
+enum GemmEpi : int { GE_F32 = 0, GE_SILU = 1 };
+
+struct GemmArgs {
+  int M, N, K;
+  int epi;               // GE_F32: out fp32 [M, ldo]; GE_SILU: out fp16 [M, ldo], ldo >= N / 2
+  int ldo;
+  void* out;
+  const float* row_scale;  // [M] or null: row m of the product is multiplied by it
+  uint32_t* err;           // error word
+};
+
+// Bounded wait on an mbarrier phase; gives up (setting the CTA's abort flag
+// and the error word) after ~2 s or when another role has given up.
+__device__ __forceinline__ bool gm_wait(uint64_t* bar, uint32_t par, volatile int* abort_flag, uint32_t* err) {
+  if (mbar_try_wait(bar, par)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, par)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > PF_WAIT) {
+      *abort_flag = 1;
+      pf_error(err, EW_MBAR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(GM_THREADS, 1)
+    gemm_f16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmArgs g) {
+  extern __shared__ uint8_t gm_raw[];
+  // the ring at a 1,024-byte aligned shared address (the 128-byte swizzle's atom)
+  uint8_t* sm = gm_raw + ((1024u - (smem_addr(gm_raw) & 1023u)) & 1023u);
+  uint8_t* sA = sm;
+  uint8_t* sB = sm + GM_ST * GM_A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + GM_ST * GM_STAGE_BYTES);
+  uint64_t* empty = full + GM_ST;
+  uint64_t* tfull = empty + GM_ST;   // accumulator b holds a finished tile
+  uint64_t* tempty = tfull + 2;      // accumulator b has been read back
+  uint64_t* done = tempty + 2;       // every MMA of this CTA has completed
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = (g.M + GM_BM - 1) / GM_BM, nt = (g.N + GM_BN - 1) / GM_BN;
+  const int ntiles = mt * nt, nkb = g.K / GM_BK;
+
+  if (threadIdx.x == 0) {
+#pragma unroll 1
+    for (int s = 0; s < GM_ST; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(tfull + 0, 1);
+    mbar_init(tfull + 1, 1);
+    mbar_init(tempty + 0, 4);
+    mbar_init(tempty + 1, 4);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&tmA);
+    tma_prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tbase, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tbase;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer: TMA loads into the ring ----
+      uint32_t it = 0;
+      bool ok = true;
+#pragma unroll 1
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int mb = t % mt, nb = t / mt;
+#pragma unroll 1
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = int(it % GM_ST);
+          if (it >= GM_ST && !gm_wait(empty + s, ((it / GM_ST) & 1u) ^ 1u, abort_flag, g.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(full + s, GM_STAGE_BYTES);
+          tma_load_2d(sA + s * GM_A_BYTES, &tmA, kb * GM_BK, mb * GM_BM, full + s);
+          tma_load_2d(sB + s * GM_B_BYTES, &tmB, kb * GM_BK, nb * GM_BN, full + s);
+        }
+      }
+      // the loads in flight land before the CTA may exit
+      const uint32_t first = it > uint32_t(GM_ST) ? it - GM_ST : 0u;
+#pragma unroll 1
+      for (uint32_t j = first; j < it; ++j) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(full + (j % GM_ST), (j / GM_ST) & 1u)) {
+          if (clock64() - t0 > PF_WAIT) {
+            pf_error(g.err, EW_DRAIN_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      uint32_t it = 0;
+      int local = 0;
+      bool ok = true;
+#pragma unroll 1
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = uint32_t(local >> 1);
+        if (local >= 2 && !gm_wait(tempty + buf, (use - 1u) & 1u, abort_flag, g.err)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + uint32_t(buf * GM_BN);
+#pragma unroll 1
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = int(it % GM_ST);
+          if (!gm_wait(full + s, (it / GM_ST) & 1u, abort_flag, g.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < GM_BK / 16; ++k) {
+            const uint64_t ad = umma_desc_sw128(sA + s * GM_A_BYTES, uint32_t(k * 32));
+            const uint64_t bd = umma_desc_sw128(sB + s * GM_B_BYTES, uint32_t(k * 32));
+            umma_f16(d, ad, bd, GM_IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(empty + s);
+        }
+        if (ok) umma_commit(tfull + buf);
+      }
+      // every MMA issued has completed before the tensor memory is freed
+      umma_commit(done);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(done, 0u)) {
+        if (clock64() - t0 > PF_WAIT) {
+          pf_error(g.err, EW_DRAIN_TIMEOUT);
+          break;
+        }
+      }
+    }
+  } else {
+    // ---- epilogue: warps 2..5, TMEM lanes 32 (warp % 4) .. + 31 ----
+    const int q = warp & 3;
+    int local = 0;
+#pragma unroll 1
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+      const int mb = t % mt, nb = t / mt;
+      const int buf = local & 1;
+      const uint32_t use = uint32_t(local >> 1);
+      if (!gm_wait(tfull + buf, use & 1u, abort_flag, g.err)) break;
+      tc_fence_after();
+      const int row = mb * GM_BM + q * 32 + lane;
+      const bool live = row < g.M;
+      const float rs = (live && g.row_scale != nullptr) ? g.row_scale[row] : 1.f;
+      const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + uint32_t(buf * GM_BN);
+#pragma unroll 1
+      for (int c = 0; c < GM_BN; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(ta + uint32_t(c), r);
+        tmem_ld_wait();
+        const int col = nb * GM_BN + c;
+        if (!live || col >= g.N) continue;
+        if (g.epi == GE_F32) {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)row * g.ldo + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o[i] = make_float4(__uint_as_float(r[4 * i]) * rs, __uint_as_float(r[4 * i + 1]) * rs,
+                               __uint_as_float(r[4 * i + 2]) * rs, __uint_as_float(r[4 * i + 3]) * rs);
+        } else {
+          // columns alternate gate j, up j: eight SwiGLU outputs
+          uint32_t h[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float g0 = __uint_as_float(r[4 * i]) * rs, u0 = __uint_as_float(r[4 * i + 1]) * rs;
+            const float g1 = __uint_as_float(r[4 * i + 2]) * rs, u1 = __uint_as_float(r[4 * i + 3]) * rs;
+            const float h0 = g0 / (1.f + expf(-g0)) * u0, h1 = g1 / (1.f + expf(-g1)) * u1;
+            h[i] = uint32_t(f16_checked(h0, g.err)) | (uint32_t(f16_checked(h1, g.err)) << 16);
+          }
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) + (size_t)row * g.ldo + col / 2) =
+              make_uint4(h[0], h[1], h[2], h[3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + buf);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Causal GQA flash attention over the prompt (mma.sync, bf16 in, fp32 softmax)
+// ---------------------------------------------------------------------------
+// CTA = 64 consecutive query positions of one query head; 4 warps of 16
+// queries.  Keys stream through shared memory in blocks of 64 positions
+// (double buffered, cp.async).  Positions before the prompt come from the
+// cache, whose rows keep their chunk permutation (16-byte chunk c of slot s at
+// c ^ (s & 7); a block's row r has r = slot mod 8, since window and block
+// start are multiples of 64, so a block never straddles the ring's wrap);
+// the prompt's own keys come from a plain buffer and are permuted the same
+// way on the way in.  The ldmatrix addressing undoes the permutation.  The
+// prompt's keys are not in the cache yet: a ring of `window` slots cannot
+// hold the windows of two consecutive queries, so they are appended after the
+// attention (kv_append_kernel).
+constexpr int FA_BQ = 64, FA_BK = 64, FA_THREADS = 128;
+
+struct FaArgs {
+  const uint16_t* q;    // bf16 [T][nq][hd]
+  const uint16_t* kc;   // this layer's K region [batch][nkv][slots][hd]: positions before the prompt
+  const uint16_t* vc;
+  const uint16_t* kn;   // the prompt's own keys / values, bf16 [nkv][T][hd] in plain order
+  const uint16_t* vn;
+  uint16_t* out;        // fp16 [T][nq][hd]
+  int T, nq, nkv, slots, window, start, seq;
+  float scale_log2;     // log2(e) / sqrt(hd)
+  uint32_t* err;
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int HD>
+__global__ void __launch_bounds__(FA_THREADS) flash_prefill_kernel(const FaArgs a) {
+  constexpr int CH = HD / 8;            // 16-byte chunks per row
+  constexpr int ROWB = HD * 2;          // bytes per key row
+  extern __shared__ __align__(128) uint8_t fa_sm[];
+  uint8_t* Ks = fa_sm;                  // [2][64][HD]
+  uint8_t* Vs = fa_sm + 2 * FA_BK * ROWB;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  const int nqb = (a.T + FA_BQ - 1) / FA_BQ;
+  const int qb = nqb - 1 - int(blockIdx.x);  // the longest rows first
+  const int h = blockIdx.y;
+  const int kvh = h / (a.nq / a.nkv);
+  const int q0 = qb * FA_BQ;                 // first query of the CTA (prompt index)
+  const int p_first = a.start + q0;
+  const int p_last = a.start + min(q0 + FA_BQ, a.T) - 1;
+  const int lo = a.window ? max(0, p_first - a.window + 1) : 0;
+  const int jb0 = lo / FA_BK, jb1 = p_last / FA_BK;  // key blocks [jb0, jb1]
+  const size_t head_base = ((size_t)a.seq * a.nkv + kvh) * a.slots;
+
+  // Q fragments of this warp's 16 queries (rows beyond T are zero)
+  uint32_t qf[HD / 16][4];
+  {
+    const int r0 = q0 + warp * 16 + g8, r1 = r0 + 8;
+#pragma unroll
+    for (int s = 0; s < HD / 16; ++s) {
+      const int c = 16 * s + 2 * t4;
+      auto ld = [&](int r, int cc) -> uint32_t {
+        if (r >= a.T) return 0u;
+        return *reinterpret_cast<const uint32_t*>(a.q + ((size_t)r * a.nq + h) * HD + cc);
+      };
+      qf[s][0] = ld(r0, c);
+      qf[s][1] = ld(r1, c);
+      qf[s][2] = ld(r0, c + 8);
+      qf[s][3] = ld(r1, c + 8);
+    }
+  }
+  const size_t new_base = (size_t)kvh * a.T;
+  const int end = a.start + a.T;
+  auto load_block = [&](int jb, int buf) {
+    uint8_t* kd = Ks + buf * FA_BK * ROWB;
+    uint8_t* vd = Vs + buf * FA_BK * ROWB;
+#pragma unroll 1
+    for (int i = threadIdx.x; i < FA_BK * CH; i += FA_THREADS) {
+      const int r = i / CH, c = i % CH;
+      const int j = jb * FA_BK + r;  // key position
+      if (j >= end) {
+        // beyond the prompt (masked keys): zeros, since a masked key's
+        // weight 0 times a NaN would still poison the sum
+        *reinterpret_cast<uint4*>(kd + r * ROWB + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(vd + r * ROWB + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+      } else if (j >= a.start) {
+        const size_t off = (new_base + (j - a.start)) * HD + c * 8;
+        const int pc = (c ^ (r & 7)) * 16;
+        cp_async16(kd + r * ROWB + pc, a.kn + off);
+        cp_async16(vd + r * ROWB + pc, a.vn + off);
+      } else {
+        const int slot = a.window ? j % a.window : j;
+        const size_t off = ((head_base + slot) * HD) + c * 8;  // stored order = shared-memory order
+        cp_async16(kd + r * ROWB + c * 16, a.kc + off);
+        cp_async16(vd + r * ROWB + c * 16, a.vc + off);
+      }
+    }
+    cp_async_commit();
+  };
+
+  float o[HD / 8][4];
+#pragma unroll
+  for (int j = 0; j < HD / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const int pq0 = a.start + q0 + warp * 16 + g8, pq1 = pq0 + 8;  // positions of this thread's two rows
+
+  load_block(jb0, 0);
+#pragma unroll 1
+  for (int jb = jb0; jb <= jb1; ++jb) {
+    const int buf = (jb - jb0) & 1;
+    if (jb < jb1) {
+      load_block(jb + 1, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint8_t* kb = Ks + buf * FA_BK * ROWB;
+    const uint8_t* vb = Vs + buf * FA_BK * ROWB;
+    // S = Q K^T: 16 queries x 64 keys (8 n-tiles of 8 keys)
+    float sc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+    const int lr = lane & 7, lm = lane >> 3;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int row = 8 * n + lr;
+#pragma unroll
+      for (int s = 0; s < HD / 16; s += 2) {
+        uint32_t k0, k1, k2, k3;
+        ldsm_x4(k0, k1, k2, k3, kb + row * ROWB + (((2 * s + lm) ^ (row & 7)) << 4));
+        mma_16816(sc[n], qf[s][0], qf[s][1], qf[s][2], qf[s][3], k0, k1);
+        mma_16816(sc[n], qf[s + 1][0], qf[s + 1][1], qf[s + 1][2], qf[s + 1][3], k2, k3);
+      }
+    }
+    // mask (causal, window) and online softmax in base 2
+    const int j0 = jb * FA_BK;
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int j = j0 + 8 * n + 2 * t4 + e;
+        const bool v0 = j <= pq0 && (a.window == 0 || pq0 - j < a.window);
+        const bool v1 = j <= pq1 && (a.window == 0 || pq1 - j < a.window);
+        sc[n][e] = v0 ? sc[n][e] * a.scale_log2 : -INFINITY;
+        sc[n][2 + e] = v1 ? sc[n][2 + e] * a.scale_log2 : -INFINITY;
+        mx0 = fmaxf(mx0, sc[n][e]);
+        mx1 = fmaxf(mx1, sc[n][2 + e]);
+      }
+    }
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float ref0 = (mn0 == -INFINITY) ? 0.f : mn0, ref1 = (mn1 == -INFINITY) ? 0.f : mn1;
+    const float al0 = exp2f(m0 - ref0), al1 = exp2f(m1 - ref1);
+    m0 = mn0;
+    m1 = mn1;
+    float s0 = 0.f, s1 = 0.f;
+    uint32_t pf[4][4];  // P as A fragments of the 4 key k-steps
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const float p00 = exp2f(sc[n][0] - ref0), p01 = exp2f(sc[n][1] - ref0);
+      const float p10 = exp2f(sc[n][2] - ref1), p11 = exp2f(sc[n][3] - ref1);
+      s0 += p00 + p01;
+      s1 += p10 + p11;
+      const uint32_t w0 = pack_bf16x2(p00, p01), w1 = pack_bf16x2(p10, p11);
+      pf[n >> 1][(n & 1) ? 2 : 0] = w0;
+      pf[n >> 1][(n & 1) ? 3 : 1] = w1;
+    }
+    l0 = l0 * al0 + s0;
+    l1 = l1 * al1 + s1;
+#pragma unroll
+    for (int j = 0; j < HD / 8; ++j) {
+      o[j][0] *= al0;
+      o[j][1] *= al0;
+      o[j][2] *= al1;
+      o[j][3] *= al1;
+    }
+    // O += P V: 4 k-steps of 16 keys, HD / 8 n-tiles of 8 dims (two per ldmatrix)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int row = 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+      for (int d2 = 0; d2 < HD / 16; ++d2) {
+        uint32_t v0, v1, v2, v3;
+        const int ch = 2 * d2 + (lane >> 4);
+        ldsm_x4_t(v0, v1, v2, v3, vb + row * ROWB + ((ch ^ (row & 7)) << 4));
+        mma_16816(o[2 * d2], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], v0, v1);
+        mma_16816(o[2 * d2 + 1], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], v2, v3);
+      }
+    }
+    __syncthreads();  // the buffer is refilled by the next iteration's load
+  }
+#pragma unroll
+  for (int off = 1; off <= 2; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+  const int r0 = q0 + warp * 16 + g8, r1 = r0 + 8;
+#pragma unroll
+  for (int j = 0; j < HD / 8; ++j) {
+    const int c = 8 * j + 2 * t4;
+    if (r0 < a.T)
+      *reinterpret_cast<uint32_t*>(a.out + ((size_t)r0 * a.nq + h) * HD + c) =
+          uint32_t(f16_checked(o[j][0] * i0, a.err)) | (uint32_t(f16_checked(o[j][1] * i0, a.err)) << 16);
+    if (r1 < a.T)
+      *reinterpret_cast<uint32_t*>(a.out + ((size_t)r1 * a.nq + h) * HD + c) =
+          uint32_t(f16_checked(o[j][2] * i1, a.err)) | (uint32_t(f16_checked(o[j][3] * i1, a.err)) << 16);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-token row kernels (one CTA of 256 threads per token)
+// ---------------------------------------------------------------------------
+constexpr int RT = 256;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < RT / 32; ++i) s += red[i];
+  return s;
+}
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < RT / 32; ++i) s = fmaxf(s, red[i]);
+  return s;
+}
+
+// fp16 copy of a residual row with the range guard: rows whose max |x|
+// reaches 2^15 are scaled by a power of two first; scale[t] undoes it.
+__device__ __forceinline__ void row_to_f16(const float* x, int d, uint16_t* x16, float* scale, float* red) {
+  float mx = 0.f;
+  for (int i = threadIdx.x; i < d; i += RT) mx = fmaxf(mx, fabsf(x[i]));
+  mx = block_max(mx, red);
+  float s = 1.f, inv = 1.f;
+  if (mx >= 32768.f) {
+    int ex;
+    frexpf(mx, &ex);
+    s = ldexpf(1.f, 15 - ex);
+    inv = ldexpf(1.f, ex - 15);
+  }
+  for (int i = threadIdx.x; i < d; i += RT) x16[i] = f32_to_f16(x[i] * s);
+  if (threadIdx.x == 0) *scale = inv;
+}
+
+__global__ void __launch_bounds__(RT) embed_rows_kernel(const int32_t* __restrict__ tokens, const uint16_t* embed,
+                                                        int vocab, int d, float* X, uint16_t* X16, float* scale,
+                                                        uint32_t* err) {
+  __shared__ float red[RT / 32];
+  const int t = blockIdx.x;
+  int tok = tokens[t];
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0) pf_error(err, EW_BAD_SHAPE);
+    tok = tok < 0 ? 0 : vocab - 1;
+  }
+  float* x = X + (size_t)t * d;
+  for (int i = threadIdx.x; i < d; i += RT) x[i] = bf16_to_f32(embed[(size_t)tok * d + i]);
+  __syncthreads();
+  row_to_f16(x, d, X16 + (size_t)t * d, scale + t, red);
+}
+
+// X[t] += RMSNorm(V[t]) * gain, then the fp16 copy for the next GEMM.
+__global__ void __launch_bounds__(RT) resid_rows_kernel(const float* __restrict__ V, const float* __restrict__ gain,
+                                                        int d, float eps, float* X, uint16_t* X16, float* scale) {
+  __shared__ float red[RT / 32];
+  const int t = blockIdx.x;
+  const float* v = V + (size_t)t * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d; i += RT) ss += v[i] * v[i];
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / float(d) + eps);
+  float* x = X + (size_t)t * d;
+  for (int i = threadIdx.x; i < d; i += RT) x[i] += v[i] * r * gain[i];
+  __syncthreads();
+  row_to_f16(x, d, X16 + (size_t)t * d, scale + t, red);
+}
+
+struct QkArgs {
+  const float* Y;         // [T][q_dim + 2 kv_dim]
+  const float* qg;        // q gains [q_dim]
+  const float* kg;        // k gains [kv_dim]
+  uint16_t* q16;          // bf16 [T][nq][hd]
+  uint16_t* kn;           // the prompt's keys / values, bf16 [nkv][T][hd]
+  uint16_t* vn;
+  double f[64];           // inverse frequencies of the layer type
+  float ms;               // attention factor
+  float eps;
+  int T, nq, nkv, hd, start;
+};
+
+// QK-norm over the whole projections, gains, rotation (pairs i, i + hd / 2),
+// the query, key and value as bf16.
+__global__ void __launch_bounds__(RT) qk_rows_kernel(const __grid_constant__ QkArgs a) {
+  __shared__ float red[RT / 32];
+  const int t = blockIdx.x;
+  const int qd = a.nq * a.hd, kd = a.nkv * a.hd, H2 = a.hd / 2;
+  const float* y = a.Y + (size_t)t * (qd + 2 * kd);
+  float sq = 0.f, sk = 0.f;
+  for (int i = threadIdx.x; i < qd; i += RT) sq += y[i] * y[i];
+  for (int i = threadIdx.x; i < kd; i += RT) sk += y[qd + i] * y[qd + i];
+  sq = block_sum(sq, red);
+  sk = block_sum(sk, red);
+  const float rq = rsqrtf(sq / float(qd) + a.eps), rk = rsqrtf(sk / float(kd) + a.eps);
+  const int pos = a.start + t;
+  for (int idx = threadIdx.x; idx < (a.nq + a.nkv) * H2; idx += RT) {
+    const bool isq = idx < a.nq * H2;
+    const int j = isq ? idx : idx - a.nq * H2;
+    const int hh = j / H2, i = j - hh * H2;
+    const double ang = double(pos) * a.f[i];
+    const double rr = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+    float sn, cs;
+    sincosf(float(rr), &sn, &cs);
+    cs *= a.ms;
+    sn *= a.ms;
+    if (isq) {
+      const int c = hh * a.hd + i;
+      const float x1 = y[c] * rq * a.qg[c], x2 = y[c + H2] * rq * a.qg[c + H2];
+      a.q16[(size_t)t * qd + c] = f32_to_bf16(x1 * cs - x2 * sn);
+      a.q16[(size_t)t * qd + c + H2] = f32_to_bf16(x2 * cs + x1 * sn);
+    } else {
+      const int c = hh * a.hd + i;
+      const float x1 = y[qd + c] * rk * a.kg[c], x2 = y[qd + c + H2] * rk * a.kg[c + H2];
+      const size_t row = ((size_t)hh * a.T + t) * a.hd;
+      a.kn[row + i] = f32_to_bf16(x1 * cs - x2 * sn);
+      a.kn[row + i + H2] = f32_to_bf16(x2 * cs + x1 * sn);
+      a.vn[row + i] = f32_to_bf16(y[qd + kd + c]);
+      a.vn[row + i + H2] = f32_to_bf16(y[qd + kd + c + H2]);
+    }
+  }
+}
+
+// The prompt's keys and values of positions start + t, t in [t0, T), into
+// the cache (slot = position, or position % window on a ring), with the
+// cache's chunk permutation; one thread per 16-byte chunk.
+__global__ void kv_append_kernel(uint16_t* __restrict__ kc, uint16_t* __restrict__ vc, const uint16_t* __restrict__ kn,
+                                 const uint16_t* __restrict__ vn, int nkv, int hd, int slots, int window, int seq,
+                                 int start, int T, int t0) {
+  const int ch = hd / 8;
+  const int64_t total = (int64_t)nkv * (T - t0) * ch;
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= total) return;
+  const int c = int(id % ch);
+  const int64_t rest = id / ch;
+  const int t = t0 + int(rest % (T - t0));
+  const int h = int(rest / (T - t0));
+  const int pos = start + t;
+  const int slot = window ? pos % window : pos;
+  const size_t src = ((size_t)h * T + t) * hd + c * 8;
+  const size_t dst = (((size_t)seq * nkv + h) * slots + slot) * hd + ((c ^ (slot & 7)) * 8);
+  *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(kn + src);
+  *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(vn + src);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// K-major fp16 matrix [rows, k] (row stride k), box of box_rows x 64 with the 128-byte swizzle.
+static cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t k, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cuuint64_t(k), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(k * 2)};
+  const cuuint32_t box[2] = {cuuint32_t(GM_BK), cuuint32_t(box_rows)};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_dequant_f16(const uint8_t* tiled, int64_t n, int64_t k, uint16_t* out, cudaStream_t st) {
+  const int64_t total = (n / RB) * (k / W4_KC) * 512;
+  dequant_f16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(tiled, n, k, out);
+  return cudaGetLastError();
+}
+
+// C = A[M, K] . B[N, K]^T; A, B fp16 K-major (16-byte aligned, K % 64 == 0).
+cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi, void* out, int ldo,
+                            const float* row_scale, uint32_t* err, int n_sms, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(gemm_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap ma, mb;
+  cudaError_t e = make_map(&ma, A, M, K, GM_BM);
+  if (e != cudaSuccess) return e;
+  e = make_map(&mb, B, N, K, GM_BN);
+  if (e != cudaSuccess) return e;
+  GemmArgs g;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.epi = epi;
+  g.ldo = ldo;
+  g.out = out;
+  g.row_scale = row_scale;
+  g.err = err;
+  const int tiles = ((M + GM_BM - 1) / GM_BM) * ((N + GM_BN - 1) / GM_BN);
+  const int grid = tiles < n_sms ? tiles : n_sms;
+  gemm_f16_kernel<<<grid, GM_THREADS, GM_SMEM, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flash_prefill(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, const uint16_t* kn,
+                                 const uint16_t* vn, uint16_t* out, int T, int nq, int nkv, int hd, int slots,
+                                 int window, int start, int seq, uint32_t* err, cudaStream_t st) {
+  FaArgs a;
+  a.q = q;
+  a.kc = kc;
+  a.vc = vc;
+  a.kn = kn;
+  a.vn = vn;
+  a.out = out;
+  a.T = T;
+  a.nq = nq;
+  a.nkv = nkv;
+  a.slots = slots;
+  a.window = window;
+  a.start = start;
+  a.seq = seq;
+  a.scale_log2 = float(1.4426950408889634 / sqrt(double(hd)));
+  a.err = err;
+  const dim3 grid((T + FA_BQ - 1) / FA_BQ, nq);
+  const int smem = 4 * FA_BK * hd * 2;
+  if (hd == 128) {
+    static bool attr = false;
+    if (!attr) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(flash_prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    flash_prefill_kernel<128><<<grid, FA_THREADS, smem, st>>>(a);
+  } else {
+    flash_prefill_kernel<64><<<grid, FA_THREADS, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_embed_rows(const int32_t* tokens, int T, const uint16_t* embed, int vocab, int d, float* X,
+                              uint16_t* X16, float* scale, uint32_t* err, cudaStream_t st) {
+  embed_rows_kernel<<<T, RT, 0, st>>>(tokens, embed, vocab, d, X, X16, scale, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_resid_rows(const float* V, const float* gain, int T, int d, float eps, float* X, uint16_t* X16,
+                              float* scale, cudaStream_t st) {
+  resid_rows_kernel<<<T, RT, 0, st>>>(V, gain, d, eps, X, X16, scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qk_rows(const float* Y, const float* qg, const float* kg, uint16_t* q16, uint16_t* kn,
+                           uint16_t* vn, const double* f, float ms, float eps, int T, int nq, int nkv, int hd,
+                           int start, cudaStream_t st) {
+  QkArgs a;
+  a.Y = Y;
+  a.qg = qg;
+  a.kg = kg;
+  a.q16 = q16;
+  a.kn = kn;
+  a.vn = vn;
+  for (int i = 0; i < 64; ++i) a.f[i] = f[i];
+  a.ms = ms;
+  a.eps = eps;
+  a.T = T;
+  a.nq = nq;
+  a.nkv = nkv;
+  a.hd = hd;
+  a.start = start;
+  qk_rows_kernel<<<T, RT, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+// Append the prompt's last rows to the cache: all of them on a full layer,
+// the last `window` on a ring (the ones it keeps).
+cudaError_t launch_kv_append(uint16_t* kc, uint16_t* vc, const uint16_t* kn, const uint16_t* vn, int nkv, int hd,
+                             int slots, int window, int seq, int start, int T, cudaStream_t st) {
+  const int t0 = (window && T > window) ? T - window : 0;
+  const int64_t total = (int64_t)nkv * (T - t0) * (hd / 8);
+  kv_append_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(kc, vc, kn, vn, nkv, hd, slots, window, seq,
+                                                                     start, T, t0);
+  return cudaGetLastError();
+}
+
+}  // namespace w4a

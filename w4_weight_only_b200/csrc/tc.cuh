@@ -1,0 +1,103 @@
+// Inline-PTX wrappers for the 5th-generation tensor cores (tcgen05, tensor
+// memory) and the tensor-map form of the TMA engine, sm_100a.  Single-CTA
+// forms only (cta_group::1); no load here uses cluster multicast.
+#pragma once
+#include "ptx.cuh"
+
+namespace w4a {
+
+// ---- TMA (tensor map) -------------------------------------------------------
+// 2-D tiled load of the box at (x, y) (x innermost, in elements) into shared
+// memory, completing on an mbarrier.  x * element size must be a multiple of
+// 16 bytes; out-of-range rows and columns read as zeros.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_addr(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_map(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ---- tensor memory --------------------------------------------------------------
+// Whole-warp operations.  The allocated base address (lane 0, first column)
+// is written to shared memory at dst.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Ordering of tcgen05 operations around thread synchronisation.
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// ---- MMA ------------------------------------------------------------------------
+// D[tmem] = A * B^T (+ D when acc != 0); A and B from shared-memory matrix
+// descriptors, fp16 or bf16 inputs (both the same, per idesc), fp32 D.
+// Issued by one thread.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// The mbarrier gets one arrival once every MMA this thread issued before has
+// completed (and its shared-memory operands have been read).
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// Instruction descriptor of kind::f16 with fp32 accumulation, both operands
+// K-major: a_bf16 / b_bf16 select bf16 (else fp16), M in {64, 128, 256},
+// N a multiple of 16 up to 256.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool bf16) {
+  return (1u << 4)                              // D format: fp32
+         | ((bf16 ? 1u : 0u) << 7)              // A format
+         | ((bf16 ? 1u : 0u) << 10)             // B format
+         | (uint32_t(N >> 3) << 17)             // N / 8
+         | (uint32_t(M >> 4) << 24);            // M / 16
+}
+
+// Shared-memory matrix descriptor of a K-major tile stored with the 128-byte
+// swizzle (rows of 64 16-bit elements, 8-row atoms of 1,024 bytes; the tile
+// base 1,024-byte aligned): start address, stride between 8-row groups
+// 1,024 bytes, descriptor version 1, layout SWIZZLE_128B.  Moving along K
+// inside the 64-element row adds the byte offset to the start address.
+__device__ __forceinline__ uint64_t umma_desc_sw128(const void* tile, uint32_t byte_off) {
+  const uint32_t a = smem_addr(tile) + byte_off;
+  uint64_t d = 0;
+  d |= uint64_t((a & 0x3FFFFu) >> 4);          // start address
+  d |= uint64_t(1) << 16;                        // leading byte offset (unused for swizzled K-major)
+  d |= uint64_t(1024 >> 4) << 32;                // stride byte offset
+  d |= uint64_t(1) << 46;                        // version
+  d |= uint64_t(2) << 61;                        // SWIZZLE_128B
+  return d;
+}
+
+// ---- TMEM -> registers ------------------------------------------------------------
+// Warp-wide: thread i reads TMEM lane (lane of taddr) + i, 32-bit columns
+// col .. col + 15 of taddr.  The warp may only address its own quarter of the
+// lanes (warp id % 4).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+}  // namespace w4a
