@@ -37,10 +37,10 @@ SEED = 3
 NOMINAL_HBM_GBS = 8000.0
 
 
-# DRAM traffic of the engine from ncu (profiles/w4a_engine_decode_4layer_full.md):
-# 4- and 8-layer launches of the benchmark model at ctx 4096 give the bytes per
-# layer and the fixed part; valid only for the engine code they were taken on
-# (its hash with comments and whitespace stripped).
+# DRAM traffic of the engine from ncu: 4- and 8-layer launches of the
+# benchmark model at ctx 4096 give the bytes per layer and the fixed part;
+# valid only for the engine code they were taken on (its hash with comments
+# and whitespace stripped).
 TRAFFIC_ENGINE_CODE = "6ff7029416b7a011"
 TRAFFIC_FIXED = 1.03557e9
 TRAFFIC_PER_LAYER = 0.270234e9
@@ -94,6 +94,34 @@ def step_bytes(cfg, pos: int) -> int:
         kv += (keys - 1) * kv_row + kv_row          # read the old keys, write the new one
     gains = cfg.n_layers * (cfg.q_dim + cfg.kv_dim + 2 * d) * 4 + d * 4
     return cfg.n_layers * per_layer + cfg.vocab * d * 2 + kv + gains + d * 2
+
+
+def linear_params_per_layer(cfg) -> int:
+    d = cfg.d_model
+    return cfg.qkv_dim * d + d * cfg.q_dim + 2 * cfg.ffn * d + d * cfg.ffn
+
+
+def prefill_flops(cfg, T: int, start: int = 0) -> int:
+    """Algorithmic FLOPs of a prompt of T tokens at positions start ..: the
+    linear layers (2 per weight per token), QK^T and PV over each token's
+    visible keys (causal; the window on SWA layers), the lm_head on the last
+    token."""
+    lin = 2 * T * cfg.n_layers * linear_params_per_layer(cfg) + 2 * cfg.vocab * cfg.d_model
+    att = 0
+    for full in cfg.full_layers:
+        keys = 0
+        for p in range(start, start + T):
+            keys += p + 1 if full else min(p + 1, cfg.window)
+        att += 4 * cfg.n_heads * cfg.head_dim * keys
+    return lin + att
+
+
+def measured_tensor_peak(sustained: bool):
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["bf16_tflops_sustained" if sustained else "bf16_tflops"]), "measured"
+    return (1400.0 if sustained else 1590.0), "fallback"
 
 
 # ---------------------------------------------------------------------------
@@ -222,7 +250,18 @@ class OracleSample:
     def describe(self, steps: int) -> str:
         return (f"{steps} passes over a sample of one ctx-{CTX} token: the first {SAMPLE_ROWS} rows of each "
                 f"int4 GEMV (dequantize + float64 matvec) and of the lm_head, one layer's QK-prep + GQA "
-                f"attention over {CTX} keys; scaled by rows and by {self.cfg.n_layers} layers")
+                f"attention over {CTX} keys; the token's time is projected from the sample by rows and by "
+                f"{self.cfg.n_layers} layers")
+
+    def sample_seconds(self) -> float:
+        """Wall time of one pass over the sample itself (what is measured)."""
+        t0 = time.perf_counter()
+        for name, W in self.mats.items():
+            W.matvec(self.xs[name])
+        q, k = self.om.qk_prep(self.ocfg, self.qr, self.kr, self.qg, self.kg, CTX, True)
+        self.om.gqa_decode(self.ocfg, q, self.kv.K[0][0], self.kv.V[0][0], CTX - 1, True)
+        _ = self.head @ self.x[: self.cfg.d_model]
+        return time.perf_counter() - t0
 
 
 def oracle_threads() -> int:
@@ -241,6 +280,7 @@ def cpu_baseline(cfg, steps: int = 3):
     ts = [S.step() for _ in range(steps)]
     per_token = statistics.median(ts)
     return {"value": 1.0 / per_token, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
+            "projected": True, "measured_sample_s": round(S.sample_seconds(), 4),
             "sample": S.describe(steps) + f"; host has {len(os.sched_getaffinity(0))} cores"}
 
 
@@ -257,11 +297,13 @@ def run_reference(args, rank, world):
     ts = [S.step() for _ in range(args.steps)]
     per_token = sum(ts) / len(ts)
     v = 1.0 / per_token
-    base = {"value": v, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
+    base = {"value": v, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle", "projected": True,
+            "measured_sample_s": round(S.sample_seconds(), 4),
             "sample": S.describe(args.steps) + f"; host has {len(os.sched_getaffinity(0))} cores"}
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * per_token,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "projected": True,
             "config": {"workload": f"OLMo-3-32B-shaped int4 (g128, fp16 scale, int4 zero) decode, "
                                    f"{cfg.n_layers} layers, batch 1, ctx {CTX}, greedy",
                        "batch": 1, "ctx": CTX, "layers": cfg.n_layers, "parallelism": "host cores"},
@@ -287,6 +329,63 @@ def job_tok_s(ms_max: float, steps: int, world: int) -> float:
     return world * steps / (ms_max / 1000.0)
 
 
+def measure_prefill(model, cfg, dev, lengths, repeats: int = 3):
+    """Time to first token of prompts of uniform ids from position 0 through
+    the public prefill call (CUDA events around the call; device-resident
+    token ids, the last token's logits out), best of `repeats` after one
+    untimed call; and the int4 GEMM alone (the gate/up matrix of layer 0,
+    its fp16 expansion included) at the longest prompt's M."""
+    import torch
+    from w4_weight_only_b200 import api, synth
+    out = {"workload": f"{cfg.n_layers}-layer model, prompts of " + " and ".join(str(T) for T in lengths)
+                       + " uniform token ids from position 0; best of %d after a warm-up" % repeats,
+           "ttft_ms": {}, "tflop": {}, "tflops": {}}
+    for T in lengths:
+        kv = api.KVCache(cfg, 1, (T + 16) // 16 * 16, device=dev)
+        toks = synth.token_ids(SEED, T, cfg.vocab, dev, "prompt")
+        model.prefill(kv, toks)
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(repeats):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            model.prefill(kv, toks)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        model.check()
+        fl = prefill_flops(cfg, T)
+        out["ttft_ms"][str(T)] = round(best, 2)
+        out["tflop"][str(T)] = round(fl / 1e12, 2)
+        out["tflops"][str(T)] = round(fl / (best / 1e3) / 1e12, 1)
+        del kv
+    M = max(lengths)
+    lin = model.layers[0]["gate_up"]
+    ws = api.gemm_workspace(lin)
+    x = torch.randn((M, cfg.d_model), device=dev).to(torch.float16)
+    api.gemm(lin, x, epilogue=2, ws=ws)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(repeats):
+        api.gemm(lin, x, epilogue=2, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    api.check(ws)
+    ms = e0.elapsed_time(e1) / repeats
+    peak, src = measured_tensor_peak(sustained=False)
+    ach = 2.0 * M * lin.n * lin.k / (ms / 1e3) / 1e12
+    out["gemm"] = {"call": "w4a_gemm (fp16 expansion of the int4 matrix + tcgen05 GEMM)",
+                   "shape": f"gate/up {lin.n}x{lin.k}, M={M}, SwiGLU epilogue", "ms": round(ms, 3),
+                   "bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                   "frac": round(ach / peak, 4), "peak_source": src + " bf16 burst (fp16 has the same dense rate)"}
+    del ws, x
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -296,6 +395,10 @@ def main():
     ap.add_argument("--layers", type=int, default=64, help="model depth (64 = the benchmark model)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (TTFT) measurement")
+    ap.add_argument("--mode", default="decode", choices=["decode", "prefill"],
+                    help="prefill: only the prefill measurement (for profiling)")
+    ap.add_argument("--prefill-tokens", default="1200,8192", help="prompt lengths of the prefill measurement")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -325,6 +428,14 @@ def main():
 
     model = api.Model.from_float(cfg, emb, head, fin, layer_fn)
     del head
+    lengths = [int(t) for t in args.prefill_tokens.split(",") if t]
+    if args.mode == "prefill":
+        pf = measure_prefill(model, cfg, dev, lengths, repeats=max(1, args.steps))
+        if rank == 0:
+            print(json.dumps({"mode": "prefill", "n_gpus": world, "prefill": pf}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     total = args.warmup + args.steps
     max_ctx = ((CTX + total + 1 + 15) // 16) * 16
     kv = api.KVCache(cfg, 1, max_ctx)
@@ -414,6 +525,12 @@ def main():
         e2e = {"value": job_tok_s(te, n_e2e, world), "unit": "tok/s",
                "h2d_bytes_per_step": 8, "d2h_bytes_per_step": 4}
 
+    pf = None
+    if not args.no_prefill:
+        del kv
+        torch.cuda.empty_cache()
+        pf = measure_prefill(model, cfg, dev, lengths)
+
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
@@ -432,7 +549,7 @@ def main():
                            "l2": "inputs larger than L2: 17.2 GB of weights streamed per token",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "clocks": clk, "gpu_launches": args.steps,
-                "e2e": e2e, "cpu_baseline": base}
+                "e2e": e2e, "cpu_baseline": base, "prefill": pf}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
