@@ -51,7 +51,7 @@ enum {
 };
 
 enum { W4A_F32 = 0, W4A_BF16 = 1 };
-enum { W4A_LAYOUT_CANONICAL = 0, W4A_LAYOUT_TILED = 1 };
+enum { W4A_LAYOUT_CANONICAL = 0, W4A_LAYOUT_TILED = 1, W4A_LAYOUT_SYM32 = 2 };
 enum { W4A_EPI_NONE = 0, W4A_EPI_SUMSQ = 1, W4A_EPI_SILU_MUL = 2 };
 
 /* Model shape.  Source: ATLAS-OLMo-3-32B-Think-v4 model card, "Architecture
@@ -66,22 +66,30 @@ typedef struct {
   double rope_theta;                   /* 500000 */
   double yarn_factor;                  /* 8 */
   int32_t yarn_orig_ctx;               /* 8192 */
-  int32_t group;                       /* quantization group, 128 */
+  int32_t group;                       /* 128: asymmetric int4 (fp16 scale, int4 zero);
+                                          32: the symmetric checkpoint format (bf16 scale) */
   double yarn_beta_fast, yarn_beta_slow; /* 32, 1 */
   double eps;                          /* 1e-6 */
   int32_t final_norm;                  /* 1: RMSNorm with gains before lm_head */
   int32_t reserved;
 } W4AConfig;
 
-/* One int4 matrix W [n, k] (n outputs, k inputs), w = (q - z) * s per group of
- * `group` consecutive inputs.  Source: ATLAS-OLMo-3-32B-Think-v4 model card,
- * "Quantization recipe" (column j in word j/8, little-endian nibble).
- *  CANONICAL: qweight uint32 [n, k/8]; scales fp16 bits [k/group, n];
- *             qzeros uint32 [k/group, n/8] (eight rows per word, same nibble order).
- *  TILED:     qweight points at the kernel layout written by w4a_tile();
- *             scales and qzeros are unused.  row_interleave = 1 means tiled
- *             rows alternate between canonical rows [0, n/2) and [n/2, n)
- *             (the fused gate/up matrix). */
+/* One int4 matrix W [n, k] (n outputs, k inputs).  Source: ATLAS-OLMo-3-32B-
+ * Think-v4 model card, "Quantization recipe" (column j in word j/8,
+ * little-endian nibble).  Two formats:
+ *  group 128, w = (q - z) * s, asymmetric (the AWQ-style g128 format):
+ *   CANONICAL: qweight uint32 [n, k/8]; scales fp16 bits [k/128, n];
+ *              qzeros uint32 [k/128, n/8] (eight rows per word, same nibble order).
+ *  group 32, w = (nibble - 8) * s, symmetric (the model card's checkpoint:
+ *  "symmetric (no zero-points), group size 32", bf16 scales, stored nibble
+ *  q + 8), ingested as stored:
+ *   SYM32:     qweight uint32 [n, k/8] (stored nibbles); scales bf16 bits
+ *              [n, k/32] (one per output row and 32-input group); qzeros unused.
+ *  TILED:     qweight points at the kernel layout written by w4a_tile() from
+ *             either canonical form (group selects which); scales and qzeros
+ *             are unused.  row_interleave = 1 means tiled rows alternate
+ *             between canonical rows [0, n/2) and [n/2, n) (the fused gate/up
+ *             matrix). */
 typedef struct {
   int64_t n, k;
   int32_t group;
@@ -143,16 +151,20 @@ W4A_API int w4a_version(void);
 W4A_API int w4a_pack(const void* W, int w_dtype, int64_t n, int64_t k, int group,
              uint32_t* qweight, uint16_t* scales, uint32_t* qzeros, void* stream);
 
-/* Exact dequantization (q - z) * s to fp32 [n, k] (device), from either
- * layout.  Bit-exact: the product of a 5-bit integer and an fp16 is exact. */
+/* Exact dequantization to fp32 [n, k] (device), from any layout: (q - z) * s,
+ * or (nibble - 8) * s for group 32.  Bit-exact: the product of a 5-bit
+ * integer and an fp16 or bf16 value is exact in fp32. */
 W4A_API int w4a_unpack(const W4ATensor* t, float* out, void* stream);
 
-/* Size of the tiled layout of an n x k int4 matrix (n % 16 == 0, k % 512 == 0). */
+/* Size of the tiled layout of an n x k int4 matrix: group 128, 16 x 512 units
+ * of 4,256 bytes (n % 16 == 0, k % 512 == 0); group 32, 16 x 256 units of
+ * 2,304 bytes (k % 256 == 0). */
 W4A_API int w4a_tiled_bytes(int64_t n, int64_t k, int group, size_t* bytes);
 
-/* Rewrite a CANONICAL tensor into the kernel layout: 16-row x 512-column
- * units of 4,256 bytes (codes in mma-fragment order, then fp16 scales, then
- * zeros), units ordered row-block-major.  row_interleave as in W4ATensor. */
+/* Rewrite a CANONICAL (group 128) or SYM32 (group 32) tensor into the kernel
+ * layout: units of 16 rows (codes in mma-fragment order, then the scales; the
+ * zeros for group 128), ordered row-block-major.  row_interleave as in
+ * W4ATensor. */
 W4A_API int w4a_tile(const W4ATensor* canonical, int row_interleave, void* tiled,
              size_t tiled_bytes, void* stream);
 

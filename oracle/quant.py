@@ -12,7 +12,14 @@ asymmetric group-128 variant with an fp16 scale and a 4-bit zero per
 (row, group), dequantized as w = (q - z) * s.  With z == 8 for every group the
 two coincide, which the tests check.
 
-Readings taken where the pages are silent (each listed in the design doc):
+The page's own checkpoint format (symmetric, group 32, bf16 scales, stored
+nibble q + 8, no zero points) is dequantized by ``dequantize_sym32``: the same
+packing, w = (nibble - 8) * s with s the bf16 scale of (row, 32-column
+group).  Its scales come from an MSE observer and AWQ's search, which need
+calibration data; checkpoints of this format are therefore taken as given
+(seeded random nibbles and scales), not produced here.
+
+Readings taken where the pages are silent:
 
 * The page's AWQ scale search needs calibration data and trained weights; the
   quantizer here is round-to-nearest min/max asymmetric (reading D1).
@@ -127,4 +134,23 @@ def dequantize(qweight, scales_bits, qzeros, N: int, K: int, group: int = 128):
     zz = z.astype(np.int64).T               # [N, K/g]
     q = codes.astype(np.int64).reshape(N, K // group, group)
     w = (q - zz[:, :, None]).astype(np.float64) * s[:, :, None]
+    return w.reshape(N, K)
+
+
+def bf16_bits_to_f64(bits):
+    """bf16 bit patterns (uint16) -> their exact values as float64."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def dequantize_sym32(qweight, scale_bits, N: int, K: int, group: int = 32):
+    """The model card's checkpoint format ("Quantization recipe": symmetric,
+    no zero points, group 32, stored nibble q + 8, bf16 scales).
+
+    qweight uint32 [N, K/8] packed as ``pack_rows`` packs; scale_bits bf16
+    bits [N, K/group] (one scale per output row and group of inputs).
+    Returns the exact float64 W~[n, k] = (nibble - 8) * s[n, k // group]."""
+    nib = unpack_rows(qweight, K).astype(np.int64)
+    s = bf16_bits_to_f64(scale_bits).reshape(N, K // group)
+    w = (nib - 8).reshape(N, K // group, group).astype(np.float64) * s[:, :, None]
     return w.reshape(N, K)

@@ -85,3 +85,45 @@ def max_rel_to_rms(got, ref) -> float:
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     return float(np.max(np.abs(got - ref)) / max(rms(ref), 1e-30))
+
+
+class Sym32Pair:
+    """The GPU model and the oracle built from the same seeded checkpoint in
+    the model card's symmetric group-32 format (cfg.group = 32): the GPU
+    tiles the stored nibbles and bf16 scales, the oracle dequantizes them
+    with its own reading of the format."""
+
+    def __init__(self, cfg: wc.Config, seed: int, gen_device: str = "cpu"):
+        from types import SimpleNamespace
+        from oracle import quant
+        from w4_weight_only_b200 import api
+        assert cfg.group == 32
+        self.cfg, self.seed = cfg, seed
+        emb, head, fin = synth.embed_head(cfg, seed, gen_device)
+        self.emb, self.head, self.fin = emb, head, fin
+
+        def layer_gpu(l):
+            raw = synth.sym32_layer(cfg, seed, l, gen_device)
+            return {k: (tuple(t.to("cuda") for t in v) if isinstance(v, tuple) else v.to("cuda"))
+                    for k, v in raw.items()}
+
+        self.gpu = api.Model.from_sym32(cfg, emb.to("cuda"), head.to("cuda"),
+                                        fin.to("cuda") if cfg.final_norm else None, layer_gpu)
+        torch.cuda.synchronize()
+        self.ocfg = oracle_config(cfg)
+
+        def dense(pair):
+            qw, sc = pair
+            n, k = qw.shape[0], qw.shape[1] * 8
+            return quant.dequantize_sym32(qw.cpu().numpy().view(np.uint32), sc.cpu().view(torch.int16).numpy()
+                                          .view(np.uint16), n, k)
+
+        def layer_oracle(l):
+            raw = synth.sym32_layer(cfg, seed, l, gen_device)
+            return SimpleNamespace(Wqkv=dense(raw["qkv"]), Wo=dense(raw["o"]), Wgu=dense(raw["gate_up"]),
+                                   Wd=dense(raw["down"]), q_norm=np64(raw["q_norm"]), k_norm=np64(raw["k_norm"]),
+                                   post_attn_norm=np64(raw["post_attn_norm"]),
+                                   post_ffn_norm=np64(raw["post_ffn_norm"]))
+
+        self.oracle = om.OracleModel(self.ocfg, np64(emb), np64(head), np64(fin) if cfg.final_norm else None,
+                                     layer_oracle, cache_dense=True)

@@ -138,3 +138,55 @@ def test_rounding_half_even_in_fp32():
     codes, s16, z = quant.quantize(row[None, :])
     assert s16[0, 0] == s and z[0, 0] == 0
     assert codes[0, 2] == 2 and codes[0, 3] == 4
+
+
+# ---- the model card's symmetric group-32 checkpoint format -----------------------
+def _bf16_bits(x):
+    """Round float32 values to bf16 (nearest-even) and return the bits."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def test_sym32_known_pattern_and_offset():
+    """Stored nibbles k % 16 (the page's packing: column j in word j / 8,
+    nibble j % 8) decode to q = k % 16 - 8, from -8 to 7."""
+    gold = json.loads((GOLD / "known_pattern_words.json").read_text())
+    want = [int(w, 16) for w in gold["codes_k_mod_16_words"]]
+    K = 64
+    qw = quant.pack_rows(np.tile(np.arange(K) % 16, (2, 1)))
+    assert list(qw[0][:2]) == want
+    s = _bf16_bits(np.full((2, K // 32), 0.5, np.float32))
+    w = quant.dequantize_sym32(qw, s, 2, K)
+    assert np.array_equal(w[0], ((np.arange(K) % 16) - 8) * 0.5)
+    assert w.min() == -4.0 and w.max() == 3.5
+
+
+def test_sym32_equals_asymmetric_with_zero_8():
+    """The symmetric format is the asymmetric dequantization with every zero
+    point 8 and group 32 (scales that fp16 holds exactly)."""
+    r = _rng(11)
+    N, K = 16, 256
+    codes = r.integers(0, 16, size=(N, K))
+    qw = quant.pack_rows(codes)
+    sf = (r.random((N, K // 32)) * 0.01 + 1e-3).astype(np.float32)
+    sb = _bf16_bits(sf)
+    sv = quant.bf16_bits_to_f64(sb)
+    s16 = sv.astype(np.float16)
+    assert np.array_equal(s16.astype(np.float64), sv)  # bf16 values in the fp16 range are fp16 values
+    zeros = quant.pack_rows(np.full((K // 32, N), 8))
+    asym = quant.dequantize(qw, np.ascontiguousarray(s16.T).view(np.uint16), zeros, N, K, group=32)
+    assert np.array_equal(quant.dequantize_sym32(qw, sb, N, K), asym)
+
+
+def test_sym32_brute_force():
+    r = _rng(12)
+    N, K = 3, 64
+    codes = r.integers(0, 16, size=(N, K))
+    sb = _bf16_bits(r.random((N, K // 32)).astype(np.float32))
+    w = quant.dequantize_sym32(quant.pack_rows(codes), sb, N, K)
+    for n in range(N):
+        for k in range(K):
+            bits = int(sb[n, k // 32]) << 16
+            s = float(np.array([bits], dtype=np.uint32).view(np.float32)[0])
+            assert w[n, k] == (int(codes[n, k]) - 8) * s

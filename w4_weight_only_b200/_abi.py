@@ -13,7 +13,7 @@ MAX_LAYERS = 128
 OK, ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_KERNEL, ERR_TIMEOUT = (
     0, -1, -2, -3, -4, -5, -6, -7, -8)
 F32, BF16 = 0, 1
-LAYOUT_CANONICAL, LAYOUT_TILED = 0, 1
+LAYOUT_CANONICAL, LAYOUT_TILED, LAYOUT_SYM32 = 0, 1, 2
 EPI_NONE, EPI_SUMSQ, EPI_SILU_MUL = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 4194304
 

@@ -99,6 +99,33 @@ def tile(qw, sc, qz, n: int, k: int, row_interleave: bool = False, group: int = 
     return W4Linear(blob, n, k, row_interleave, group)
 
 
+def tile_sym32(qweight: torch.Tensor, scales: torch.Tensor, row_interleave: bool = False) -> W4Linear:
+    """The model card's checkpoint format (symmetric int4, group 32, stored
+    nibble q + 8): qweight int32 [n, k/8], scales bf16 [n, k/32], as stored,
+    rewritten into the kernel's group-32 units."""
+    _need(qweight, torch.int32, "qweight")
+    _need(scales, torch.bfloat16, "scales")
+    n, k = qweight.shape[0], qweight.shape[1] * 8
+    nbytes = _size_out("w4a_tiled_bytes", n, k, 32)
+    blob = torch.empty(nbytes, dtype=torch.uint8, device=qweight.device)
+    t = _abi.W4ATensor()
+    t.n, t.k, t.group, t.layout, t.row_interleave = n, k, 32, _abi.LAYOUT_SYM32, 0
+    t.qweight, t.scales, t.qzeros = qweight.data_ptr(), scales.data_ptr(), None
+    call("w4a_tile", C.byref(t), 1 if row_interleave else 0, _p(blob), nbytes, _stream())
+    return W4Linear(blob, n, k, row_interleave, 32)
+
+
+def unpack_sym32(qweight: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+    """Exact fp32 dequantization of a symmetric group-32 checkpoint matrix."""
+    n, k = qweight.shape[0], qweight.shape[1] * 8
+    out = torch.empty((n, k), dtype=torch.float32, device=qweight.device)
+    t = _abi.W4ATensor()
+    t.n, t.k, t.group, t.layout, t.row_interleave = n, k, 32, _abi.LAYOUT_SYM32, 0
+    t.qweight, t.scales, t.qzeros = qweight.data_ptr(), scales.data_ptr(), None
+    call("w4a_unpack", C.byref(t), _p(out), _stream())
+    return out
+
+
 def quantize_linear(W: torch.Tensor, row_interleave: bool = False, group: int = 128) -> W4Linear:
     """pack() then tile(): the kernel-layout int4 form of W [n, k]."""
     n, k = W.shape
@@ -326,6 +353,25 @@ class Model:
             L = {"qkv": quantize_linear(raw["qkv"]), "o": quantize_linear(raw["o"]),
                  "gate_up": quantize_linear(raw["gate_up"], row_interleave=True),
                  "down": quantize_linear(raw["down"])}
+            for g in ("q_norm", "k_norm", "post_attn_norm", "post_ffn_norm"):
+                L[g] = raw[g].float().contiguous()
+            del raw
+            layers.append(L)
+        return cls(cfg, embed.contiguous(), tile_bf16(lm_head.contiguous()),
+                   None if final_norm is None else final_norm.float().contiguous(), layers)
+
+    @classmethod
+    def from_sym32(cls, cfg: Config, embed: torch.Tensor, lm_head: torch.Tensor, final_norm, layer_fn):
+        """layer_fn(l) -> dict of (qweight int32, scales bf16) checkpoint pairs
+        for qkv, o, gate_up, down in the symmetric group-32 format (cfg.group
+        must be 32) and the four fp32 gains."""
+        if cfg.group != 32:
+            raise ValueError("from_sym32 needs cfg.group == 32")
+        layers = []
+        for l in range(cfg.n_layers):
+            raw = layer_fn(l)
+            L = {"qkv": tile_sym32(*raw["qkv"]), "o": tile_sym32(*raw["o"]),
+                 "gate_up": tile_sym32(*raw["gate_up"], row_interleave=True), "down": tile_sym32(*raw["down"])}
             for g in ("q_norm", "k_norm", "post_attn_norm", "post_ffn_norm"):
                 L[g] = raw[g].float().contiguous()
             del raw

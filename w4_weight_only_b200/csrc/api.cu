@@ -23,7 +23,9 @@ cudaError_t launch_qk_prep(int, int, int, int, float, const double*, float, cons
                            const float*, const float*, const int32_t*, uint16_t*, uint16_t*, uint16_t*, int,
                            cudaStream_t);
 cudaError_t launch_sample(const float*, int, int, float, float, const float*, int32_t*, double*, cudaStream_t);
-cudaError_t launch_dequant_f16(const uint8_t*, int64_t, int64_t, uint16_t*, cudaStream_t);
+cudaError_t launch_dequant_f16(const uint8_t*, int64_t, int64_t, int, uint16_t*, cudaStream_t);
+cudaError_t launch_tile_s32(const uint32_t*, const uint16_t*, int64_t, int64_t, int, uint8_t*, cudaStream_t);
+cudaError_t launch_unpack_s32(const uint32_t*, const uint16_t*, const uint8_t*, int64_t, int64_t, int, float*, cudaStream_t);
 cudaError_t launch_gemm_f16(const uint16_t*, const uint16_t*, int, int, int, int, void*, int, const float*, uint32_t*,
                             int, cudaStream_t);
 cudaError_t launch_flash_prefill(const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*,
@@ -197,6 +199,7 @@ struct WsLayout {
 
 struct Dims {
   int d, nq, nkv, hd, ffn, vocab, n_layers;
+  int fmt;  // W4Fmt of the int4 matrices
 };
 
 // A GEMV geometry the engine can run: some k-split fits shared memory and no
@@ -224,7 +227,7 @@ static int decode_geos(const Dims& dm, int B, int nc, Geo* g) {
   // argmax reads each logit once
   const int readers[5] = {nc, nc, nc, nc, 1};
   for (int i = 0; i < 5; ++i) {
-    g[i] = gemv_geo(n[i], k[i], i == 4 ? BF_KC : W4_KC, B, nb, nc, readers[i]);
+    g[i] = gemv_geo(n[i], k[i], i == 4 ? BF_KC : fmt_kc(dm.fmt), B, nb, nc, readers[i]);
     const int rc = geo_check(g[i], n[i], k[i], B);
     if (rc) return rc;
   }
@@ -242,7 +245,7 @@ static int ws_layout(int B, int nc, const Dims& dm, int attn, int decode, long l
   }
   Geo gs = {};
   if (gemv_n > 0) {
-    gs = gemv_geo(gemv_n, gemv_k, W4_KC, B, nb_for(B), nc, 1);
+    gs = gemv_geo(gemv_n, gemv_k, fmt_kc(dm.fmt), B, nb_for(B), nc, 1);
     const int rc = geo_check(gs, gemv_n, gemv_k, B);
     if (rc) return rc;
   }
@@ -361,7 +364,8 @@ static int check_config(const W4AConfig* c) {
   if (c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads || c->n_heads / c->n_kv_heads > MAX_GQ ||
       c->n_kv_heads > 16)
     return fail(W4A_ERR_SHAPE, "heads %d / kv heads %d", c->n_heads, c->n_kv_heads);
-  if (c->group != GROUP) return fail(W4A_ERR_UNSUPPORTED, "group %d (only 128)", c->group);
+  if (c->group != GROUP && c->group != S32_GROUP)
+    return fail(W4A_ERR_UNSUPPORTED, "group %d (128: asymmetric, 32: the symmetric checkpoint format)", c->group);
   const int qd = c->n_heads * c->head_dim;
   if (c->d_model % W4_KC || qd % W4_KC || c->ffn % W4_KC)
     return fail(W4A_ERR_SHAPE, "d_model, heads*head_dim and ffn must be multiples of 512");
@@ -371,7 +375,8 @@ static int check_config(const W4AConfig* c) {
 }
 
 static Dims dims_of(const W4AConfig& c) {
-  return Dims{c.d_model, c.n_heads, c.n_kv_heads, c.head_dim, c.ffn, c.vocab, c.n_layers};
+  return Dims{c.d_model, c.n_heads, c.n_kv_heads, c.head_dim, c.ffn, c.vocab, c.n_layers,
+              c.group == S32_GROUP ? FMT_SYM32 : FMT_ASYM128};
 }
 
 static int kv_regions(const W4AConfig* c, int batch, int max_ctx, uint64_t* off, int* slots, size_t* total) {
@@ -407,14 +412,23 @@ int w4a_pack(const void* W, int w_dtype, int64_t n, int64_t k, int group, uint32
   return W4A_OK;
 }
 
+static int tensor_fmt(const W4ATensor* t) { return t->group == S32_GROUP ? FMT_SYM32 : FMT_ASYM128; }
+
 static int check_tensor(const W4ATensor* t) {
   if (!t || !t->qweight) return fail(W4A_ERR_ARG, "null tensor");
-  if (t->group != GROUP) return fail(W4A_ERR_UNSUPPORTED, "group %d (only 128)", t->group);
+  if (t->group != GROUP && t->group != S32_GROUP)
+    return fail(W4A_ERR_UNSUPPORTED, "group %d (128: asymmetric, 32: the symmetric checkpoint format)", t->group);
+  const int kc = fmt_kc(tensor_fmt(t));
   if (t->layout == W4A_LAYOUT_CANONICAL) {
+    if (t->group != GROUP) return fail(W4A_ERR_ARG, "group 32 tensors use W4A_LAYOUT_SYM32");
     if (!t->scales || !t->qzeros) return fail(W4A_ERR_ARG, "canonical tensor needs scales and qzeros");
     if (t->n <= 0 || t->k <= 0 || t->n % 8 || t->k % GROUP) return fail(W4A_ERR_SHAPE, "bad canonical shape");
+  } else if (t->layout == W4A_LAYOUT_SYM32) {
+    if (t->group != S32_GROUP) return fail(W4A_ERR_ARG, "W4A_LAYOUT_SYM32 needs group 32");
+    if (!t->scales) return fail(W4A_ERR_ARG, "the symmetric format needs its scales");
+    if (t->n <= 0 || t->k <= 0 || t->n % 8 || t->k % S32_GROUP) return fail(W4A_ERR_SHAPE, "bad canonical shape");
   } else if (t->layout == W4A_LAYOUT_TILED) {
-    if (t->n <= 0 || t->k <= 0 || t->n % RB || t->k % W4_KC) return fail(W4A_ERR_SHAPE, "bad tiled shape");
+    if (t->n <= 0 || t->k <= 0 || t->n % RB || t->k % kc) return fail(W4A_ERR_SHAPE, "bad tiled shape");
     if (t->row_interleave && (t->n % (2 * RB))) return fail(W4A_ERR_SHAPE, "interleaved n must be a multiple of 32");
   } else {
     return fail(W4A_ERR_ARG, "layout %d", t->layout);
@@ -430,6 +444,12 @@ int w4a_unpack(const W4ATensor* t, float* out, void* stream) {
   if (t->layout == W4A_LAYOUT_CANONICAL)
     CK(launch_unpack(static_cast<const uint32_t*>(t->qweight), static_cast<const uint16_t*>(t->scales),
                      static_cast<const uint32_t*>(t->qzeros), nullptr, t->n, t->k, 0, out, S(stream)));
+  else if (t->layout == W4A_LAYOUT_SYM32)
+    CK(launch_unpack_s32(static_cast<const uint32_t*>(t->qweight), static_cast<const uint16_t*>(t->scales), nullptr,
+                         t->n, t->k, 0, out, S(stream)));
+  else if (t->group == S32_GROUP)
+    CK(launch_unpack_s32(nullptr, nullptr, static_cast<const uint8_t*>(t->qweight), t->n, t->k, t->row_interleave,
+                         out, S(stream)));
   else
     CK(launch_unpack(nullptr, nullptr, nullptr, static_cast<const uint8_t*>(t->qweight), t->n, t->k,
                      t->row_interleave, out, S(stream)));
@@ -438,7 +458,12 @@ int w4a_unpack(const W4ATensor* t, float* out, void* stream) {
 
 int w4a_tiled_bytes(int64_t n, int64_t k, int group, size_t* bytes) {
   if (!bytes) return fail(W4A_ERR_ARG, "null output");
-  if (group != GROUP) return fail(W4A_ERR_UNSUPPORTED, "group %d (only 128)", group);
+  if (group == S32_GROUP) {
+    if (n <= 0 || k <= 0 || n % RB || k % S32_KC) return fail(W4A_ERR_SHAPE, "n %% 16 and k %% 256 must be 0");
+    *bytes = (size_t)(n / RB) * (k / S32_KC) * S32_UNIT;
+    return W4A_OK;
+  }
+  if (group != GROUP) return fail(W4A_ERR_UNSUPPORTED, "group %d (128 or 32)", group);
   if (n <= 0 || k <= 0 || n % RB || k % W4_KC) return fail(W4A_ERR_SHAPE, "n %% 16 and k %% 512 must be 0");
   *bytes = (size_t)(n / RB) * (k / W4_KC) * W4_UNIT;
   return W4A_OK;
@@ -447,7 +472,7 @@ int w4a_tiled_bytes(int64_t n, int64_t k, int group, size_t* bytes) {
 int w4a_tile(const W4ATensor* c, int row_interleave, void* tiled, size_t tiled_bytes, void* stream) {
   int rc = check_tensor(c);
   if (rc) return rc;
-  if (c->layout != W4A_LAYOUT_CANONICAL) return fail(W4A_ERR_ARG, "w4a_tile takes a canonical tensor");
+  if (c->layout == W4A_LAYOUT_TILED) return fail(W4A_ERR_ARG, "w4a_tile takes a canonical tensor");
   if (!tiled) return fail(W4A_ERR_ARG, "null output");
   size_t need;
   rc = w4a_tiled_bytes(c->n, c->k, c->group, &need);
@@ -455,9 +480,13 @@ int w4a_tile(const W4ATensor* c, int row_interleave, void* tiled, size_t tiled_b
   if (row_interleave && c->n % (2 * RB)) return fail(W4A_ERR_SHAPE, "interleaved n must be a multiple of 32");
   if (tiled_bytes < need) return fail(W4A_ERR_WORKSPACE, "tiled buffer %zu < %zu bytes", tiled_bytes, need);
   if (!aligned16(tiled)) return fail(W4A_ERR_ALIGN, "tiled buffer not 16-byte aligned");
-  CK(launch_tile(static_cast<const uint32_t*>(c->qweight), static_cast<const uint16_t*>(c->scales),
-                 static_cast<const uint32_t*>(c->qzeros), c->n, c->k, row_interleave ? 1 : 0,
-                 static_cast<uint8_t*>(tiled), S(stream)));
+  if (c->layout == W4A_LAYOUT_SYM32)
+    CK(launch_tile_s32(static_cast<const uint32_t*>(c->qweight), static_cast<const uint16_t*>(c->scales), c->n, c->k,
+                       row_interleave ? 1 : 0, static_cast<uint8_t*>(tiled), S(stream)));
+  else
+    CK(launch_tile(static_cast<const uint32_t*>(c->qweight), static_cast<const uint16_t*>(c->scales),
+                   static_cast<const uint32_t*>(c->qzeros), c->n, c->k, row_interleave ? 1 : 0,
+                   static_cast<uint8_t*>(tiled), S(stream)));
   return W4A_OK;
 }
 
@@ -489,7 +518,7 @@ int w4a_gemv_workspace_bytes(const W4ATensor* W, int batch, size_t* bytes) {
   rc = nc_for_sizing(&nc);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, nc, Dims{0, 0, 0, 128, 0, 0, 0}, 0, 0, W->n, W->k, &L);
+  rc = ws_layout(batch, nc, Dims{0, 0, 0, 128, 0, 0, 0, tensor_fmt(W)}, 0, 0, W->n, W->k, &L);
   if (rc) return rc;
   *bytes = L.total;
   return W4A_OK;
@@ -511,15 +540,17 @@ int w4a_gemv(const W4ATensor* W, const uint16_t* x, int batch, void* out, int ep
   rc = device_info(&di);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, 128, 0, 0, 0}, 0, 0, W->n, W->k, &L);
+  const int fmt = tensor_fmt(W);
+  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, 128, 0, 0, 0, fmt}, 0, 0, W->n, W->k, &L);
   if (rc) return rc;
   if (ws_bytes < L.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   static thread_local EngineParams P;
   memset(&P, 0, sizeof(P));
   P.mode = MODE_GEMV;
+  P.fmt = fmt;
   P.phase_begin = 0;
   // with K split into slabs a second phase sums them and applies the epilogue
-  P.geo[0] = gemv_geo(W->n, W->k, W4_KC, batch, nb_for(batch), di->sms, 1);
+  P.geo[0] = gemv_geo(W->n, W->k, fmt_kc(fmt), batch, nb_for(batch), di->sms, 1);
   P.phase_end = (P.geo[0].ns > 1 || epilogue == W4A_EPI_SUMSQ) ? 2 : 1;
   P.B = batch;
   P.pos_const = -1;
@@ -580,7 +611,7 @@ int w4a_attn_workspace_bytes(int batch, int n_heads, int n_kv_heads, int head_di
   int rc = nc_for_sizing(&nc);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, nc, Dims{0, 0, 0, head_dim, 0, 0, 0}, 1, 0, 0, 0, &L);
+  rc = ws_layout(batch, nc, Dims{0, 0, 0, head_dim, 0, 0, 0, 0}, 1, 0, 0, 0, &L);
   if (rc) return rc;
   *bytes = L.total;
   return W4A_OK;
@@ -601,7 +632,7 @@ int w4a_attn_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_t* 
   int rc = device_info(&di);
   if (rc) return rc;
   WsLayout L;
-  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, head_dim, 0, 0, 0}, 1, 0, 0, 0, &L);
+  rc = ws_layout(batch, di->sms, Dims{0, 0, 0, head_dim, 0, 0, 0, 0}, 1, 0, 0, 0, &L);
   if (rc) return rc;
   if (ws_bytes < L.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   static thread_local EngineParams P;
@@ -766,6 +797,7 @@ static int decode_common(W4AModel* m, const int32_t* tokens, const W4AKVCache* k
   static thread_local EngineParams P;
   memset(&P, 0, sizeof(P));
   P.mode = MODE_DECODE;
+  P.fmt = c.group == S32_GROUP ? FMT_SYM32 : FMT_ASYM128;
   P.d = c.d_model;
   P.nq = c.n_heads;
   P.nkv = c.n_kv_heads;
@@ -929,6 +961,7 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   rc = kv_regions(&c, kv->batch, kv->max_ctx, off, slots, &total);
   if (rc) return rc;
   const float eps = float(c.eps);
+  const Dims dm = dims_of(c);
   CK(launch_embed_rows(tokens, Tp, m->embed, c.vocab, d, X, X16, scale, err, st));
   for (int l = 0; l < nl; ++l) {
     const LayerPtrs& L = m->layers[l];
@@ -937,18 +970,18 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
     uint16_t* kc = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(kv->base) + off[l]);
     uint16_t* vc = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(kc) +
                                                al256((size_t)kv->batch * nkv * slots[l] * hd * 2));
-    CK(launch_dequant_f16(L.qkv, qkv, d, W16, st));
+    CK(launch_dequant_f16(L.qkv, qkv, d, dm.fmt, W16, st));
     CK(launch_gemm_f16(X16, W16, Tp, qkv, d, 0, Y, qkv, scale, err, di->sms, st));
     CK(launch_qk_rows(Y, L.q_norm, L.k_norm, Q16, Kn, Vn, m->inv_freq[full], m->ms[full], eps, Tp, nq, nkv, hd,
                       start_pos, st));
     CK(launch_flash_prefill(Q16, kc, vc, Kn, Vn, O16, Tp, nq, nkv, hd, slots[l], win, start_pos, seq, err, st));
     CK(launch_kv_append(kc, vc, Kn, Vn, nkv, hd, slots[l], win, seq, start_pos, Tp, st));
-    CK(launch_dequant_f16(L.o, d, qd, W16, st));
+    CK(launch_dequant_f16(L.o, d, qd, dm.fmt, W16, st));
     CK(launch_gemm_f16(O16, W16, Tp, d, qd, 0, Y, d, nullptr, err, di->sms, st));
     CK(launch_resid_rows(Y, L.attn_norm, Tp, d, eps, X, X16, scale, st));
-    CK(launch_dequant_f16(L.gu, 2LL * ffn, d, W16, st));
+    CK(launch_dequant_f16(L.gu, 2LL * ffn, d, dm.fmt, W16, st));
     CK(launch_gemm_f16(X16, W16, Tp, 2 * ffn, d, 1, H16, ffn, scale, err, di->sms, st));
-    CK(launch_dequant_f16(L.down, d, ffn, W16, st));
+    CK(launch_dequant_f16(L.down, d, ffn, dm.fmt, W16, st));
     CK(launch_gemm_f16(H16, W16, Tp, d, ffn, 0, Y, d, nullptr, err, di->sms, st));
     CK(launch_resid_rows(Y, L.ffn_norm, Tp, d, eps, X, X16, scale, st));
   }
@@ -990,7 +1023,7 @@ int w4a_gemm(const W4ATensor* W, const uint16_t* x, int M, const float* row_scal
   uint16_t* W16 = reinterpret_cast<uint16_t*>(b + 256);
   uint32_t* err = reinterpret_cast<uint32_t*>(b) + 2;
   cudaStream_t st = S(stream);
-  CK(launch_dequant_f16(static_cast<const uint8_t*>(W->qweight), W->n, W->k, W16, st));
+  CK(launch_dequant_f16(static_cast<const uint8_t*>(W->qweight), W->n, W->k, tensor_fmt(W), W16, st));
   const int silu = epilogue == W4A_EPI_SILU_MUL ? 1 : 0;
   CK(launch_gemm_f16(x, W16, M, int(W->n), int(W->k), silu, out, silu ? int(W->n / 2) : int(W->n), row_scale, err,
                      di->sms, st));

@@ -284,6 +284,103 @@ __global__ void qk_prep_kernel(int nq, int nkv, int hd, float eps, const RopeTab
   }
 }
 
+// ---- the symmetric group-32 checkpoint format ----------------------------------
+// Canonical: qweight uint32 [n, k/8] with column j in word j/8, nibble j % 8
+// holding q + 8; scales bf16 [n, k/32] (row-major, one per output row and
+// 32-column group).  w = (nibble - 8) * s.  Tiled: 16-row x 256-column units
+// of S32_UNIT bytes, codes as in the int4 unit (fragment order, the same
+// in-unit column permutation), then the scales [row % 8][group 8][row / 8].
+
+// One thread per 32-bit word of codes in the tiled layout.
+__global__ void tile_s32_codes_kernel(const uint32_t* __restrict__ qw, int64_t n, int64_t k, int interleave,
+                                      uint8_t* __restrict__ out) {
+  const int64_t nkc = k / S32_KC;
+  const int64_t total = (n / RB) * nkc * (S32_KC / 16) * 32;
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= total) return;
+  const int lane = int(id % 32);
+  const int s = int((id / 32) % (S32_KC / 16));
+  const int64_t unit = id / (32 * (S32_KC / 16));
+  const int64_t rb = unit / nkc, kc = unit % nkc;
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t r0 = canon_row(rb * RB + g, n, interleave), r1 = canon_row(rb * RB + g + 8, n, interleave);
+  uint32_t w = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t row = (j & 1) ? r1 : r0;
+    const int64_t col = kc * S32_KC + unit_col(s, t, ((j & 2) ? 2 : 0) + ((j & 4) ? 1 : 0));
+    w |= canon_code(qw, k, row, col) << (4 * j);
+  }
+  uint8_t* u = out + unit * S32_UNIT;
+  reinterpret_cast<uint32_t*>(u + ((s >> 2) * 32 + lane) * 16)[s & 3] = w;
+}
+
+// One thread per (unit, 32-column group, tiled row of the block): its scale.
+__global__ void tile_s32_meta_kernel(const uint16_t* __restrict__ sc, int64_t n, int64_t k, int interleave,
+                                     uint8_t* __restrict__ out) {
+  const int64_t nkc = k / S32_KC;
+  const int64_t total = (n / RB) * nkc * 8 * RB;
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= total) return;
+  const int i = int(id % RB);
+  const int grp = int((id / RB) % 8);
+  const int64_t unit = id / (8 * RB);
+  const int64_t rb = unit / nkc, kc = unit % nkc;
+  const int64_t row = canon_row(rb * RB + i, n, interleave);
+  const int64_t gi = kc * 8 + grp;  // 32-column group along k
+  reinterpret_cast<uint16_t*>(out + unit * S32_UNIT + 2048)[(i & 7) * 16 + grp * 2 + (i >> 3)] =
+      sc[row * (k / S32_GROUP) + gi];
+}
+
+// Exact dequantization of the symmetric group-32 format to fp32 [n, k],
+// canonical (tiled == nullptr) or tiled.
+__global__ void unpack_s32_kernel(const uint32_t* __restrict__ qw, const uint16_t* __restrict__ sc,
+                                  const uint8_t* __restrict__ tiled, int64_t n, int64_t k, int interleave,
+                                  float* __restrict__ out) {
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= n * k) return;
+  const int64_t row = id / k, col = id - row * k;
+  uint32_t q;
+  uint16_t sb;
+  if (tiled == nullptr) {
+    q = canon_code(qw, k, row, col);
+    sb = sc[row * (k / S32_GROUP) + col / S32_GROUP];
+  } else {
+    int64_t r = row;
+    if (interleave) r = (row < n / 2) ? 2 * row : 2 * (row - n / 2) + 1;
+    const int64_t rb = r / RB;
+    const int i = int(r % RB), g = i & 7, hi = i >> 3;
+    const int64_t nkc = k / S32_KC, kc = col / S32_KC;
+    const int kk = int(col % S32_KC);
+    const int m = kk / 32, t = (kk % 32) / 8, e = (kk % 8) / 4, j = kk % 4;
+    const int s = 2 * m + e;
+    const int lane = g * 4 + t;
+    const int nib = ((j & 1) ? 4 : 0) + ((j & 2) ? 2 : 0) + hi;
+    const uint8_t* u = tiled + (rb * nkc + kc) * S32_UNIT;
+    const uint32_t w = reinterpret_cast<const uint32_t*>(u + ((s >> 2) * 32 + lane) * 16)[s & 3];
+    q = (w >> (4 * nib)) & 15u;
+    sb = reinterpret_cast<const uint16_t*>(u + 2048)[g * 16 + m * 2 + hi];
+  }
+  out[id] = float(int(q) - 8) * bf16_to_f32(sb);
+}
+
+// ---- launchers (called from api.cu) ------------------------------------------
+cudaError_t launch_tile_s32(const uint32_t* qw, const uint16_t* sc, int64_t n, int64_t k, int interleave,
+                            uint8_t* out, cudaStream_t st) {
+  const int64_t nw = (n / RB) * (k / S32_KC) * (S32_KC / 16) * 32;
+  tile_s32_codes_kernel<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(qw, n, k, interleave, out);
+  const int64_t nm = (n / RB) * (k / S32_KC) * 8 * RB;
+  tile_s32_meta_kernel<<<(unsigned)((nm + 255) / 256), 256, 0, st>>>(sc, n, k, interleave, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_s32(const uint32_t* qw, const uint16_t* sc, const uint8_t* tiled, int64_t n, int64_t k,
+                              int interleave, float* out, cudaStream_t st) {
+  const int64_t total = n * k;
+  unpack_s32_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(qw, sc, tiled, n, k, interleave, out);
+  return cudaGetLastError();
+}
+
 // ---- launchers (called from api.cu) ------------------------------------------
 cudaError_t launch_pack(const void* W, int w_dtype, int64_t n, int64_t k, uint32_t* qw, uint16_t* sc, uint32_t* qz,
                         cudaStream_t st) {

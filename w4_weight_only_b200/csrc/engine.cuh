@@ -101,7 +101,7 @@ inline Geo gemv_geo(long long n, long long k, int kcw, int B, int nb, int nc, in
   const int kmax = choose_kps(g.nkc, kcw, B, nb);
   if (kmax <= 0 || nc <= 0) return g;
   const int ns0 = g.nkc / kmax;
-  const int ub = kcw == W4_KC ? W4_UNIT : BF_UNIT;
+  const int ub = kcw == W4_KC ? W4_UNIT : (kcw == S32_KC ? S32_UNIT : BF_UNIT);
   const double slab_cost = double(readers) * B * double(n) * 4.0 / L2_VS_SM_HBM;
   double best = 0.0;
   for (int ns = ns0; ns <= g.nkc && (ns == ns0 || ns <= ns_cap); ++ns) {
@@ -165,6 +165,10 @@ struct alignas(16) PD {
   int gi;                        // GEMV: index of its geometry in the launch's table
 };
 static_assert(sizeof(PD) == 256, "phase descriptor size");
+
+__host__ __device__ __forceinline__ bool is_gemv_kind(int k) {
+  return k == PK_GEMV_W4 || k == PK_GEMV_BF16 || k == PK_GEMV_S32;
+}
 
 // Launch constants (shared memory).
 struct LC {
@@ -344,12 +348,12 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
   PD& d = *out;
   const int B = P.B;
   if (P.mode == MODE_GEMV) {
-    d.kind = (p == 0) ? PK_GEMV_W4 : PK_REDUCE;
+    d.kind = (p == 0) ? (P.fmt == FMT_SYM32 ? PK_GEMV_S32 : PK_GEMV_W4) : PK_REDUCE;
     d.blob = P.g_blob;
     d.n = P.g_n;
     d.k = P.g_k;
-    d.kcw = W4_KC;
-    d.ub = W4_UNIT;
+    d.kcw = fmt_kc(P.fmt);
+    d.ub = fmt_unit(P.fmt);
     d.xsrc = XS_BF16;
     d.xbf = P.g_x;
     d.xbf_stride = P.g_k;
@@ -440,9 +444,9 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.knorm = lw.k_norm;
     return;
   }
-  d.kind = PK_GEMV_W4;
-  d.kcw = W4_KC;
-  d.ub = W4_UNIT;
+  d.kind = P.fmt == FMT_SYM32 ? PK_GEMV_S32 : PK_GEMV_W4;
+  d.kcw = fmt_kc(P.fmt);
+  d.ub = fmt_unit(P.fmt);
   d.rows_valid = 1 << 30;
   d.epi = EPI_PART;
   if (sub == 0) {
@@ -635,7 +639,7 @@ __device__ __forceinline__ void cur_enter(Cursor* c, int q, int w) {
   }
   const PD& d = pd_slot(q);
   c->kind = d.kind;
-  if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_BF16) {
+  if (is_gemv_kind(d.kind)) {
     const int4* e = ctab(d.gi, w);
     const int4 e0 = e[0], e1 = e[1];
     c->p0 = d.blob;
@@ -675,7 +679,7 @@ __device__ __forceinline__ void cur_normalize(Cursor* c, int w) {
       cur_enter(c, c->p, w);
       continue;
     }
-    if (kind == PK_GEMV_W4 || kind == PK_GEMV_BF16) {
+    if (is_gemv_kind(kind)) {
       if (c->i < c->end) return;
     } else if (kind == PK_ATTN) {
       const int* st = sst(c->x2);
@@ -721,7 +725,7 @@ __device__ __forceinline__ void cur_store(Cursor* s, const Cursor& c) {
 // Next unit of a copy-warp lane's cursor: the common GEMV step in registers,
 // everything else through the lane's shared-memory copy.
 __device__ __forceinline__ void cur_adv(Cursor& c, int w) {
-  if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
+  if (is_gemv_kind(c.kind)) {
     ++c.i;
     if (++c.x6 == c.x2) {
       c.x6 = 0;
@@ -743,7 +747,7 @@ __device__ __forceinline__ void cur_adv(Cursor& c, int w) {
 // Source range(s) of the unit under a cursor.
 __device__ __forceinline__ void cur_src(const Cursor& c, int warp, const uint8_t*& s1, const uint8_t*& s2,
                                         uint32_t& bytes, int hd) {
-  if (c.kind == PK_GEMV_W4 || c.kind == PK_GEMV_BF16) {
+  if (is_gemv_kind(c.kind)) {
     const uint32_t idx = uint32_t(c.x5 * c.x1 + c.x4 * c.x2 + c.x6);
     s1 = c.p0 + (size_t)idx * uint32_t(c.x0);
     s2 = nullptr;
@@ -1205,7 +1209,7 @@ __device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
   LC& L = lc();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = L.B, dm = L.d;
-  const bool f16 = (d.kind == PK_GEMV_W4);
+  const bool f16 = (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_S32);
   float* rd = red();
   float* wsum = sm_at<float>(sm_wsp(NB));  // [NW][MAX_B] per-warp sums of squares (reset by stage_reset)
   const int xrow_b = klen * 2 + 64;
@@ -1561,6 +1565,89 @@ __device__ __forceinline__ void w4_unit(const uint8_t* slot, const uint8_t* xl, 
   w4_math<NB>(r, xl, xrow_b, xsg, acc, B, g);
 }
 
+// Symmetric group-32 unit (16 rows x 256 columns): codes [grp 2][half 2]
+// [lane 32][4 words] as in the int4 unit, then bf16 scales at +2048 ordered
+// [row % 8][32-column group 8][row / 8] (a lane's 16 scales are 32 contiguous
+// bytes).  The zero point is 8 for every group, so the LOP3 forms 1024 + q
+// (rows g) / 1024 + 16 q (rows g + 8) are moved to q - 8 / 16 (q - 8) by one
+// exact fp16 subtraction, and every 32-column group (two k-steps) closes as
+// s * acc (s / 16 for the 16x rows); no per-group sums of x are needed.
+struct S32Regs {
+  uint4 q[4];   // codes of this lane: [grp][half]
+  uint4 s0, s1; // scales of rows g, g + 8: groups 0..3, 4..7
+};
+__device__ __forceinline__ void s32_load(const uint8_t* slot, int g, int lane, S32Regs& r) {
+  const uint4* qw = reinterpret_cast<const uint4*>(slot) + lane;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r.q[i] = qw[i * 32];
+  r.s0 = *reinterpret_cast<const uint4*>(slot + 2048 + g * 32);
+  r.s1 = *reinterpret_cast<const uint4*>(slot + 2048 + g * 32 + 16);
+}
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <int NB>
+__device__ __forceinline__ void s32_math(const S32Regs& r, const uint8_t* xl, int xrow_b, float (&acc)[NB][4], int B,
+                                         int g) {
+  constexpr uint32_t Z_LO = 0x64086408u;  // fp16 pair 1032 = 1024 + 8
+  constexpr uint32_t Z_HI = 0x64806480u;  // fp16 pair 1152 = 1024 + 16 * 8
+#pragma unroll
+  for (int grp = 0; grp < 2; ++grp) {
+    const uint4 w0 = r.q[grp * 2];
+    const uint4 w1 = r.q[grp * 2 + 1];
+    uint4 xv[NB][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int pr = 0; pr < 4; ++pr)
+        xv[nb][pr] = (g + 8 * nb < B)
+                         ? *reinterpret_cast<const uint4*>(xl + nb * 8 * xrow_b + grp * 256 + pr * 64)
+                         : make_uint4(0u, 0u, 0u, 0u);
+    const uint4 sv = grp ? r.s1 : r.s0;
+#pragma unroll
+    for (int sub = 0; sub < 4; ++sub) {
+      float c[NB][4];
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) c[nb][0] = c[nb][1] = c[nb][2] = c[nb][3] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = 2 * sub + e;
+        const uint32_t w = u4_word(i < 4 ? w0 : w1, i & 3);
+        const uint32_t a0 = hsub2_bits(lop3_and_or(w, 0x000F000Fu, 0x64006400u), Z_LO);
+        const uint32_t a1 = hsub2_bits(lop3_and_or(w, 0x00F000F0u, 0x64006400u), Z_HI);
+        const uint32_t w8 = w >> 8;
+        const uint32_t a2 = hsub2_bits(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), Z_LO);
+        const uint32_t a3 = hsub2_bits(lop3_and_or(w8, 0x00F000F0u, 0x64006400u), Z_HI);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const uint4& x = xv[nb][i >> 1];
+          mma_16816_f16(c[nb], a0, a1, a2, a3, (i & 1) ? x.z : x.x, (i & 1) ? x.w : x.y);
+        }
+      }
+      // scales of group grp * 4 + sub: rows g (low half) and g + 8 (high half)
+      const uint32_t sw = u4_word(sv, sub);
+      const float sl = bf16_to_f32(uint16_t(sw & 0xffffu));
+      const float shi = bf16_to_f32(uint16_t(sw >> 16)) * 0.0625f;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        acc[nb][0] = fmaf(sl, c[nb][0], acc[nb][0]);
+        acc[nb][1] = fmaf(sl, c[nb][1], acc[nb][1]);
+        acc[nb][2] = fmaf(shi, c[nb][2], acc[nb][2]);
+        acc[nb][3] = fmaf(shi, c[nb][3], acc[nb][3]);
+      }
+    }
+  }
+}
+template <int NB>
+__device__ __forceinline__ void s32_unit(const uint8_t* slot, const uint8_t* xl, int xrow_b, float (&acc)[NB][4],
+                                         int B, int g, int lane) {
+  S32Regs r;
+  s32_load(slot, g, lane, r);
+  s32_math<NB>(r, xl, xrow_b, acc, B, g);
+}
+
 // bf16 unit: A fragments [k-step 8][lane 32][4 words].
 struct BfRegs {
   uint4 a[8];
@@ -1730,7 +1817,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     klen = 0;
   }
   stage_x<NB>(d, kbase, klen);
-  if (d.kind == PK_GEMV_W4) {
+  if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_S32) {
     const uint32_t* xmax = reinterpret_cast<const uint32_t*>(red() + 32);
     bool any = false;
 #pragma unroll 1
@@ -1744,7 +1831,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     Cons C;
     cons_load(C, warp);
     const int kps = d.g.kps, nrb = d.g.nrb, kcw = d.kcw;
-    const bool w4 = (d.kind == PK_GEMV_W4);
+    const bool w4 = (d.kind == PK_GEMV_W4), s32 = (d.kind == PK_GEMV_S32);
     const int xrow_b = klen * 2 + 64;
     const uint8_t* xl = sm_at<uint8_t>(SM_XS + g * xrow_b + t * 16);
     const float* xsg = sm_at<float>(sm_xsum(NB)) + 2 * t;
@@ -1775,9 +1862,16 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
         // two batch tiles: the math reads the slot (registers are short)
         if (w4)
           w4_unit<NB>(slot, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g, lane);
+        else if (s32)
+          s32_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
         else
           bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
         cons_release(C, warp, lane, false);
+      } else if (s32) {
+        S32Regs sr;
+        s32_load(slot, g, lane, sr);
+        cons_release(C, warp, lane, false);
+        s32_math<NB>(sr, xl + koff * 2, xrow_b, acc, B, g);
       } else if (w4) {
         // copy the unit to registers and hand the slot back before the math
         W4Regs ur;
@@ -2613,7 +2707,7 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     // the CTA's x range: the slabs its segments touch
     int kbase = 0, klen = 0;
     if (a < b) {
-      const int upsl = g.nrb * g.kps, KS = g.kps * (gi == 4 ? BF_KC : W4_KC);
+      const int upsl = g.nrb * g.kps, KS = g.kps * (gi == 4 ? BF_KC : fmt_kc(P.fmt));
       const int s0 = a / upsl, s1 = (b - 1) / upsl;
       kbase = s0 * KS;
       klen = (s1 - s0 + 1) * KS;
@@ -2706,7 +2800,7 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
     mark(1);
     const PD& d = pd_slot(p);
     const int kind = d.kind;
-    if (kind == PK_GEMV_W4 || kind == PK_GEMV_BF16)
+    if (is_gemv_kind(kind))
       gemv_phase<NB, HD>(d);
     else if (kind == PK_ATTN) {
       attn_phase<HD>(d);

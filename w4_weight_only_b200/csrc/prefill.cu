@@ -95,6 +95,53 @@ __global__ void dequant_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n,
   *reinterpret_cast<uint4*>(out + (r0 + 8) * k + col) = b;
 }
 
+// The symmetric group-32 units (16 x 256, bf16 scales, zero 8) -> fp16 [n, k].
+__global__ void dequant_s32_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n, int64_t k,
+                                       uint16_t* __restrict__ out) {
+  const int64_t nkc = k / S32_KC;
+  const int64_t total = (n / RB) * nkc * 8 * 32;
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= total) return;
+  const int lane = int(id & 31);
+  const int m = int((id >> 5) & 7);
+  const int64_t unit = id >> 8;
+  const int64_t rb = unit / nkc, kc = unit - rb * nkc;
+  const int g = lane >> 2, t = lane & 3;
+  const uint8_t* u = tiled + unit * S32_UNIT;
+  const int s0 = 2 * m, s1 = 2 * m + 1;
+  const uint32_t w0 = reinterpret_cast<const uint32_t*>(u + ((s0 >> 2) * 32 + lane) * 16)[s0 & 3];
+  const uint32_t w1 = reinterpret_cast<const uint32_t*>(u + ((s1 >> 2) * 32 + lane) * 16)[s1 & 3];
+  const uint16_t* sc = reinterpret_cast<const uint16_t*>(u + 2048);
+  const float s_lo = bf16_to_f32(sc[g * 16 + m * 2 + 0]), s_hi = bf16_to_f32(sc[g * 16 + m * 2 + 1]);
+  uint16_t lo[8], hi[8];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const uint32_t w = e ? w1 : w0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int q = int((w >> (4 * j)) & 15u) - 8;
+      const int c = 4 * e + ((j & 2) ? 2 : 0) + ((j & 4) ? 1 : 0);
+      if (j & 1)
+        hi[c] = f32_to_f16(float(q) * s_hi);
+      else
+        lo[c] = f32_to_f16(float(q) * s_lo);
+    }
+  }
+  const int64_t col = kc * S32_KC + 32 * m + 8 * t;
+  const int64_t r0 = rb * RB + g;
+  uint4 a, b;
+  a.x = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
+  a.y = uint32_t(lo[2]) | (uint32_t(lo[3]) << 16);
+  a.z = uint32_t(lo[4]) | (uint32_t(lo[5]) << 16);
+  a.w = uint32_t(lo[6]) | (uint32_t(lo[7]) << 16);
+  b.x = uint32_t(hi[0]) | (uint32_t(hi[1]) << 16);
+  b.y = uint32_t(hi[2]) | (uint32_t(hi[3]) << 16);
+  b.z = uint32_t(hi[4]) | (uint32_t(hi[5]) << 16);
+  b.w = uint32_t(hi[6]) | (uint32_t(hi[7]) << 16);
+  *reinterpret_cast<uint4*>(out + r0 * k + col) = a;
+  *reinterpret_cast<uint4*>(out + (r0 + 8) * k + col) = b;
+}
+
 // ---------------------------------------------------------------------------
 // GEMM on the tcgen05 tensor cores: D[M, N] = A[M, K] . B[N, K]^T, fp16 in,
 // fp32 accumulation in tensor memory
@@ -722,9 +769,14 @@ static cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int6
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_dequant_f16(const uint8_t* tiled, int64_t n, int64_t k, uint16_t* out, cudaStream_t st) {
-  const int64_t total = (n / RB) * (k / W4_KC) * 512;
-  dequant_f16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(tiled, n, k, out);
+cudaError_t launch_dequant_f16(const uint8_t* tiled, int64_t n, int64_t k, int fmt, uint16_t* out, cudaStream_t st) {
+  if (fmt == FMT_SYM32) {
+    const int64_t total = (n / RB) * (k / S32_KC) * 256;
+    dequant_s32_f16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(tiled, n, k, out);
+  } else {
+    const int64_t total = (n / RB) * (k / W4_KC) * 512;
+    dequant_f16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(tiled, n, k, out);
+  }
   return cudaGetLastError();
 }
 

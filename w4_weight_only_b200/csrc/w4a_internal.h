@@ -22,6 +22,12 @@ constexpr int BF_KC = 128;             // k per bf16 unit
 constexpr int GROUP = 128;             // quantization group (the only one supported)
 constexpr int W4_UNIT = RB * W4_KC / 2 + (W4_KC / GROUP) * RB * 2 + (W4_KC / GROUP) * RB / 2;  // 4256
 constexpr int BF_UNIT = RB * BF_KC * 2;                                                      // 4096
+// The model card's own checkpoint format: symmetric int4, group 32, bf16
+// scales, stored nibble q + 8 (w = (nibble - 8) * s).  Its unit holds 16 rows
+// x 256 columns: the codes in the same fragment order, then the 16 x 8 scales.
+constexpr int S32_GROUP = 32;
+constexpr int S32_KC = 256;
+constexpr int S32_UNIT = RB * S32_KC / 2 + (S32_KC / S32_GROUP) * RB * 2;                    // 2304
 constexpr int ATT_KEYS = 8;            // keys per warp unit
 constexpr int ATT_CTA_KEYS = ATT_KEYS * NW;  // keys per CTA unit (120)
 // Shared-memory budget per CTA (bytes).  x fragments shrink when two
@@ -34,7 +40,8 @@ constexpr int MAX_LAYERS = 128;
 constexpr int MAX_GQ = 8;              // query heads per KV head supported by the attention tile
 
 static_assert(W4_UNIT == 4256, "int4 unit size");
-static_assert(W4_UNIT <= SLOT_BYTES && BF_UNIT <= SLOT_BYTES, "slot too small");
+static_assert(W4_UNIT <= SLOT_BYTES && BF_UNIT <= SLOT_BYTES && S32_UNIT <= SLOT_BYTES, "slot too small");
+static_assert(S32_UNIT == 2304, "sym32 unit size");
 
 // ---- device error word bits -----------------------------------------------
 enum : uint32_t {
@@ -48,7 +55,12 @@ enum : uint32_t {
 
 // ---- engine modes / phase kinds --------------------------------------------
 enum Mode : int { MODE_DECODE = 0, MODE_GEMV = 1, MODE_ATTN = 2 };
-enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_ATTN = 2, PK_ARGMAX = 3, PK_REDUCE = 4 };
+enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_ATTN = 2, PK_ARGMAX = 3, PK_REDUCE = 4, PK_GEMV_S32 = 5 };
+// int4 weight formats of a launch: asymmetric group 128 (fp16 scale, int4
+// zero) or the symmetric group-32 checkpoint format (bf16 scale, zero 8)
+enum W4Fmt : int { FMT_ASYM128 = 0, FMT_SYM32 = 1 };
+__host__ __device__ constexpr int fmt_kc(int fmt) { return fmt == FMT_SYM32 ? S32_KC : W4_KC; }
+__host__ __device__ constexpr int fmt_unit(int fmt) { return fmt == FMT_SYM32 ? S32_UNIT : W4_UNIT; }
 enum XSrc : int { XS_BF16 = 0, XS_EMBED = 1, XS_RESID = 2, XS_FINAL = 3, XS_F16 = 4, XS_SILU = 5 };
 enum Epi : int { EPI_Y = 0, EPI_Y_SUMSQ = 1, EPI_SILU = 2, EPI_PART = 3 };
 
@@ -97,6 +109,7 @@ struct EngineParams {
   int phase_begin, phase_end;
   int nc;               // CTAs in the grid
   long long wait_bar;   // bound in cycles on waits for other CTAs (<= 0: the default, ~2 s)
+  int fmt;              // W4Fmt of every int4 matrix of the launch
   // model dims
   int d, nq, nkv, hd, ffn, vocab, window, n_layers;
   float eps;

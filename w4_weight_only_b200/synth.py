@@ -13,7 +13,9 @@ Recipes (the pages' shapes with random-init values; no checkpoint is used):
 * embedding, lm_head N(0, 0.02) rounded to bf16;
 * prompts         uniform token ids in [0, vocab);
 * a pre-filled KV cache N(0, 1) bf16 (already-rotated keys);
-* GEMV activations N(0, 1) bf16; raw attention projections N(0, 1) fp32.
+* GEMV activations N(0, 1) bf16; raw attention projections N(0, 1) fp32;
+* checkpoints in the model card's symmetric group-32 format: uniform random
+  packed nibbles and bf16 scales 0.004 * |1 + 0.25 N(0, 1)| (+ 0.0002).
 """
 from __future__ import annotations
 
@@ -100,3 +102,31 @@ def uniforms(seed: int, n: int, device="cpu") -> torch.Tensor:
     """fp32 [n] uniform in [0, 1): the draws of the sampler."""
     g = _gen(device, seed, "uniform")
     return torch.rand((n,), generator=g, device=device, dtype=torch.float32)
+
+
+def sym32_matrix(seed: int, n: int, k: int, device="cpu", *keys):
+    """A checkpoint matrix in the symmetric group-32 format: (qweight int32
+    [n, k/8] of uniform random bits, i.e. eight uniform 4-bit nibbles per
+    word; scales bf16 [n, k/32] drawn as 0.004 * (1 + 0.25 N(0, 1)), kept
+    positive)."""
+    g = _gen(device, seed, "sym32_q", n, k, *keys)
+    qw = torch.randint(-(2 ** 31), 2 ** 31, (n, k // 8), generator=g, device=device, dtype=torch.int64)
+    s = normal((n, k // 32), device, 0.25, 1.0, seed, "sym32_s", n, k, *keys).abs_().add_(0.05).mul_(0.004)
+    return qw.to(torch.int32), s.to(torch.bfloat16)
+
+
+def sym32_layer(cfg, seed: int, l: int, device="cpu") -> dict:
+    """Layer l in the symmetric group-32 format: checkpoint pairs for qkv
+    [q+2kv, d] ([Q; K; V]), o, gate_up [2 ffn, d] ([gate; up]) and down,
+    and the four gains (1 + N(0, 0.1))."""
+    d, qd, kvd, f = cfg.d_model, cfg.n_heads * cfg.head_dim, cfg.n_kv_heads * cfg.head_dim, cfg.ffn
+    return {
+        "qkv": sym32_matrix(seed, qd + 2 * kvd, d, device, "qkv", l),
+        "o": sym32_matrix(seed, d, qd, device, "o", l),
+        "gate_up": sym32_matrix(seed, 2 * f, d, device, "gate_up", l),
+        "down": sym32_matrix(seed, d, f, device, "down", l),
+        "q_norm": normal((qd,), device, 0.1, 1.0, seed, "q_norm", l),
+        "k_norm": normal((kvd,), device, 0.1, 1.0, seed, "k_norm", l),
+        "post_attn_norm": normal((d,), device, 0.1, 1.0, seed, "post_attn_norm", l),
+        "post_ffn_norm": normal((d,), device, 0.1, 1.0, seed, "post_ffn_norm", l),
+    }
