@@ -193,8 +193,8 @@ static int launch_engine(EngineParams& P, int nb, int hd, cudaStream_t st) {
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t ctl, seg, apart, amax_v, amax_i, y_part, o, a_part, gu_part, h, f_part, lg_part, xA, xB, g_part, plan,
-      total;
+  size_t ctl, seg, apart, amax_v, amax_i, y_part, o, a_part, gu_part, h, f_part, lg_part, xA, xB, g_part, a_red,
+      f_red, rb_ctr, plan, total;
 };
 
 struct Dims {
@@ -271,6 +271,9 @@ static int ws_layout(int B, int nc, const Dims& dm, int attn, int decode, long l
   L->xA = put(decode ? (size_t)B * dm.d * 4 : 0);
   L->xB = put(decode ? (size_t)B * dm.d * 4 : 0);
   L->g_part = put(gemv_n > 0 ? (size_t)gs.ns * B * gemv_n * 4 : 0);
+  L->a_red = put(decode && g[1].ns > RED_NS ? (size_t)B * dm.d * 4 : 0);
+  L->f_red = put(decode && g[3].ns > RED_NS ? (size_t)B * dm.d * 4 : 0);
+  L->rb_ctr = put(decode ? (size_t)2 * MAX_RBC * 4 : 0);
   // phase descriptors: every phase of a decode step (standalone ops use at most two)
   L->plan = put(decode ? (size_t)(5 * dm.n_layers + 2) * sizeof(PD) : 2 * sizeof(PD));
   L->total = off;
@@ -294,6 +297,9 @@ static void ws_bind(EngineParams& P, void* ws, const WsLayout& L) {
   P.ws.xA = reinterpret_cast<float*>(b + L.xA);
   P.ws.xB = reinterpret_cast<float*>(b + L.xB);
   P.ws.g_part = reinterpret_cast<float*>(b + L.g_part);
+  P.ws.a_red = reinterpret_cast<float*>(b + L.a_red);
+  P.ws.f_red = reinterpret_cast<float*>(b + L.f_red);
+  P.ws.rb_ctr = reinterpret_cast<uint32_t*>(b + L.rb_ctr);
   P.ws.plan = b + L.plan;
 }
 
@@ -370,6 +376,7 @@ static int check_config(const W4AConfig* c) {
   if (c->d_model % W4_KC || qd % W4_KC || c->ffn % W4_KC)
     return fail(W4A_ERR_SHAPE, "d_model, heads*head_dim and ffn must be multiples of 512");
   if (c->window < 16 || c->window % 16) return fail(W4A_ERR_SHAPE, "window %d (multiple of 16)", c->window);
+  if (c->d_model / RB > MAX_RBC) return fail(W4A_ERR_SHAPE, "d_model %d (at most %d)", c->d_model, MAX_RBC * RB);
   if (c->vocab < 1) return fail(W4A_ERR_SHAPE, "vocab %d", c->vocab);
   return W4A_OK;
 }

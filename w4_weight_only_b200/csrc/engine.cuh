@@ -154,11 +154,11 @@ struct alignas(16) PD {
   float* aux;                    // reduce: per-16-row sums of squares
   int xbf_stride, vns, vstride, out_f16;
   int type, newkv, slots, seqoff;  // attention: layer type, append new k/v, cache slots, first sequence
-  const uint8_t* kc;             // attention K region
+  const uint8_t* kc;             // attention K region; a GEMV summing its own slabs: its row-block counters
   const uint8_t* vc;             // attention V region
   uint16_t* aout;                // attention output [B][nq][hd]
   const float* qpart;            // QKV slabs [qns][B][qkv_dim]
-  const float* lpart;            // lm_head slabs [lns][B][vocab]
+  const float* lpart;            // lm_head slabs [lns][B][vocab]; a GEMV summing its own slabs: the sums [B][ostride]
   const float* qnorm;            // QK-norm gains
   const float* knorm;
   int qns, lns, red_epi;
@@ -246,7 +246,9 @@ constexpr int SM_ROPE = SM_LC + 256;                // inverse frequencies, fp64
 constexpr int SM_PD = SM_ROPE + 2 * 64 * 8;         // descriptor slots
 constexpr int SM_WST = SM_PD + PD_SLOTS * (int)sizeof(PD);  // ring state per warp
 constexpr int SM_CTAB = SM_WST + NW * (int)sizeof(Ring);  // GEMV unit ranges [5 geometries][NW][4] int4
-constexpr int SM_TOTAL = SM_CTAB + 5 * NW * 64;
+constexpr int SM_RBL = SM_CTAB + 5 * NW * 64;          // row blocks this CTA sums at the phase end [1 + RBL_MAX]
+constexpr int RBL_MAX = 127;
+constexpr int SM_TOTAL = SM_RBL + (1 + RBL_MAX) * 4;
 static_assert(SM_TOTAL <= 232448, "shared memory budget");
 // attention views of the x region
 constexpr int ATT_PW = MAX_GQ * (128 + 2);                // floats of one warp's partial
@@ -396,6 +398,10 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
   const Geo& g_gu = P.geo[2];
   const Geo& g_dn = P.geo[3];
   const Geo& g_lm = P.geo[4];
+  // the O and down phases sum their own slabs when K is cut into many
+  const bool red_o = g_o.ns > RED_NS, red_dn = g_dn.ns > RED_NS;
+  const float* f_src = red_dn ? P.ws.f_red : P.ws.f_part;
+  const int f_ns = red_dn ? 1 : g_dn.ns;
   if (p == 5 * nl) {
     d.kind = PK_GEMV_BF16;
     d.blob = P.lm_head;
@@ -407,8 +413,8 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.gi = 4;
     d.xsrc = XS_FINAL;
     d.xres = P.ws.xB;
-    d.vpart = P.ws.f_part;
-    d.vns = g_dn.ns;
+    d.vpart = f_src;
+    d.vns = f_ns;
     d.vstride = dm;
     d.gain = P.layers[nl - 1].ffn_norm;
     d.gain2 = P.final_norm ? P.final_gain : nullptr;
@@ -460,8 +466,8 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     } else {
       d.xsrc = XS_RESID;
       d.xres = P.ws.xB;
-      d.vpart = P.ws.f_part;
-      d.vns = g_dn.ns;
+      d.vpart = f_src;
+      d.vns = f_ns;
       d.vstride = dm;
       d.gain = P.layers[l - 1].ffn_norm;
     }
@@ -480,6 +486,10 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.xbf_stride = qd;
     d.out = P.ws.a_part;
     d.ostride = dm;
+    if (red_o) {
+      d.kc = reinterpret_cast<const uint8_t*>(P.ws.rb_ctr);
+      d.lpart = P.ws.a_red;
+    }
   } else if (sub == 3) {
     d.blob = lw.gu;
     d.n = 2 * P.ffn;
@@ -488,8 +498,8 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.gi = 2;
     d.xsrc = XS_RESID;
     d.xres = P.ws.xA;
-    d.vpart = P.ws.a_part;
-    d.vns = g_o.ns;
+    d.vpart = red_o ? P.ws.a_red : P.ws.a_part;
+    d.vns = red_o ? 1 : g_o.ns;
     d.vstride = dm;
     d.gain = lw.attn_norm;
     d.xdst = P.ws.xB;
@@ -520,6 +530,10 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     }
     d.out = P.ws.f_part;
     d.ostride = dm;
+    if (red_dn) {
+      d.kc = reinterpret_cast<const uint8_t*>(P.ws.rb_ctr + MAX_RBC);
+      d.lpart = P.ws.f_red;
+    }
   }
 }
 
@@ -1343,6 +1357,14 @@ __device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
 #pragma unroll 1
     for (int j = 0; warp * 32 + j * NT < total8; ++j) {
       const int c = warp * 32 + j * NT + lane, bb = (warp * 32 + j * NT) / n8, k0 = (c - bb * n8) * 8;
+      if (!two) {
+        // the warp's 32 chunks (256 columns of one row): skip them unless they
+        // meet the CTA's k-range or its share of the residual copy (warp-uniform)
+        const int cw = warp * 32 + j * NT, kw = (cw - bb * n8) * 8;
+        const bool in_k = kw + 256 > kbase && kw < kbase + klen;
+        const bool in_out = has_out && cw + 32 > o0 && cw < o1;
+        if (!in_k && !in_out) continue;
+      }
       float x[8];
       if (two) {
         if (j == 0)
@@ -1745,6 +1767,82 @@ __device__ __forceinline__ void emit_rows(const PD& d, int s, int rb, Acc<NB> A,
   }
 }
 
+// Sum of the ns slabs of outputs (b, r) of a GEMV that sums its own slabs,
+// in slab order, eight L2 loads in flight.
+__device__ __forceinline__ float slab_total(const PD& d, int b, int r, int B) {
+  const float* p = reinterpret_cast<const float*>(d.out) + (size_t)b * d.ostride + r;
+  const size_t sstride = (size_t)B * d.ostride;
+  const int ns = d.g.ns;
+  float v = 0.f;
+  int sl = 0;
+#pragma unroll 1
+  for (; sl + 8 <= ns; sl += 8) {
+    float t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = __ldcg(p + (sl + i) * sstride);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v += t[i];
+  }
+#pragma unroll 1
+  for (; sl < ns; ++sl) v += __ldcg(p + sl * sstride);
+  return v;
+}
+
+// After a warp has written the partial rows of segment (slab, row block rb)
+// of a GEMV that sums its own slabs: count the row block's arrivals; the CTA
+// whose arrival completes the row block sums its ns slabs in slab order (the
+// same order whichever CTA arrives last, so the sums are bit-reproducible),
+// at the end of its unit loop with all its threads (rb_sum_pending), and
+// clears the counter for the next layer.  Release: every lane's stores, a
+// fence each, the warp barrier, one atomic add; acquire: the atomic, a fence,
+// the CTA barrier, L2 loads.
+__device__ __forceinline__ void rb_sum(const PD& d, int rb, int B, int lane) {
+  if (d.lpart == nullptr || d.epi != EPI_PART) return;
+  uint32_t* ctr = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(d.kc)) + rb;
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) {
+    last = int(atomicAdd(ctr, 1u)) == d.g.ns - 1;
+    if (last) {
+      __threadfence();
+      *ctr = 0u;
+      int* list = sm_at<int>(SM_RBL);
+      const int i = atomicAdd(list, 1);
+      if (i < RBL_MAX) {
+        list[1 + i] = rb;
+        last = 0;  // summed at the phase end
+      }
+    }
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  // the CTA's list is full: this warp sums the row block now
+  float* sum = const_cast<float*>(d.lpart);
+#pragma unroll 1
+  for (int i = lane; i < RB * B; i += 32) {
+    const int r = rb * RB + (i & (RB - 1)), b = i / RB;
+    if (r < d.rows_valid) sum[(size_t)b * d.ostride + r] = slab_total(d, b, r, B);
+  }
+}
+
+// The row blocks this CTA completed: every math thread takes (row block,
+// output) pairs.  Called by all math threads after a CTA barrier.
+__device__ __forceinline__ void rb_sum_pending(const PD& d) {
+  int* list = sm_at<int>(SM_RBL);
+  const int n = min(list[0], RBL_MAX);
+  const int B = lc().B, per = RB * B;
+  float* sum = const_cast<float*>(d.lpart);
+#pragma unroll 1
+  for (int i = threadIdx.x; i < n * per; i += NT) {
+    const int rb = list[1 + i / per], j = i - (i / per) * per;
+    const int r = rb * RB + (j & (RB - 1)), b = j / RB;
+    if (r < d.rows_valid) sum[(size_t)b * d.ostride + r] = slab_total(d, b, r, B);
+  }
+  cbar();
+  if (threadIdx.x == 0) list[0] = 0;
+}
+
 // A segment piece leaves the warp: undo the range scaling, then emit it
 // (segment wholly inside this warp) or park it in the warp's slot.
 // whole: the warp ran all of the segment's units; first: it is the warp's
@@ -1766,6 +1864,7 @@ __device__ __forceinline__ void seg_done(const PD& d, int s, int rb, bool whole,
   }
   if (whole) {
     emit_rows<NB>(d, s, rb, acc_of<NB>(acc), B, lane);
+    rb_sum(d, rb, B, lane);
   } else {
     float* q = park + (first ? 0 : 32 * 4 * NB);
 #pragma unroll
@@ -1801,6 +1900,7 @@ __device__ __forceinline__ void cta_combine(const PD& d) {
     }
   }
   emit_rows<NB>(d, c.z, c.w, acc_of<NB>(sum), lc().B, lane);
+  rb_sum(d, c.w, lc().B, lane);
 }
 
 template <int NB, int HD>
@@ -1867,17 +1967,17 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
         else
           bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
         cons_release(C, warp, lane, false);
-      } else if (s32) {
-        S32Regs sr;
-        s32_load(slot, g, lane, sr);
-        cons_release(C, warp, lane, false);
-        s32_math<NB>(sr, xl + koff * 2, xrow_b, acc, B, g);
       } else if (w4) {
         // copy the unit to registers and hand the slot back before the math
         W4Regs ur;
         w4_load(slot, g, lane, ur);
         cons_release(C, warp, lane, false);
         w4_math<NB>(ur, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g);
+      } else if (s32) {
+        S32Regs sr;
+        s32_load(slot, g, lane, sr);
+        cons_release(C, warp, lane, false);
+        s32_math<NB>(sr, xl + koff * 2, xrow_b, acc, B, g);
       } else {
         BfRegs br;
         bf_load(slot, lane, br);
@@ -1898,6 +1998,10 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
   cbar();
   mark(4);
   if (a < b) cta_combine<NB>(d);
+  if (d.lpart != nullptr && d.epi == EPI_PART) {
+    cbar();
+    rb_sum_pending(d);
+  }
   mark(5);
 }
 
@@ -2607,6 +2711,7 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     fence_mbar_init();
   }
   if (tid < 128) sm_at<double>(SM_ROPE)[tid] = P.inv_freq[tid >> 6][tid & 63];
+  if (tid == 0) sm_at<int>(SM_RBL)[0] = 0;
   const int B = P.B;
   if (P.mode != MODE_GEMV && tid < B) posb()[tid] = (P.pos_const >= 0) ? P.pos_const : P.pos[tid];
   __syncthreads();

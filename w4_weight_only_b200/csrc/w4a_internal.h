@@ -38,6 +38,11 @@ __host__ __device__ constexpr int wsp_bytes(int nb) { return NW * 2 * 32 * 4 * n
 constexpr int MAX_B = 16;
 constexpr int MAX_LAYERS = 128;
 constexpr int MAX_GQ = 8;              // query heads per KV head supported by the attention tile
+// A GEMV phase whose K is split into more than RED_NS slabs (batch > 1) sums
+// them itself: the last CTA to finish a row block adds the slabs in order, so
+// the consuming phase reads one copy of the vector instead of ns.
+constexpr int RED_NS = 4;
+constexpr int MAX_RBC = 2048;          // row blocks with a counter (d <= 32,768)
 
 static_assert(W4_UNIT == 4256, "int4 unit size");
 static_assert(W4_UNIT <= SLOT_BYTES && BF_UNIT <= SLOT_BYTES && S32_UNIT <= SLOT_BYTES, "slot too small");
@@ -101,6 +106,9 @@ struct Workspace {
   float* xA;            // residual at the layer input [B][d]
   float* xB;            // residual after attention [B][d]
   float* g_part;        // standalone GEMV output when split [ns][B][n]
+  float* a_red;         // O output with its slabs summed by the producer [B][d] (many slabs)
+  float* f_red;         // down output with its slabs summed by the producer [B][d]
+  uint32_t* rb_ctr;     // producer-side slab sums: arrivals per row block [2][MAX_RBC]
   void* plan;           // phase descriptors, one per phase of the launch
 };
 
