@@ -396,8 +396,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (TTFT) measurement")
-    ap.add_argument("--mode", default="decode", choices=["decode", "prefill"],
-                    help="prefill: only the prefill measurement (for profiling)")
+    ap.add_argument("--no-sampled", action="store_true", help="skip the sampled-decode measurement")
+    ap.add_argument("--mode", default="decode", choices=["decode", "prefill", "sample"],
+                    help="prefill / sample: only that measurement (for profiling)")
     ap.add_argument("--prefill-tokens", default="1200,8192", help="prompt lengths of the prefill measurement")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -419,6 +420,29 @@ def main():
     from w4_weight_only_b200 import api, synth
     from w4_weight_only_b200 import config as wc
     cfg = wc.olmo3_32b(args.layers)
+
+    if args.mode == "sample":
+        # the sampler alone over the full vocabulary (temperature 0.6, top-p 0.95)
+        out = {}
+        for Bs in (1, 16):
+            lgs = synth.logits_rows(SEED, Bs, cfg.vocab, 3.0, str(dev))
+            us = synth.uniforms(SEED + 1, Bs, str(dev))
+            for _ in range(args.warmup):
+                api.sample(lgs, 0.6, 0.95, us)
+            torch.cuda.synchronize()
+            c0 = torch.cuda.Event(enable_timing=True)
+            c1 = torch.cuda.Event(enable_timing=True)
+            c0.record()
+            for _ in range(args.steps):
+                api.sample(lgs, 0.6, 0.95, us)
+            c1.record()
+            torch.cuda.synchronize()
+            out[str(Bs)] = round(1000.0 * c0.elapsed_time(c1) / args.steps, 1)
+        if rank == 0:
+            print(json.dumps({"mode": "sample", "vocab": cfg.vocab, "us_per_call": out}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     # ---- model and cache (not timed) ----
     emb, head, fin = synth.embed_head(cfg, SEED, "cuda")
@@ -525,6 +549,51 @@ def main():
         e2e = {"value": job_tok_s(te, n_e2e, world), "unit": "tok/s",
                "h2d_bytes_per_step": 8, "d2h_bytes_per_step": 4}
 
+    # ---- sampled decode: the same steps with temperature 0.6 / top-p 0.95 ----
+    sampled = None
+    if not args.no_sampled:
+        u_all = synth.uniforms(SEED, args.steps, str(dev)).contiguous()
+        lg1 = torch.empty((1, cfg.vocab), dtype=torch.float32, device=dev)
+        stok = torch.zeros((args.steps + 1,), dtype=torch.int32, device=dev)
+        stok[0] = 1
+        spos = torch.arange(CTX, CTX + args.steps, dtype=torch.int32, device=dev)
+
+        def sstep(i):
+            model.decode_step(kv, stok[i:i + 1], spos[i:i + 1], logits=lg1, want_next=False)
+            stok[i + 1:i + 2].copy_(api.sample(lg1, 0.6, 0.95, u_all[i:i + 1]))
+
+        for i in range(3):
+            sstep(i)
+        torch.cuda.synchronize()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(args.steps):
+            sstep(i)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        api.check(ws)
+        ms_s = max_over_ranks(s0.elapsed_time(s1), world, dev)
+        # the sampler alone at batch 1 and 16 over the full vocabulary
+        per_call = {}
+        for Bs in (1, 16):
+            lgs = synth.logits_rows(SEED, Bs, cfg.vocab, 3.0, str(dev))
+            us = synth.uniforms(SEED + 1, Bs, str(dev))
+            api.sample(lgs, 0.6, 0.95, us)
+            torch.cuda.synchronize()
+            c0 = torch.cuda.Event(enable_timing=True)
+            c1 = torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            for _ in range(20):
+                api.sample(lgs, 0.6, 0.95, us)
+            c1.record(stream)
+            torch.cuda.synchronize()
+            per_call[str(Bs)] = round(1000.0 * c0.elapsed_time(c1) / 20, 1)
+        sampled = {"value": job_tok_s(ms_s, args.steps, world), "unit": "tok/s",
+                   "how": "each step: decode_step (logits) then w4a_sample (temperature 0.6, top-p 0.95, seeded "
+                          "draws) feeding the next token, device-timed like the greedy steps",
+                   "sample_us_per_call": per_call}
+
     pf = None
     if not args.no_prefill:
         del kv
@@ -549,7 +618,7 @@ def main():
                            "l2": "inputs larger than L2: 17.2 GB of weights streamed per token",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roof, "clocks": clk, "gpu_launches": args.steps,
-                "e2e": e2e, "cpu_baseline": base, "prefill": pf}
+                "e2e": e2e, "cpu_baseline": base, "sampled_decode": sampled, "prefill": pf}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

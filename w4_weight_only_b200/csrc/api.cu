@@ -858,11 +858,42 @@ int w4a_decode_step(W4AModel* m, const int32_t* token_ids, const W4AKVCache* kv,
 }
 
 // ---- dense prefill -------------------------------------------------------------
+// A second stream per device for the fp16 expansion of the next matrix, and
+// the events that order it against the GEMMs (created once per device).
+struct PfSide {
+  cudaStream_t st = nullptr;
+  cudaEvent_t ready[2] = {nullptr, nullptr};  // buffer b holds its matrix
+  cudaEvent_t used[2] = {nullptr, nullptr};   // buffer b's last GEMM has run
+};
+static PfSide g_side[64];
+static std::mutex g_side_mu;
+
+static int pf_side(PfSide** out) {
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(W4A_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  PfSide& s = g_side[dev];
+  if (!s.st) {
+    // the lowest priority: the GEMM's persistent CTAs (on the caller's
+    // stream) are placed first, the expansion's short blocks fill the rest
+    int lo = 0, hi = 0;
+    CK(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+    CK(cudaStreamCreateWithPriority(&s.st, cudaStreamNonBlocking, lo));
+    for (int i = 0; i < 2; ++i) {
+      CK(cudaEventCreateWithFlags(&s.ready[i], cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&s.used[i], cudaEventDisableTiming));
+    }
+  }
+  *out = &s;
+  return W4A_OK;
+}
+
 // Workspace: the batch-1 decode workspace (its control words, error word
 // included, come first; the prompt's last token runs as a decode step), then
 // the prefill buffers for Tp = T - 1 tokens.
 struct PfLayout {
-  size_t dec, X, X16, scale, Y, Q16, O16, H16, Kn, Vn, W16, total;
+  size_t dec, X, X16, scale, Y, Q16, O16, H16, Kn, Vn, W16, W16b, total;
 };
 static int pf_layout(const W4AConfig& c, int T, int nc, PfLayout* P) {
   WsLayout L;
@@ -892,6 +923,7 @@ static int pf_layout(const W4AConfig& c, int T, int nc, PfLayout* P) {
   if (2 * ffn * d > w) w = 2 * ffn * d;
   if (d * ffn > w) w = d * ffn;
   P->W16 = put(Tp ? w * 2 : 0);
+  P->W16b = put(Tp ? w * 2 : 0);
   P->total = off;
   return W4A_OK;
 }
@@ -957,7 +989,7 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   uint16_t* Q16 = reinterpret_cast<uint16_t*>(b + P.Q16);
   uint16_t* O16 = reinterpret_cast<uint16_t*>(b + P.O16);
   uint16_t* H16 = reinterpret_cast<uint16_t*>(b + P.H16);
-  uint16_t* W16 = reinterpret_cast<uint16_t*>(b + P.W16);
+  uint16_t* Wbuf[2] = {reinterpret_cast<uint16_t*>(b + P.W16), reinterpret_cast<uint16_t*>(b + P.W16b)};
   uint16_t* Kn = reinterpret_cast<uint16_t*>(b + P.Kn);
   uint16_t* Vn = reinterpret_cast<uint16_t*>(b + P.Vn);
   const int d = c.d_model, nq = c.n_heads, nkv = c.n_kv_heads, hd = c.head_dim;
@@ -969,6 +1001,48 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   if (rc) return rc;
   const float eps = float(c.eps);
   const Dims dm = dims_of(c);
+  // The int4 matrices are expanded to fp16 on a second stream, one matrix
+  // ahead, into two alternating buffers: the expansion (memory-bound) of
+  // matrix i + 1 runs under the GEMM (tensor-bound) of matrix i.
+  PfSide* side;
+  rc = pf_side(&side);
+  if (rc) return rc;
+  const int nmat = 4 * nl;
+  auto mat = [&](int i, const uint8_t*& blob, long long& n, long long& k) {
+    const LayerPtrs& L = m->layers[i / 4];
+    switch (i % 4) {
+      case 0: blob = L.qkv; n = qkv; k = d; break;
+      case 1: blob = L.o; n = d; k = qd; break;
+      case 2: blob = L.gu; n = 2LL * ffn; k = d; break;
+      default: blob = L.down; n = d; k = ffn; break;
+    }
+  };
+  auto expand = [&](int i) -> int {
+    const uint8_t* blob;
+    long long n, k;
+    mat(i, blob, n, k);
+    CK(cudaStreamWaitEvent(side->st, side->used[i & 1], 0));   // the GEMM that read this buffer last
+    CK(launch_dequant_f16(blob, n, k, dm.fmt, Wbuf[i & 1], side->st));
+    CK(cudaEventRecord(side->ready[i & 1], side->st));
+    return W4A_OK;
+  };
+  auto gemm = [&](int i, const uint16_t* A, int epi, void* out, int ldo, const float* rsc) -> int {
+    const uint8_t* blob;
+    long long n, k;
+    mat(i, blob, n, k);
+    if (i + 1 < nmat) {
+      const int r = expand(i + 1);
+      if (r) return r;
+    }
+    CK(cudaStreamWaitEvent(st, side->ready[i & 1], 0));
+    CK(launch_gemm_f16(A, Wbuf[i & 1], Tp, int(n), int(k), epi, out, ldo, rsc, err, di->sms, st));
+    CK(cudaEventRecord(side->used[i & 1], st));
+    return W4A_OK;
+  };
+  CK(cudaEventRecord(side->used[0], st));  // the side stream starts after the caller's earlier work
+  CK(cudaEventRecord(side->used[1], st));
+  rc = expand(0);
+  if (rc) return rc;
   CK(launch_embed_rows(tokens, Tp, m->embed, c.vocab, d, X, X16, scale, err, st));
   for (int l = 0; l < nl; ++l) {
     const LayerPtrs& L = m->layers[l];
@@ -977,19 +1051,16 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
     uint16_t* kc = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(kv->base) + off[l]);
     uint16_t* vc = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(kc) +
                                                al256((size_t)kv->batch * nkv * slots[l] * hd * 2));
-    CK(launch_dequant_f16(L.qkv, qkv, d, dm.fmt, W16, st));
-    CK(launch_gemm_f16(X16, W16, Tp, qkv, d, 0, Y, qkv, scale, err, di->sms, st));
+    const int i = 4 * l;
+    if ((rc = gemm(i, X16, 0, Y, qkv, scale))) return rc;
     CK(launch_qk_rows(Y, L.q_norm, L.k_norm, Q16, Kn, Vn, m->inv_freq[full], m->ms[full], eps, Tp, nq, nkv, hd,
                       start_pos, st));
     CK(launch_flash_prefill(Q16, kc, vc, Kn, Vn, O16, Tp, nq, nkv, hd, slots[l], win, start_pos, seq, err, st));
     CK(launch_kv_append(kc, vc, Kn, Vn, nkv, hd, slots[l], win, seq, start_pos, Tp, st));
-    CK(launch_dequant_f16(L.o, d, qd, dm.fmt, W16, st));
-    CK(launch_gemm_f16(O16, W16, Tp, d, qd, 0, Y, d, nullptr, err, di->sms, st));
+    if ((rc = gemm(i + 1, O16, 0, Y, d, nullptr))) return rc;
     CK(launch_resid_rows(Y, L.attn_norm, Tp, d, eps, X, X16, scale, st));
-    CK(launch_dequant_f16(L.gu, 2LL * ffn, d, dm.fmt, W16, st));
-    CK(launch_gemm_f16(X16, W16, Tp, 2 * ffn, d, 1, H16, ffn, scale, err, di->sms, st));
-    CK(launch_dequant_f16(L.down, d, ffn, dm.fmt, W16, st));
-    CK(launch_gemm_f16(H16, W16, Tp, d, ffn, 0, Y, d, nullptr, err, di->sms, st));
+    if ((rc = gemm(i + 2, X16, 1, H16, ffn, scale))) return rc;
+    if ((rc = gemm(i + 3, H16, 0, Y, d, nullptr))) return rc;
     CK(launch_resid_rows(Y, L.ffn_norm, Tp, d, eps, X, X16, scale, st));
   }
   // the last token: one decode step over the cache the prompt has filled

@@ -400,7 +400,7 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 template <int HD>
-__global__ void __launch_bounds__(FA_THREADS) flash_prefill_kernel(const FaArgs a) {
+__global__ void __launch_bounds__(FA_THREADS, 3) flash_prefill_kernel(const FaArgs a) {
   constexpr int CH = HD / 8;            // 16-byte chunks per row
   constexpr int ROWB = HD * 2;          // bytes per key row
   extern __shared__ __align__(128) uint8_t fa_sm[];
@@ -500,20 +500,36 @@ __global__ void __launch_bounds__(FA_THREADS) flash_prefill_kernel(const FaArgs 
         mma_16816(sc[n], qf[s + 1][0], qf[s + 1][1], qf[s + 1][2], qf[s + 1][3], k2, k3);
       }
     }
-    // mask (causal, window) and online softmax in base 2
+    // mask (causal, window) and online softmax in base 2; a block that every
+    // row of the warp sees whole needs no mask (warp-uniform test)
     const int j0 = jb * FA_BK;
+    const int wq_lo = a.start + q0 + warp * 16, wq_hi = wq_lo + 15;
+    const bool whole = j0 + FA_BK - 1 <= wq_lo && (a.window == 0 || wq_hi - j0 < a.window);
     float mx0 = -INFINITY, mx1 = -INFINITY;
+    if (whole) {
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
+      for (int n = 0; n < 8; ++n) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int j = j0 + 8 * n + 2 * t4 + e;
-        const bool v0 = j <= pq0 && (a.window == 0 || pq0 - j < a.window);
-        const bool v1 = j <= pq1 && (a.window == 0 || pq1 - j < a.window);
-        sc[n][e] = v0 ? sc[n][e] * a.scale_log2 : -INFINITY;
-        sc[n][2 + e] = v1 ? sc[n][2 + e] * a.scale_log2 : -INFINITY;
-        mx0 = fmaxf(mx0, sc[n][e]);
-        mx1 = fmaxf(mx1, sc[n][2 + e]);
+        for (int e = 0; e < 2; ++e) {
+          sc[n][e] *= a.scale_log2;
+          sc[n][2 + e] *= a.scale_log2;
+          mx0 = fmaxf(mx0, sc[n][e]);
+          mx1 = fmaxf(mx1, sc[n][2 + e]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int j = j0 + 8 * n + 2 * t4 + e;
+          const bool v0 = j <= pq0 && (a.window == 0 || pq0 - j < a.window);
+          const bool v1 = j <= pq1 && (a.window == 0 || pq1 - j < a.window);
+          sc[n][e] = v0 ? sc[n][e] * a.scale_log2 : -INFINITY;
+          sc[n][2 + e] = v1 ? sc[n][2 + e] * a.scale_log2 : -INFINITY;
+          mx0 = fmaxf(mx0, sc[n][e]);
+          mx1 = fmaxf(mx1, sc[n][2 + e]);
+        }
       }
     }
 #pragma unroll

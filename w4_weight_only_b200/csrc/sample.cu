@@ -4,18 +4,23 @@
 // top-p 0.95; nucleus sampling as published by Holtzman et al., 2019).
 //
 // One CTA per row.  Tokens are ordered by logit, largest first, equal logits
-// by the lower index (the order of their probabilities).  With
-// e_i = exp((z_i - max z) / T) in fp64 and Z = sum e_i:
+// by the lower index (the order of their probabilities).  Each token's weight
+// e_i = exp((z_i - max z) / T) is evaluated in fp64 and held as a 64-bit
+// fixed-point integer E_i = round(e_i 2^F), F = 63 - ceil(log2 V), so that
+// any sum of them fits 64 bits and is exact: sums in any order, by shared
+// atomics, give the same bits.  With Z = sum E_i:
 //  1. the nucleus is the shortest prefix of that order whose mass reaches
-//     top_p * Z: the largest logit key t with mass(key >= t) >= top_p Z is
-//     found by bisection over the 32-bit order-preserving keys of the fp32
-//     logits, and the first k tokens of key t (by index) complete the prefix;
+//     need = top_p Z: the largest 32-bit order-preserving logit key t with
+//     mass(key >= t) >= need, found by radix selection, eight bits of the key
+//     per pass (a 256-bin histogram of masses per pass, bins taken from the
+//     top until the mass reaches need); then the first k tokens of key t (by
+//     index) complete the prefix, k = ceil((need - mass(key > t)) / E_t);
 //  2. the drawn token is the first of the nucleus whose cumulative mass
-//     exceeds u * M (M = the nucleus mass): again the largest key s whose
-//     nucleus mass from the top through s exceeds u M, then the j-th token of
-//     key s by index.
-// Every mass is a fixed-order sum (per thread, then a shuffle tree, then the
-// warps in order), so the result does not depend on scheduling.
+//     exceeds target = floor(u M) (M = the nucleus mass): the largest key s
+//     whose nucleus mass from the top through s exceeds target (again radix
+//     selection, over the keys above t, or s = t), then the j-th token of key
+//     s by index.
+// About ten passes over the row, against ~66 for a bisection over the keys.
 #include <math.h>
 #include <stdint.h>
 
@@ -32,55 +37,155 @@ __device__ __forceinline__ uint32_t zkey(float z) {
   const uint32_t u = __float_as_uint(z + 0.0f);  // -0 and +0 are one logit
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending with z
 }
-__device__ __forceinline__ float key_z(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
 
-// Block-wide sum of one double per thread in a fixed order.
-__device__ double block_sum(double v, double* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();  // red is free again
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  double s = lane < SW ? red[lane] : 0.0;
-  if (warp == 0) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) red[SW] = s;
-  }
-  __syncthreads();
-  return red[SW];
-}
+struct Shared {
+  unsigned long long mass[256];  // histogram of masses of one radix pass (all warps)
+  unsigned int count[256];       // and of token counts
+  unsigned long long red[SW];
+  float fred[SW];
+  int ired[SW + 1];
+  // the selection in progress (written by warp 0)
+  unsigned long long above;      // mass of the keys above the current prefix range
+  unsigned long long bin_mass;   // mass of the chosen bin
+  unsigned int bin_count;
+  uint32_t prefix;
+  int found;
+};
 
-__device__ int block_sum_int(int v, int* red) {
+__device__ unsigned long long block_sum_u64(unsigned long long v, Shared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   __syncthreads();
-  if (lane == 0) red[warp] = v;
+  if (lane == 0) sh.red[warp] = v;
   __syncthreads();
-  int s = lane < SW ? red[lane] : 0;
-  if (warp == 0) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) red[SW] = s;
-  }
-  __syncthreads();
-  return red[SW];
+  unsigned long long s = 0;
+#pragma unroll 1
+  for (int w = 0; w < SW; ++w) s += sh.red[w];
+  return s;
 }
 
-// mass of the tokens whose key is at least x
-__device__ double mass_ge(const float* z, const double* e, int V, uint32_t x, double* red) {
-  double s = 0.0;
-  for (int i = threadIdx.x; i < V; i += ST)
-    if (zkey(z[i]) >= x) s += e[i];
-  return block_sum(s, red);
+// One radix pass: histogram (mass, count) by key byte `shift` of the tokens
+// whose key bits above that byte equal `hi` (all tokens at the top byte) and
+// whose key exceeds `floor_key` (all when floor_key < 0).  Lanes of a warp
+// that hit one bin are added up first (match.any groups; the 64-bit weights
+// in three 23-bit parts, so the 32-bit group sums cannot overflow), then one
+// shared atomic per group.  Then warp 0 takes bins from the top down: the
+// first bin at which (above + masses so far) reaches `need` is chosen; the
+// masses of the bins above it join `above`.
+__device__ void radix_pass(const float* z, const unsigned long long* E, int V, int shift, uint32_t hi,
+                           long long floor_key, unsigned long long need, Shared& sh) {
+  // per-warp histograms in dynamic shared memory: [SW][256] masses, then
+  // [SW][256] counts; only the warp's group leaders touch its own, so no
+  // atomics are needed
+  extern __shared__ unsigned long long wh[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long* hm = wh + warp * 256;
+  unsigned int* hc = reinterpret_cast<unsigned int*>(wh + SW * 256) + warp * 256;
+#pragma unroll
+  for (int b = lane; b < 256; b += 32) {
+    hm[b] = 0ull;
+    hc[b] = 0u;
+  }
+  __syncwarp();
+  const bool top = shift == 24;
+#pragma unroll 2
+  for (int i0 = warp * 32; i0 < V; i0 += ST) {  // warp-uniform
+    const int i = i0 + lane;
+    bool ok = i < V;
+    const uint32_t k = ok ? zkey(z[i]) : 0u;
+    if (ok && !top && (k >> (shift + 8)) != hi) ok = false;
+    if (ok && (long long)k <= floor_key) ok = false;
+    if (__ballot_sync(0xffffffffu, ok) == 0u) continue;
+    const int b = ok ? int((k >> shift) & 255u) : 256;
+    const unsigned long long e = ok ? E[i] : 0ull;
+    const unsigned peers = __match_any_sync(0xffffffffu, b);
+    const uint32_t p0 = __reduce_add_sync(peers, uint32_t(e & 0x7FFFFFull));
+    const uint32_t p1 = __reduce_add_sync(peers, uint32_t((e >> 23) & 0x7FFFFFull));
+    const uint32_t p2 = __reduce_add_sync(peers, uint32_t(e >> 46));
+    if (ok && lane == __ffs(peers) - 1) {
+      hm[b] += (unsigned long long)p0 + ((unsigned long long)p1 << 23) + ((unsigned long long)p2 << 46);
+      hc[b] += (unsigned)__popc(peers);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  // merge the warps' histograms (integer sums)
+  if (threadIdx.x < 256) {
+    const int b = threadIdx.x;
+    unsigned long long m = 0;
+    unsigned int c = 0;
+#pragma unroll 4
+    for (int w = 0; w < SW; ++w) {
+      m += wh[w * 256 + b];
+      c += reinterpret_cast<const unsigned int*>(wh + SW * 256)[w * 256 + b];
+    }
+    sh.mass[b] = m;
+    sh.count[b] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    // lane l holds bins 255 - 8 l .. 248 - 8 l (from the top)
+    unsigned long long local = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) local += sh.mass[255 - 8 * lane - j];
+    // inclusive sum over the lanes from the top (lower lane = higher bins)
+    unsigned long long incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const unsigned long long base = sh.above, excl = incl - local;
+    const unsigned mask = __ballot_sync(0xffffffffu, base + incl >= need);
+    // the lane whose range reaches need (callers guarantee one does; else the
+    // lowest non-empty bin is taken)
+    const int first = mask ? __ffs(mask) - 1 : 31;
+    if (lane == first) {
+      unsigned long long cum = base + excl;
+      int pick = -1;
+#pragma unroll 1
+      for (int j = 0; j < 8; ++j) {
+        const int b = 255 - 8 * lane - j;
+        if (sh.count[b] == 0u) continue;
+        if (cum + sh.mass[b] >= need) {
+          pick = b;
+          break;
+        }
+        cum += sh.mass[b];
+        pick = b;
+      }
+      if (pick < 0) {
+        pick = 255 - 8 * lane;
+      } else if (cum + sh.mass[pick] < need) {
+        cum -= sh.mass[pick];  // not reached: the picked bin's mass is not above it
+      }
+      sh.above = cum;
+      sh.bin_mass = sh.mass[pick];
+      sh.bin_count = sh.count[pick];
+      sh.prefix = (top ? 0u : (hi << 8)) | uint32_t(pick);
+    }
+  }
+  __syncthreads();
+}
+
+// Largest key x (over the keys above floor_key) with mass(key >= x) >= need;
+// returns x, and mass(key > x), the mass and count of key x in sh.
+__device__ uint32_t radix_select(const float* z, const unsigned long long* E, int V, long long floor_key,
+                                 unsigned long long need, unsigned long long start_above, Shared& sh) {
+  if (threadIdx.x == 0) sh.above = start_above;
+  __syncthreads();
+  uint32_t hi = 0;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    radix_pass(z, E, V, shift, hi, floor_key, need, sh);
+    hi = sh.prefix;
+  }
+  return hi;
 }
 
 // index of the j-th (1-based) token of key x, by index
-__device__ int nth_of_key(const float* z, int V, uint32_t x, int j, int* ired, int* out) {
+__device__ int nth_of_key(const float* z, int V, uint32_t x, int j, Shared& sh) {
   const int chunk = (V + ST - 1) / ST, i0 = threadIdx.x * chunk, i1 = min(V, i0 + chunk);
   int c = 0;
   for (int i = i0; i < i1; ++i) c += zkey(z[i]) == x;
@@ -93,124 +198,122 @@ __device__ int nth_of_key(const float* z, int V, uint32_t x, int j, int* ired, i
     if (lane >= o) incl += t;
   }
   __syncthreads();
-  if (lane == 31) ired[warp] = incl;
+  if (lane == 31) sh.ired[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < SW ? ired[lane] : 0;
+    int w = lane < SW ? sh.ired[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int t = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += t;
     }
-    if (lane < SW) ired[lane] = w;  // inclusive totals per warp
+    if (lane < SW) sh.ired[lane] = w;  // inclusive totals per warp
   }
   __syncthreads();
-  const int before = (warp ? ired[warp - 1] : 0) + incl - c;
+  const int before = (warp ? sh.ired[warp - 1] : 0) + incl - c;
   if (j > before && j <= before + c) {
     int seen = before;
     for (int i = i0; i < i1; ++i)
       if (zkey(z[i]) == x && ++seen == j) {
-        *out = i;
+        sh.found = i;
         break;
       }
   }
   __syncthreads();
-  return *out;
+  return sh.found;
 }
 
 __global__ void __launch_bounds__(ST, 1) sample_kernel(const float* __restrict__ logits, int V, float temperature,
                                                         float top_p, const float* __restrict__ u,
-                                                        int32_t* __restrict__ tokens, double* __restrict__ ebuf) {
-  __shared__ double red[SW + 1];
-  __shared__ int ired[SW + 1];
-  __shared__ float fred[SW];
-  __shared__ int found;
+                                                        int32_t* __restrict__ tokens,
+                                                        unsigned long long* __restrict__ ebuf, int fbits) {
+  __shared__ Shared sh;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* z = logits + (size_t)row * V;
-  double* e = ebuf + (size_t)row * V;
-  if (tid == 0) found = 0;
-  // the largest and smallest logits (their keys bound the searches)
-  float mx = -INFINITY, mn = INFINITY;
-  for (int i = tid; i < V; i += ST) {
-    mx = fmaxf(mx, z[i]);
-    mn = fminf(mn, z[i]);
-  }
+  unsigned long long* E = ebuf + (size_t)row * V;
+  if (tid == 0) sh.found = 0;
+  // the largest logit
+  float mx = -INFINITY;
+  for (int i = tid; i < V; i += ST) mx = fmaxf(mx, z[i]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-  }
-  if (lane == 0) fred[warp] = mx;
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) sh.fred[warp] = mx;
   __syncthreads();
   float m = -INFINITY;
-  for (int w = 0; w < SW; ++w) m = fmaxf(m, fred[w]);
-  __syncthreads();
-  if (lane == 0) fred[warp] = mn;
-  __syncthreads();
-  float lo_z = INFINITY;
-  for (int w = 0; w < SW; ++w) lo_z = fminf(lo_z, fred[w]);
-  // unnormalized probabilities
+  for (int w = 0; w < SW; ++w) m = fmaxf(m, sh.fred[w]);
+  // fixed-point weights
   const double invT = 1.0 / double(temperature);
-  double zs = 0.0;
+  const double scale = ldexp(1.0, fbits);
+  unsigned long long zs = 0;
   for (int i = tid; i < V; i += ST) {
-    const double v = exp((double(z[i]) - double(m)) * invT);
-    e[i] = v;
-    zs += v;
+    const double e = exp((double(z[i]) - double(m)) * invT);
+    const unsigned long long q = (unsigned long long)(e * scale + 0.5);
+    E[i] = q;
+    zs += q;
+  }
+  const unsigned long long Z = block_sum_u64(zs, sh);
+  __syncthreads();  // E is visible to the CTA
+  // 1. the nucleus
+  unsigned long long need = (unsigned long long)ceil(double(top_p) * double(Z));
+  if (need > Z) need = Z;
+  if (need < 1) need = 1;
+  const uint32_t t = radix_select(z, E, V, -1, need, 0ull, sh);
+  const unsigned long long A = sh.above;  // mass of the keys above t
+  const unsigned long long mt = sh.bin_mass;
+  const unsigned int nt = sh.bin_count;
+  const unsigned long long et = nt ? mt / nt : 0ull;  // one logit, one weight
+  unsigned long long k = nt;
+  if (et > 0 && need > A) {
+    k = (need - A + et - 1) / et;
+    if (k < 1) k = 1;
+    if (k > nt) k = nt;
+  } else if (et > 0) {
+    k = 1;
+  }
+  const unsigned long long M = A + k * et;
+  // 2. the draw: first nucleus token whose cumulative mass exceeds target
+  unsigned long long target = (unsigned long long)floor(double(u[row]) * double(M));
+  if (M > 0 && target >= M) target = M - 1;
+  uint32_t s = t;
+  unsigned long long above_s = A, es = et, ns = k;
+  if (target < A) {
+    __syncthreads();
+    s = radix_select(z, E, V, (long long)t, target + 1, 0ull, sh);
+    above_s = sh.above;
+    ns = sh.bin_count;
+    es = ns ? sh.bin_mass / ns : 0ull;
+  }
+  unsigned long long j = 1;
+  if (es > 0) {
+    j = (target - above_s) / es + 1;
+    if (j < 1) j = 1;
+    if (j > ns) j = ns;
   }
   __syncthreads();
-  const double Z = block_sum(zs, red);
-  // 1. the nucleus: largest key t with mass(key >= t) >= top_p Z
-  const double need = double(top_p) * Z;
-  uint64_t lo = zkey(lo_z), hi = uint64_t(zkey(m)) + 1;  // mass_ge(lo) = Z >= need; mass_ge(hi) = 0
-  while (hi - lo > 1) {
-    const uint64_t mid = lo + (hi - lo) / 2;
-    if (mass_ge(z, e, V, uint32_t(mid), red) >= need) lo = mid;
-    else hi = mid;
-  }
-  const uint32_t t = uint32_t(lo);
-  const double A = t == 0xffffffffu ? 0.0 : mass_ge(z, e, V, t + 1, red);
-  int nt_local = 0;
-  for (int i = tid; i < V; i += ST) nt_local += zkey(z[i]) == t;
-  const int nt = block_sum_int(nt_local, ired);
-  // the tokens of key t share one logit, hence one e (the same expression)
-  const double et = exp((double(key_z(t)) - double(m)) * invT);
-  int k = nt;
-  if (et > 0.0) {
-    const double kk = ceil((need - A) / et);
-    k = kk < 1.0 ? 1 : (kk > double(nt) ? nt : int(kk));
-  }
-  const double M = A + double(k) * et;
-  // 2. the draw: largest key s whose nucleus mass from the top through s
-  // exceeds u M (every key above t: mass_ge; t itself: M)
-  const double target = double(u[row]) * M;
-  lo = t;
-  hi = uint64_t(zkey(m)) + 1;
-  while (hi - lo > 1) {
-    const uint64_t mid = lo + (hi - lo) / 2;
-    if (mass_ge(z, e, V, uint32_t(mid), red) > target) lo = mid;
-    else hi = mid;
-  }
-  const uint32_t s = uint32_t(lo);
-  const double above = s == 0xffffffffu ? 0.0 : mass_ge(z, e, V, s + 1, red);
-  int ns_local = 0;
-  for (int i = tid; i < V; i += ST) ns_local += zkey(z[i]) == s;
-  int ns = block_sum_int(ns_local, ired);
-  const double es = exp((double(key_z(s)) - double(m)) * invT);
-  if (s == t) ns = k;  // only the first k tokens of key t are in the nucleus
-  int j = 1;
-  if (es > 0.0) {
-    const double jj = floor((target - above) / es) + 1.0;
-    j = jj < 1.0 ? 1 : (jj > double(ns) ? ns : int(jj));
-  }
-  const int tok = nth_of_key(z, V, s, j, ired, &found);
+  const int tok = nth_of_key(z, V, s, int(j), sh);
   if (tid == 0) tokens[row] = tok;
 }
 
 }  // namespace
 
+// Bits of the fixed-point weights for a row of V tokens: V e_i <= V < 2^63.
+int sample_fbits(int vocab) {
+  int lg = 0;
+  while ((1ll << lg) < (long long)vocab) ++lg;
+  return 63 - lg;
+}
+
 cudaError_t launch_sample(const float* logits, int batch, int vocab, float temperature, float top_p, const float* u,
                           int32_t* tokens, double* ebuf, cudaStream_t st) {
-  sample_kernel<<<batch, ST, 0, st>>>(logits, vocab, temperature, top_p, u, tokens, ebuf);
+  constexpr int dyn = SW * 256 * (8 + 4);  // per-warp histograms
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  sample_kernel<<<batch, ST, dyn, st>>>(logits, vocab, temperature, top_p, u, tokens,
+                                        reinterpret_cast<unsigned long long*>(ebuf), sample_fbits(vocab));
   return cudaGetLastError();
 }
 
