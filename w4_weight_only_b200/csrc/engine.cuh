@@ -166,9 +166,7 @@ struct alignas(16) PD {
 };
 static_assert(sizeof(PD) == 256, "phase descriptor size");
 
-__host__ __device__ __forceinline__ bool is_gemv_kind(int k) {
-  return k == PK_GEMV_W4 || k == PK_GEMV_BF16 || k == PK_GEMV_S32;
-}
+__host__ __device__ __forceinline__ bool is_gemv_kind(int k) { return unsigned(k) <= unsigned(PK_GEMV_S32); }
 
 // Launch constants (shared memory).
 struct LC {
@@ -246,9 +244,7 @@ constexpr int SM_ROPE = SM_LC + 256;                // inverse frequencies, fp64
 constexpr int SM_PD = SM_ROPE + 2 * 64 * 8;         // descriptor slots
 constexpr int SM_WST = SM_PD + PD_SLOTS * (int)sizeof(PD);  // ring state per warp
 constexpr int SM_CTAB = SM_WST + NW * (int)sizeof(Ring);  // GEMV unit ranges [5 geometries][NW][4] int4
-constexpr int SM_RBL = SM_CTAB + 5 * NW * 64;          // row blocks this CTA sums at the phase end [1 + RBL_MAX]
-constexpr int RBL_MAX = 127;
-constexpr int SM_TOTAL = SM_RBL + (1 + RBL_MAX) * 4;
+constexpr int SM_TOTAL = SM_CTAB + 5 * NW * 64;
 static_assert(SM_TOTAL <= 232448, "shared memory budget");
 // attention views of the x region
 constexpr int ATT_PW = MAX_GQ * (128 + 2);                // floats of one warp's partial
@@ -257,6 +253,11 @@ constexpr int SM_QF = SM_XS + NW * ATT_PW * 4;            // q fragments (4 KB)
 constexpr int SM_ASCR = SM_QF + 4096;                     // k, v rows fp32 [2][128], sums [2][NW]
 static_assert(NW * 64 * 3 * 4 <= NW * ATT_PW * 4, "piece-merge scratch inside the warp partials");
 static_assert(SM_ASCR + 2 * 128 * 4 + 2 * NW * 4 <= SM_XS + X_REGION, "attention scratch");
+// row blocks a GEMV phase's CTA sums at its end [1 + RBL_MAX]: in the q
+// region, which only attention phases use
+constexpr int SM_RBL = SM_QS;
+constexpr int RBL_MAX = 127;
+static_assert((1 + RBL_MAX) * 4 <= MAX_GQ * 128 * 4, "row-block list");
 
 extern __shared__ __align__(128) uint8_t w4a_smem[];
 
@@ -1903,7 +1904,85 @@ __device__ __forceinline__ void cta_combine(const PD& d) {
   rb_sum(d, c.w, lc().B, lane);
 }
 
-template <int NB, int HD>
+// The unit loop of a GEMV phase over this CTA's segments (S32: the
+// symmetric group-32 units; else group-128 int4 or bf16 units).
+template <int NB, bool S32>
+__device__ __forceinline__ void gemv_units(const PD& d, int4 e0, int4 e1, int kbase, int klen) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int wa = e0.x, wb = e0.y;
+  const int B = lc().B;
+  Cons C;
+  cons_load(C, warp);
+  const int kps = d.g.kps, nrb = d.g.nrb, kcw = d.kcw;
+  const bool w4 = (d.kind == PK_GEMV_W4);
+  const int xrow_b = klen * 2 + 64;
+  const uint8_t* xl = sm_at<uint8_t>(SM_XS + g * xrow_b + t * 16);
+  const float* xsg = sm_at<float>(sm_xsum(NB)) + 2 * t;
+  float* park = sm_at<float>(sm_wsp(NB)) + warp * (2 * 32 * 4 * NB) + lane * 4 * NB;
+  int u = wa;
+  int sl = e0.z, rb = e0.w, kci = e1.x;
+  float acc[NB][4];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+  // the segment in progress: its slab and row block, units run, first?
+  int cs = sl, crb = rb, cn = 0;
+  bool cfirst = true;
+#pragma unroll 1
+  for (; u < wb; ++u) {
+    if (sl != cs || rb != crb) {
+      seg_done<NB>(d, cs, crb, cn == kps, cfirst, acc, park, B, lane);
+      cs = sl;
+      crb = rb;
+      cn = 0;
+      cfirst = false;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+    }
+    ++cn;
+    const int koff = (sl * kps + kci) * kcw - kbase;
+    const uint8_t* slot = cons_wait(C, warp, lane);
+    if (NB > 1) {
+      // two batch tiles: the math reads the slot (registers are short)
+      if (S32)
+        s32_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
+      else if (w4)
+        w4_unit<NB>(slot, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g, lane);
+      else
+        bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
+      cons_release(C, warp, lane, false);
+    } else if (S32) {
+      S32Regs sr;
+      s32_load(slot, g, lane, sr);
+      cons_release(C, warp, lane, false);
+      s32_math<NB>(sr, xl + koff * 2, xrow_b, acc, B, g);
+    } else if (w4) {
+      // copy the unit to registers and hand the slot back before the math
+      W4Regs ur;
+      w4_load(slot, g, lane, ur);
+      cons_release(C, warp, lane, false);
+      w4_math<NB>(ur, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g);
+    } else {
+      BfRegs br;
+      bf_load(slot, lane, br);
+      cons_release(C, warp, lane, false);
+      bf_math<NB>(br, xl + koff * 2, xrow_b, acc, B, g);
+    }
+    if (++kci == kps) {
+      kci = 0;
+      if (++rb == nrb) {
+        rb = 0;
+        ++sl;
+      }
+    }
+  }
+  seg_done<NB>(d, cs, crb, cn == kps, cfirst, acc, park, B, lane);
+  cons_store(C, warp, lane);
+}
+
+// S32: the symmetric group-32 format's instantiation, a separate function,
+// so that the group-128 / bf16 one carries none of its code.
+template <int NB, int HD, bool S32>
 __device__ __noinline__ void gemv_phase(const PD& d) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -1916,6 +1995,9 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     a = b = 0;
     klen = 0;
   }
+  // the list of row blocks to sum shares memory with attention phases: clear
+  // it here (the staging's closing barrier orders this before any append)
+  if (tid == 0 && d.lpart != nullptr && d.epi == EPI_PART) sm_at<int>(SM_RBL)[0] = 0;
   stage_x<NB>(d, kbase, klen);
   if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_S32) {
     const uint32_t* xmax = reinterpret_cast<const uint32_t*>(red() + 32);
@@ -1926,74 +2008,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
   }
   mark(3);
   if (a < b) {
-    const int wa = e0.x, wb = e0.y;
-    const int B = lc().B;
-    Cons C;
-    cons_load(C, warp);
-    const int kps = d.g.kps, nrb = d.g.nrb, kcw = d.kcw;
-    const bool w4 = (d.kind == PK_GEMV_W4), s32 = (d.kind == PK_GEMV_S32);
-    const int xrow_b = klen * 2 + 64;
-    const uint8_t* xl = sm_at<uint8_t>(SM_XS + g * xrow_b + t * 16);
-    const float* xsg = sm_at<float>(sm_xsum(NB)) + 2 * t;
-    float* park = sm_at<float>(sm_wsp(NB)) + warp * (2 * 32 * 4 * NB) + lane * 4 * NB;
-    int u = wa;
-    int sl = e0.z, rb = e0.w, kci = e1.x;
-    float acc[NB][4];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-    // the segment in progress: its slab and row block, units run, first?
-    int cs = sl, crb = rb, cn = 0;
-    bool cfirst = true;
-#pragma unroll 1
-    for (; u < wb; ++u) {
-      if (sl != cs || rb != crb) {
-        seg_done<NB>(d, cs, crb, cn == kps, cfirst, acc, park, B, lane);
-        cs = sl;
-        crb = rb;
-        cn = 0;
-        cfirst = false;
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-      }
-      ++cn;
-      const int koff = (sl * kps + kci) * kcw - kbase;
-      const uint8_t* slot = cons_wait(C, warp, lane);
-      if (NB > 1) {
-        // two batch tiles: the math reads the slot (registers are short)
-        if (w4)
-          w4_unit<NB>(slot, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g, lane);
-        else if (s32)
-          s32_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
-        else
-          bf_unit<NB>(slot, xl + koff * 2, xrow_b, acc, B, g, lane);
-        cons_release(C, warp, lane, false);
-      } else if (w4) {
-        // copy the unit to registers and hand the slot back before the math
-        W4Regs ur;
-        w4_load(slot, g, lane, ur);
-        cons_release(C, warp, lane, false);
-        w4_math<NB>(ur, xl + koff * 2, xrow_b, xsg + (koff >> 7) * (8 * NB), acc, B, g);
-      } else if (s32) {
-        S32Regs sr;
-        s32_load(slot, g, lane, sr);
-        cons_release(C, warp, lane, false);
-        s32_math<NB>(sr, xl + koff * 2, xrow_b, acc, B, g);
-      } else {
-        BfRegs br;
-        bf_load(slot, lane, br);
-        cons_release(C, warp, lane, false);
-        bf_math<NB>(br, xl + koff * 2, xrow_b, acc, B, g);
-      }
-      if (++kci == kps) {
-        kci = 0;
-        if (++rb == nrb) {
-          rb = 0;
-          ++sl;
-        }
-      }
-    }
-    seg_done<NB>(d, cs, crb, cn == kps, cfirst, acc, park, B, lane);
-    cons_store(C, warp, lane);
+    gemv_units<NB, S32>(d, e0, e1, kbase, klen);
   }
   cbar();
   mark(4);
@@ -2905,8 +2920,10 @@ __global__ void __launch_bounds__(NTH, 1) w4a_engine_kernel(const __grid_constan
     mark(1);
     const PD& d = pd_slot(p);
     const int kind = d.kind;
-    if (is_gemv_kind(kind))
-      gemv_phase<NB, HD>(d);
+    if (kind == PK_GEMV_S32)
+      gemv_phase<NB, HD, true>(d);
+    else if (is_gemv_kind(kind))
+      gemv_phase<NB, HD, false>(d);
     else if (kind == PK_ATTN) {
       attn_phase<HD>(d);
       // every CTA advances the equal-split counters' target (see attn_combine);

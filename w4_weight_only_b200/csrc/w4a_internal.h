@@ -60,7 +60,8 @@ enum : uint32_t {
 
 // ---- engine modes / phase kinds --------------------------------------------
 enum Mode : int { MODE_DECODE = 0, MODE_GEMV = 1, MODE_ATTN = 2 };
-enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_ATTN = 2, PK_ARGMAX = 3, PK_REDUCE = 4, PK_GEMV_S32 = 5 };
+// the GEMV kinds come first: "is a GEMV" is one unsigned comparison
+enum PhaseKind : int { PK_GEMV_W4 = 0, PK_GEMV_BF16 = 1, PK_GEMV_S32 = 2, PK_ATTN = 3, PK_ARGMAX = 4, PK_REDUCE = 5 };
 // int4 weight formats of a launch: asymmetric group 128 (fp16 scale, int4
 // zero) or the symmetric group-32 checkpoint format (bf16 scale, zero 8)
 enum W4Fmt : int { FMT_ASYM128 = 0, FMT_SYM32 = 1 };
