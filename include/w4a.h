@@ -285,8 +285,9 @@ W4A_API int w4a_decode_step(W4AModel* model, const int32_t* token_ids, const W4A
  * prompt's tokens taken through each layer together (model card
  * "Limitations & roadmap": batched / tiled prefill, GEMV -> GEMM): the int4
  * projections as tcgen05 GEMMs on weights expanded to fp16, causal attention
- * with the sliding window as a flash-attention kernel, the last token as one
- * decode step.  Prompts of fewer than 9 tokens run token by token.
+ * with the sliding window as a flash-attention kernel, then the final norm
+ * and the lm_head for the last token only.  Prompts of fewer than 9 tokens
+ * run token by token.
  * last_logits: fp32 [vocab] of the last token, or NULL.  ws: device scratch
  * of w4a_prefill_workspace_bytes(model, T) bytes, zero-filled once before its
  * first use (its leading part is a decode workspace, whose error word

@@ -9,11 +9,20 @@ YaRN layer), the full vocabulary (seed 5).  Prompts of 1,200 uniform token ids
 * continuing at position 3,500 after a pre-filled N(0, 1) history, so that
   the 4,096-slot ring of the sliding-window layer wraps during the prompt.
 
-Checks: the last token's logits within 3e-2 (and its greedy token when the
-oracle's top-2 gap exceeds 2 x 3e-2), and the K and V rows the prefill wrote
+Checks: the last token's logits, and its greedy token when the oracle's
+top-2 gap exceeds 2 x the logit bound, and the K and V rows the prefill wrote
 for sampled positions of both layers, within 2e-2 of the RMS of the oracle's
 rows (they are bf16 roundings of values derived from the layer inputs).  The
 oracle runs its layer-at-a-time prefill, pinned against sequential decode.
+
+The logit bound: every prompt token, the last one included, runs through the
+dense path, whose tensor-core products take q and the attention
+probabilities rounded once to bf16 (relative 2^-9 each, uniform), where the
+decode step carries both as hi + lo bf16 pairs.  The logits' error is then
+roughly normal with an RMS near 7e-3 (the final hidden state's ~0.5 %
+relative error times the lm_head's gain, 0.02 sqrt(d) ~ 1.4), so its maximum
+over 100,278 logits sits near 4.4 RMS ~ 3e-2: the test bounds the RMS at
+1e-2 and the maximum at 4.5e-2.
 """
 import numpy as np
 import pytest
@@ -26,7 +35,8 @@ from helpers import Pair
 
 pytestmark = pytest.mark.gpu
 
-LOGIT_TOL = 3e-2
+LOGIT_TOL = 4.5e-2
+LOGIT_RMS = 1e-2
 KV_TOL = 2e-2
 T = 1200
 
@@ -62,7 +72,8 @@ def test_prefill_1200_tokens_full_shape(pair, start):
     ref, _ = om.prefill_layers(P.oracle, okv, toks.numpy(), b=0, start_pos=start)
     got = last.cpu().numpy().astype(np.float64)
     err = float(np.max(np.abs(got - ref)))
-    assert err <= LOGIT_TOL, err
+    rms = float(np.sqrt(np.mean((got - ref) ** 2)))
+    assert err <= LOGIT_TOL and rms <= LOGIT_RMS, (err, rms)
     top2 = np.sort(ref)[-2:]
     if top2[1] - top2[0] >= 2 * LOGIT_TOL:
         assert int(np.argmax(got)) == int(np.argmax(ref))

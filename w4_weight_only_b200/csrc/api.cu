@@ -35,6 +35,8 @@ cudaError_t launch_kv_append(uint16_t*, uint16_t*, const uint16_t*, const uint16
 cudaError_t launch_embed_rows(const int32_t*, int, const uint16_t*, int, int, float*, uint16_t*, float*, uint32_t*,
                               cudaStream_t);
 cudaError_t launch_resid_rows(const float*, const float*, int, int, float, float*, uint16_t*, float*, cudaStream_t);
+cudaError_t launch_final_row(const float*, const float*, int, float, uint16_t*, cudaStream_t);
+cudaError_t launch_head_gemv(const uint8_t*, int, int, const uint16_t*, float*, int*, int, cudaStream_t);
 cudaError_t launch_qk_rows(const float*, const float*, const float*, uint16_t*, uint16_t*, uint16_t*, const double*,
                            float, float, int, int, int, int, int, cudaStream_t);
 }  // namespace w4a
@@ -890,16 +892,16 @@ static int pf_side(PfSide** out) {
 }
 
 // Workspace: the batch-1 decode workspace (its control words, error word
-// included, come first; the prompt's last token runs as a decode step), then
-// the prefill buffers for Tp = T - 1 tokens.
+// included, come first; prompts too short for the dense path run as decode
+// steps), then the dense path's buffers for `rows` prompt tokens.
 struct PfLayout {
-  size_t dec, X, X16, scale, Y, Q16, O16, H16, Kn, Vn, W16, W16b, total;
+  size_t dec, X, X16, scale, Y, Q16, O16, H16, Kn, Vn, XB, ctr, W16, W16b, total;
 };
-static int pf_layout(const W4AConfig& c, int T, int nc, PfLayout* P) {
+static int pf_layout(const W4AConfig& c, int rows, int nc, PfLayout* P) {
   WsLayout L;
   int rc = ws_layout(1, nc, dims_of(c), 1, 1, 0, 0, &L);
   if (rc) return rc;
-  const size_t Tp = T > 1 ? (size_t)(T - 1) : 0;
+  const size_t Tp = rows > 0 ? (size_t)rows : 0;
   const size_t d = c.d_model, qd = (size_t)c.n_heads * c.head_dim, kvd = (size_t)c.n_kv_heads * c.head_dim;
   const size_t qkv = qd + 2 * kvd, ffn = c.ffn;
   size_t off = 0;
@@ -918,6 +920,8 @@ static int pf_layout(const W4AConfig& c, int T, int nc, PfLayout* P) {
   P->H16 = put(Tp * ffn * 2);
   P->Kn = put(Tp * kvd * 2);
   P->Vn = put(Tp * kvd * 2);
+  P->XB = put(Tp ? d * 2 : 0);
+  P->ctr = put(Tp ? 4 : 0);
   size_t w = qkv * d;
   if (d * qd > w) w = d * qd;
   if (2 * ffn * d > w) w = 2 * ffn * d;
@@ -939,7 +943,7 @@ int w4a_prefill_workspace_bytes(const W4AModel* m, int T, size_t* bytes) {
   int rc = nc_for_sizing(&nc);
   if (rc) return rc;
   PfLayout P;
-  rc = pf_layout(m->cfg, T - 1 >= PF_MIN_DENSE ? T : 1, nc, &P);
+  rc = pf_layout(m->cfg, T - 1 >= PF_MIN_DENSE ? T : 0, nc, &P);
   if (rc) return rc;
   *bytes = P.total;
   return W4A_OK;
@@ -963,10 +967,10 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   int rc = device_info(&di);
   if (rc) return rc;
   const int nl = c.n_layers;
-  const int Tp = T - 1;
-  const bool dense = Tp >= PF_MIN_DENSE;
+  const bool dense = T - 1 >= PF_MIN_DENSE;
+  const int Tp = T;  // the dense path runs every prompt token, the last one included
   PfLayout P;
-  rc = pf_layout(c, dense ? T : 1, di->sms, &P);
+  rc = pf_layout(c, dense ? T : 0, di->sms, &P);
   if (rc) return rc;
   if (ws_bytes < P.total) return fail(W4A_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, P.total);
   uint8_t* b = static_cast<uint8_t*>(ws);
@@ -992,6 +996,8 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   uint16_t* Wbuf[2] = {reinterpret_cast<uint16_t*>(b + P.W16), reinterpret_cast<uint16_t*>(b + P.W16b)};
   uint16_t* Kn = reinterpret_cast<uint16_t*>(b + P.Kn);
   uint16_t* Vn = reinterpret_cast<uint16_t*>(b + P.Vn);
+  uint16_t* XB = reinterpret_cast<uint16_t*>(b + P.XB);
+  int* hctr = reinterpret_cast<int*>(b + P.ctr);
   const int d = c.d_model, nq = c.n_heads, nkv = c.n_kv_heads, hd = c.head_dim;
   const int qd = nq * hd, qkv = qd + 2 * nkv * hd, ffn = c.ffn;
   uint64_t off[MAX_LAYERS];
@@ -1063,11 +1069,12 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
     if ((rc = gemm(i + 3, H16, 0, Y, d, nullptr))) return rc;
     CK(launch_resid_rows(Y, L.ffn_norm, Tp, d, eps, X, X16, scale, st));
   }
-  // the last token: one decode step over the cache the prompt has filled
-  // (its K / V appended, the final norm, the lm_head)
-  const bool want = last_logits != nullptr;
-  return decode_common(m, tokens + Tp, kv, seq, 1, nullptr, start_pos + Tp, want ? last_logits : nullptr, nullptr,
-                       nullptr, want ? 5 * nl + 2 : 5 * nl, b + P.dec, dec_bytes, st);
+  // the last token's logits: the final norm of its residual, then the lm_head
+  if (last_logits != nullptr) {
+    CK(launch_final_row(X + (size_t)(T - 1) * d, c.final_norm ? m->final_norm : nullptr, d, eps, XB, st));
+    CK(launch_head_gemv(m->lm_head, c.vocab, d, XB, last_logits, hctr, di->sms, st));
+  }
+  return W4A_OK;
 }
 
 // ---- int4 GEMM (the prefill's projections) ---------------------------------------

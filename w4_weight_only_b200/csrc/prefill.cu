@@ -146,20 +146,29 @@ __global__ void dequant_s32_f16_kernel(const uint8_t* __restrict__ tiled, int64_
 // GEMM on the tcgen05 tensor cores: D[M, N] = A[M, K] . B[N, K]^T, fp16 in,
 // fp32 accumulation in tensor memory
 // ---------------------------------------------------------------------------
-// Persistent: one CTA per SM walks output tiles of 128 x 256 (M-blocks of one
+// Persistent: one CTA per SM walks output tiles of 128 x BN (M-blocks of one
 // N-column consecutive, so the CTAs running together share the B panels in
-// L2).  Warp 0 (one thread) issues the TMA loads of a 4-stage ring of
-// 64-column K slices, warp 1 (one thread) issues the MMAs (four of K = 16 per
-// slice) and owns the 512 tensor-memory columns (two 256-column accumulators,
-// so the epilogue of a tile overlaps the MMAs of the next), warps 2..5 read
-// an accumulator back (each its own 32 TMEM lanes = 32 rows) and write it.
-constexpr int GM_BM = 128, GM_BN = 256, GM_BK = 64, GM_ST = 4;
+// L2).  Warp 0 (one thread) issues the TMA loads of a ring of 64-column K
+// slices, warp 1 (one thread) issues the MMAs (four of K = 16 per slice) and
+// owns 2 BN tensor-memory columns (two accumulators, so the epilogue of a
+// tile overlaps the MMAs of the next), warps 2..5 read an accumulator back
+// (each its own 32 TMEM lanes = 32 rows) and write it.
+constexpr int GM_BM = 128, GM_BK = 64;
+constexpr double GM_NARROW_COST = 0.77;  // time of a 128-wide tile / a 256-wide one (measured)
 constexpr int GM_A_BYTES = GM_BM * GM_BK * 2;
-constexpr int GM_B_BYTES = GM_BN * GM_BK * 2;
-constexpr int GM_STAGE_BYTES = GM_A_BYTES + GM_B_BYTES;
 constexpr int GM_THREADS = 192;
-constexpr int GM_SMEM = GM_ST * GM_STAGE_BYTES + 256 + 1024;  // ring, barriers, alignment slack
-constexpr uint32_t GM_IDESC = umma_idesc_f16(GM_BM, GM_BN, false);
+// Tile widths: 256 columns (4 stages), or 128 (6 stages) where the wider
+// tile would leave too much of the last wave of tiles idle.
+template <int BN>
+struct GmTile {
+  static constexpr int ST = BN == 256 ? 4 : 6;
+  static constexpr int B_BYTES = BN * GM_BK * 2;
+  static constexpr int STAGE_BYTES = GM_A_BYTES + B_BYTES;
+  static constexpr int SMEM = ST * STAGE_BYTES + 256 + 1024;  // ring, barriers, alignment slack
+  static constexpr int TMEM_COLS = 2 * BN;                    // two accumulators
+  static constexpr uint32_t IDESC = umma_idesc_f16(GM_BM, BN, false);
+};
+static_assert(GmTile<256>::SMEM <= 232448 && GmTile<128>::SMEM <= 232448, "GEMM shared memory");
 
 enum GemmEpi : int { GE_F32 = 0, GE_SILU = 1 };
 
@@ -188,9 +197,12 @@ __device__ __forceinline__ bool gm_wait(uint64_t* bar, uint32_t par, volatile in
   return true;
 }
 
+template <int BN>
 __global__ void __launch_bounds__(GM_THREADS, 1)
     gemm_f16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmArgs g) {
+  using TL = GmTile<BN>;
+  constexpr int GM_ST = TL::ST, GM_BN = BN, GM_B_BYTES = TL::B_BYTES, GM_STAGE_BYTES = TL::STAGE_BYTES;
   extern __shared__ uint8_t gm_raw[];
   // the ring at a 1,024-byte aligned shared address (the 128-byte swizzle's atom)
   uint8_t* sm = gm_raw + ((1024u - (smem_addr(gm_raw) & 1023u)) & 1023u);
@@ -225,7 +237,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
     tma_prefetch_map(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tbase, 512);
+    tmem_alloc(tbase, TL::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -291,7 +303,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
           for (int k = 0; k < GM_BK / 16; ++k) {
             const uint64_t ad = umma_desc_sw128(sA + s * GM_A_BYTES, uint32_t(k * 32));
             const uint64_t bd = umma_desc_sw128(sB + s * GM_B_BYTES, uint32_t(k * 32));
-            umma_f16(d, ad, bd, GM_IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d, ad, bd, TL::IDESC, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit(empty + s);
         }
@@ -358,12 +370,13 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, TL::TMEM_COLS);
   }
 }
 
 // ---------------------------------------------------------------------------
-// Causal GQA flash attention over the prompt (mma.sync, bf16 in, fp32 softmax)
+// Causal GQA flash attention over the prompt for head_dim 64 (mma.sync, bf16
+// in, fp32 softmax; head_dim 128 runs on the tensor-memory kernel below)
 // ---------------------------------------------------------------------------
 // CTA = 64 consecutive query positions of one query head; 4 warps of 16
 // queries.  Keys stream through shared memory in blocks of 64 positions
@@ -598,6 +611,393 @@ __global__ void __launch_bounds__(FA_THREADS, 3) flash_prefill_kernel(const FaAr
 }
 
 // ---------------------------------------------------------------------------
+// Causal GQA flash attention on the tcgen05 tensor cores (head_dim 128)
+// ---------------------------------------------------------------------------
+// CTA = two tiles of 128 consecutive queries of one query head (tile 0 the
+// earlier); they share every key / value block of 128 positions.  Per block:
+// S_i = Q_i K^T into tensor memory, the softmax warps of tile i turn their
+// rows of S_i into bf16 P_i in shared memory, O_i += P_i V accumulates in
+// tensor memory.  The two tiles alternate on the tensor core, so one tile's
+// softmax runs under the other's MMAs.  Warp roles: warps 0-3 the softmax of
+// tile 0 and 4-7 of tile 1 (thread = query row = TMEM lane), warp 8 the
+// loads (Q, K and V by tensor copies; a block that reaches back into the
+// cache is gathered row by row by the whole warp, since the ring's slots
+// and the prompt's buffer interleave there), warp 9 the MMAs (one thread)
+// and the 512 TMEM columns (S_0, S_1, O_0, O_1).  K and V tiles are stored
+// alike (rows = keys, 128-byte swizzle, two 64-column panels): S reads K as
+// a K-major operand, O reads V as an MN-major one.  The online softmax keeps
+// a row's reference maximum until a block raises it by more than 2^8, so O is
+// rescaled (read, scaled, written back in TMEM) only on those rare blocks;
+// P <= 2^8 meanwhile, exact enough in bf16 and fp32.
+constexpr int FT_BQ = 128, FT_BK = 128, FT_HD = 128;
+constexpr int FT_PANEL = 128 * 128;       // 128 rows x 64 bf16
+constexpr int FT_TILE = 2 * FT_PANEL;     // 128 x 128 bf16
+constexpr int FT_NS = 3;                  // K / V ring slots (K_j, V_j, K_j+1, ... in load order)
+constexpr int FT_THREADS = 320;
+constexpr int FT_SMEM = (4 + FT_NS) * FT_TILE + 128 + 1024;
+constexpr float FT_RESCALE = 8.f;
+static_assert(FT_SMEM <= 232448, "flash shared memory");
+
+struct FtArgs {
+  const uint16_t* kc;   // this layer's cache region [batch][nkv][slots][hd] (rows chunk-permuted)
+  const uint16_t* vc;
+  const uint16_t* kn;   // the prompt's keys / values, bf16 [nkv][T][hd]
+  const uint16_t* vn;
+  uint16_t* out;        // fp16 [T][nq][hd]
+  int T, nq, nkv, slots, window, start, seq;
+  float scale_log2;
+  uint32_t* err;
+};
+
+// Bounded wait by every lane of a warp; false (the abort flag and the error
+// word set) on a timeout or when another role has given up.
+__device__ __forceinline__ bool ft_wait(uint64_t* bar, uint32_t par, volatile int* abort_flag, uint32_t* err) {
+  if (mbar_wait_sleep(bar, par)) return true;
+  const long long t0 = clock64();
+  while (!mbar_wait_sleep(bar, par)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > PF_WAIT) {
+      *abort_flag = 1;
+      pf_error(err, EW_MBAR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Rows of a key / value block that reaches back into the cache, gathered by
+// the 32 lanes into the tile layout (row r = position pb + r): cache rows
+// verbatim but for their chunk order, prompt rows, zeros past the prompt.
+__device__ __forceinline__ void ft_gather(uint8_t* dst, const uint16_t* cache, const uint16_t* prompt, int pb, int kvh,
+                                          const FtArgs& a, int lane) {
+#pragma unroll 1
+  for (int idx = lane; idx < FT_BK * 16; idx += 32) {
+    const int r = idx >> 4, c = idx & 15;
+    uint8_t* d = dst + (c >> 3) * FT_PANEL + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+    const int p = pb + r;
+    if (p < a.start) {
+      const int slot = a.window ? p % a.window : p;
+      const size_t row = ((size_t)a.seq * a.nkv + kvh) * a.slots + slot;
+      cp_async16(d, cache + row * FT_HD + ((c ^ (slot & 7)) << 3));
+    } else if (p < a.start + a.T) {
+      cp_async16(d, prompt + ((size_t)kvh * a.T + (p - a.start)) * FT_HD + (c << 3));
+    } else {
+      *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  cp_async_commit();
+}
+
+__global__ void __launch_bounds__(FT_THREADS, 1)
+    flash_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FtArgs a) {
+  extern __shared__ uint8_t ft_raw[];
+  uint8_t* sm = ft_raw + ((1024u - (smem_addr(ft_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = sm;                  // Q_0, Q_1
+  uint8_t* sP = sm + 2 * FT_TILE;    // P_0, P_1
+  uint8_t* sR = sm + 4 * FT_TILE;    // ring
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(sm + (4 + FT_NS) * FT_TILE);
+  uint64_t* kv_full = q_full + 1;          // [FT_NS]
+  uint64_t* kv_empty = kv_full + FT_NS;    // [FT_NS]
+  uint64_t* s_full = kv_empty + FT_NS;     // [2]: S_i computed (and every earlier MMA done)
+  uint64_t* p_full = s_full + 2;           // [2]: P_i written, O_i rescaled (4 warps arrive)
+  uint64_t* o_done = p_full + 2;           // every MMA of the CTA done
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(o_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tbase + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int npair = (a.T + 2 * FT_BQ - 1) / (2 * FT_BQ);
+  const int q0 = (npair - 1 - int(blockIdx.x)) * 2 * FT_BQ;  // the longest rows first
+  const int h = blockIdx.y, kvh = h / (a.nq / a.nkv);
+  const int p_first = a.start + q0;
+  const int p_last = a.start + min(q0 + 2 * FT_BQ, a.T) - 1;
+  const int lo = a.window ? max(0, p_first - a.window + 1) : 0;
+  const int b0 = lo / FT_BK, nb = p_last / FT_BK - b0 + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+#pragma unroll 1
+    for (int s = 0; s < FT_NS; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    mbar_init(s_full + 0, 1);
+    mbar_init(s_full + 1, 1);
+    mbar_init(p_full + 0, 4);
+    mbar_init(p_full + 1, 4);
+    mbar_init(o_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmV);
+  }
+  if (warp == 9) {
+    tmem_alloc(tbase, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tbase;
+
+  if (warp == 8) {
+    // ---- loads ----
+    if (lane == 0) {
+      mbar_expect_tx(q_full, 2 * FT_TILE);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        tma_load_3d(sQ + i * FT_TILE, &tmQ, 0, h, q0 + i * FT_BQ, q_full);
+        tma_load_3d(sQ + i * FT_TILE + FT_PANEL, &tmQ, 64, h, q0 + i * FT_BQ, q_full);
+      }
+    }
+    uint32_t it = 0;
+    bool ok = true;
+#pragma unroll 1
+    for (int j = 0; j < nb && ok; ++j) {
+      const int pb = (b0 + j) * FT_BK;
+#pragma unroll 1
+      for (int kv = 0; kv < 2; ++kv, ++it) {
+        const int s = int(it % FT_NS);
+        if (it >= FT_NS) {
+          int good = 1;
+          if (lane == 0) good = ft_wait(kv_empty + s, ((it / FT_NS) - 1u) & 1u, abort_flag, a.err) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, good, 0)) {
+            ok = false;
+            break;
+          }
+        }
+        uint8_t* dst = sR + s * FT_TILE;
+        if (pb >= a.start) {
+          if (lane == 0) {
+            const CUtensorMap* m = kv ? &tmV : &tmK;
+            mbar_expect_tx(kv_full + s, FT_TILE);
+            tma_load_3d(dst, m, 0, pb - a.start, kvh, kv_full + s);
+            tma_load_3d(dst + FT_PANEL, m, 64, pb - a.start, kvh, kv_full + s);
+          }
+        } else {
+          ft_gather(dst, kv ? a.vc : a.kc, kv ? a.vn : a.kn, pb, kvh, a, lane);
+          cp_async_wait<0>();
+          fence_proxy_async();  // the rows are read by the tensor core
+          __syncwarp();
+          if (lane == 0) mbar_arrive(kv_full + s);
+        }
+      }
+    }
+    // tensor copies still in flight land before the CTA may exit
+    if (lane == 0) {
+      const uint32_t first = it > uint32_t(FT_NS) ? it - FT_NS : 0u;
+#pragma unroll 1
+      for (uint32_t j = first; j < it; ++j) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(kv_full + (j % FT_NS), (j / FT_NS) & 1u)) {
+          if (clock64() - t0 > PF_WAIT) {
+            pf_error(a.err, EW_DRAIN_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ---- MMAs (one thread) ----
+    if (lane == 0) {
+      const uint32_t idS = umma_idesc_f16(128, 128, true);
+      const uint32_t idO = idS | UMMA_B_MN;
+      auto tile_ready = [&](uint32_t i) {
+        return ft_wait(kv_full + i % FT_NS, (i / FT_NS) & 1u, abort_flag, a.err);
+      };
+      // S_qi = Q_qi K^T, K = ring tile ki
+      auto issue_s = [&](int qi, uint32_t ki) {
+        const uint8_t* q = sQ + qi * FT_TILE;
+        const uint8_t* k = sR + (ki % FT_NS) * FT_TILE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = uint32_t((ks >> 2) * FT_PANEL + (ks & 3) * 32);
+          umma_f16(tmem + uint32_t(qi * 128), umma_desc_sw128(q, off), umma_desc_sw128(k, off), idS,
+                   ks > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + qi);
+      };
+      // O_qi (+)= P_qi V, V = ring tile vi (MN-major: 64-column atoms a panel apart, 8-key groups 1 KB apart)
+      auto issue_pv = [&](int qi, uint32_t vi, bool first) {
+        const uint8_t* pm = sP + qi * FT_TILE;
+        const uint8_t* v = sR + (vi % FT_NS) * FT_TILE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = uint32_t((ks >> 2) * FT_PANEL + (ks & 3) * 32);
+          umma_f16(tmem + uint32_t(256 + qi * 128), umma_desc_sw128(pm, off),
+                   umma_desc_mn_sw128(v + ks * 16 * 128, FT_PANEL, 1024), idO, (first && ks == 0) ? 0u : 1u);
+        }
+      };
+      bool ok = ft_wait(q_full, 0u, abort_flag, a.err) && tile_ready(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(kv_empty + 0);
+      }
+#pragma unroll 1
+      for (int j = 0; j < nb && ok; ++j) {
+        const uint32_t vt = 2u * j + 1u, kn = 2u * j + 2u;
+        const bool more = j + 1 < nb;
+        if (!tile_ready(vt) || !ft_wait(p_full + 0, uint32_t(j) & 1u, abort_flag, a.err)) break;
+        tc_fence_after();
+        issue_pv(0, vt, j == 0);
+        if (more) {
+          if (!tile_ready(kn)) break;
+          tc_fence_after();
+          issue_s(0, kn);
+        }
+        if (!ft_wait(p_full + 1, uint32_t(j) & 1u, abort_flag, a.err)) break;
+        tc_fence_after();
+        issue_pv(1, vt, j == 0);
+        umma_commit(kv_empty + vt % FT_NS);
+        if (more) {
+          issue_s(1, kn);
+          umma_commit(kv_empty + kn % FT_NS);
+        }
+      }
+      umma_commit(o_done);
+      // every MMA issued has completed before the tensor memory is freed
+      const long long t0 = clock64();
+      while (!mbar_try_wait(o_done, 0u)) {
+        if (clock64() - t0 > PF_WAIT) {
+          pf_error(a.err, EW_DRAIN_TIMEOUT);
+          break;
+        }
+      }
+    }
+  } else {
+    // ---- softmax of tile qi: thread = query row = TMEM lane ----
+    const int qi = warp >> 2, r = (warp & 3) * 32 + lane;
+    const int t = q0 + qi * FT_BQ + r;
+    const int p = a.start + t;
+    const uint32_t tl = tmem + (uint32_t((warp & 3) * 32) << 16);
+    const uint32_t tS = tl + uint32_t(qi * 128), tO = tl + uint32_t(256 + qi * 128);
+    uint8_t* prow = sP + qi * FT_TILE + r * 128;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+#pragma unroll 1
+    for (int j = 0; j < nb; ++j) {
+      if (!__all_sync(0xffffffffu, ft_wait(s_full + qi, uint32_t(j) & 1u, abort_flag, a.err))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // keys pb + i visible to this row: i in [ilo, ihi] (the whole block on
+      // most blocks); two passes over S in 32-column chunks keep the code
+      // small enough for the instruction cache
+      const int pb = (b0 + j) * FT_BK;
+      const int ilo = a.window ? max(0, p - a.window + 1 - pb) : 0;
+      const int ihi = min(FT_BK - 1, p - pb);
+      const bool whole = ilo == 0 && ihi == FT_BK - 1;
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c0 = 0; c0 < FT_BK; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tS + uint32_t(c0), v);
+        tmem_ld_wait();
+        if (whole) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i >= ilo && c0 + i <= ihi) mx = fmaxf(mx, __uint_as_float(v[i]));
+        }
+      }
+      mx *= a.scale_log2;  // a positive scale commutes with the maximum
+      float alpha = 1.f;
+      if (mx > m_run + FT_RESCALE) {  // also the first finite maximum of the row
+        alpha = exp2f(m_run - mx);    // 0 while the reference was -inf
+        m_run = mx;
+      }
+      const float nref = m_run == -INFINITY ? 0.f : -m_run;
+      float sum = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < FT_BK; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tS + uint32_t(c0), v);
+        tmem_ld_wait();
+        uint32_t w[16];
+        if (whole) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float p0 = exp2f(fmaf(__uint_as_float(v[i]), a.scale_log2, nref));
+            const float p1 = exp2f(fmaf(__uint_as_float(v[i + 1]), a.scale_log2, nref));
+            sum += p0 + p1;
+            w[i >> 1] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float p0 = exp2f(fmaf(__uint_as_float(v[i]), a.scale_log2, nref));
+            float p1 = exp2f(fmaf(__uint_as_float(v[i + 1]), a.scale_log2, nref));
+            if (c0 + i < ilo || c0 + i > ihi) p0 = 0.f;
+            if (c0 + i + 1 < ilo || c0 + i + 1 > ihi) p1 = 0.f;
+            sum += p0 + p1;
+            w[i >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c8 = (c0 >> 3) + k;
+          *reinterpret_cast<uint4*>(prow + (c8 >> 3) * FT_PANEL + (((c8 & 7) ^ (r & 7)) << 4)) =
+              make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        }
+      }
+      l_run = l_run * alpha + sum;
+      // O rows whose reference moved (the previous block's P V has completed:
+      // S_qi's barrier follows it)
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + uint32_t(c), o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + uint32_t(c), o);
+        }
+        tmem_st_wait();
+      }
+      fence_proxy_async();  // P is read by the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + qi);
+    }
+    if (ok && __all_sync(0xffffffffu, ft_wait(o_done, 0u, abort_flag, a.err))) {
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      uint16_t* orow = a.out + ((size_t)t * a.nq + h) * FT_HD;
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + uint32_t(c), o);
+        tmem_ld_wait();
+        if (t < a.T) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = uint32_t(f16_checked(__uint_as_float(o[i + 2 * e]) * inv, a.err)) |
+                     (uint32_t(f16_checked(__uint_as_float(o[i + 2 * e + 1]) * inv, a.err)) << 16);
+            *reinterpret_cast<uint4*>(orow + c + i) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Per-token row kernels (one CTA of 256 threads per token)
 // ---------------------------------------------------------------------------
 constexpr int RT = 256;
@@ -674,6 +1074,76 @@ __global__ void __launch_bounds__(RT) resid_rows_kernel(const float* __restrict_
   for (int i = threadIdx.x; i < d; i += RT) x[i] += v[i] * r * gain[i];
   __syncthreads();
   row_to_f16(x, d, X16 + (size_t)t * d, scale + t, red);
+}
+
+// The last prompt token's input to the lm_head: RMSNorm with the final gains
+// (none when `gain` is null), rounded to bf16.  One CTA.
+__global__ void __launch_bounds__(RT) final_row_kernel(const float* __restrict__ x, const float* __restrict__ gain,
+                                                       int d, float eps, uint16_t* __restrict__ xb) {
+  __shared__ float red[RT / 32];
+  float r = 1.f;
+  if (gain != nullptr) {
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < d; i += RT) ss += x[i] * x[i];
+    ss = block_sum(ss, red);
+    r = rsqrtf(ss / float(d) + eps);
+  }
+  for (int i = threadIdx.x; i < d; i += RT) xb[i] = f32_to_bf16(gain != nullptr ? x[i] * r * gain[i] : x[i]);
+}
+
+// logits = W . x for one bf16 row x and the bf16 lm_head W in 16-row x
+// 128-column units of mma A fragments (the decode layout).  HBM-bound: each
+// warp takes whole 16-row blocks from a counter (so every row's sum runs in
+// one fixed order) and streams the block's units with two in flight; x sits
+// in shared memory and enters the mma as the n = 0 column (the other seven
+// columns are zero).
+constexpr int HG_THREADS = 256;
+__global__ void __launch_bounds__(HG_THREADS) head_gemv_kernel(const uint8_t* __restrict__ W, int n, int k,
+                                                               const uint16_t* __restrict__ xb, float* __restrict__ out,
+                                                               int* __restrict__ counter) {
+  extern __shared__ __align__(16) uint16_t hg_x[];
+  for (int i = threadIdx.x * 8; i < k; i += HG_THREADS * 8)
+    *reinterpret_cast<uint4*>(hg_x + i) = *reinterpret_cast<const uint4*>(xb + i);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int nrb = (n + RB - 1) / RB, nkc = k / BF_KC;
+#pragma unroll 1
+  for (;;) {
+    int rb = 0;
+    if (lane == 0) rb = atomicAdd(counter, 1);
+    rb = __shfl_sync(0xffffffffu, rb, 0);
+    if (rb >= nrb) break;
+    const uint4* u = reinterpret_cast<const uint4*>(W + (size_t)rb * nkc * BF_UNIT) + lane;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    auto math = [&](const uint4 (&av)[8], int kc) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        // k-step s holds columns 32 m + 8 t + 4 e + (0..3), m = s / 2, e = s % 2
+        const int c = kc * BF_KC + 32 * (s >> 1) + 8 * t + 4 * (s & 1);
+        const uint2 xv = g == 0 ? *reinterpret_cast<const uint2*>(hg_x + c) : make_uint2(0u, 0u);
+        mma_16816(acc, av[s].x, av[s].y, av[s].z, av[s].w, xv.x, xv.y);
+      }
+    };
+    auto load = [&](uint4 (&av)[8], int kc) {
+      const uint4* un = u + (size_t)kc * (BF_UNIT / 16);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) av[i] = __ldcs(un + i * 32);
+    };
+    uint4 a0[8], a1[8];
+    load(a0, 0);
+#pragma unroll 1
+    for (int kc = 0; kc < nkc; kc += 2) {
+      if (kc + 1 < nkc) load(a1, kc + 1);
+      math(a0, kc);
+      if (kc + 2 < nkc) load(a0, kc + 2);
+      if (kc + 1 < nkc) math(a1, kc + 1);
+    }
+    if (t == 0) {
+      const int r0 = rb * RB + g, r1 = r0 + 8;
+      if (r0 < n) out[r0] = acc[0];
+      if (r1 < n) out[r1] = acc[2];
+    }
+  }
 }
 
 struct QkArgs {
@@ -785,6 +1255,60 @@ static cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int6
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// bf16 3-D tensor [d2][d1][d0] (d0 contiguous; row strides in bytes), box of
+// 64 x b1 x b2 with the 128-byte swizzle.
+static cudaError_t make_map3(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2, int64_t s1,
+                             int64_t s2, int b1, int b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {cuuint64_t(d0), cuuint64_t(d1), cuuint64_t(d2)};
+  const cuuint64_t strides[2] = {cuuint64_t(s1), cuuint64_t(s2)};
+  const cuuint32_t box[3] = {64u, cuuint32_t(b1), cuuint32_t(b2)};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+static cudaError_t launch_flash_tc(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, const uint16_t* kn,
+                                   const uint16_t* vn, uint16_t* out, int T, int nq, int nkv, int slots, int window,
+                                   int start, int seq, uint32_t* err, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FT_SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap mq, mk, mv;
+  // q [T][nq][128]: boxes of 64 dims x 1 head x 128 tokens
+  cudaError_t e = make_map3(&mq, q, FT_HD, nq, T, (int64_t)FT_HD * 2, (int64_t)nq * FT_HD * 2, 1, FT_BQ);
+  if (e != cudaSuccess) return e;
+  // the prompt's K / V [nkv][T][128]: boxes of 64 dims x 128 keys x 1 head
+  e = make_map3(&mk, kn, FT_HD, T, nkv, (int64_t)FT_HD * 2, (int64_t)T * FT_HD * 2, FT_BK, 1);
+  if (e != cudaSuccess) return e;
+  e = make_map3(&mv, vn, FT_HD, T, nkv, (int64_t)FT_HD * 2, (int64_t)T * FT_HD * 2, FT_BK, 1);
+  if (e != cudaSuccess) return e;
+  FtArgs a;
+  a.kc = kc;
+  a.vc = vc;
+  a.kn = kn;
+  a.vn = vn;
+  a.out = out;
+  a.T = T;
+  a.nq = nq;
+  a.nkv = nkv;
+  a.slots = slots;
+  a.window = window;
+  a.start = start;
+  a.seq = seq;
+  a.scale_log2 = float(1.4426950408889634 / sqrt(double(FT_HD)));
+  a.err = err;
+  const dim3 grid((T + 2 * FT_BQ - 1) / (2 * FT_BQ), nq);
+  flash_tc_kernel<<<grid, FT_THREADS, FT_SMEM, st>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequant_f16(const uint8_t* tiled, int64_t n, int64_t k, int fmt, uint16_t* out, cudaStream_t st) {
   if (fmt == FMT_SYM32) {
     const int64_t total = (n / RB) * (k / S32_KC) * 256;
@@ -796,19 +1320,42 @@ cudaError_t launch_dequant_f16(const uint8_t* tiled, int64_t n, int64_t k, int f
   return cudaGetLastError();
 }
 
-// C = A[M, K] . B[N, K]^T; A, B fp16 K-major (16-byte aligned, K % 64 == 0).
-cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi, void* out, int ldo,
-                            const float* row_scale, uint32_t* err, int n_sms, cudaStream_t st) {
+template <int BN>
+static cudaError_t launch_gemm_tile(const CUtensorMap& ma, const uint16_t* B, int M, int N, int K, const GemmArgs& g,
+                                   int n_sms, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM);
+    const cudaError_t e =
+        cudaFuncSetAttribute(gemm_f16_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, GmTile<BN>::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  CUtensorMap ma, mb;
-  cudaError_t e = make_map(&ma, A, M, K, GM_BM);
+  CUtensorMap mb;
+  const cudaError_t e = make_map(&mb, B, N, K, BN);
   if (e != cudaSuccess) return e;
-  e = make_map(&mb, B, N, K, GM_BN);
+  const int tiles = ((M + GM_BM - 1) / GM_BM) * ((N + BN - 1) / BN);
+  const int grid = tiles < n_sms ? tiles : n_sms;
+  gemm_f16_kernel<BN><<<grid, GM_THREADS, GmTile<BN>::SMEM, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+// Tile width of a GEMM: the persistent CTAs take tiles round-robin, so the
+// time goes as the number of waves of tiles times a tile's time.  A 128-wide
+// tile takes about 0.77 of a 256-wide one (its A slice is read from shared
+// memory for half the columns); it is chosen when its waves cost less, which
+// happens for short prompts whose tiles do not fill one wave.
+int gemm_tile_width(int M, int N, int n_sms) {
+  const int64_t mt = (M + GM_BM - 1) / GM_BM;
+  const int64_t w256 = (mt * ((N + 255) / 256) + n_sms - 1) / n_sms;
+  const int64_t w128 = (mt * ((N + 127) / 128) + n_sms - 1) / n_sms;
+  return double(w128) * GM_NARROW_COST < double(w256) ? 128 : 256;
+}
+
+// C = A[M, K] . B[N, K]^T; A, B fp16 K-major (16-byte aligned, K % 64 == 0).
+cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi, void* out, int ldo,
+                            const float* row_scale, uint32_t* err, int n_sms, cudaStream_t st) {
+  CUtensorMap ma;
+  const cudaError_t e = make_map(&ma, A, M, K, GM_BM);
   if (e != cudaSuccess) return e;
   GemmArgs g;
   g.M = M;
@@ -819,10 +1366,8 @@ cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, 
   g.out = out;
   g.row_scale = row_scale;
   g.err = err;
-  const int tiles = ((M + GM_BM - 1) / GM_BM) * ((N + GM_BN - 1) / GM_BN);
-  const int grid = tiles < n_sms ? tiles : n_sms;
-  gemm_f16_kernel<<<grid, GM_THREADS, GM_SMEM, st>>>(ma, mb, g);
-  return cudaGetLastError();
+  if (gemm_tile_width(M, N, n_sms) == 128) return launch_gemm_tile<128>(ma, B, M, N, K, g, n_sms, st);
+  return launch_gemm_tile<256>(ma, B, M, N, K, g, n_sms, st);
 }
 
 cudaError_t launch_flash_prefill(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, const uint16_t* kn,
@@ -844,20 +1389,10 @@ cudaError_t launch_flash_prefill(const uint16_t* q, const uint16_t* kc, const ui
   a.seq = seq;
   a.scale_log2 = float(1.4426950408889634 / sqrt(double(hd)));
   a.err = err;
+  if (hd == 128) return launch_flash_tc(q, kc, vc, kn, vn, out, T, nq, nkv, slots, window, start, seq, err, st);
   const dim3 grid((T + FA_BQ - 1) / FA_BQ, nq);
   const int smem = 4 * FA_BK * hd * 2;
-  if (hd == 128) {
-    static bool attr = false;
-    if (!attr) {
-      const cudaError_t e =
-          cudaFuncSetAttribute(flash_prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    flash_prefill_kernel<128><<<grid, FA_THREADS, smem, st>>>(a);
-  } else {
-    flash_prefill_kernel<64><<<grid, FA_THREADS, smem, st>>>(a);
-  }
+  flash_prefill_kernel<64><<<grid, FA_THREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -870,6 +1405,25 @@ cudaError_t launch_embed_rows(const int32_t* tokens, int T, const uint16_t* embe
 cudaError_t launch_resid_rows(const float* V, const float* gain, int T, int d, float eps, float* X, uint16_t* X16,
                               float* scale, cudaStream_t st) {
   resid_rows_kernel<<<T, RT, 0, st>>>(V, gain, d, eps, X, X16, scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_final_row(const float* x, const float* gain, int d, float eps, uint16_t* xb, cudaStream_t st) {
+  final_row_kernel<<<1, RT, 0, st>>>(x, gain, d, eps, xb);
+  return cudaGetLastError();
+}
+
+// counter: one int of device memory, reset here.
+cudaError_t launch_head_gemv(const uint8_t* W, int n, int k, const uint16_t* xb, float* out, int* counter, int n_sms,
+                             cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)k * 2;
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(head_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  head_gemv_kernel<<<2 * n_sms, HG_THREADS, smem, st>>>(W, n, k, xb, out, counter);
   return cudaGetLastError();
 }
 
