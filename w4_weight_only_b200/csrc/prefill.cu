@@ -620,9 +620,9 @@ __global__ void __launch_bounds__(FA_THREADS, 3) flash_prefill_kernel(const FaAr
 // tensor memory.  The two tiles alternate on the tensor core, so one tile's
 // softmax runs under the other's MMAs.  Warp roles: warps 0-3 the softmax of
 // tile 0 and 4-7 of tile 1 (thread = query row = TMEM lane), warp 8 the
-// loads (Q, K and V by tensor copies; a block that reaches back into the
-// cache is gathered row by row by the whole warp, since the ring's slots
-// and the prompt's buffer interleave there), warp 9 the MMAs (one thread)
+// loads (Q, K and V by tensor copies, from the prompt's buffers or from the
+// cache; the one block that straddles the prompt's start, or a ring's wrap,
+// is gathered row by row by the whole warp), warp 9 the MMAs (one thread)
 // and the 512 TMEM columns (S_0, S_1, O_0, O_1).  K and V tiles are stored
 // alike (rows = keys, 128-byte swizzle, two 64-column panels): S reads K as
 // a K-major operand, O reads V as an MN-major one.  The online softmax keeps
@@ -690,7 +690,8 @@ __device__ __forceinline__ void ft_gather(uint8_t* dst, const uint16_t* cache, c
 
 __global__ void __launch_bounds__(FT_THREADS, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FtArgs a) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
+                    const __grid_constant__ CUtensorMap tmVc, const FtArgs a) {
   extern __shared__ uint8_t ft_raw[];
   uint8_t* sm = ft_raw + ((1024u - (smem_addr(ft_raw) & 1023u)) & 1023u);
   uint8_t* sQ = sm;                  // Q_0, Q_1
@@ -731,6 +732,8 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
     tma_prefetch_map(&tmQ);
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
+    tma_prefetch_map(&tmKc);
+    tma_prefetch_map(&tmVc);
   }
   if (warp == 9) {
     tmem_alloc(tbase, 512);
@@ -774,6 +777,17 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
             mbar_expect_tx(kv_full + s, FT_TILE);
             tma_load_3d(dst, m, 0, pb - a.start, kvh, kv_full + s);
             tma_load_3d(dst + FT_PANEL, m, 64, pb - a.start, kvh, kv_full + s);
+          }
+        } else if (pb + FT_BK <= a.start && (a.window == 0 || pb % a.window + FT_BK <= a.window)) {
+          // history only, in consecutive slots: the cache rows already carry
+          // the tile's chunk order (chunk c of slot s at c ^ (s & 7), and
+          // s = pb + r mod 8), so a plain tensor copy lays the tile out
+          if (lane == 0) {
+            const CUtensorMap* m = kv ? &tmVc : &tmKc;
+            const int slot0 = a.window ? pb % a.window : pb;
+            mbar_expect_tx(kv_full + s, FT_TILE);
+            tma_load_3d(dst, m, 0, slot0, a.seq * a.nkv + kvh, kv_full + s);
+            tma_load_3d(dst + FT_PANEL, m, 64, slot0, a.seq * a.nkv + kvh, kv_full + s);
           }
         } else {
           ft_gather(dst, kv ? a.vc : a.kc, kv ? a.vn : a.kn, pb, kvh, a, lane);
@@ -884,28 +898,34 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
         break;
       }
       tc_fence_after();
-      // keys pb + i visible to this row: i in [ilo, ihi] (the whole block on
-      // most blocks); two passes over S in 32-column chunks keep the code
-      // small enough for the instruction cache
+      // the row of S in four 32-column register groups, one wait; keys pb + i
+      // visible to this row: i in [ilo, ihi] (the whole block on most blocks;
+      // the others get -inf where hidden)
       const int pb = (b0 + j) * FT_BK;
       const int ilo = a.window ? max(0, p - a.window + 1 - pb) : 0;
       const int ihi = min(FT_BK - 1, p - pb);
-      const bool whole = ilo == 0 && ihi == FT_BK - 1;
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c0 = 0; c0 < FT_BK; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tS + uint32_t(c0), v);
-        tmem_ld_wait();
-        if (whole) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[i]));
-        } else {
+      uint32_t v0[32], v1[32], v2[32], v3[32];
+      tmem_ld32(tS + 0u, v0);
+      tmem_ld32(tS + 32u, v1);
+      tmem_ld32(tS + 64u, v2);
+      tmem_ld32(tS + 96u, v3);
+      tmem_ld_wait();
+      if (ilo > 0 || ihi < FT_BK - 1) {
+        auto hide = [&](uint32_t (&v)[32], int c0) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c0 + i >= ilo && c0 + i <= ihi) mx = fmaxf(mx, __uint_as_float(v[i]));
-        }
+            if (c0 + i < ilo || c0 + i > ihi) v[i] = 0xff800000u;  // -inf
+        };
+        hide(v0, 0);
+        hide(v1, 32);
+        hide(v2, 64);
+        hide(v3, 96);
       }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        mx = fmaxf(fmaxf(mx, fmaxf(__uint_as_float(v0[i]), __uint_as_float(v1[i]))),
+                   fmaxf(__uint_as_float(v2[i]), __uint_as_float(v3[i])));
       mx *= a.scale_log2;  // a positive scale commutes with the maximum
       float alpha = 1.f;
       if (mx > m_run + FT_RESCALE) {  // also the first finite maximum of the row
@@ -914,38 +934,27 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
       }
       const float nref = m_run == -INFINITY ? 0.f : -m_run;
       float sum = 0.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < FT_BK; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tS + uint32_t(c0), v);
-        tmem_ld_wait();
-        uint32_t w[16];
-        if (whole) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float p0 = exp2f(fmaf(__uint_as_float(v[i]), a.scale_log2, nref));
-            const float p1 = exp2f(fmaf(__uint_as_float(v[i + 1]), a.scale_log2, nref));
-            sum += p0 + p1;
-            w[i >> 1] = pack_bf16x2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float p0 = exp2f(fmaf(__uint_as_float(v[i]), a.scale_log2, nref));
-            float p1 = exp2f(fmaf(__uint_as_float(v[i + 1]), a.scale_log2, nref));
-            if (c0 + i < ilo || c0 + i > ihi) p0 = 0.f;
-            if (c0 + i + 1 < ilo || c0 + i + 1 > ihi) p1 = 0.f;
-            sum += p0 + p1;
-            w[i >> 1] = pack_bf16x2(p0, p1);
-          }
-        }
+      // P = 2^(s scale - m) rounded to bf16, 16 bytes (8 keys) per store
+      auto emit = [&](const uint32_t (&v)[32], int c0) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = exp2f(fmaf(__uint_as_float(v[8 * k + 2 * e]), a.scale_log2, nref));
+            const float p1 = exp2f(fmaf(__uint_as_float(v[8 * k + 2 * e + 1]), a.scale_log2, nref));
+            sum += p0 + p1;
+            w[e] = pack_bf16x2(p0, p1);
+          }
           const int c8 = (c0 >> 3) + k;
           *reinterpret_cast<uint4*>(prow + (c8 >> 3) * FT_PANEL + (((c8 & 7) ^ (r & 7)) << 4)) =
-              make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
-      }
+      };
+      emit(v0, 0);
+      emit(v1, 32);
+      emit(v2, 64);
+      emit(v3, 96);
       l_run = l_run * alpha + sum;
       // O rows whose reference moved (the previous block's P V has completed:
       // S_qi's barrier follows it)
@@ -1258,7 +1267,7 @@ static cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int6
 // bf16 3-D tensor [d2][d1][d0] (d0 contiguous; row strides in bytes), box of
 // 64 x b1 x b2 with the 128-byte swizzle.
 static cudaError_t make_map3(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2, int64_t s1,
-                             int64_t s2, int b1, int b2) {
+                             int64_t s2, int b1, int b2, bool swizzle = true) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   const cuuint64_t dims[3] = {cuuint64_t(d0), cuuint64_t(d1), cuuint64_t(d2)};
@@ -1266,8 +1275,8 @@ static cudaError_t make_map3(CUtensorMap* m, const void* base, int64_t d0, int64
   const cuuint32_t box[3] = {64u, cuuint32_t(b1), cuuint32_t(b2)};
   const cuuint32_t es[3] = {1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -1289,6 +1298,14 @@ static cudaError_t launch_flash_tc(const uint16_t* q, const uint16_t* kc, const 
   if (e != cudaSuccess) return e;
   e = make_map3(&mv, vn, FT_HD, T, nkv, (int64_t)FT_HD * 2, (int64_t)T * FT_HD * 2, FT_BK, 1);
   if (e != cudaSuccess) return e;
+  // the cache regions [.. seq][nkv][slots][128], rows as stored (no swizzle)
+  CUtensorMap mkc, mvc;
+  e = make_map3(&mkc, kc, FT_HD, slots, (int64_t)(seq + 1) * nkv, (int64_t)FT_HD * 2, (int64_t)slots * FT_HD * 2, FT_BK,
+                1, false);
+  if (e != cudaSuccess) return e;
+  e = make_map3(&mvc, vc, FT_HD, slots, (int64_t)(seq + 1) * nkv, (int64_t)FT_HD * 2, (int64_t)slots * FT_HD * 2, FT_BK,
+                1, false);
+  if (e != cudaSuccess) return e;
   FtArgs a;
   a.kc = kc;
   a.vc = vc;
@@ -1305,7 +1322,7 @@ static cudaError_t launch_flash_tc(const uint16_t* q, const uint16_t* kc, const 
   a.scale_log2 = float(1.4426950408889634 / sqrt(double(FT_HD)));
   a.err = err;
   const dim3 grid((T + 2 * FT_BQ - 1) / (2 * FT_BQ), nq);
-  flash_tc_kernel<<<grid, FT_THREADS, FT_SMEM, st>>>(mq, mk, mv, a);
+  flash_tc_kernel<<<grid, FT_THREADS, FT_SMEM, st>>>(mq, mk, mv, mkc, mvc, a);
   return cudaGetLastError();
 }
 
