@@ -5,9 +5,11 @@ out = x . W~^T for fp16 x [M, k].  The kernel multiplies weights expanded to
 fp16, (q - z) * s rounded to nearest (relative error <= 2^-11 per weight),
 with fp32 accumulation; over k products of random sign that is ~2^-11 / sqrt(3)
 of RMS(y) per output, so the bound on the max error is 3e-3 * RMS(y_ref).
-SwiGLU outputs are fp16: element-wise, the GEMM bound carried through
-silu(g) * u to first order plus fp16 rounding (2^-11 |ref|).  M covers
-partial 128-row tiles (9, 77, 200, 300, 1200).
+M covers partial 128-row tiles (9, 77, 200, 300, 1200), both tile widths
+and, at the O shape with 1,200 rows, K cut in two halves whose sums are
+added into the output.  SwiGLU outputs are fp16: element-wise, the GEMM
+bound carried through silu(g) * u to first order plus fp16 rounding
+(2^-11 |ref|).
 
 w4a_attn_prefill (causal GQA attention of a prompt over the cache, the
 sliding window as a ring): compared with the oracle's per-query attention
@@ -39,7 +41,7 @@ def _api():
 
 @pytest.mark.parametrize("n,k,M,scaled", [(768, 512, 9, False), (768, 512, 200, True), (512, 1536, 77, False),
                                           (7168, 5120, 1200, True), (5120, 27648, 300, False),
-                                          (5120, 5120, 130, False)])
+                                          (5120, 5120, 130, False), (5120, 5120, 1200, True)])
 def test_gemm_against_oracle(built_lib, cuda, n, k, M, scaled):
     api, _ = _api()
     dev = "cuda" if n * k > 4_000_000 else "cpu"

@@ -155,6 +155,7 @@ __global__ void dequant_s32_f16_kernel(const uint8_t* __restrict__ tiled, int64_
 // (each its own 32 TMEM lanes = 32 rows) and write it.
 constexpr int GM_BM = 128, GM_BK = 64;
 constexpr double GM_NARROW_COST = 0.77;  // time of a 128-wide tile / a 256-wide one (measured)
+constexpr double GM_SPLIT_COST = 1.1;    // time of a half-K tile / half a whole one (the reduction)
 constexpr int GM_A_BYTES = GM_BM * GM_BK * 2;
 constexpr int GM_THREADS = 192;
 // Tile widths: 256 columns (4 stages), or 128 (6 stages) where the wider
@@ -179,6 +180,7 @@ struct GemmArgs {
   void* out;
   const float* row_scale;  // [M] or null: row m of the product is multiplied by it
   uint32_t* err;           // error word
+  int ksplit;              // 1, or 2 (GE_F32 only): halves of K added into a zeroed out
 };
 
 // Bounded wait on an mbarrier phase; gives up (setting the CTA's abort flag
@@ -218,7 +220,13 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = (g.M + GM_BM - 1) / GM_BM, nt = (g.N + GM_BN - 1) / GM_BN;
-  const int ntiles = mt * nt, nkb = g.K / GM_BK;
+  const int ntiles = mt * nt * g.ksplit, nkb = g.K / GM_BK;
+  // tile t: M-block t % mt, N-block (t / mt) % nt, K part t / (mt nt)
+  auto krange = [&](int t, int& kb0, int& kb1) {
+    const int ks = t / (mt * nt);
+    kb0 = ks * nkb / g.ksplit;
+    kb1 = (ks + 1) * nkb / g.ksplit;
+  };
 
   if (threadIdx.x == 0) {
 #pragma unroll 1
@@ -252,9 +260,11 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
       bool ok = true;
 #pragma unroll 1
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int mb = t % mt, nb = t / mt;
+        const int mb = t % mt, nb = (t / mt) % nt;
+        int kb0, kb1;
+        krange(t, kb0, kb1);
 #pragma unroll 1
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = int(it % GM_ST);
           if (it >= GM_ST && !gm_wait(empty + s, ((it / GM_ST) & 1u) ^ 1u, abort_flag, g.err)) {
             ok = false;
@@ -291,8 +301,10 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
         if (local >= 2 && !gm_wait(tempty + buf, (use - 1u) & 1u, abort_flag, g.err)) break;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(buf * GM_BN);
+        int kb0, kb1;
+        krange(t, kb0, kb1);
 #pragma unroll 1
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = int(it % GM_ST);
           if (!gm_wait(full + s, (it / GM_ST) & 1u, abort_flag, g.err)) {
             ok = false;
@@ -303,7 +315,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
           for (int k = 0; k < GM_BK / 16; ++k) {
             const uint64_t ad = umma_desc_sw128(sA + s * GM_A_BYTES, uint32_t(k * 32));
             const uint64_t bd = umma_desc_sw128(sB + s * GM_B_BYTES, uint32_t(k * 32));
-            umma_f16(d, ad, bd, TL::IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d, ad, bd, TL::IDESC, (kb != kb0 || k != 0) ? 1u : 0u);
           }
           umma_commit(empty + s);
         }
@@ -325,7 +337,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
     int local = 0;
 #pragma unroll 1
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
-      const int mb = t % mt, nb = t / mt;
+      const int mb = t % mt, nb = (t / mt) % nt;
       const int buf = local & 1;
       const uint32_t use = uint32_t(local >> 1);
       if (!gm_wait(tfull + buf, use & 1u, abort_flag, g.err)) break;
@@ -342,11 +354,23 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
         const int col = nb * GM_BN + c;
         if (!live || col >= g.N) continue;
         if (g.epi == GE_F32) {
-          float4* o = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)row * g.ldo + col);
+          float* o = static_cast<float*>(g.out) + (size_t)row * g.ldo + col;
+          if (g.ksplit > 1) {
+            // this half of K's sum added into the zeroed output: with two
+            // halves, 0 + a + b is the same in either order
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o[i] = make_float4(__uint_as_float(r[4 * i]) * rs, __uint_as_float(r[4 * i + 1]) * rs,
-                               __uint_as_float(r[4 * i + 2]) * rs, __uint_as_float(r[4 * i + 3]) * rs);
+            for (int i = 0; i < 4; ++i)
+              asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o + 4 * i),
+                           "f"(__uint_as_float(r[4 * i]) * rs), "f"(__uint_as_float(r[4 * i + 1]) * rs),
+                           "f"(__uint_as_float(r[4 * i + 2]) * rs), "f"(__uint_as_float(r[4 * i + 3]) * rs)
+                           : "memory");
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              reinterpret_cast<float4*>(o)[i] =
+                  make_float4(__uint_as_float(r[4 * i]) * rs, __uint_as_float(r[4 * i + 1]) * rs,
+                              __uint_as_float(r[4 * i + 2]) * rs, __uint_as_float(r[4 * i + 3]) * rs);
+          }
         } else {
           // columns alternate gate j, up j: eight SwiGLU outputs
           uint32_t h[4];
@@ -1381,6 +1405,16 @@ int gemm_tile_width(int M, int N, int n_sms) {
   return double(w128) * GM_NARROW_COST < double(w256) ? 128 : 256;
 }
 
+// K in two halves (the tile count doubles, each tile does half the work) when
+// that fills the last wave of tiles better: long K, few tiles (short prompts
+// through O and down).  Only the plain fp32 output sums partial products.
+int gemm_ksplit(int M, int N, int K, int bn, int epi, int n_sms) {
+  if (epi != GE_F32 || K / GM_BK < 16) return 1;
+  const int64_t tiles = (int64_t)((M + GM_BM - 1) / GM_BM) * ((N + bn - 1) / bn);
+  const int64_t w1 = (tiles + n_sms - 1) / n_sms, w2 = (2 * tiles + n_sms - 1) / n_sms;
+  return double(w2) * 0.5 * GM_SPLIT_COST < double(w1) ? 2 : 1;
+}
+
 // C = A[M, K] . B[N, K]^T; A, B fp16 K-major (16-byte aligned, K % 64 == 0).
 cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi, void* out, int ldo,
                             const float* row_scale, uint32_t* err, int n_sms, cudaStream_t st) {
@@ -1396,7 +1430,13 @@ cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, 
   g.out = out;
   g.row_scale = row_scale;
   g.err = err;
-  if (gemm_tile_width(M, N, n_sms) == 128) return launch_gemm_tile<128>(ma, B, M, N, K, g, n_sms, st);
+  const int bn = gemm_tile_width(M, N, n_sms);
+  g.ksplit = gemm_ksplit(M, N, K, bn, epi, n_sms);
+  if (g.ksplit > 1) {
+    const cudaError_t z = cudaMemset2DAsync(out, (size_t)ldo * 4, 0, (size_t)N * 4, (size_t)M, st);
+    if (z != cudaSuccess) return z;
+  }
+  if (bn == 128) return launch_gemm_tile<128>(ma, B, M, N, K, g, n_sms, st);
   return launch_gemm_tile<256>(ma, B, M, N, K, g, n_sms, st);
 }
 
