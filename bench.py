@@ -397,7 +397,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (TTFT) measurement")
     ap.add_argument("--no-sampled", action="store_true", help="skip the sampled-decode measurement")
-    ap.add_argument("--mode", default="decode", choices=["decode", "prefill", "sample"],
+    ap.add_argument("--mode", default="decode", choices=["decode", "prefill", "sample", "attn"],
                     help="prefill / sample: only that measurement (for profiling)")
     ap.add_argument("--prefill-tokens", default="1200,8192", help="prompt lengths of the prefill measurement")
     args = ap.parse_args()
@@ -420,6 +420,43 @@ def main():
     from w4_weight_only_b200 import api, synth
     from w4_weight_only_b200 import config as wc
     cfg = wc.olmo3_32b(args.layers)
+
+    if args.mode == "attn":
+        # the prompt attention alone at the 32B shape: 8,192 tokens from
+        # position 0 through a 4,096 window, and through full attention
+        out = {}
+        nq, nkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+        T = max(int(t) for t in args.prefill_tokens.split(",") if t)
+        for window in (cfg.window, 0):
+            slots = window if window else (T + 15) // 16 * 16
+            kreg = torch.zeros((1, nkv, slots, hd), dtype=torch.bfloat16, device=dev)
+            vreg = torch.zeros_like(kreg)
+            K = synth.normal((nkv, T, hd), str(dev), 1.0, 0.0, SEED, "attn_k", T).to(torch.bfloat16)
+            V = synth.normal((nkv, T, hd), str(dev), 1.0, 0.0, SEED, "attn_v", T).to(torch.bfloat16)
+            q = synth.normal((T, nq, hd), str(dev), 1.0, 0.0, SEED, "attn_q", T).to(torch.bfloat16)
+            ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+            o = torch.empty((T, nq, hd), dtype=torch.float16, device=dev)
+            for _ in range(args.warmup):
+                api.attn_prefill(q, kreg, vreg, K, V, 1, 0, slots, window, 0, ws=ws, out=o)
+            torch.cuda.synchronize()
+            c0 = torch.cuda.Event(enable_timing=True)
+            c1 = torch.cuda.Event(enable_timing=True)
+            c0.record()
+            for _ in range(args.steps):
+                api.attn_prefill(q, kreg, vreg, K, V, 1, 0, slots, window, 0, ws=ws, out=o)
+            c1.record()
+            torch.cuda.synchronize()
+            api.check(ws)
+            ms = c0.elapsed_time(c1) / args.steps
+            vis = sum(min(t + 1, window) if window else t + 1 for t in range(T))
+            fl = 4.0 * hd * nq * vis
+            out["window %d" % window if window else "full"] = {"ms": round(ms, 4), "tflop": round(fl / 1e12, 4),
+                                                              "tflops": round(fl / (ms / 1e3) / 1e12, 1)}
+        if rank == 0:
+            print(json.dumps({"mode": "attn", "tokens": T, "heads": [nq, nkv, hd], "attention": out}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     if args.mode == "sample":
         # the sampler alone over the full vocabulary (temperature 0.6, top-p 0.95)

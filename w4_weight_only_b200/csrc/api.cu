@@ -27,7 +27,8 @@ cudaError_t launch_dequant_f16(const uint8_t*, int64_t, int64_t, int, uint16_t*,
 cudaError_t launch_tile_s32(const uint32_t*, const uint16_t*, int64_t, int64_t, int, uint8_t*, cudaStream_t);
 cudaError_t launch_unpack_s32(const uint32_t*, const uint16_t*, const uint8_t*, int64_t, int64_t, int, float*, cudaStream_t);
 cudaError_t launch_gemm_f16(const uint16_t*, const uint16_t*, int, int, int, int, void*, int, const float*, uint32_t*,
-                            int, cudaStream_t);
+                            int, cudaStream_t, int, const uint8_t* const*, const int64_t*, const int64_t*, int,
+                            uint16_t* const*);
 cudaError_t launch_flash_prefill(const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*,
                                  uint16_t*, int, int, int, int, int, int, int, int, uint32_t*, cudaStream_t);
 cudaError_t launch_kv_append(uint16_t*, uint16_t*, const uint16_t*, const uint16_t*, int, int, int, int, int, int, int,
@@ -862,40 +863,11 @@ int w4a_decode_step(W4AModel* m, const int32_t* token_ids, const W4AKVCache* kv,
 // ---- dense prefill -------------------------------------------------------------
 // A second stream per device for the fp16 expansion of the next matrix, and
 // the events that order it against the GEMMs (created once per device).
-struct PfSide {
-  cudaStream_t st = nullptr;
-  cudaEvent_t ready[2] = {nullptr, nullptr};  // buffer b holds its matrix
-  cudaEvent_t used[2] = {nullptr, nullptr};   // buffer b's last GEMM has run
-};
-static PfSide g_side[64];
-static std::mutex g_side_mu;
-
-static int pf_side(PfSide** out) {
-  int dev = 0;
-  CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return fail(W4A_ERR_UNSUPPORTED, "device index %d", dev);
-  std::lock_guard<std::mutex> lk(g_side_mu);
-  PfSide& s = g_side[dev];
-  if (!s.st) {
-    // the lowest priority: the GEMM's persistent CTAs (on the caller's
-    // stream) are placed first, the expansion's short blocks fill the rest
-    int lo = 0, hi = 0;
-    CK(cudaDeviceGetStreamPriorityRange(&lo, &hi));
-    CK(cudaStreamCreateWithPriority(&s.st, cudaStreamNonBlocking, lo));
-    for (int i = 0; i < 2; ++i) {
-      CK(cudaEventCreateWithFlags(&s.ready[i], cudaEventDisableTiming));
-      CK(cudaEventCreateWithFlags(&s.used[i], cudaEventDisableTiming));
-    }
-  }
-  *out = &s;
-  return W4A_OK;
-}
-
 // Workspace: the batch-1 decode workspace (its control words, error word
 // included, come first; prompts too short for the dense path run as decode
 // steps), then the dense path's buffers for `rows` prompt tokens.
 struct PfLayout {
-  size_t dec, X, X16, scale, Y, Q16, O16, H16, Kn, Vn, XB, ctr, W16, W16b, total;
+  size_t dec, X, X16, scale, Y, Q16, O16, H16, Kn, Vn, XB, ctr, Wq, Wo, Wg, Wd, total;
 };
 static int pf_layout(const W4AConfig& c, int rows, int nc, PfLayout* P) {
   WsLayout L;
@@ -922,12 +894,11 @@ static int pf_layout(const W4AConfig& c, int rows, int nc, PfLayout* P) {
   P->Vn = put(Tp * kvd * 2);
   P->XB = put(Tp ? d * 2 : 0);
   P->ctr = put(Tp ? 4 : 0);
-  size_t w = qkv * d;
-  if (d * qd > w) w = d * qd;
-  if (2 * ffn * d > w) w = 2 * ffn * d;
-  if (d * ffn > w) w = d * ffn;
-  P->W16 = put(Tp ? w * 2 : 0);
-  P->W16b = put(Tp ? w * 2 : 0);
+  // each of a layer's four matrices expanded to fp16 in its own buffer
+  P->Wq = put(Tp ? qkv * d * 2 : 0);
+  P->Wo = put(Tp ? d * qd * 2 : 0);
+  P->Wg = put(Tp ? 2 * ffn * d * 2 : 0);
+  P->Wd = put(Tp ? d * ffn * 2 : 0);
   P->total = off;
   return W4A_OK;
 }
@@ -993,7 +964,8 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   uint16_t* Q16 = reinterpret_cast<uint16_t*>(b + P.Q16);
   uint16_t* O16 = reinterpret_cast<uint16_t*>(b + P.O16);
   uint16_t* H16 = reinterpret_cast<uint16_t*>(b + P.H16);
-  uint16_t* Wbuf[2] = {reinterpret_cast<uint16_t*>(b + P.W16), reinterpret_cast<uint16_t*>(b + P.W16b)};
+  uint16_t* Wbuf[4] = {reinterpret_cast<uint16_t*>(b + P.Wq), reinterpret_cast<uint16_t*>(b + P.Wo),
+                       reinterpret_cast<uint16_t*>(b + P.Wg), reinterpret_cast<uint16_t*>(b + P.Wd)};
   uint16_t* Kn = reinterpret_cast<uint16_t*>(b + P.Kn);
   uint16_t* Vn = reinterpret_cast<uint16_t*>(b + P.Vn);
   uint16_t* XB = reinterpret_cast<uint16_t*>(b + P.XB);
@@ -1007,14 +979,14 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
   if (rc) return rc;
   const float eps = float(c.eps);
   const Dims dm = dims_of(c);
-  // The int4 matrices are expanded to fp16 on a second stream, one matrix
-  // ahead, into two alternating buffers: the expansion (memory-bound) of
-  // matrix i + 1 runs under the GEMM (tensor-bound) of matrix i.
-  PfSide* side;
-  rc = pf_side(&side);
-  if (rc) return rc;
+  // The int4 matrices are expanded to fp16, each into its own buffer, by
+  // spare warps of an earlier GEMM (memory-bound work under a tensor-bound
+  // product): the gate/up GEMM of layer l expands its down matrix, the down
+  // GEMM expands layer l + 1's QKV, O and gate/up; layer 0's first three are
+  // expanded up front.  Matrix i (4 per layer) goes to buffer i % 4, last
+  // read by the same matrix of the layer before, whose GEMM has finished.
   const int nmat = 4 * nl;
-  auto mat = [&](int i, const uint8_t*& blob, long long& n, long long& k) {
+  auto mat = [&](int i, const uint8_t*& blob, int64_t& n, int64_t& k) {
     const LayerPtrs& L = m->layers[i / 4];
     switch (i % 4) {
       case 0: blob = L.qkv; n = qkv; k = d; break;
@@ -1023,32 +995,36 @@ int w4a_prefill(W4AModel* m, const int32_t* tokens, int T, const W4AKVCache* kv,
       default: blob = L.down; n = d; k = ffn; break;
     }
   };
-  auto expand = [&](int i) -> int {
-    const uint8_t* blob;
-    long long n, k;
-    mat(i, blob, n, k);
-    CK(cudaStreamWaitEvent(side->st, side->used[i & 1], 0));   // the GEMM that read this buffer last
-    CK(launch_dequant_f16(blob, n, k, dm.fmt, Wbuf[i & 1], side->st));
-    CK(cudaEventRecord(side->ready[i & 1], side->st));
-    return W4A_OK;
-  };
   auto gemm = [&](int i, const uint16_t* A, int epi, void* out, int ldo, const float* rsc) -> int {
     const uint8_t* blob;
-    long long n, k;
+    int64_t n, k;
     mat(i, blob, n, k);
-    if (i + 1 < nmat) {
-      const int r = expand(i + 1);
-      if (r) return r;
+    const uint8_t* nb[3];
+    int64_t nn[3], nk[3];
+    uint16_t* nd[3];
+    int cnt = 0;
+    auto add = [&](int j) {
+      if (j >= nmat) return;
+      mat(j, nb[cnt], nn[cnt], nk[cnt]);
+      nd[cnt] = Wbuf[j % 4];
+      ++cnt;
+    };
+    if (i % 4 == 2) add(i + 1);
+    if (i % 4 == 3) {
+      add(i + 1);
+      add(i + 2);
+      add(i + 3);
     }
-    CK(cudaStreamWaitEvent(st, side->ready[i & 1], 0));
-    CK(launch_gemm_f16(A, Wbuf[i & 1], Tp, int(n), int(k), epi, out, ldo, rsc, err, di->sms, st));
-    CK(cudaEventRecord(side->used[i & 1], st));
+    CK(launch_gemm_f16(A, Wbuf[i % 4], Tp, int(n), int(k), epi, out, ldo, rsc, err, di->sms, st, cnt, nb, nn, nk,
+                       dm.fmt, nd));
     return W4A_OK;
   };
-  CK(cudaEventRecord(side->used[0], st));  // the side stream starts after the caller's earlier work
-  CK(cudaEventRecord(side->used[1], st));
-  rc = expand(0);
-  if (rc) return rc;
+  for (int i = 0; i < 3 && i < nmat; ++i) {
+    const uint8_t* blob;
+    int64_t n, k;
+    mat(i, blob, n, k);
+    CK(launch_dequant_f16(blob, n, k, dm.fmt, Wbuf[i], st));
+  }
   CK(launch_embed_rows(tokens, Tp, m->embed, c.vocab, d, X, X16, scale, err, st));
   for (int l = 0; l < nl; ++l) {
     const LayerPtrs& L = m->layers[l];
@@ -1111,7 +1087,7 @@ int w4a_gemm(const W4ATensor* W, const uint16_t* x, int M, const float* row_scal
   CK(launch_dequant_f16(static_cast<const uint8_t*>(W->qweight), W->n, W->k, tensor_fmt(W), W16, st));
   const int silu = epilogue == W4A_EPI_SILU_MUL ? 1 : 0;
   CK(launch_gemm_f16(x, W16, M, int(W->n), int(W->k), silu, out, silu ? int(W->n / 2) : int(W->n), row_scale, err,
-                     di->sms, st));
+                     di->sms, st, 0, nullptr, nullptr, nullptr, 0, nullptr));
   return W4A_OK;
 }
 

@@ -43,29 +43,16 @@ __device__ __forceinline__ uint16_t f16_checked(float v, uint32_t* err) {
 // ---------------------------------------------------------------------------
 // int4 tiled units -> fp16 [n, k] (tiled row order)
 // ---------------------------------------------------------------------------
-// One thread per (unit, 32-column slice m, lane): the two code words of
-// k-steps 2m and 2m + 1 hold rows g and g + 8 at columns 32 m + 8 t .. + 7.
-__global__ void dequant_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n, int64_t k,
-                                   uint16_t* __restrict__ out) {
-  const int64_t nkc = k / W4_KC;
-  const int64_t total = (n / RB) * nkc * 16 * 32;
-  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= total) return;
-  const int lane = int(id & 31);
-  const int m = int((id >> 5) & 15);
-  const int64_t unit = id >> 9;
-  const int64_t rb = unit / nkc, kc = unit - rb * nkc;
-  const int g = lane >> 2, t = lane & 3;
-  const uint8_t* u = tiled + unit * W4_UNIT;
-  const int s0 = 2 * m, s1 = 2 * m + 1;
-  const uint32_t w0 = reinterpret_cast<const uint32_t*>(u + ((s0 >> 2) * 32 + lane) * 16)[s0 & 3];
-  const uint32_t w1 = reinterpret_cast<const uint32_t*>(u + ((s1 >> 2) * 32 + lane) * 16)[s1 & 3];
-  const int grp = m >> 2;
-  const uint16_t* sc = reinterpret_cast<const uint16_t*>(u + 4096);
-  const uint32_t* zw = reinterpret_cast<const uint32_t*>(u + 4224);
-  const float s_lo = half_bits_to_f32(sc[g * 8 + grp * 2 + 0]), s_hi = half_bits_to_f32(sc[g * 8 + grp * 2 + 1]);
-  const int z_lo = int((zw[grp * 2 + 0] >> (4 * g)) & 15u), z_hi = int((zw[grp * 2 + 1] >> (4 * g)) & 15u);
-  // nibble j of a word: row g (+8 when j odd), column offset 2 [j & 2] + [j & 4]
+// One unit per warp: lane (g, t) holds, for every k-step s of the unit, the
+// code word of rows g and g + 8 at columns 32 (s / 2) + 8 t + 4 (s % 2) ..
+// + 3 (eight nibbles: row g + 8 when the nibble index is odd, column offset
+// 2 [j & 2] + [j & 4]); its words are eight (four) 16-byte loads, coalesced
+// across the warp.  Both formats: asymmetric group 128 (16 x 512 units, fp16
+// scales, int4 zeros) and the symmetric group-32 checkpoint (16 x 256 units,
+// bf16 scales, zero 8).  Streaming loads and stores: the int4 units are read
+// once and the fp16 rows are read back by a later GEMM, not from L2.
+__device__ __forceinline__ void dq_pair(uint32_t w0, uint32_t w1, float s_lo, float s_hi, int z_lo, int z_hi,
+                                        uint16_t* __restrict__ dst, int64_t k) {
   uint16_t lo[8], hi[8];
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
@@ -80,8 +67,6 @@ __global__ void dequant_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n,
         lo[c] = f32_to_f16(float(q - z_lo) * s_lo);
     }
   }
-  const int64_t col = kc * W4_KC + 32 * m + 8 * t;
-  const int64_t r0 = rb * RB + g;
   uint4 a, b;
   a.x = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
   a.y = uint32_t(lo[2]) | (uint32_t(lo[3]) << 16);
@@ -91,55 +76,65 @@ __global__ void dequant_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n,
   b.y = uint32_t(hi[2]) | (uint32_t(hi[3]) << 16);
   b.z = uint32_t(hi[4]) | (uint32_t(hi[5]) << 16);
   b.w = uint32_t(hi[6]) | (uint32_t(hi[7]) << 16);
-  *reinterpret_cast<uint4*>(out + r0 * k + col) = a;
-  *reinterpret_cast<uint4*>(out + (r0 + 8) * k + col) = b;
+  __stcs(reinterpret_cast<uint4*>(dst), a);
+  __stcs(reinterpret_cast<uint4*>(dst + 8 * k), b);
 }
+__device__ __forceinline__ uint32_t u4c(const uint4& v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
 
-// The symmetric group-32 units (16 x 256, bf16 scales, zero 8) -> fp16 [n, k].
-__global__ void dequant_s32_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n, int64_t k,
-                                       uint16_t* __restrict__ out) {
-  const int64_t nkc = k / S32_KC;
-  const int64_t total = (n / RB) * nkc * 8 * 32;
-  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= total) return;
-  const int lane = int(id & 31);
-  const int m = int((id >> 5) & 7);
-  const int64_t unit = id >> 8;
-  const int64_t rb = unit / nkc, kc = unit - rb * nkc;
+__device__ __forceinline__ void dq_unit(const uint8_t* __restrict__ tiled, int64_t k, int fmt, int unit, int lane,
+                                        uint16_t* __restrict__ out) {
   const int g = lane >> 2, t = lane & 3;
-  const uint8_t* u = tiled + unit * S32_UNIT;
-  const int s0 = 2 * m, s1 = 2 * m + 1;
-  const uint32_t w0 = reinterpret_cast<const uint32_t*>(u + ((s0 >> 2) * 32 + lane) * 16)[s0 & 3];
-  const uint32_t w1 = reinterpret_cast<const uint32_t*>(u + ((s1 >> 2) * 32 + lane) * 16)[s1 & 3];
-  const uint16_t* sc = reinterpret_cast<const uint16_t*>(u + 2048);
-  const float s_lo = bf16_to_f32(sc[g * 16 + m * 2 + 0]), s_hi = bf16_to_f32(sc[g * 16 + m * 2 + 1]);
-  uint16_t lo[8], hi[8];
+  if (fmt == FMT_SYM32) {
+    const int nkc = int(k / S32_KC), rb = unit / nkc, kc = unit - rb * nkc;
+    const uint8_t* u = tiled + (size_t)unit * S32_UNIT;
+    uint4 wv[4];
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const uint32_t w = e ? w1 : w0;
+    for (int q = 0; q < 4; ++q) wv[q] = __ldcs(reinterpret_cast<const uint4*>(u) + q * 32 + lane);
+    const uint4 sa = __ldcs(reinterpret_cast<const uint4*>(u + 2048) + 2 * g);
+    const uint4 sb = __ldcs(reinterpret_cast<const uint4*>(u + 2048) + 2 * g + 1);
+    uint16_t* row = out + ((size_t)rb * RB + g) * k + (size_t)kc * S32_KC + 8 * t;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int q = int((w >> (4 * j)) & 15u) - 8;
-      const int c = 4 * e + ((j & 2) ? 2 : 0) + ((j & 4) ? 1 : 0);
-      if (j & 1)
-        hi[c] = f32_to_f16(float(q) * s_hi);
-      else
-        lo[c] = f32_to_f16(float(q) * s_lo);
+    for (int m = 0; m < 8; ++m) {
+      // scales of group m: bf16 (row g, row g + 8) in word m of the row's 32 bytes
+      const uint32_t sw = m < 4 ? u4c(sa, m) : u4c(sb, m - 4);
+      dq_pair(u4c(wv[m >> 1], (2 * m) & 3), u4c(wv[m >> 1], (2 * m + 1) & 3), bf16_to_f32(uint16_t(sw & 0xffffu)),
+              bf16_to_f32(uint16_t(sw >> 16)), 8, 8, row + 32 * m, k);
+    }
+  } else {
+    const int nkc = int(k / W4_KC), rb = unit / nkc, kc = unit - rb * nkc;
+    const uint8_t* u = tiled + (size_t)unit * W4_UNIT;
+    uint4 wv[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) wv[q] = __ldcs(reinterpret_cast<const uint4*>(u) + q * 32 + lane);
+    const uint4 sc = __ldcs(reinterpret_cast<const uint4*>(u + 4096) + g);  // fp16 (row g, row g + 8) per group
+    const uint4 z0 = __ldcs(reinterpret_cast<const uint4*>(u + 4224));       // zero words: group, row half
+    const uint4 z1 = __ldcs(reinterpret_cast<const uint4*>(u + 4224) + 1);
+    uint16_t* row = out + ((size_t)rb * RB + g) * k + (size_t)kc * W4_KC + 8 * t;
+#pragma unroll
+    for (int grp = 0; grp < 4; ++grp) {
+      const uint32_t sw = u4c(sc, grp);
+      const float s_lo = half_bits_to_f32(uint16_t(sw & 0xffffu)), s_hi = half_bits_to_f32(uint16_t(sw >> 16));
+      const uint32_t zl = grp < 2 ? u4c(z0, 2 * grp) : u4c(z1, 2 * grp - 4);
+      const uint32_t zh = grp < 2 ? u4c(z0, 2 * grp + 1) : u4c(z1, 2 * grp - 3);
+      const int z_lo = int((zl >> (4 * g)) & 15u), z_hi = int((zh >> (4 * g)) & 15u);
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        const int m = 4 * grp + mm;
+        dq_pair(u4c(wv[m >> 1], (2 * m) & 3), u4c(wv[m >> 1], (2 * m + 1) & 3), s_lo, s_hi, z_lo, z_hi,
+                row + 32 * m, k);
+      }
     }
   }
-  const int64_t col = kc * S32_KC + 32 * m + 8 * t;
-  const int64_t r0 = rb * RB + g;
-  uint4 a, b;
-  a.x = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
-  a.y = uint32_t(lo[2]) | (uint32_t(lo[3]) << 16);
-  a.z = uint32_t(lo[4]) | (uint32_t(lo[5]) << 16);
-  a.w = uint32_t(lo[6]) | (uint32_t(lo[7]) << 16);
-  b.x = uint32_t(hi[0]) | (uint32_t(hi[1]) << 16);
-  b.y = uint32_t(hi[2]) | (uint32_t(hi[3]) << 16);
-  b.z = uint32_t(hi[4]) | (uint32_t(hi[5]) << 16);
-  b.w = uint32_t(hi[6]) | (uint32_t(hi[7]) << 16);
-  *reinterpret_cast<uint4*>(out + r0 * k + col) = a;
-  *reinterpret_cast<uint4*>(out + (r0 + 8) * k + col) = b;
+}
+
+// Units of a matrix.
+__host__ __device__ __forceinline__ int dequant_units(int64_t n, int64_t k, int fmt) {
+  return int((n / RB) * (k / (fmt == FMT_SYM32 ? S32_KC : W4_KC)));
+}
+__global__ void __launch_bounds__(256) dequant_f16_kernel(const uint8_t* __restrict__ tiled, int64_t n, int64_t k,
+                                                          int fmt, uint16_t* __restrict__ out) {
+  const int unit = int(blockIdx.x) * 8 + int(threadIdx.x >> 5);
+  if (unit < dequant_units(n, k, fmt)) dq_unit(tiled, k, fmt, unit, threadIdx.x & 31, out);
 }
 
 // ---------------------------------------------------------------------------
@@ -152,12 +147,14 @@ __global__ void dequant_s32_f16_kernel(const uint8_t* __restrict__ tiled, int64_
 // slices, warp 1 (one thread) issues the MMAs (four of K = 16 per slice) and
 // owns 2 BN tensor-memory columns (two accumulators, so the epilogue of a
 // tile overlaps the MMAs of the next), warps 2..5 read an accumulator back
-// (each its own 32 TMEM lanes = 32 rows) and write it.
+// (each its own 32 TMEM lanes = 32 rows) and write it, and warps 6..13 expand
+// later matrices of the sequence from int4 to fp16 meanwhile.
 constexpr int GM_BM = 128, GM_BK = 64;
 constexpr double GM_NARROW_COST = 0.77;  // time of a 128-wide tile / a 256-wide one (measured)
 constexpr double GM_SPLIT_COST = 1.1;    // time of a half-K tile / half a whole one (the reduction)
 constexpr int GM_A_BYTES = GM_BM * GM_BK * 2;
-constexpr int GM_THREADS = 192;
+constexpr int GM_EXP = 256;  // threads expanding later matrices (warps 6 ..)
+constexpr int GM_THREADS = 192 + GM_EXP;
 // Tile widths: 256 columns (4 stages), or 128 (6 stages) where the wider
 // tile would leave too much of the last wave of tiles idle.
 template <int BN>
@@ -181,6 +178,12 @@ struct GemmArgs {
   const float* row_scale;  // [M] or null: row m of the product is multiplied by it
   uint32_t* err;           // error word
   int ksplit;              // 1, or 2 (GE_F32 only): halves of K added into a zeroed out
+  // matrices to expand to fp16 while this product runs (their int4 units,
+  // shapes, fp16 destinations; nx_count of them, 0 .. 3)
+  int nx_count, nx_fmt;
+  const uint8_t* nx_blob[3];
+  int64_t nx_n[3], nx_k[3];
+  uint16_t* nx_out[3];
 };
 
 // Bounded wait on an mbarrier phase; gives up (setting the CTA's abort flag
@@ -330,6 +333,17 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
           break;
         }
       }
+    }
+  } else if (warp >= 6) {
+    // ---- warps 6..13: later matrices' fp16 expansion, this CTA's share ----
+    // (HBM-bound work under the tensor-bound product; the GEMMs that read
+    // them run later on the same stream).  One unit per warp at a time.
+    const int ew = int(blockIdx.x) * (GM_EXP / 32) + (warp - 6), nw = int(gridDim.x) * (GM_EXP / 32);
+#pragma unroll 1
+    for (int mi = 0; mi < g.nx_count; ++mi) {
+      const int units = dequant_units(g.nx_n[mi], g.nx_k[mi], g.nx_fmt);
+#pragma unroll 1
+      for (int unit = ew; unit < units; unit += nw) dq_unit(g.nx_blob[mi], g.nx_k[mi], g.nx_fmt, unit, lane, g.nx_out[mi]);
     }
   } else {
     // ---- epilogue: warps 2..5, TMEM lanes 32 (warp % 4) .. + 31 ----
@@ -1364,13 +1378,8 @@ static cudaError_t launch_flash_tc(const uint16_t* q, const uint16_t* kc, const 
 }
 
 cudaError_t launch_dequant_f16(const uint8_t* tiled, int64_t n, int64_t k, int fmt, uint16_t* out, cudaStream_t st) {
-  if (fmt == FMT_SYM32) {
-    const int64_t total = (n / RB) * (k / S32_KC) * 256;
-    dequant_s32_f16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(tiled, n, k, out);
-  } else {
-    const int64_t total = (n / RB) * (k / W4_KC) * 512;
-    dequant_f16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(tiled, n, k, out);
-  }
+  const int units = dequant_units(n, k, fmt);
+  dequant_f16_kernel<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(tiled, n, k, fmt, out);
   return cudaGetLastError();
 }
 
@@ -1417,7 +1426,9 @@ int gemm_ksplit(int M, int N, int K, int bn, int epi, int n_sms) {
 
 // C = A[M, K] . B[N, K]^T; A, B fp16 K-major (16-byte aligned, K % 64 == 0).
 cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, int K, int epi, void* out, int ldo,
-                            const float* row_scale, uint32_t* err, int n_sms, cudaStream_t st) {
+                            const float* row_scale, uint32_t* err, int n_sms, cudaStream_t st, int nx_count,
+                            const uint8_t* const* nx_blob, const int64_t* nx_n, const int64_t* nx_k, int nx_fmt,
+                            uint16_t* const* nx_out) {
   CUtensorMap ma;
   const cudaError_t e = make_map(&ma, A, M, K, GM_BM);
   if (e != cudaSuccess) return e;
@@ -1430,6 +1441,15 @@ cudaError_t launch_gemm_f16(const uint16_t* A, const uint16_t* B, int M, int N, 
   g.out = out;
   g.row_scale = row_scale;
   g.err = err;
+  if (nx_count < 0 || nx_count > 3) return cudaErrorInvalidValue;
+  g.nx_count = nx_count;
+  g.nx_fmt = nx_fmt;
+  for (int i = 0; i < 3; ++i) {
+    g.nx_blob[i] = i < nx_count ? nx_blob[i] : nullptr;
+    g.nx_n[i] = i < nx_count ? nx_n[i] : 0;
+    g.nx_k[i] = i < nx_count ? nx_k[i] : 0;
+    g.nx_out[i] = i < nx_count ? nx_out[i] : nullptr;
+  }
   const int bn = gemm_tile_width(M, N, n_sms);
   g.ksplit = gemm_ksplit(M, N, K, bn, epi, n_sms);
   if (g.ksplit > 1) {
