@@ -141,9 +141,9 @@ __global__ void __launch_bounds__(256) dequant_f16_kernel(const uint8_t* __restr
 // GEMM on the tcgen05 tensor cores: D[M, N] = A[M, K] . B[N, K]^T, fp16 in,
 // fp32 accumulation in tensor memory
 // ---------------------------------------------------------------------------
-// Persistent: one CTA per SM walks output tiles of 128 x BN (M-blocks of one
-// N-column consecutive, so the CTAs running together share the B panels in
-// L2).  Warp 0 (one thread) issues the TMA loads of a ring of 64-column K
+// Persistent: one CTA per SM walks output tiles of 128 x BN (groups of 16
+// M-blocks, M-block-fastest, so the CTAs running together share the A and B
+// panels in L2).  Warp 0 (one thread) issues the TMA loads of a ring of 64-column K
 // slices, warp 1 (one thread) issues the MMAs (four of K = 16 per slice) and
 // owns 2 BN tensor-memory columns (two accumulators, so the epilogue of a
 // tile overlaps the MMAs of the next), warps 2..5 read an accumulator back
@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(256) dequant_f16_kernel(const uint8_t* __restr
 constexpr int GM_BM = 128, GM_BK = 64;
 constexpr double GM_NARROW_COST = 0.77;  // time of a 128-wide tile / a 256-wide one (measured)
 constexpr double GM_SPLIT_COST = 1.1;    // time of a half-K tile / half a whole one (the reduction)
+constexpr int GM_GROUP = 16;             // M-blocks per group of the tile order
 constexpr int GM_A_BYTES = GM_BM * GM_BK * 2;
 constexpr int GM_EXP = 256;  // threads expanding later matrices (warps 6 ..)
 constexpr int GM_THREADS = 192 + GM_EXP;
@@ -224,7 +225,18 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = (g.M + GM_BM - 1) / GM_BM, nt = (g.N + GM_BN - 1) / GM_BN;
   const int ntiles = mt * nt * g.ksplit, nkb = g.K / GM_BK;
-  // tile t: M-block t % mt, N-block (t / mt) % nt, K part t / (mt nt)
+  // tile t: K part t / (mt nt); within a part, groups of GM_GROUP M-blocks
+  // walk their N-blocks M-block-fastest, so the ~148 tiles in flight cover a
+  // block of about 16 x 9 tiles and read about half the operand bytes of a
+  // whole column of M-blocks
+  auto tile_mn = [&](int t, int& mb, int& nb) {
+    const int r = t % (mt * nt);
+    const int grp = r / (GM_GROUP * nt), first = grp * GM_GROUP;
+    const int gm = min(GM_GROUP, mt - first);
+    const int rr = r - first * nt;
+    mb = first + rr % gm;
+    nb = rr / gm;
+  };
   auto krange = [&](int t, int& kb0, int& kb1) {
     const int ks = t / (mt * nt);
     kb0 = ks * nkb / g.ksplit;
@@ -263,8 +275,8 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
       bool ok = true;
 #pragma unroll 1
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const int mb = t % mt, nb = (t / mt) % nt;
-        int kb0, kb1;
+        int mb, nb, kb0, kb1;
+        tile_mn(t, mb, nb);
         krange(t, kb0, kb1);
 #pragma unroll 1
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -351,7 +363,8 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
     int local = 0;
 #pragma unroll 1
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
-      const int mb = t % mt, nb = (t / mt) % nt;
+      int mb, nb;
+      tile_mn(t, mb, nb);
       const int buf = local & 1;
       const uint32_t use = uint32_t(local >> 1);
       if (!gm_wait(tfull + buf, use & 1u, abort_flag, g.err)) break;
@@ -1233,16 +1246,21 @@ __global__ void __launch_bounds__(RT) qk_rows_kernel(const __grid_constant__ QkA
   sk = block_sum(sk, red);
   const float rq = rsqrtf(sq / float(qd) + a.eps), rk = rsqrtf(sk / float(kd) + a.eps);
   const int pos = a.start + t;
-  for (int idx = threadIdx.x; idx < (a.nq + a.nkv) * H2; idx += RT) {
-    const bool isq = idx < a.nq * H2;
-    const int j = isq ? idx : idx - a.nq * H2;
-    const int hh = j / H2, i = j - hh * H2;
+  // the rotation of pair i at this position, shared by every head
+  __shared__ float2 rot[64];
+  for (int i = threadIdx.x; i < H2; i += RT) {
     const double ang = double(pos) * a.f[i];
     const double rr = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
     float sn, cs;
     sincosf(float(rr), &sn, &cs);
-    cs *= a.ms;
-    sn *= a.ms;
+    rot[i] = make_float2(cs * a.ms, sn * a.ms);
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < (a.nq + a.nkv) * H2; idx += RT) {
+    const bool isq = idx < a.nq * H2;
+    const int j = isq ? idx : idx - a.nq * H2;
+    const int hh = j / H2, i = j - hh * H2;
+    const float cs = rot[i].x, sn = rot[i].y;
     if (isq) {
       const int c = hh * a.hd + i;
       const float x1 = y[c] * rq * a.qg[c], x2 = y[c + H2] * rq * a.qg[c + H2];
