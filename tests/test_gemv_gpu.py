@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import quant
+from oracle import fast, quant
 from w4_weight_only_b200 import synth
 from helpers import max_rel_to_rms, np64
 
@@ -53,15 +53,20 @@ FULL = [("qkv", 7168, 5120), ("o", 5120, 5120), ("gate_up", 55296, 5120), ("down
 @pytest.mark.parametrize("name,n,k", FULL)
 @pytest.mark.parametrize("batch", [1, 4, 16])
 def test_gemv_full_size_sampled(built_lib, cuda, name, n, k, batch):
-    """Full-size launch (the benchmark's configuration); the oracle computes 96
-    sampled output rows one by one, including the first and last row blocks."""
+    """Full-size launch (the benchmark's configuration): every output row
+    against the oracle's vectorised dequantization (``oracle.fast``, equal
+    bit for bit to ``oracle.quant``), and 96 sampled rows, the first and last
+    row blocks included, through ``oracle.quant`` itself."""
     api, _ = _api()
     W, x = synth.gemv_case(21, n, k, batch, "cuda")
     lin = api.quantize_linear(W)
     y = api.gemv(lin, x).cpu().numpy()
+    Wc, xc = W.cpu(), x.cpu()
+    ref_all = np64(xc) @ fast.dense_matrix(Wc).T
+    assert max_rel_to_rms(y, ref_all) <= TOL
     g = torch.Generator().manual_seed(n + k)
     rows = torch.cat([torch.arange(16), torch.arange(n - 16, n), torch.randint(0, n, (64,), generator=g)])
-    ref = _ref_rows(W.cpu(), x.cpu(), rows.numpy())
+    ref = _ref_rows(Wc, xc, rows.numpy())
     assert max_rel_to_rms(y[:, rows.numpy()], ref) <= TOL
 
 
