@@ -253,11 +253,7 @@ constexpr int SM_QF = SM_XS + NW * ATT_PW * 4;            // q fragments (4 KB)
 constexpr int SM_ASCR = SM_QF + 4096;                     // k, v rows fp32 [2][128], sums [2][NW]
 static_assert(NW * 64 * 3 * 4 <= NW * ATT_PW * 4, "piece-merge scratch inside the warp partials");
 static_assert(SM_ASCR + 2 * 128 * 4 + 2 * NW * 4 <= SM_XS + X_REGION, "attention scratch");
-// row blocks a GEMV phase's CTA sums at its end [1 + RBL_MAX]: in the q
-// region, which only attention phases use
-constexpr int SM_RBL = SM_QS;
-constexpr int RBL_MAX = 127;
-static_assert((1 + RBL_MAX) * 4 <= MAX_GQ * 128 * 4, "row-block list");
+
 
 extern __shared__ __align__(128) uint8_t w4a_smem[];
 
@@ -1790,58 +1786,57 @@ __device__ __forceinline__ float slab_total(const PD& d, int b, int r, int B) {
 }
 
 // After a warp has written the partial rows of segment (slab, row block rb)
-// of a GEMV that sums its own slabs: count the row block's arrivals; the CTA
-// whose arrival completes the row block sums its ns slabs in slab order (the
-// same order whichever CTA arrives last, so the sums are bit-reproducible),
-// at the end of its unit loop with all its threads (rb_sum_pending), and
-// clears the counter for the next layer.  Release: every lane's stores, a
-// fence each, the warp barrier, one atomic add; acquire: the atomic, a fence,
-// the CTA barrier, L2 loads.
+// of a GEMV that sums its own slabs: count the row block's arrivals (release:
+// every lane's stores, a fence each, the warp barrier, one atomic add).
 __device__ __forceinline__ void rb_sum(const PD& d, int rb, int B, int lane) {
   if (d.lpart == nullptr || d.epi != EPI_PART) return;
   uint32_t* ctr = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(d.kc)) + rb;
   __threadfence();
   __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    last = int(atomicAdd(ctr, 1u)) == d.g.ns - 1;
-    if (last) {
-      __threadfence();
-      *ctr = 0u;
-      int* list = sm_at<int>(SM_RBL);
-      const int i = atomicAdd(list, 1);
-      if (i < RBL_MAX) {
-        list[1 + i] = rb;
-        last = 0;  // summed at the phase end
-      }
-    }
-  }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (!last) return;
-  // the CTA's list is full: this warp sums the row block now
-  float* sum = const_cast<float*>(d.lpart);
-#pragma unroll 1
-  for (int i = lane; i < RB * B; i += 32) {
-    const int r = rb * RB + (i & (RB - 1)), b = i / RB;
-    if (r < d.rows_valid) sum[(size_t)b * d.ostride + r] = slab_total(d, b, r, B);
-  }
+  if (lane == 0) atomicAdd(ctr, 1u);
 }
 
-// The row blocks this CTA completed: every math thread takes (row block,
-// output) pairs.  Called by all math threads after a CTA barrier.
+// At the phase end, CTA c sums row blocks c, c + nc, ... (all its math
+// threads, each block's ns slabs in slab order, so the sums are the same
+// whichever CTA runs them): thread 0 waits (bounded) until every slab of the
+// block has arrived (acquire), then the block is summed and its counter
+// cleared for the next layer.  A fixed share per CTA: the CTAs that emit a
+// block's last slab are not the ones left to sum it, so no CTA gathers a long
+// tail of blocks.  Called by all math threads after a CTA barrier.
 __device__ __forceinline__ void rb_sum_pending(const PD& d) {
-  int* list = sm_at<int>(SM_RBL);
-  const int n = min(list[0], RBL_MAX);
-  const int B = lc().B, per = RB * B;
+  const LC& L = lc();
+  const int B = L.B, per = RB * B, nrb = d.g.nrb;
+  uint32_t* ctr = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(d.kc));
   float* sum = const_cast<float*>(d.lpart);
 #pragma unroll 1
-  for (int i = threadIdx.x; i < n * per; i += NT) {
-    const int rb = list[1 + i / per], j = i - (i / per) * per;
-    const int r = rb * RB + (j & (RB - 1)), b = j / RB;
-    if (r < d.rows_valid) sum[(size_t)b * d.ostride + r] = slab_total(d, b, r, B);
+  for (int rb = blockIdx.x; rb < nrb; rb += gridDim.x) {
+    if (threadIdx.x == 0) {
+      int ok = 1;
+      const long long t0 = clock64();
+      while (ld_acquire(ctr + rb) < uint32_t(d.g.ns)) {
+        if (ld_volatile_u32(L.ctl + 2) != 0u) {  // another CTA gave up: its slab may never come
+          ok = 0;
+          break;
+        }
+        if (clock64() - t0 > L.wait_bar) {
+          set_error(EW_BARRIER_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+      flags()[2] = ok;
+    }
+    cbar();
+    if (flags()[2]) {
+#pragma unroll 1
+      for (int i = threadIdx.x; i < per; i += NT) {
+        const int r = rb * RB + (i & (RB - 1)), b = i / RB;
+        if (r < d.rows_valid) sum[(size_t)b * d.ostride + r] = slab_total(d, b, r, B);
+      }
+    }
+    cbar();
+    if (threadIdx.x == 0) ctr[rb] = 0u;
   }
-  cbar();
-  if (threadIdx.x == 0) list[0] = 0;
 }
 
 // A segment piece leaves the warp: undo the range scaling, then emit it
@@ -1995,9 +1990,6 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
     a = b = 0;
     klen = 0;
   }
-  // the list of row blocks to sum shares memory with attention phases: clear
-  // it here (the staging's closing barrier orders this before any append)
-  if (tid == 0 && d.lpart != nullptr && d.epi == EPI_PART) sm_at<int>(SM_RBL)[0] = 0;
   stage_x<NB>(d, kbase, klen);
   if (d.kind == PK_GEMV_W4 || d.kind == PK_GEMV_S32) {
     const uint32_t* xmax = reinterpret_cast<const uint32_t*>(red() + 32);
@@ -2726,7 +2718,6 @@ __device__ __noinline__ void setup(const EngineParams& P) {
     fence_mbar_init();
   }
   if (tid < 128) sm_at<double>(SM_ROPE)[tid] = P.inv_freq[tid >> 6][tid & 63];
-  if (tid == 0) sm_at<int>(SM_RBL)[0] = 0;
   const int B = P.B;
   if (P.mode != MODE_GEMV && tid < B) posb()[tid] = (P.pos_const >= 0) ? P.pos_const : P.pos[tid];
   __syncthreads();
