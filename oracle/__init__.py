@@ -27,12 +27,12 @@ pages that define the method:
   terms and wrong indices.
 * ``sampling`` -- temperature / top-p (nucleus) sampling of one token with the
   draw passed in (ATLAS model card, "Benchmarks" and "Prompting guide for
-  Think models": temperature 0.6, top-p 0.95); the device side is not built
-  yet.
+  Think models": temperature 0.6, top-p 0.95).
 
 Parity status per function is stated in each module header.  Every function is
-pinned by a ``-m "not gpu"`` test except the end-to-end logits, whose
-conventions (rotation pairing, YaRN ramp, final norm) are readings of pages
-that print no worked example: "parity unpinned" beyond the invariants listed in
-``model``.
+pinned by a ``-m "not gpu"`` test.  The decoder's conventions that the pages
+state only in prose (rotation pairing, YaRN ramp, where RMSNorm adds eps, the
+final norm, the window counting the current token) are pinned, besides the
+invariants listed in ``model``, against the independent OLMo 3 implementation
+of the ``transformers`` package run in float64 on the same weights.
 """
