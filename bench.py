@@ -230,22 +230,67 @@ class OracleSample:
         self.qg = synth.normal((qd,), "cpu", 0.1, 1.0, SEED, "oracle_sample_qg").double().numpy()
         self.kg = synth.normal((kvd,), "cpu", 0.1, 1.0, SEED, "oracle_sample_kg").double().numpy()
 
-    def step(self) -> float:
-        """Seconds of one token, estimated from one pass over the sample."""
-        om, cfg = self.om, self.cfg
+    def _attention(self) -> None:
+        q, k = self.om.qk_prep(self.ocfg, self.qr, self.kr, self.qg, self.kg, CTX, True)
+        self.om.gqa_decode(self.ocfg, q, self.kv.K[0][0], self.kv.V[0][0], CTX - 1, True)
+
+    def layer_seconds(self) -> float:
+        """Seconds of one layer, projected from one pass over the sample."""
         t_layer = 0.0
         for name, W in self.mats.items():
             t0 = time.perf_counter()
             W.matvec(self.xs[name])
             t_layer += (time.perf_counter() - t0) * self.scale[name]
         t0 = time.perf_counter()
-        q, k = om.qk_prep(self.ocfg, self.qr, self.kr, self.qg, self.kg, CTX, True)
-        om.gqa_decode(self.ocfg, q, self.kv.K[0][0], self.kv.V[0][0], CTX - 1, True)
-        t_layer += time.perf_counter() - t0
+        self._attention()
+        return t_layer + time.perf_counter() - t0
+
+    def step(self) -> float:
+        """Seconds of one token, estimated from one pass over the sample."""
+        t_layer = self.layer_seconds()
         t0 = time.perf_counter()
-        _ = self.head @ self.x[: cfg.d_model]
+        _ = self.head @ self.x[: self.cfg.d_model]
         t_head = (time.perf_counter() - t0) * self.head_scale
-        return cfg.n_layers * t_layer + t_head
+        return self.cfg.n_layers * t_layer + t_head
+
+    def full_token_check(self) -> dict:
+        """One token's work measured rather than projected by rows: one whole
+        layer through the oracle (each int4 matrix at its full size,
+        dequantize + float64 matvec, one at a time, then the layer's
+        attention over CTX keys) and the whole bf16 lm_head, timed once; the
+        token is that layer times the layer count (every layer has the same
+        shapes, and at CTX = the window a sliding-window layer attends as many
+        keys as a full one) plus the head.  Also returns the ratio to the
+        sample's projection (median of three), which the reference arm uses
+        to calibrate its per-step samples."""
+        from w4_weight_only_b200 import synth
+        projected = statistics.median(self.step() for _ in range(3))
+        cfg = self.cfg
+        d, qd, kvd, f = cfg.d_model, cfg.q_dim, cfg.kv_dim, cfg.ffn
+        shapes = {"qkv": (qd + 2 * kvd, d), "o": (d, qd), "gate_up": (2 * f, d), "down": (d, f)}
+        layer = 0.0
+        for name, (n, k) in shapes.items():
+            qw, sb, qz = (t.numpy() for t in synth.g128_storage(SEED, n, k, "oracle_full_layer", name))
+            W = self.om.W4Matrix(qw, sb.view(self.np.uint16), qz, n, k, cfg.group)
+            x = synth.normal((k,), "cpu", 1.0, 0.0, SEED, "oracle_full_layer_x", name).double().numpy()
+            t0 = time.perf_counter()
+            W.matvec(x)
+            layer += time.perf_counter() - t0
+            del W, qw, sb, qz
+        t0 = time.perf_counter()
+        self._attention()
+        layer += time.perf_counter() - t0
+        import torch
+        head = synth.normal((cfg.vocab, d), "cpu", 0.02, 0.0, SEED, "oracle_full_head").to(
+            torch.bfloat16).double().numpy()
+        t0 = time.perf_counter()
+        _ = head @ self.x[:d]
+        t_head = time.perf_counter() - t0
+        del head
+        token = cfg.n_layers * layer + t_head
+        return {"full_layer_s": round(layer, 3), "full_lm_head_s": round(t_head, 3), "token_s": round(token, 3),
+                "sample_projected_token_s": round(projected, 3),
+                "measured_over_projected": round(token / projected, 3)}
 
     def describe(self, steps: int) -> str:
         return (f"{steps} passes over a sample of one ctx-{CTX} token: the first {SAMPLE_ROWS} rows of each "
@@ -258,8 +303,7 @@ class OracleSample:
         t0 = time.perf_counter()
         for name, W in self.mats.items():
             W.matvec(self.xs[name])
-        q, k = self.om.qk_prep(self.ocfg, self.qr, self.kr, self.qg, self.kg, CTX, True)
-        self.om.gqa_decode(self.ocfg, q, self.kv.K[0][0], self.kv.V[0][0], CTX - 1, True)
+        self._attention()
         _ = self.head @ self.x[: self.cfg.d_model]
         return time.perf_counter() - t0
 
@@ -274,14 +318,16 @@ def oracle_threads() -> int:
         return torch.get_num_threads()
 
 
-def cpu_baseline(cfg, steps: int = 3):
+def cpu_baseline(cfg):
     S = OracleSample(cfg)
     S.step()
-    ts = [S.step() for _ in range(steps)]
-    per_token = statistics.median(ts)
-    return {"value": 1.0 / per_token, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
-            "projected": True, "measured_sample_s": round(S.sample_seconds(), 4),
-            "sample": S.describe(steps) + f"; host has {len(os.sched_getaffinity(0))} cores"}
+    chk = S.full_token_check()
+    return {"value": 1.0 / chk["token_s"], "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
+            "projected": "by layer count only", "full_token": chk,
+            "sample": f"one whole layer of the ctx-{CTX} token (the four int4 GEMVs at full size, dequantize + "
+                      f"float64 matvec, and the layer's QK-prep + GQA attention over {CTX} keys) and the whole "
+                      f"lm_head, timed once; the token is {cfg.n_layers} such layers plus the head; "
+                      f"host has {len(os.sched_getaffinity(0))} cores"}
 
 
 # ---------------------------------------------------------------------------
@@ -292,18 +338,24 @@ def run_reference(args, rank, world):
         return
     cfg = wc.olmo3_32b(args.layers)
     S = OracleSample(cfg)
+    S.step()
+    chk = S.full_token_check()          # once, before the steps: the calibration
+    factor = chk["measured_over_projected"]
     for _ in range(args.warmup):
         S.step()
-    ts = [S.step() for _ in range(args.steps)]
+    t_region = time.perf_counter()
+    ts = [S.step() * factor for _ in range(args.steps)]
+    t_region = time.perf_counter() - t_region
     per_token = sum(ts) / len(ts)
     v = 1.0 / per_token
     base = {"value": v, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle", "projected": True,
-            "measured_sample_s": round(S.sample_seconds(), 4),
-            "sample": S.describe(args.steps) + f"; host has {len(os.sched_getaffinity(0))} cores"}
+            "measured_sample_s": round(S.sample_seconds(), 4), "full_token": chk,
+            "sample": S.describe(args.steps) + f", times the ratio {factor} of one measured whole-layer token "
+                                                f"to its projection; host has {len(os.sched_getaffinity(0))} cores"}
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * per_token,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "projected": True,
+            "projected": True, "timed_region_wall_s": round(t_region, 3),
             "config": {"workload": f"OLMo-3-32B-shaped int4 (g128, fp16 scale, int4 zero) decode, "
                                    f"{cfg.n_layers} layers, batch 1, ctx {CTX}, greedy",
                        "batch": 1, "ctx": CTX, "layers": cfg.n_layers, "parallelism": "host cores"},

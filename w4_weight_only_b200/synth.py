@@ -115,6 +115,18 @@ def sym32_matrix(seed: int, n: int, k: int, device="cpu", *keys):
     return qw.to(torch.int32), s.to(torch.bfloat16)
 
 
+def g128_storage(seed: int, n: int, k: int, *keys):
+    """Storage of an int4 group-128 matrix with random contents, for timing
+    only: (qweight int32 [n, k/8] and qzeros int32 [k/128, n/8] of uniform
+    random bits, scales as fp16 bits [k/128, n] of 0.003 * (1 + 0.25 N(0, 1)),
+    kept positive), the size and layout of a quantized N(0, 0.02) matrix."""
+    g = _gen("cpu", seed, "g128_q", n, k, *keys)
+    qw = torch.randint(-(2 ** 31), 2 ** 31, (n, k // 8), generator=g, dtype=torch.int64).to(torch.int32)
+    qz = torch.randint(-(2 ** 31), 2 ** 31, (k // 128, n // 8), generator=g, dtype=torch.int64).to(torch.int32)
+    s = normal((k // 128, n), "cpu", 0.25, 1.0, seed, "g128_s", n, k, *keys).abs_().add_(0.05).mul_(0.003)
+    return qw, s.to(torch.float16).view(torch.int16), qz
+
+
 def sym32_layer(cfg, seed: int, l: int, device="cpu") -> dict:
     """Layer l in the symmetric group-32 format: checkpoint pairs for qkv
     [q+2kv, d] ([Q; K; V]), o, gate_up [2 ffn, d] ([gate; up]) and down,
