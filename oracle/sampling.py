@@ -19,7 +19,9 @@ token for token:
 
 Parity: pinned by tests/test_oracle_sampling.py (hand-computed cases,
 brute-force enumeration of tiny rows, the greedy limits, shift and
-temperature invariances, exact draw frequencies).
+temperature invariances, exact draw frequencies) and, for the nucleus and its
+renormalised probabilities, by the ``transformers`` package's own temperature
+and top-p logits processors (tests/test_oracle_library_sampling.py).
 """
 from __future__ import annotations
 
