@@ -274,8 +274,10 @@ static int ws_layout(int B, int nc, const Dims& dm, int attn, int decode, long l
   L->xA = put(decode ? (size_t)B * dm.d * 4 : 0);
   L->xB = put(decode ? (size_t)B * dm.d * 4 : 0);
   L->g_part = put(gemv_n > 0 ? (size_t)gs.ns * B * gemv_n * 4 : 0);
-  L->a_red = put(decode && g[1].ns > RED_NS ? (size_t)B * dm.d * 4 : 0);
-  L->f_red = put(decode && g[3].ns > RED_NS ? (size_t)B * dm.d * 4 : 0);
+  // summed rows [B][d], then the 16-row blocks' sums of squares [B][d / 16]
+  const size_t red_bytes = (size_t)B * dm.d * 4 + (size_t)B * ((dm.d + RB - 1) / RB) * 4;
+  L->a_red = put(decode && g[1].ns > RED_NS ? red_bytes : 0);
+  L->f_red = put(decode && g[3].ns > RED_NS ? red_bytes : 0);
   L->rb_ctr = put(decode ? (size_t)2 * MAX_RBC * 4 : 0);
   // phase descriptors: every phase of a decode step (standalone ops use at most two)
   L->plan = put(decode ? (size_t)(5 * dm.n_layers + 2) * sizeof(PD) : 2 * sizeof(PD));

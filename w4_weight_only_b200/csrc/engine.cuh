@@ -157,7 +157,12 @@ struct alignas(16) PD {
   const uint8_t* kc;             // attention K region; a GEMV summing its own slabs: its row-block counters
   const uint8_t* vc;             // attention V region
   uint16_t* aout;                // attention output [B][nq][hd]
-  const float* qpart;            // QKV slabs [qns][B][qkv_dim]
+  union {
+    const float* qpart;          // attention: QKV slabs [qns][B][qkv_dim]
+    const float* vsq;            // XS_RESID / XS_FINAL GEMV above 8 rows: the branch's sums of squares
+                                 // per (row, 16-row block) [B][nrb], published by a producer that sums
+                                 // its own slabs (null otherwise)
+  };
   const float* lpart;            // lm_head slabs [lns][B][vocab]; a GEMV summing its own slabs: the sums [B][ostride]
   const float* qnorm;            // QK-norm gains
   const float* knorm;
@@ -412,6 +417,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.xres = P.ws.xB;
     d.vpart = f_src;
     d.vns = f_ns;
+    d.vsq = red_dn ? P.ws.f_red + (size_t)B * dm : nullptr;
     d.vstride = dm;
     d.gain = P.layers[nl - 1].ffn_norm;
     d.gain2 = P.final_norm ? P.final_gain : nullptr;
@@ -465,6 +471,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
       d.xres = P.ws.xB;
       d.vpart = f_src;
       d.vns = f_ns;
+      d.vsq = red_dn ? P.ws.f_red + (size_t)B * dm : nullptr;
       d.vstride = dm;
       d.gain = P.layers[l - 1].ffn_norm;
     }
@@ -486,6 +493,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     if (red_o) {
       d.kc = reinterpret_cast<const uint8_t*>(P.ws.rb_ctr);
       d.lpart = P.ws.a_red;
+      d.aux = P.ws.a_red + (size_t)B * dm;  // its blocks' sums of squares (above 8 rows)
     }
   } else if (sub == 3) {
     d.blob = lw.gu;
@@ -497,6 +505,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     d.xres = P.ws.xA;
     d.vpart = red_o ? P.ws.a_red : P.ws.a_part;
     d.vns = red_o ? 1 : g_o.ns;
+    d.vsq = red_o ? P.ws.a_red + (size_t)B * dm : nullptr;
     d.vstride = dm;
     d.gain = lw.attn_norm;
     d.xdst = P.ws.xB;
@@ -530,6 +539,7 @@ __device__ __noinline__ void build_pd(const EngineParams& P, int p, PD* out) {
     if (red_dn) {
       d.kc = reinterpret_cast<const uint8_t*>(P.ws.rb_ctr + MAX_RBC);
       d.lpart = P.ws.f_red;
+      d.aux = P.ws.f_red + (size_t)B * dm;  // its blocks' sums of squares (above 8 rows)
     }
   }
 }
@@ -1236,7 +1246,7 @@ __device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
     // row (d % 256 == 0).  Up to two chunks per thread stay in registers.
     const int n8 = dm / 8, total8 = B * n8;
     const bool fin = (d.xsrc == XS_FINAL) && d.gain2 != nullptr;
-    const bool two = total8 <= 2 * NT;
+    const bool two = NB == 1 && total8 <= 2 * NT;  // never above 8 rows (B * d / 8 > 2 NT)
     const size_t sstride = (size_t)B * d.vstride;
     const int c0 = warp * 32 + lane, c1 = c0 + NT;
     const bool h0 = warp * 32 < total8, h1 = two && warp * 32 + NT < total8;
@@ -1246,7 +1256,31 @@ __device__ __forceinline__ void stage_x(const PD& d, int kbase, int klen) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) v0[i] = v1[i] = x0[i] = x1[i] = g0[i] = g1[i] = 0.f;
     // pass 1: branch sums (and, for up to two chunks, residual and gains in flight together)
-    if (two) {
+    if (NB > 1 && d.vsq != nullptr) {
+      // the producer published its blocks' sums of squares: warp w adds those
+      // of rows w, w + NW, ... (eight loads in flight per lane, then a fixed
+      // shuffle tree), so no CTA reads the whole branch output here
+      const int nrb = (dm + RB - 1) / RB;
+#pragma unroll 1
+      for (int bb = warp; bb < B; bb += NW) {
+        const float* q = d.vsq + (size_t)bb * nrb;
+        float sq = 0.f;
+#pragma unroll 1
+        for (int r0 = 0; r0 < nrb; r0 += 8 * 32) {
+          float t[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rb = r0 + i * 32 + lane;
+            t[i] = rb < nrb ? __ldcg(q + rb) : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sq += t[i];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) wsum[warp * MAX_B + bb] = sq;
+      }
+    } else if (two) {
       // the residual and gain only where this CTA uses x: its k-range and
       // its share of the residual copy (all of it for the final norm); the
       // sums of squares need every branch value
@@ -1802,7 +1836,12 @@ __device__ __forceinline__ void rb_sum(const PD& d, int rb, int B, int lane) {
 // block has arrived (acquire), then the block is summed and its counter
 // cleared for the next layer.  A fixed share per CTA: the CTAs that emit a
 // block's last slab are not the ones left to sum it, so no CTA gathers a long
-// tail of blocks.  Called by all math threads after a CTA barrier.
+// tail of blocks.  Above 8 rows the CTA also publishes the block's sum of
+// squares per row (the 16 summed values of a row, squared and added by a fixed
+// shuffle tree), so that the consumer's RMSNorm reads B * n / 16 floats
+// instead of the whole B x n output.  Called by all math threads after a CTA
+// barrier.
+template <int NB>
 __device__ __forceinline__ void rb_sum_pending(const PD& d) {
   const LC& L = lc();
   const int B = L.B, per = RB * B, nrb = d.g.nrb;
@@ -1828,10 +1867,29 @@ __device__ __forceinline__ void rb_sum_pending(const PD& d) {
     }
     cbar();
     if (flags()[2]) {
+      if constexpr (NB > 1) {
+        static_assert(RB * MAX_B <= NT && RB == 16, "one (row, block row) per math thread");
+        const int i = threadIdx.x;
+        float v = 0.f;
+        if (i < per) {
+          const int r = rb * RB + (i & (RB - 1)), b = i / RB;
+          if (r < d.rows_valid) {
+            v = slab_total(d, b, r, B);
+            sum[(size_t)b * d.ostride + r] = v;
+          }
+        }
+        if (d.aux != nullptr && i < ((per + 31) & ~31)) {  // whole warps; a half-warp holds one row's block
+          float q = v * v;
+#pragma unroll
+          for (int o = RB / 2; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+          if (i < per && (i & (RB - 1)) == 0) d.aux[(size_t)(i / RB) * nrb + rb] = q;
+        }
+      } else {
 #pragma unroll 1
-      for (int i = threadIdx.x; i < per; i += NT) {
-        const int r = rb * RB + (i & (RB - 1)), b = i / RB;
-        if (r < d.rows_valid) sum[(size_t)b * d.ostride + r] = slab_total(d, b, r, B);
+        for (int i = threadIdx.x; i < per; i += NT) {
+          const int r = rb * RB + (i & (RB - 1)), b = i / RB;
+          if (r < d.rows_valid) sum[(size_t)b * d.ostride + r] = slab_total(d, b, r, B);
+        }
       }
     }
     cbar();
@@ -2007,7 +2065,7 @@ __device__ __noinline__ void gemv_phase(const PD& d) {
   if (a < b) cta_combine<NB>(d);
   if (d.lpart != nullptr && d.epi == EPI_PART) {
     cbar();
-    rb_sum_pending(d);
+    rb_sum_pending<NB>(d);
   }
   mark(5);
 }

@@ -107,8 +107,9 @@ struct Workspace {
   float* xA;            // residual at the layer input [B][d]
   float* xB;            // residual after attention [B][d]
   float* g_part;        // standalone GEMV output when split [ns][B][n]
-  float* a_red;         // O output with its slabs summed by the producer [B][d] (many slabs)
-  float* f_red;         // down output with its slabs summed by the producer [B][d]
+  float* a_red;         // O output with its slabs summed by the producer [B][d] (many slabs), then the
+                        // 16-row blocks' sums of squares [B][d / 16] (written above 8 rows)
+  float* f_red;         // down output, the same layout
   uint32_t* rb_ctr;     // producer-side slab sums: arrivals per row block [2][MAX_RBC]
   void* plan;           // phase descriptors, one per phase of the launch
 };
