@@ -41,9 +41,9 @@ NOMINAL_HBM_GBS = 8000.0
 # benchmark model at ctx 4096 give the bytes per layer and the fixed part;
 # valid only for the engine code they were taken on (its hash with comments
 # and whitespace stripped).
-TRAFFIC_ENGINE_CODE = "57e2d32492d894c9"
-TRAFFIC_FIXED = 1.032719e9
-TRAFFIC_PER_LAYER = 0.270604e9
+TRAFFIC_ENGINE_CODE = "fd2d498d3fad205a"
+TRAFFIC_FIXED = 1.033945e9
+TRAFFIC_PER_LAYER = 0.270434e9
 
 
 def engine_code_hash(text: str) -> str:
