@@ -43,7 +43,7 @@ enum {
   W4A_ERR_ARG = -1,          /* null pointer or invalid enum */
   W4A_ERR_SHAPE = -2,        /* sizes the kernels do not support */
   W4A_ERR_ALIGN = -3,        /* pointer not 16-byte aligned */
-  W4A_ERR_UNSUPPORTED = -4,  /* valid request this build does not implement */
+  W4A_ERR_UNSUPPORTED = -4,  /* valid request the library does not implement */
   W4A_ERR_CUDA = -5,         /* a CUDA runtime call failed */
   W4A_ERR_WORKSPACE = -6,    /* workspace too small */
   W4A_ERR_KERNEL = -7,       /* device error word set (bad shape / position / fp16 overflow) */
