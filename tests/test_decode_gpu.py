@@ -188,6 +188,29 @@ def test_engine_32b_shape_batch16_ragged(pair32):
         _check_step(cfg, lg[b].cpu().numpy(), dump[:, b].cpu().numpy(), ref_lg[b], ref_hid[:, b], f"32b seq {b}")
 
 
+def test_engine_32b_shape_batch9_ragged(pair32):
+    """Nine sequences, the smallest batch of the two-tile path: O in 5 and
+    down in 27 k-slabs, both summed by the producing CTAs, which also publish
+    the row blocks' sums of squares for the next RMSNorm; with an odd batch
+    the last warp of those sums is half idle."""
+    from w4_weight_only_b200 import api
+    P = pair32
+    cfg = P.cfg
+    lens = [1 + 113 * b for b in range(9)]
+    cap = (max(lens) + 16) // 16 * 16
+    kv = api.KVCache(cfg, 9, cap)
+    okv = om.OracleKV(P.ocfg, 9, cap)
+    _fill_kv(P, kv, okv, lens)
+    toks = [int(t) for t in synth.token_ids(P.seed + 4, 9, cfg.vocab, "cpu")]
+    dump = torch.zeros((cfg.n_layers + 1, 9, cfg.d_model), dtype=torch.float32, device="cuda")
+    lg, nxt = P.gpu.decode_step(kv, torch.tensor(toks, dtype=torch.int32, device="cuda"),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), hidden_dump=dump)
+    ref_lg, ref_hid = om.decode_step(P.oracle, okv, toks, lens)
+    P.gpu.check(9)
+    for b in range(9):
+        _check_step(cfg, lg[b].cpu().numpy(), dump[:, b].cpu().numpy(), ref_lg[b], ref_hid[:, b], f"32b b9 seq {b}")
+
+
 def test_engine_32b_shape_batch4_ragged(pair32):
     """Batch 4 at the full shape, ragged cached lengths: the geometry changes
     with the batch (the down projection in nine k-slabs)."""
